@@ -1,0 +1,115 @@
+// Internal helpers shared by the libmoe.so translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/moe.h"
+
+#define MOE_CUDA_TRY(expr)                                  \
+    do {                                                    \
+        cudaError_t _e = (expr);                            \
+        if (_e != cudaSuccess) return MOE_ERR_CUDA;         \
+    } while (0)
+
+#define MOE_LAUNCH_CHECK() MOE_CUDA_TRY(cudaGetLastError())
+
+namespace moe {
+
+constexpr int kMaxExperts = 4096;
+constexpr int kMaxCapacity = 8192;
+constexpr int kMaxTopK = 32;
+
+static inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+__host__ __device__ static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+static inline bool shape_ok(const moe_shape* s)
+{
+    if (!s) return false;
+    if (s->layers <= 0 || s->experts <= 0 || s->experts > kMaxExperts) return false;
+    if ((int64_t)s->layers * s->experts >= 65536) return false;
+    if (s->hidden <= 0 || s->hidden % 64 || s->ffn <= 0 || s->ffn % 64) return false;
+    if (s->top_k <= 0 || s->top_k > s->experts || s->top_k > kMaxTopK) return false;
+    if (s->wfmt < MOE_W_BF16 || s->wfmt > MOE_W_NVFP4) return false;
+    return true;
+}
+
+// ---------------------------------------------------------------- blob layout
+// One packed expert (= one slot).  Matrices are cut into tiles of 16 rows x
+// 64 columns; tile (rt, kt) of a [R][K] matrix sits at index rt*(K/64)+kt.
+// Inside a tile, lane L = 4g+t of a warp owns rows g and g+8, columns
+// [16t, 16t+16): FP4 tiles store for each lane 8 bytes of row g then 8
+// bytes of row g+8 (512 B per tile), BF16 tiles 32 bytes of row g then 32
+// bytes of row g+8 (2048 B per tile).  The W13 rows are reordered so that
+// row tile rt holds gate rows f = 8rt..8rt+7 in its rows 0..7 and the
+// matching up rows in rows 8..15.  FP4 scale tiles: MXFP4 32 B
+// [g][(g,b0),(g,b1),(g+8,b0),(g+8,b1)], NVFP4 64 B
+// [g][(g,b0..b3),(g+8,b0..b3)] with b the 32- or 16-column block inside
+// the tile.  NVFP4 ends with the two fp32 tensor scales.
+struct BlobLayout {
+    size_t w13, w2, s13, s2, ts, bytes;
+    int tile_bytes;    // 512 (FP4) or 2048 (BF16)
+    int stile_bytes;   // 32 (MXFP4), 64 (NVFP4), 0 (BF16)
+};
+
+static inline BlobLayout blob_layout(const moe_shape* s)
+{
+    BlobLayout b{};
+    size_t H = s->hidden, F = s->ffn;
+    if (s->wfmt == MOE_W_BF16) {
+        b.tile_bytes = 2048;
+        b.stile_bytes = 0;
+        b.w13 = 0;
+        b.w2 = 2 * F * H * 2;
+        b.s13 = b.s2 = b.ts = b.w2 + H * F * 2;
+        b.bytes = align_up(b.s13, 128);
+        return b;
+    }
+    size_t per_scale = (s->wfmt == MOE_W_MXFP4) ? 32 : 16;
+    b.tile_bytes = 512;
+    b.stile_bytes = (s->wfmt == MOE_W_MXFP4) ? 32 : 64;
+    b.w13 = 0;
+    b.w2 = 2 * F * H / 2;
+    b.s13 = b.w2 + H * F / 2;
+    b.s2 = b.s13 + 2 * F * H / per_scale;
+    b.ts = b.s2 + H * F / per_scale;
+    b.bytes = align_up(b.ts + (s->wfmt == MOE_W_NVFP4 ? 8 : 0), 128);
+    return b;
+}
+
+// ---------------------------------------------------------------- device helpers
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f)
+{
+    __nv_bfloat16 h = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t lane_id()
+{
+    uint32_t l;
+    asm volatile("mov.u32 %0, %%laneid;" : "=r"(l));
+    return l;
+}
+
+}  // namespace moe
+
+// ---------------------------------------------------------------- internal launchers
+namespace moe {
+int launch_router(const void* x, int x_dtype, const uint16_t* wg, const float* bias, int n, int H,
+                  int E, int k, float* logits, int32_t* idx, float* w, cudaStream_t st);
+size_t permute_ws_bytes(int n, int E, int k);
+int launch_permute(const int32_t* idx, int n, int E, int k, const void* x, int x_dtype, int H,
+                   int32_t* offsets, int32_t* row_of, int32_t* assign_of, uint16_t* x_perm, void* ws,
+                   cudaStream_t st);
+size_t ffn_ws_bytes(const moe_shape* s, int rows);
+int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
+               const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,
+               cudaStream_t st);
+int launch_combine(const uint16_t* y_perm, const int32_t* row_of, const float* w, int n, int k, int H,
+                   void* out, int out_dtype, cudaStream_t st);
+}  // namespace moe

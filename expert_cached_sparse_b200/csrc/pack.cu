@@ -1,0 +1,131 @@
+// Host-side packing of one expert from the canonical layout into the slot
+// blob the kernels stream.  The pages describe a runtime weight format that
+// stores expert banks "in the runtime's layout" so start-up needs no tensor
+// discovery or repacking ("FreeToken linux", section "Prepara los pesos del
+// modelo"; "FreeToken 290b model", section "Identifica el modelo y el
+// formato de expertos").  This is that layout for this library; one fill is
+// one contiguous copy of it.  The layout is described in common.cuh
+// (BlobLayout).
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+
+namespace {
+
+// canonical row of packed W13 row p: tile rows 0..7 gate f, 8..15 up f
+inline int w13_canon_row(int p, int F)
+{
+    int rt = p / 16, r = p % 16;
+    int f = 8 * rt + (r & 7);
+    return r < 8 ? f : F + f;
+}
+
+void pack_fp4_matrix(const uint8_t* q, int R, int K, bool w13, int F, uint8_t* out)
+{
+    const int KT = K / 64;
+    for (int rt = 0; rt < R / 16; rt++)
+        for (int kt = 0; kt < KT; kt++) {
+            uint8_t* tile = out + ((size_t)rt * KT + kt) * 512;
+            for (int L = 0; L < 32; L++) {
+                int g = L >> 2, t = L & 3;
+                for (int half = 0; half < 2; half++) {
+                    int p = 16 * rt + g + 8 * half;
+                    int cr = w13 ? w13_canon_row(p, F) : p;
+                    const uint8_t* src = q + (size_t)cr * (K / 2) + (64 * kt + 16 * t) / 2;
+                    memcpy(tile + 16 * L + 8 * half, src, 8);
+                }
+            }
+        }
+}
+
+void pack_fp4_scales(const uint8_t* sc, int R, int K, bool w13, int F, bool mx, uint8_t* out)
+{
+    const int KT = K / 64, per = mx ? 32 : 16, nb = K / per, bpt = 64 / per, stile = mx ? 32 : 64;
+    for (int rt = 0; rt < R / 16; rt++)
+        for (int kt = 0; kt < KT; kt++) {
+            uint8_t* tile = out + ((size_t)rt * KT + kt) * stile;
+            for (int g = 0; g < 8; g++)
+                for (int half = 0; half < 2; half++) {
+                    int p = 16 * rt + g + 8 * half;
+                    int cr = w13 ? w13_canon_row(p, F) : p;
+                    for (int b = 0; b < bpt; b++)
+                        tile[2 * bpt * g + bpt * half + b] = sc[(size_t)cr * nb + bpt * kt + b];
+                }
+        }
+}
+
+void pack_bf16_matrix(const uint16_t* w, int R, int K, bool w13, int F, uint8_t* out)
+{
+    const int KT = K / 64;
+    for (int rt = 0; rt < R / 16; rt++)
+        for (int kt = 0; kt < KT; kt++) {
+            uint8_t* tile = out + ((size_t)rt * KT + kt) * 2048;
+            for (int j = 0; j < 4; j++)
+                for (int L = 0; L < 32; L++) {
+                    int g = L >> 2, t = L & 3;
+                    for (int half = 0; half < 2; half++) {
+                        int p = 16 * rt + g + 8 * half;
+                        int cr = w13 ? w13_canon_row(p, F) : p;
+                        const uint16_t* src = w + (size_t)cr * K + 64 * kt + 16 * t + 4 * j;
+                        memcpy(tile + 512 * j + 16 * L + 8 * half, src, 8);
+                    }
+                }
+        }
+}
+
+bool mx_codes_ok(const uint8_t* sc, size_t n)
+{
+    for (size_t i = 0; i < n; i++)
+        if (sc[i] < 2 || sc[i] > 142) return false;
+    return true;
+}
+
+bool nv_codes_ok(const uint8_t* sc, size_t n)
+{
+    for (size_t i = 0; i < n; i++)
+        if ((sc[i] & 0x7F) == 0x7F) return false;   // S.1111.111 is NaN
+    return true;
+}
+
+}  // namespace
+
+extern "C" size_t moe_slot_bytes(const moe_shape* shape)
+{
+    if (!moe::shape_ok(shape)) return 0;
+    return moe::blob_layout(shape).bytes;
+}
+
+extern "C" int moe_pack_expert(const moe_shape* s, const void* h_w13, const uint8_t* h_w13_scales,
+                               const void* h_w2, const uint8_t* h_w2_scales, const float* h_tensor_scales,
+                               void* h_blob_out)
+{
+    if (!moe::shape_ok(s) || !h_w13 || !h_w2 || !h_blob_out) return MOE_ERR_INVALID_ARG;
+    const int H = s->hidden, F = s->ffn;
+    moe::BlobLayout bl = moe::blob_layout(s);
+    uint8_t* out = static_cast<uint8_t*>(h_blob_out);
+    memset(out, 0, bl.bytes);
+    if (s->wfmt == MOE_W_BF16) {
+        pack_bf16_matrix(static_cast<const uint16_t*>(h_w13), 2 * F, H, true, F, out + bl.w13);
+        pack_bf16_matrix(static_cast<const uint16_t*>(h_w2), H, F, false, F, out + bl.w2);
+        return MOE_OK;
+    }
+    if (!h_w13_scales || !h_w2_scales) return MOE_ERR_INVALID_ARG;
+    const bool mx = s->wfmt == MOE_W_MXFP4;
+    const size_t per = mx ? 32 : 16;
+    const size_t n13 = (size_t)2 * F * H / per, n2 = (size_t)H * F / per;
+    if (mx) {
+        if (!mx_codes_ok(h_w13_scales, n13) || !mx_codes_ok(h_w2_scales, n2)) return MOE_ERR_UNSUPPORTED;
+    } else {
+        if (!h_tensor_scales) return MOE_ERR_INVALID_ARG;
+        if (!nv_codes_ok(h_w13_scales, n13) || !nv_codes_ok(h_w2_scales, n2)) return MOE_ERR_UNSUPPORTED;
+        for (int i = 0; i < 2; i++)
+            if (!isfinite(h_tensor_scales[i])) return MOE_ERR_UNSUPPORTED;
+    }
+    pack_fp4_matrix(static_cast<const uint8_t*>(h_w13), 2 * F, H, true, F, out + bl.w13);
+    pack_fp4_matrix(static_cast<const uint8_t*>(h_w2), H, F, false, F, out + bl.w2);
+    pack_fp4_scales(h_w13_scales, 2 * F, H, true, F, mx, out + bl.s13);
+    pack_fp4_scales(h_w2_scales, H, F, false, F, mx, out + bl.s2);
+    if (!mx) memcpy(out + bl.ts, h_tensor_scales, 2 * sizeof(float));
+    return MOE_OK;
+}

@@ -1,0 +1,217 @@
+// Router: logits in a fixed fp32 order, then top-k and renormalised softmax
+// weights.  "A router activates only a small subset of experts per token"
+// ("FreeToken linux", section "Como gestiona FreeToken la memoria MoE").
+//
+// The logit order is part of the contract (it decides integer outputs):
+// for one (token, expert) pair, 32 lanes; lane l owns the 8-element chunks
+// l, l+32, ... of the hidden dimension and accumulates them with fused
+// multiply-adds in ascending order; an xor butterfly (16, 8, 4, 2, 1)
+// then sums the lanes, leaving the same value in all of them.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+// 8 activations of chunk c of token row xrow, widened exactly to fp32.
+template <bool XF32>
+__device__ __forceinline__ void load_x8(const void* xrow, int c, float v[8])
+{
+    if (XF32) {
+        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(xrow) + 8 * c);
+        float4 a = __ldg(p), b = __ldg(p + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+        uint4 q = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(xrow) + 8 * c));
+        uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+}
+
+// Warp per (token, group of EB experts).  TB tokens share each gate-row load.
+template <bool XF32, int TB, int EB>
+__global__ void __launch_bounds__(256) router_logits_kernel(const void* __restrict__ x,
+                                                            const uint16_t* __restrict__ wg,
+                                                            const float* __restrict__ bias, int n,
+                                                            int H, int E, float* __restrict__ logits)
+{
+    const int lane = threadIdx.x & 31;
+    const int warps_total = gridDim.x * (blockDim.x >> 5);
+    const int egroups = (E + EB - 1) / EB;
+    const int tgroups = (n + TB - 1) / TB;
+    const int chunks = H / 8;
+    const size_t xrow_bytes = (size_t)H * (XF32 ? 4 : 2);
+    for (int wi = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); wi < egroups * tgroups;
+         wi += warps_total) {
+        const int eg = wi % egroups, tg = wi / egroups;
+        float acc[TB][EB];
+#pragma unroll
+        for (int a = 0; a < TB; a++)
+#pragma unroll
+            for (int b = 0; b < EB; b++) acc[a][b] = 0.0f;
+        for (int c = lane; c < chunks; c += 32) {
+            float xv[TB][8];
+#pragma unroll
+            for (int a = 0; a < TB; a++) {
+                int t = tg * TB + a;
+                if (t < n) load_x8<XF32>(static_cast<const char*>(x) + (size_t)t * xrow_bytes, c, xv[a]);
+                else
+#pragma unroll
+                    for (int i = 0; i < 8; i++) xv[a][i] = 0.0f;
+            }
+#pragma unroll
+            for (int b = 0; b < EB; b++) {
+                int e = eg * EB + b;
+                if (e >= E) break;
+                uint4 q = __ldg(reinterpret_cast<const uint4*>(wg + (size_t)e * H + 8 * c));
+                uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+                float wv[8];
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    wv[2 * i] = __uint_as_float(w4[i] << 16);
+                    wv[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+                }
+#pragma unroll
+                for (int a = 0; a < TB; a++)
+#pragma unroll
+                    for (int i = 0; i < 8; i++) acc[a][b] = __fmaf_rn(xv[a][i], wv[i], acc[a][b]);
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < TB; a++)
+#pragma unroll
+            for (int b = 0; b < EB; b++)
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1)
+                    acc[a][b] = __fadd_rn(acc[a][b], __shfl_xor_sync(0xffffffffu, acc[a][b], off));
+        if (lane == 0) {
+#pragma unroll
+            for (int a = 0; a < TB; a++) {
+                int t = tg * TB + a;
+                if (t >= n) break;
+#pragma unroll
+                for (int b = 0; b < EB; b++) {
+                    int e = eg * EB + b;
+                    if (e >= E) break;
+                    logits[(size_t)t * E + e] = bias ? __fadd_rn(acc[a][b], __ldg(bias + e)) : acc[a][b];
+                }
+            }
+        }
+    }
+}
+
+// a ranks above b: larger logit; ties -> lower index; NaN below everything.
+__device__ __forceinline__ bool ranks_above(float a, int ia, float b, int ib)
+{
+    bool na = isnan(a), nb = isnan(b);
+    if (na != nb) return nb;
+    if (na) return ia < ib;
+    if (a != b) return a > b;
+    return ia < ib;
+}
+
+// Warp per token: k rounds of arg-max, then exp(l - lmax) renormalised.
+__global__ void __launch_bounds__(128) router_topk_kernel(const float* __restrict__ logits, int n,
+                                                          int E, int k, int32_t* __restrict__ idx,
+                                                          float* __restrict__ w)
+{
+    extern __shared__ unsigned char s_taken[];  // [warps][E]
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    unsigned char* taken = s_taken + (size_t)wib * E;
+    const int t = blockIdx.x * (blockDim.x >> 5) + wib;
+    if (t >= n) return;
+    const float* lt = logits + (size_t)t * E;
+    for (int e = lane; e < E; e += 32) taken[e] = 0;
+    __syncwarp();
+    float my_l = 0.0f;
+    int my_i = 0;
+    for (int r = 0; r < k; r++) {
+        float bv = 0.0f;
+        int bi = -1;
+        for (int e = lane; e < E; e += 32) {
+            if (taken[e]) continue;
+            float v = __ldg(lt + e);
+            if (bi < 0 || ranks_above(v, e, bv, bi)) { bv = v; bi = e; }
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (oi >= 0 && (bi < 0 || ranks_above(ov, oi, bv, bi))) { bv = ov; bi = oi; }
+        }
+        if (lane == 0) taken[bi] = 1;
+        if (lane == r) { my_l = bv; my_i = bi; }
+        __syncwarp();
+    }
+    const float lmax = __shfl_sync(0xffffffffu, my_l, 0);
+    float p = (lane < k) ? expf(my_l - lmax) : 0.0f;
+    float z = p;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+    if (lane < k) {
+        idx[(size_t)t * k + lane] = my_i;
+        w[(size_t)t * k + lane] = p / z;
+    }
+}
+
+template <bool XF32>
+int launch_logits(const void* x, const uint16_t* wg, const float* bias, int n, int H, int E,
+                  float* logits, cudaStream_t st)
+{
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int threads = 256, wpb = threads / 32;
+    if (n >= 64) {
+        constexpr int TB = 4, EB = 8;
+        long units = (long)((E + EB - 1) / EB) * ((n + TB - 1) / TB);
+        int grid = (int)((units + wpb - 1) / wpb);
+        if (grid > sms * 8) grid = sms * 8;
+        router_logits_kernel<XF32, TB, EB><<<grid, threads, 0, st>>>(x, wg, bias, n, H, E, logits);
+    } else {
+        constexpr int TB = 1, EB = 1;
+        long units = (long)E * n;
+        int grid = (int)((units + wpb - 1) / wpb);
+        if (grid > sms * 8) grid = sms * 8;
+        router_logits_kernel<XF32, TB, EB><<<grid, threads, 0, st>>>(x, wg, bias, n, H, E, logits);
+    }
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+}  // namespace
+
+int launch_router(const void* x, int x_dtype, const uint16_t* wg, const float* bias, int n, int H,
+                  int E, int k, float* logits, int32_t* idx, float* w, cudaStream_t st)
+{
+    if (n == 0) return MOE_OK;
+    int rc = (x_dtype == MOE_DT_F32) ? launch_logits<true>(x, wg, bias, n, H, E, logits, st)
+                                     : launch_logits<false>(x, wg, bias, n, H, E, logits, st);
+    if (rc) return rc;
+    const int wpb = 4;
+    size_t smem = (size_t)wpb * E;
+    router_topk_kernel<<<(n + wpb - 1) / wpb, wpb * 32, smem, st>>>(logits, n, E, k, idx, w);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+}  // namespace moe
+
+extern "C" int moe_router_topk(const void* d_x, int32_t x_dtype, const uint16_t* d_wg,
+                               const float* d_bias, int32_t n, int32_t hidden, int32_t experts,
+                               int32_t k, float* d_logits, int32_t* d_topk_idx, float* d_topk_w,
+                               void* stream)
+{
+    if (n < 0 || hidden <= 0 || hidden % 8 || experts <= 0 || experts > moe::kMaxExperts || k <= 0 ||
+        k > experts || k > moe::kMaxTopK)
+        return MOE_ERR_INVALID_ARG;
+    if (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
+    if (n > 0 && (!d_x || !d_wg || !d_logits || !d_topk_idx || !d_topk_w)) return MOE_ERR_INVALID_ARG;
+    if (((uintptr_t)d_x | (uintptr_t)d_wg) & 15) return MOE_ERR_INVALID_ARG;
+    return moe::launch_router(d_x, x_dtype, d_wg, d_bias, n, hidden, experts, k, d_logits,
+                              d_topk_idx, d_topk_w, moe::as_stream(stream));
+}

@@ -1,0 +1,299 @@
+/*
+ * moe.h -- C ABI of libmoe.so: a routed mixture-of-experts layer whose expert
+ * weights live in pinned host memory and are cached, whole (layer, expert)
+ * pair by pair, in a GPU-resident slot pool with one LRU policy shared by all
+ * layers.  Single GPU (NVIDIA B200, sm_100a).
+ *
+ * What the layer computes, and where the FreeToken pages state it:
+ *  - a router picks a few of many experts per token ("FreeToken linux",
+ *    section "Como gestiona FreeToken la memoria MoE": 6 of 256 routed
+ *    experts per layer for DeepSeek-V4-Flash);
+ *  - the full expert set stays in host RAM, VRAM holds expert slots used as
+ *    an LRU cache shared across MoE layers; a hit runs on the GPU, a miss is
+ *    brought in over PCIe (same section and its memory-tier table;
+ *    "FreeToken 290b model", section "Como gestiona FreeToken el prellenado
+ *    y la decodificacion");
+ *  - a cache entry is a logical (layer, expert) pair ("FreeToken rtx 4090",
+ *    section "Como funciona la jerarquia de memoria MoE");
+ *  - the cache can be resized at a scheduler safe point ("FreeToken
+ *    quantization", section "Flujo de configuracion de la cuantizacion de
+ *    FreeToken");
+ *  - expert weights come as MXFP4, NVFP4 or BF16 ("FreeToken quantization",
+ *    section "Formatos compatibles, hardware y perfil de rendimiento");
+ *  - host expert banks are stored in the runtime's own layout so no
+ *    repacking happens at start-up ("FreeToken linux", section "Prepara los
+ *    pesos del modelo", the FTW format): moe_pack_expert produces that layout.
+ * The pages print no formulas.  This library reads them as: softmax router
+ * followed by top-k and renormalisation over the chosen k; SwiGLU experts
+ * h = silu(W1 x) * (W3 x), y = W2 h; out = sum_j w_j y_j.
+ *
+ * Conventions for every entry point:
+ *  - d_ marks a device pointer, h_ a host pointer.  The caller allocates and
+ *    owns every buffer, device or host; the library never calls cudaMalloc,
+ *    cudaFree or cudaHostAlloc.  It creates CUDA events for the cache.
+ *  - `stream` arguments are cudaStream_t values passed as void*; NULL is the
+ *    legacy default stream.
+ *  - Work is enqueued asynchronously on the given stream unless stated.
+ *  - Every function returns a moe_status; nothing aborts or prints.
+ *    Argument errors are detected on the host before anything is enqueued.
+ *  - Row-major everywhere.  Integer tensors are int32.  bf16 tensors are
+ *    passed as uint16_t bit patterns.
+ *  - Limits: hidden % 64 == 0, ffn % 64 == 0, 1 <= top_k <= experts <= 4096,
+ *    capacity <= 8192, layers * experts < 65536.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,
+    MOE_ERR_CAPACITY = -2,   /* a call requests more distinct experts than slots */
+    MOE_ERR_CUDA = -3,       /* a CUDA runtime call or kernel launch failed */
+    MOE_ERR_FILL = -4,       /* a miss fill could not be issued */
+    MOE_ERR_TIMEOUT = -5,    /* reserved: a bounded device-side wait gave up */
+    MOE_ERR_UNSUPPORTED = -6,/* shape or scale codes outside what the kernels handle */
+    MOE_ERR_STATE = -7       /* the cache is in an unusable state */
+} moe_status;
+
+typedef enum { MOE_W_BF16 = 0, MOE_W_MXFP4 = 1, MOE_W_NVFP4 = 2 } moe_wfmt;
+typedef enum { MOE_DT_F32 = 0, MOE_DT_BF16 = 1 } moe_dtype;
+
+typedef struct {
+    int32_t layers;   /* L: MoE layers sharing one cache */
+    int32_t experts;  /* E: routed experts per layer */
+    int32_t hidden;   /* H */
+    int32_t ffn;      /* F: expert FFN width */
+    int32_t top_k;    /* k */
+    int32_t wfmt;     /* moe_wfmt */
+} moe_shape;
+
+typedef struct moe_cache moe_cache; /* opaque host-side handle */
+
+/* Cache trace events, in the order one lookup emits them: every HIT in
+ * ascending expert id, then for each miss in ascending expert id an EVICT
+ * of its victim (if the slot was taken) followed by its MISS.  A resize
+ * emits EVICT records for the surplus, then MOVE records for survivors
+ * whose slot number changes. */
+typedef enum { MOE_EV_HIT = 0, MOE_EV_MISS = 1, MOE_EV_EVICT = 2, MOE_EV_MOVE = 3 } moe_event;
+
+typedef struct {
+    uint32_t call;   /* LRU clock value of the call (1-based count of successful lookups) */
+    int32_t slot;    /* slot the event refers to (for MOVE: the new slot) */
+    uint16_t layer;  /* (layer, expert) key the event refers to */
+    uint16_t expert;
+    uint8_t event;   /* moe_event */
+    uint8_t pad[3];
+} moe_trace_rec;     /* 16 bytes */
+
+typedef struct {
+    uint64_t lookups;      /* successful lookup calls */
+    uint64_t hits;         /* requested (layer, expert) pairs found resident */
+    uint64_t misses;       /* requested pairs brought in */
+    uint64_t evictions;
+    uint64_t fill_bytes;   /* bytes copied host -> device by fills */
+    uint64_t host_syncs;   /* lookups that had to read the miss list on the host */
+    uint64_t trace_dropped;/* records lost because the trace buffer was full */
+} moe_cache_stats;
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_str(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int moe_version(void);
+
+/* ---------------------------------------------------------------- sizes */
+
+/* Bytes of one packed expert blob (= one slot), a multiple of 128.
+ * MXFP4, H=4096, F=2048: 13,369,344.  0 for an invalid shape. */
+size_t moe_slot_bytes(const moe_shape* shape);
+
+/* Device bytes the cache bookkeeping needs for `capacity` slots and a
+ * trace buffer of `trace_capacity` records. */
+size_t moe_cache_meta_bytes(const moe_shape* shape, int32_t capacity, int32_t trace_capacity);
+
+/* Device workspace bytes of moe_permute for n tokens. */
+size_t moe_permute_workspace_bytes(int32_t n, int32_t experts, int32_t top_k);
+
+/* Device workspace bytes of moe_grouped_ffn for `rows` permuted rows. */
+size_t moe_ffn_workspace_bytes(const moe_shape* shape, int32_t rows);
+
+/* Device workspace bytes of moe_layer_forward for n tokens. */
+size_t moe_layer_workspace_bytes(const moe_shape* shape, int32_t n);
+
+/* ---------------------------------------------------------------- packing */
+
+/*
+ * Host only.  Converts one expert from the canonical layout into the packed
+ * slot blob (the device layout the kernels stream; its internal order is
+ * private to this library and may change between versions).
+ * Canonical layout:
+ *   w13 [2F][H]: rows 0..F-1 gate W1, rows F..2F-1 up W3;  w2 [H][F].
+ *   FP4 formats: two E2M1 codes per byte along a row, even column in the low
+ *   nibble; w13_scales [2F][H/32] E8M0 (MXFP4) or [2F][H/16] E4M3 (NVFP4),
+ *   w2_scales likewise over F.  NVFP4 also takes tensor_scales = {s13, s2}
+ *   (fp32 scales of the whole W13 and W2); other formats ignore it (may be
+ *   NULL).  BF16: w13/w2 are uint16 bit patterns, scales NULL.
+ * blob_out: moe_slot_bytes(shape) bytes.
+ * Errors: MOE_ERR_UNSUPPORTED for NaN scale codes, MXFP4 scale codes
+ * outside [2, 142] (block scales 2^-125 .. 2^15) or non-finite NVFP4 tensor
+ * scales.
+ */
+int moe_pack_expert(const moe_shape* shape, const void* h_w13, const uint8_t* h_w13_scales,
+                    const void* h_w2, const uint8_t* h_w2_scales, const float* h_tensor_scales,
+                    void* h_blob_out);
+
+/* ---------------------------------------------------------------- cache */
+
+/*
+ * Creates a cache of `capacity` slots over the caller's device memory:
+ *   d_meta: moe_cache_meta_bytes() bytes, 256-byte aligned;
+ *   d_slot_pool: capacity * moe_slot_bytes() bytes, 256-byte aligned;
+ *   h_blobs: layers*experts pointers, h_blobs[l*E+e] = packed blob of expert
+ *   e of layer l in pinned host memory (the caller keeps the array and the
+ *   blobs alive and unchanged for the life of the cache; several keys may
+ *   point to the same blob).
+ * All slots start free (cold cache).  Initialises d_meta on `stream` and
+ * synchronises it.
+ */
+int moe_cache_create(const moe_shape* shape, void* d_meta, size_t meta_bytes, void* d_slot_pool,
+                     int32_t capacity, int32_t trace_capacity, const void* const* h_blobs,
+                     void* stream, moe_cache** out);
+
+/*
+ * Looks up the experts that `d_idx` (count entries, device, any order,
+ * duplicates allowed) requests for `layer`, updates the LRU state (the
+ * policy is stated on moe_trace_rec and below), records the trace, and
+ * brings every miss into its slot.
+ *   LRU: the clock advances by one per successful call; hits get the new
+ *   clock value; each miss (ascending expert id) takes the lowest free slot,
+ *   else evicts the resident key with the smallest (last use, slot) that
+ *   this call does not request.
+ * d_slot_of_expert [E] (device) receives the slot of each requested expert,
+ * -1 for the others.  Fills are issued on copy_stream after everything
+ * already on `stream` is done, and `stream` waits for them, so work enqueued
+ * on `stream` afterwards sees the weights.
+ * Blocks the host until the miss list is known, except when every expert of
+ * `layer` is already resident (then nothing is read back).
+ * MOE_ERR_CAPACITY if more distinct experts are requested than slots exist;
+ * the state is unchanged (the host learns this at the same sync point).
+ */
+int moe_cache_lookup_update(moe_cache* cache, int32_t layer, const int32_t* d_idx, int32_t count,
+                            int32_t* d_slot_of_expert, void* stream, void* copy_stream);
+
+/*
+ * Resizes the cache to new_capacity slots at a safe point: synchronises
+ * `stream`, evicts the least recently used surplus (by (last use, slot)),
+ * copies the survivors, packed to the front in old-slot order, into
+ * d_pool_new, and moves the bookkeeping to d_meta_new (either may equal the
+ * old buffer when large enough; the survivors only ever move to lower
+ * slots, so an in-place pool works).  Emits EVICT / MOVE trace records.
+ */
+int moe_cache_resize(moe_cache* cache, void* d_meta_new, size_t meta_bytes, void* d_pool_new,
+                     int32_t new_capacity, void* stream);
+
+/* Copies up to `cap` trace records, oldest first, into h_buf, reports how
+ * many in *n_out, and clears the device trace buffer.  Synchronous. */
+int moe_cache_read_trace(moe_cache* cache, moe_trace_rec* h_buf, size_t cap, size_t* n_out);
+
+/* Counters since creation.  Synchronous. */
+int moe_cache_get_stats(moe_cache* cache, moe_cache_stats* out);
+
+/* Host copies of the slot table [L*E], slot keys [C] (l*E+e or -1) and
+ * last-use stamps [C].  Any pointer may be NULL.  Synchronous. */
+int moe_cache_snapshot(moe_cache* cache, int32_t* h_slot_of, int32_t* h_key_of, uint64_t* h_stamp);
+
+int32_t moe_cache_capacity(const moe_cache* cache);
+
+/* Releases the host-side handle and its events (not the caller's memory). */
+int moe_cache_destroy(moe_cache* cache);
+
+/* ---------------------------------------------------------------- steps */
+
+/*
+ * Router.  d_x [n][hidden] (float32 or bf16 per x_dtype), d_wg [experts]
+ * [hidden] bf16, d_bias [experts] float32 or NULL.
+ *   logit[t][e] = fp32(sum_h x[t][h] * wg[e][h]) + bias[e], the sum formed in
+ *   a fixed order: 32 lanes, lane l accumulating with fused multiply-adds
+ *   over the 8-element chunks l, l+32, ... in ascending order, then an xor
+ *   butterfly (16, 8, 4, 2, 1) across the lanes.
+ *   d_topk_idx [n][k]: the k largest logits, descending; ties go to the
+ *   lower expert id; NaN ranks below -inf.
+ *   d_topk_w [n][k]: exp(l_j - l_max) / sum over the chosen k (softmax over
+ *   all experts renormalised over the top-k).
+ * d_logits [n][experts] float32 is scratch the caller provides, and holds
+ * the logits afterwards.
+ */
+int moe_router_topk(const void* d_x, int32_t x_dtype, const uint16_t* d_wg, const float* d_bias,
+                    int32_t n, int32_t hidden, int32_t experts, int32_t k, float* d_logits,
+                    int32_t* d_topk_idx, float* d_topk_w, void* stream);
+
+/*
+ * Token -> expert permutation.  Assignment a = t*k + j goes to expert
+ * idx[a].  d_expert_offsets [experts+1]: exclusive prefix sum of the
+ * per-expert counts; d_row_of [n*k]: row_of[a] = offsets[e] + number of
+ * earlier assignments to the same expert (stable); d_assign_of [n*k]: the
+ * inverse; d_x_perm [n*k][hidden] bf16: x_perm[row_of[a]] = bf16(x[a/k])
+ * (round to nearest even when x is float32).  d_ws: workspace of
+ * moe_permute_workspace_bytes() bytes.  An index outside [0, experts) is
+ * the caller's error: that assignment gets row_of = -1 and no row, and
+ * offsets[experts] counts only the valid ones.
+ */
+int moe_permute(const int32_t* d_topk_idx, int32_t n, int32_t experts, int32_t k, const void* d_x,
+                int32_t x_dtype, int32_t hidden, int32_t* d_expert_offsets, int32_t* d_row_of,
+                int32_t* d_assign_of, uint16_t* d_x_perm, void* d_ws, size_t ws_bytes,
+                void* stream);
+
+/*
+ * Grouped SwiGLU expert FFN over the permuted rows.  d_slot_pool holds
+ * pool_slots packed blobs of moe_slot_bytes() each.  For every expert e
+ * with rows [offsets[e], offsets[e+1]) (clipped to [0, rows)) and
+ * 0 <= d_slot_of_expert[e] < pool_slots, the weights are read from that
+ * slot and
+ *   h = silu(x W1^T) * (x W3^T)   (fp32 accumulation, h rounded to bf16),
+ *   y = h W2^T                    (fp32 accumulation, y rounded to bf16)
+ * is written to d_y_perm rows.  Rows of experts with any other slot value
+ * (-1 in particular) are left untouched, so hits and misses can run as two
+ * passes.  d_ws: moe_ffn_workspace_bytes() bytes (holds h).  FP4 weights are
+ * expanded exactly to bf16 (E2M1 times its block scale is exact there); the
+ * NVFP4 tensor scales are applied in fp32.
+ */
+int moe_grouped_ffn(const moe_shape* shape, const void* d_slot_pool, int32_t pool_slots,
+                    const int32_t* d_slot_of_expert, const int32_t* d_expert_offsets,
+                    const uint16_t* d_x_perm, int32_t rows, uint16_t* d_y_perm, void* d_ws,
+                    size_t ws_bytes, void* stream);
+
+/*
+ * Combine.  out[t] = sum over j = 0..k-1, in that order, of
+ * w[t][j] * y_perm[row_of[t*k+j]], accumulated in fp32 and stored as
+ * out_dtype.  Deterministic (no atomics).
+ */
+int moe_combine(const uint16_t* d_y_perm, const int32_t* d_row_of, const float* d_topk_w, int32_t n,
+                int32_t k, int32_t hidden, void* d_out, int32_t out_dtype, void* stream);
+
+/*
+ * The whole layer for `layer`: router -> cache lookup -> permute -> grouped
+ * FFN over the hits -> (fills of the misses on copy_stream, overlapped with
+ * the hit FFN) -> grouped FFN over the misses -> combine.
+ * d_x [n][H] (x_dtype), d_wg [E][H] bf16, d_bias [E] or NULL; d_out [n][H]
+ * in x_dtype.  d_ws: moe_layer_workspace_bytes() bytes.  d_topk_idx_out /
+ * d_topk_w_out ([n][k], device) receive the routing when not NULL.
+ * Blocks the host once, for the miss list, unless every expert of the layer
+ * is resident; in that case nothing is read back and the call can be
+ * captured in a CUDA graph.
+ */
+int moe_layer_forward(moe_cache* cache, int32_t layer, const void* d_x, int32_t x_dtype,
+                      const uint16_t* d_wg, const float* d_bias, int32_t n, void* d_out,
+                      void* d_ws, size_t ws_bytes, void* stream, void* copy_stream,
+                      int32_t* d_topk_idx_out, float* d_topk_w_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

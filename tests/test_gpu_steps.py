@@ -1,0 +1,195 @@
+"""GPU parity of the individual steps, called through the C ABI, against the
+CPU oracle on the same seeded inputs.
+
+Router: logits and top-k indices bit-exact, weights within tolerance.
+Permute: offsets / row_of / assign_of bit-exact, x_perm bit-exact.
+Grouped FFN: per-expert relative L2 against the fp64 oracle, all formats,
+ragged groups (0, 1, 7, 8, 9, 33, 70 rows), permuted slots, two passes.
+Combine: against the oracle combine of the same bf16 rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+from expert_cached_sparse_b200 import api as A
+from expert_cached_sparse_b200 import workloads as W
+
+from helpers import ALARM_REL_L2, TOL_REL_L2, Layer, bf16_bits, dev, host, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _x_dev(cfg, x):
+    return dev(x) if cfg.x_dtype == "bf16" else dev(x.astype(np.float32))
+
+
+# ------------------------------------------------------------------ router
+ROUTER_CASES = [(W.TINY, 64), (W.TINY, 1), (W.DS_DECODE, 1), (W.DS_DECODE, 4), (W.DS_DECODE, 16),
+                (W.DS_DECODE, 37), (W.DS_PREFILL, 300), (W.QWEN_BF16, 512), (W.QWEN_BF16, 8),
+                (W.TRACE40, 1)]
+
+
+@pytest.mark.parametrize("cfg,n", ROUTER_CASES, ids=lambda v: getattr(v, "name", str(v)))
+def test_router_parity(orc, cfg, n):
+    x = W.gen_x(cfg, 0, n, "router")
+    wg = W.gen_wg(cfg, 0, 0)
+    bias = W.gen_bias(cfg, 0, 0)
+    l_ref, i_ref, w_ref = orc.router(x, wg, bias, cfg.top_k)
+    E, k = cfg.experts, cfg.top_k
+    logits = torch.empty(n, E, dtype=torch.float32, device="cuda")
+    idx = torch.empty(n, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(n, k, dtype=torch.float32, device="cuda")
+    A.moe_router_topk(_x_dev(cfg, x), dev(wg), None if bias is None else dev(bias), n, cfg.hidden, E, k,
+                      logits, idx, w)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(logits).view(np.uint32), l_ref.view(np.uint32))
+    np.testing.assert_array_equal(host(idx), i_ref)
+    assert rel_l2(host(w), w_ref) < 1e-5
+
+
+def test_router_ties_nan_and_empty(orc):
+    cfg = W.scaled(W.TINY, hidden=64, experts=8, top_k=3)
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((6, 64)).astype(np.float32)
+    x[2, 5] = np.nan
+    wg = W.gen_wg(cfg, 0, 0)
+    wg[3] = wg[6]
+    wg[1] = wg[4]
+    l_ref, i_ref, w_ref = orc.router(x, wg, None, 3)
+    logits = torch.empty(6, 8, device="cuda")
+    idx = torch.empty(6, 3, dtype=torch.int32, device="cuda")
+    w = torch.empty(6, 3, device="cuda")
+    A.moe_router_topk(dev(x), dev(wg), None, 6, 64, 8, 3, logits, idx, w)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(idx), i_ref)
+    assert list(host(idx)[2]) == [0, 1, 2]
+    ok = ~np.isnan(w_ref)
+    np.testing.assert_allclose(host(w)[ok], w_ref[ok], rtol=1e-5)
+    A.moe_router_topk(dev(x), dev(wg), None, 0, 64, 8, 3, logits, idx, w)   # n = 0: no work
+
+
+# ------------------------------------------------------------------ permute
+PERM_CASES = [(1, 8, 2, "f32"), (64, 8, 2, "f32"), (5, 256, 6, "bf16"), (16, 256, 6, "bf16"),
+              (333, 128, 8, "bf16"), (4096, 256, 6, "bf16")]
+
+
+@pytest.mark.parametrize("n,E,k,xd", PERM_CASES)
+def test_permute_parity(orc, n, E, k, xd):
+    rng = np.random.default_rng(n * E)
+    H = 256
+    if n > 100:
+        # Zipf-like skew: a few experts take most rows
+        idx = np.minimum(E - 1, rng.zipf(1.3, size=(n, k)) - 1).astype(np.int32)
+    else:
+        idx = rng.integers(0, E, size=(n, k)).astype(np.int32)
+    xf = rng.standard_normal((n, H)).astype(np.float32)
+    x = xf if xd == "f32" else W.f32_to_bf16_bits(xf)
+    off_ref, row_ref, asg_ref = orc.permute(idx, E)
+    offs = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    row_of = torch.empty(n * k, dtype=torch.int32, device="cuda")
+    asg = torch.empty(n * k, dtype=torch.int32, device="cuda")
+    xp = torch.empty(n * k, H, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(A.moe_permute_workspace_bytes(n, E, k), dtype=torch.uint8, device="cuda")
+    A.moe_permute(dev(idx), n, E, k, dev(x), H, offs, row_of, asg, xp, ws)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(offs), off_ref)
+    np.testing.assert_array_equal(host(row_of), row_ref)
+    np.testing.assert_array_equal(host(asg), asg_ref)
+    xb = W.f32_to_bf16_bits(xf) if xd == "f32" else x
+    np.testing.assert_array_equal(bf16_bits(xp), xb[asg_ref // k])
+
+
+# ------------------------------------------------------------------ grouped FFN
+def _ffn_case(orc, cfg, counts, slots, pool_slots, seed=0, passes=1):
+    E = cfg.experts
+    L = Layer(cfg, seed)
+    shape = A.shape_of(cfg)
+    sb = A.moe_slot_bytes(shape)
+    pool = torch.zeros(pool_slots * sb, dtype=torch.uint8, device="cuda")
+    for e in range(E):
+        if slots[e] >= 0:
+            pool[slots[e] * sb:(slots[e] + 1) * sb].copy_(L.blob(0, e), non_blocking=False)
+    rows = int(sum(counts))
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    rng = np.random.default_rng(seed + 7)
+    xb = W.f32_to_bf16_bits(rng.standard_normal((rows, cfg.hidden)).astype(np.float32))
+    y = torch.full((rows, cfg.hidden), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(A.moe_ffn_workspace_bytes(shape, rows), dtype=torch.uint8, device="cuda")
+    sl = np.asarray(slots, np.int32)
+    if passes == 1:
+        A.moe_grouped_ffn(shape, pool, pool_slots, dev(sl), dev(offsets), dev(xb), rows, y, ws)
+    else:
+        half = np.where(np.arange(E) % 2 == 0, sl, -1).astype(np.int32)
+        other = np.where(np.arange(E) % 2 == 1, sl, -1).astype(np.int32)
+        A.moe_grouped_ffn(shape, pool, pool_slots, dev(half), dev(offsets), dev(xb), rows, y, ws)
+        A.moe_grouped_ffn(shape, pool, pool_slots, dev(other), dev(offsets), dev(xb), rows, y, ws)
+    torch.cuda.synchronize()
+    yg = host(y)
+    xf = W.bf16_bits_to_f32(xb).astype(np.float64)
+    worst = 0.0
+    for e in range(E):
+        r0, r1 = offsets[e], offsets[e + 1]
+        if r0 == r1:
+            continue
+        if slots[e] < 0:
+            assert np.all(np.isnan(yg[r0:r1])), "rows of a skipped expert were written"
+            continue
+        w13, w2 = orc.dequant_expert(cfg.wfmt, L.expert(0, e), cfg.hidden, cfg.ffn)
+        ref = np.stack([orc.expert_ffn(w13, w2, xf[r]) for r in range(r0, r1)])
+        err = rel_l2(yg[r0:r1], ref)
+        worst = max(worst, err)
+        assert err < TOL_REL_L2, (e, err)
+    return worst
+
+
+SMALL = dict(hidden=256, ffn=128, experts=8, top_k=2, layers=1)
+
+
+@pytest.mark.parametrize("base", [W.TINY, W.DS_DECODE, W.TRACE40], ids=["bf16", "mxfp4", "nvfp4"])
+@pytest.mark.parametrize("passes", [1, 2])
+def test_grouped_ffn_ragged(orc, base, passes):
+    cfg = W.scaled(base, **SMALL)
+    counts = [0, 1, 7, 8, 9, 33, 70, 3]
+    slots = [3, 9, 0, -1, 5, 2, 7, 1]        # permuted, one expert not resident
+    worst = _ffn_case(orc, cfg, counts, slots, pool_slots=10, passes=passes)
+    assert worst < ALARM_REL_L2, worst
+
+
+@pytest.mark.parametrize("base", [W.DS_DECODE, W.TRACE40, W.QWEN_BF16], ids=["mxfp4", "nvfp4", "bf16"])
+def test_grouped_ffn_full_size(orc, base):
+    """Full expert shapes (H, F of the workload), decode-like group sizes."""
+    cfg = W.scaled(base, experts=6, top_k=2, layers=1)
+    counts = [1, 0, 2, 16, 5, 1]
+    slots = [4, 1, 0, 2, 5, 3]
+    worst = _ffn_case(orc, cfg, counts, slots, pool_slots=6, seed=3)
+    assert worst < ALARM_REL_L2, worst
+
+
+def test_grouped_ffn_slot_out_of_range_is_skipped(orc):
+    cfg = W.scaled(W.DS_DECODE, **SMALL)
+    counts = [2, 2, 0, 0, 0, 0, 0, 1]
+    slots = [0, 50, -1, -1, -1, -1, -1, 1]   # 50 >= pool_slots: skipped, not read
+    _ffn_case(orc, cfg, counts, slots, pool_slots=2)
+
+
+# ------------------------------------------------------------------ combine
+@pytest.mark.parametrize("n,k,H,out", [(64, 2, 256, "f32"), (16, 6, 4096, "bf16"), (37, 8, 2048, "bf16")])
+def test_combine_parity(orc, n, k, H, out):
+    rng = np.random.default_rng(n)
+    yb = W.f32_to_bf16_bits(rng.standard_normal((n * k, H)).astype(np.float32) * 100)
+    perm = rng.permutation(n * k).astype(np.int32)       # row_of
+    w = rng.random((n, k)).astype(np.float32)
+    w /= w.sum(1, keepdims=True)
+    ref_rows = W.bf16_bits_to_f32(yb).astype(np.float64)[perm]   # assignment order
+    ref = orc.combine(ref_rows, w.astype(np.float64))
+    o = torch.empty(n, H, dtype=torch.float32 if out == "f32" else torch.bfloat16, device="cuda")
+    A.moe_combine(dev(yb), dev(perm), dev(w), n, k, H, o)
+    torch.cuda.synchronize()
+    err = rel_l2(host(o), ref)
+    assert err < (1e-6 if out == "f32" else 4e-3), err
+    # deterministic: a second run is bitwise identical
+    o2 = torch.empty_like(o)
+    A.moe_combine(dev(yb), dev(perm), dev(w), n, k, H, o2)
+    torch.cuda.synchronize()
+    assert torch.equal(o.view(torch.int16) if o.dtype == torch.bfloat16 else o,
+                       o2.view(torch.int16) if o2.dtype == torch.bfloat16 else o2)
