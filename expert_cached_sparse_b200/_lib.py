@@ -33,8 +33,9 @@ EXPORTS = [
     "moe_pack_expert", "moe_cache_create", "moe_cache_lookup_update", "moe_cache_resize",
     "moe_cache_read_trace", "moe_cache_get_stats", "moe_cache_snapshot", "moe_cache_capacity",
     "moe_cache_destroy", "moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine",
-    "moe_layer_forward",
+    "moe_layer_forward", "moe_profile_enable", "moe_profile_read",
 ]
+PROF_KINDS = ["router", "lookup", "permute", "ffn", "combine", "fill"]
 
 TRACE_DTYPE = np.dtype([("call", "<u4"), ("slot", "<i4"), ("layer", "<u2"), ("expert", "<u2"),
                         ("event", "u1"), ("pad", "u1", 3)])
@@ -48,6 +49,10 @@ class MoeShape(C.Structure):
 class MoeStats(C.Structure):
     _fields_ = [(n, C.c_uint64) for n in ("lookups", "hits", "misses", "evictions", "fill_bytes",
                                            "host_syncs", "trace_dropped")]
+
+
+class MoeProf(C.Structure):
+    _fields_ = [("launches", C.c_uint64), ("timed", C.c_uint64), ("ms", C.c_double)]
 
 
 class MoeError(RuntimeError):
@@ -84,6 +89,8 @@ def _load():
         "moe_grouped_ffn": (C.c_int, [SP, P, I32, P, P, P, I32, P, P, SZ, P]),
         "moe_combine": (C.c_int, [P, P, P, I32, I32, I32, P, I32, P]),
         "moe_layer_forward": (C.c_int, [P, I32, P, I32, P, P, I32, P, P, SZ, P, P, P, P]),
+        "moe_profile_enable": (C.c_int, [C.c_int]),
+        "moe_profile_read": (C.c_int, [C.POINTER(MoeProf), C.c_int, C.c_int]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)

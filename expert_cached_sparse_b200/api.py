@@ -186,3 +186,16 @@ def moe_layer_forward(cache: MoeCache, layer, x, wg, bias, out, ws, stream=None,
                                  ws.numel() * ws.element_size(), stream_handle(stream),
                                  stream_handle(copy_stream), ptr(topk_idx_out), ptr(topk_w_out))
     check("moe_layer_forward", rc)
+
+
+# ------------------------------------------------------------------ profiling
+def moe_profile_enable(timing: bool) -> None:
+    check("moe_profile_enable", L.lib.moe_profile_enable(1 if timing else 0))
+
+
+def moe_profile_read(reset: bool = False) -> dict:
+    """{kind: {"launches", "timed", "ms"}} for router/lookup/permute/ffn/combine/fill."""
+    arr = (L.MoeProf * len(L.PROF_KINDS))()
+    check("moe_profile_read", L.lib.moe_profile_read(arr, len(L.PROF_KINDS), 1 if reset else 0))
+    return {k: {"launches": arr[i].launches, "timed": arr[i].timed, "ms": arr[i].ms}
+            for i, k in enumerate(L.PROF_KINDS)}

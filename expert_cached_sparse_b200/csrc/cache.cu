@@ -394,9 +394,13 @@ static int lookup_smem_bytes(int E, int C)
 int cache_launch_lookup(moe_cache* c, int layer, const int32_t* idx, int count, int32_t* slot_user,
                         cudaStream_t st)
 {
-    lookup_kernel<<<1, kLookupThreads, c->lookup_smem, st>>>(c->m, layer, idx, count, c->shape.experts,
+    {
+        ProfScope ps(MOE_PROF_LOOKUP, st);
+        prof_count(MOE_PROF_LOOKUP, 1);
+        lookup_kernel<<<1, kLookupThreads, c->lookup_smem, st>>>(c->m, layer, idx, count, c->shape.experts,
                                                              c->C, c->trace_cap, slot_user);
-    MOE_LAUNCH_CHECK();
+        MOE_LAUNCH_CHECK();
+    }
     // everything before this point on `st` (earlier readers of any victim
     // slot included) is complete once ev_lookup fires
     MOE_CUDA_TRY(cudaEventRecord(c->ev_lookup, st));
@@ -443,6 +447,8 @@ int cache_read_and_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t c
         MOE_CUDA_TRY(cudaStreamSynchronize(st));
         return MOE_ERR_FILL;
     }
+    ProfScope ps(MOE_PROF_FILL, copy);
+    prof_count(MOE_PROF_FILL, h->n_miss);
     for (int i = 0; i < h->n_miss; i++) {
         const void* src = c->blobs[(size_t)layer * E + ms[i].expert];
         if (!src) return MOE_ERR_STATE;

@@ -49,6 +49,8 @@ int launch_combine(const uint16_t* y_perm, const int32_t* row_of, const float* w
                    int out_dtype, cudaStream_t st)
 {
     if (n == 0) return MOE_OK;
+    ProfScope ps(MOE_PROF_COMBINE, st);
+    prof_count(MOE_PROF_COMBINE, 1);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -98,6 +98,25 @@ __device__ __forceinline__ uint32_t lane_id()
 
 }  // namespace moe
 
+// ---------------------------------------------------------------- profiling
+namespace moe {
+void prof_count(int kind, int launches);
+// Brackets the work enqueued on `st` during its lifetime with two events
+// when timing is enabled (moe_profile_enable); a no-op otherwise.
+class ProfScope {
+  public:
+    ProfScope(int kind, cudaStream_t st);
+    ~ProfScope();
+    ProfScope(const ProfScope&) = delete;
+    ProfScope& operator=(const ProfScope&) = delete;
+
+  private:
+    int kind_;
+    cudaStream_t st_;
+    cudaEvent_t a_;
+};
+}  // namespace moe
+
 // ---------------------------------------------------------------- internal launchers
 namespace moe {
 int launch_router(const void* x, int x_dtype, const uint16_t* wg, const float* bias, int n, int H,

@@ -322,6 +322,8 @@ int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool
                cudaStream_t st)
 {
     if (rows == 0) return MOE_OK;
+    ProfScope ps(MOE_PROF_FFN, st);
+    prof_count(MOE_PROF_FFN, 2);
     BlobLayout bl = blob_layout(s);
     uint16_t* h = static_cast<uint16_t*>(ws);
     FfnArgs a1{};

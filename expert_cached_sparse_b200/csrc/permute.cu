@@ -179,6 +179,8 @@ int launch_permute(const int32_t* idx, int n, int E, int k, const void* x, int x
         MOE_CUDA_TRY(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st));
         return MOE_OK;
     }
+    ProfScope ps(MOE_PROF_PERMUTE, st);
+    prof_count(MOE_PROF_PERMUTE, 3);
     PermWs p;
     ws_layout(A, E, &p, ws);
     const int W = warps_per_chunk(E);

@@ -189,6 +189,8 @@ int launch_router(const void* x, int x_dtype, const uint16_t* wg, const float* b
                   int E, int k, float* logits, int32_t* idx, float* w, cudaStream_t st)
 {
     if (n == 0) return MOE_OK;
+    ProfScope ps(MOE_PROF_ROUTER, st);
+    prof_count(MOE_PROF_ROUTER, 2);
     int rc = (x_dtype == MOE_DT_F32) ? launch_logits<true>(x, wg, bias, n, H, E, logits, st)
                                      : launch_logits<false>(x, wg, bias, n, H, E, logits, st);
     if (rc) return rc;

@@ -102,6 +102,23 @@ typedef struct {
     uint64_t trace_dropped;/* records lost because the trace buffer was full */
 } moe_cache_stats;
 
+/* Profiling categories: kernels of each step, and the host->device fills. */
+typedef enum {
+    MOE_PROF_ROUTER = 0,  /* router logits + top-k kernels */
+    MOE_PROF_LOOKUP = 1,  /* cache lookup kernel */
+    MOE_PROF_PERMUTE = 2, /* histogram, scan, scatter/gather kernels */
+    MOE_PROF_FFN = 3,     /* grouped FFN kernels (gate-up, down) */
+    MOE_PROF_COMBINE = 4, /* combine kernel */
+    MOE_PROF_FILL = 5,    /* miss fills: host->device copies (not kernels) */
+    MOE_PROF_COUNT = 6
+} moe_prof_kind;
+
+typedef struct {
+    uint64_t launches;  /* kernels launched (copies issued for MOE_PROF_FILL) */
+    uint64_t timed;     /* bracketed steps whose duration is in ms */
+    double ms;          /* summed device time of the bracketed steps */
+} moe_prof_entry;
+
 /* Human-readable name of a status code (static string). */
 const char* moe_status_str(int status);
 
@@ -292,6 +309,22 @@ int moe_layer_forward(moe_cache* cache, int32_t layer, const void* d_x, int32_t 
                       const uint16_t* d_wg, const float* d_bias, int32_t n, void* d_out,
                       void* d_ws, size_t ws_bytes, void* stream, void* copy_stream,
                       int32_t* d_topk_idx_out, float* d_topk_w_out);
+
+/* ---------------------------------------------------------------- profiling */
+
+/*
+ * Launch counters are always kept (process-wide).  With timing != 0, every
+ * step an entry point enqueues (the router's two kernels, the lookup, the
+ * permutation's three kernels, each grouped-FFN pass, the combine, each
+ * call's batch of fills) is bracketed by two CUDA events recorded on the
+ * stream it runs on.  Not thread-safe with respect to moe_profile_read.
+ */
+int moe_profile_enable(int timing);
+
+/* Waits for the pending events, then copies min(count, MOE_PROF_COUNT)
+ * entries (indexed by moe_prof_kind) to h_out; reset != 0 zeroes all
+ * counters afterwards.  Synchronous. */
+int moe_profile_read(moe_prof_entry* h_out, int count, int reset);
 
 #ifdef __cplusplus
 }

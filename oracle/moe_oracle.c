@@ -98,10 +98,12 @@ static int fp4_code(const uint8_t* q, int cols, int r, int c)
  * along a row. */
 void orc_dequant_mxfp4(const uint8_t* q, const uint8_t* sc, int rows, int cols, double* out)
 {
+    double v[16], s[256];  /* the decoders above, tabulated once */
+    for (int i = 0; i < 16; i++) v[i] = orc_e2m1(i);
+    for (int i = 0; i < 256; i++) s[i] = orc_e8m0(i);
     for (int r = 0; r < rows; r++)
         for (int c = 0; c < cols; c++)
-            out[(size_t)r * cols + c] =
-                orc_e2m1(fp4_code(q, cols, r, c)) * orc_e8m0(sc[(size_t)r * (cols / 32) + c / 32]);
+            out[(size_t)r * cols + c] = v[fp4_code(q, cols, r, c)] * s[sc[(size_t)r * (cols / 32) + c / 32]];
 }
 
 /* NVFP4 -> real: w = e2m1 * e4m3(scale) * s_tensor, one E4M3 scale per 16
@@ -109,11 +111,13 @@ void orc_dequant_mxfp4(const uint8_t* q, const uint8_t* sc, int rows, int cols, 
 void orc_dequant_nvfp4(const uint8_t* q, const uint8_t* sc, float s_tensor, int rows, int cols,
                        double* out)
 {
+    double v[16], s[256];  /* the decoders above, tabulated once */
+    for (int i = 0; i < 16; i++) v[i] = orc_e2m1(i);
+    for (int i = 0; i < 256; i++) s[i] = orc_e4m3(i);
     for (int r = 0; r < rows; r++)
         for (int c = 0; c < cols; c++)
-            out[(size_t)r * cols + c] = orc_e2m1(fp4_code(q, cols, r, c)) *
-                                        orc_e4m3(sc[(size_t)r * (cols / 16) + c / 16]) *
-                                        (double)s_tensor;
+            out[(size_t)r * cols + c] =
+                v[fp4_code(q, cols, r, c)] * s[sc[(size_t)r * (cols / 16) + c / 16]] * (double)s_tensor;
 }
 
 void orc_dequant_bf16(const uint16_t* w, size_t count, double* out)

@@ -107,7 +107,7 @@ def _ffn_case(orc, cfg, counts, slots, pool_slots, seed=0, passes=1):
     sb = A.moe_slot_bytes(shape)
     pool = torch.zeros(pool_slots * sb, dtype=torch.uint8, device="cuda")
     for e in range(E):
-        if slots[e] >= 0:
+        if 0 <= slots[e] < pool_slots:
             pool[slots[e] * sb:(slots[e] + 1) * sb].copy_(L.blob(0, e), non_blocking=False)
     rows = int(sum(counts))
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
@@ -131,7 +131,7 @@ def _ffn_case(orc, cfg, counts, slots, pool_slots, seed=0, passes=1):
         r0, r1 = offsets[e], offsets[e + 1]
         if r0 == r1:
             continue
-        if slots[e] < 0:
+        if not 0 <= slots[e] < pool_slots:
             assert np.all(np.isnan(yg[r0:r1])), "rows of a skipped expert were written"
             continue
         w13, w2 = orc.dequant_expert(cfg.wfmt, L.expert(0, e), cfg.hidden, cfg.ffn)
