@@ -33,7 +33,7 @@ EXPORTS = [
     "moe_pack_expert", "moe_cache_create", "moe_cache_lookup_update", "moe_cache_resize",
     "moe_cache_read_trace", "moe_cache_get_stats", "moe_cache_snapshot", "moe_cache_capacity",
     "moe_cache_destroy", "moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine",
-    "moe_layer_forward", "moe_profile_enable", "moe_profile_read",
+    "moe_layer_forward", "moe_profile_enable", "moe_profile_read", "moe_get_device_error",
 ]
 PROF_KINDS = ["router", "lookup", "permute", "ffn", "combine", "fill"]
 
@@ -91,6 +91,7 @@ def _load():
         "moe_layer_forward": (C.c_int, [P, I32, P, I32, P, P, I32, P, P, SZ, P, P, P, P]),
         "moe_profile_enable": (C.c_int, [C.c_int]),
         "moe_profile_read": (C.c_int, [C.POINTER(MoeProf), C.c_int, C.c_int]),
+        "moe_get_device_error": (C.c_int, [C.c_int]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)

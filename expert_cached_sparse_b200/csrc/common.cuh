@@ -129,6 +129,10 @@ size_t ffn_ws_bytes(const moe_shape* s, int rows);
 int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
                const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,
                cudaStream_t st);
+bool ffn_tc_supported(const moe_shape* s);
+int launch_ffn_tc(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
+                  const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, uint16_t* h,
+                  cudaStream_t st);
 int launch_combine(const uint16_t* y_perm, const int32_t* row_of, const float* w, int n, int k, int H,
                    void* out, int out_dtype, cudaStream_t st);
 }  // namespace moe

@@ -19,6 +19,9 @@
 //    SwiGLU epilogue is lane-local: h = silu(gate) * up, rounded to bf16;
 //  - phase 2 writes y rows in bf16; the NVFP4 tensor scales multiply the
 //    fp32 accumulators.
+#include <stdlib.h>
+#include <string.h>
+
 #include "common.cuh"
 
 namespace moe {
@@ -315,6 +318,18 @@ int launch_ffn_fmt(const moe_shape* s, const BlobLayout& bl, FfnArgs a1, FfnArgs
 
 }  // namespace
 
+// Grouped GEMM on tcgen05 when groups are large (prefill: rows >= 4 per
+// expert on average) and the weights are FP4; the weight-streaming mma.sync
+// kernel otherwise.  MOE_FFN_PATH=mma|tc overrides the choice.
+static bool use_tc_path(const moe_shape* s, int rows)
+{
+    if (!ffn_tc_supported(s)) return false;
+    const char* force = getenv("MOE_FFN_PATH");
+    if (force && !strcmp(force, "mma")) return false;
+    if (force && !strcmp(force, "tc")) return true;
+    return rows >= 4 * s->experts;
+}
+
 size_t ffn_ws_bytes(const moe_shape* s, int rows) { return align_up((size_t)rows * s->ffn * 2, 256) + 256; }
 
 int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
@@ -348,6 +363,8 @@ int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool
     a2.K = s->ffn;
     a2.in = h;
     a2.out = y_perm;
+    if (use_tc_path(s, rows))
+        return launch_ffn_tc(s, pool, slot_bytes, pool_slots, slot_of, offsets, x_perm, rows, y_perm, h, st);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -1,0 +1,615 @@
+// Prefill grouped SwiGLU GEMM on the fifth-generation tensor cores (tcgen05).
+//
+// Prefill touches nearly every expert with tens to hundreds of rows each, so
+// the expert FFN becomes a grouped GEMM ("FreeToken 290b model", section
+// "Como gestiona FreeToken el prellenado y la decodificacion": prefill runs
+// whole layers; the pages' own design streams the next layer's experts over
+// PCIe, here every expert is already resident).  Design for sm_100a:
+//  - swap-AB: the expert's weight rows are the MMA's M side (128 rows per
+//    tile), tokens the N side (up to 256 per tile), K in chunks of 64;
+//  - weights stay packed FP4 in HBM; a bulk copy brings each 128 x 64 FP4
+//    chunk (4 KB + scales) to shared memory, four warps expand it exactly to
+//    bf16 (E2M1 x block scale is exact in bf16) and write it with
+//    tcgen05.st straight into tensor memory, where the MMA reads its A
+//    operand; no bf16 weight tile ever touches shared memory;
+//  - tokens (x_perm, or h for the down projection) arrive by TMA in 16-row
+//    boxes with the 128-byte swizzle the MMA's shared-memory descriptor
+//    expects; rows past the expert's block are loaded but never stored;
+//  - the accumulator lives in tensor memory (128 lanes x N fp32 columns);
+//    the same four warps read it back with tcgen05.ld for the epilogue:
+//    SwiGLU (gate and up rows are 8 lanes apart, one shuffle) into h, or the
+//    NVFP4 tensor scale into y;
+//  - warp 0 issues copies, warp 1 issues MMAs (one thread each); mbarriers
+//    chain the roles; every wait is bounded and a timeout sets an error word
+//    and drains the CTA instead of hanging.
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+__device__ int g_tc_error;   // first device-side error of the tensor-core FFN (0: none)
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN_MAX = 256;
+constexpr int BK = 64;
+constexpr int SA = 4;              // FP4 A stages
+constexpr int SB = 4;              // token (B) stages
+constexpr int NABUF = 2;           // tensor-memory A buffers
+constexpr int THREADS = 192;       // warp 0 copies, warp 1 MMA, warps 2..5 expand + epilogue
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t D_COL = 0;      // accumulator columns [0, 256)
+constexpr uint32_t A_COL = 256;    // A buffers: 32 columns each
+constexpr uint32_t B_STAGE_BYTES = BN_MAX * 128;
+constexpr uint32_t A_STAGE_BYTES = 8 * 512;
+constexpr uint32_t S_STAGE_BYTES = 8 * 64;
+constexpr unsigned long long WAIT_LIMIT = 1ull << 22;   // tries (each >= ~0.5 us) before giving up
+
+struct TcArgs {
+    const char* pool;
+    size_t slot_bytes;
+    size_t w_off, s_off, ts_off;
+    int R, K, E;
+    const int32_t* slot_of;
+    const int32_t* offsets;
+    int pool_slots, rows;
+    uint16_t* out;
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+// Bounded wait; on timeout records MOE_ERR_TIMEOUT and raises the CTA's abort flag.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag)
+{
+    for (unsigned long long i = 0; i < WAIT_LIMIT; i++) {
+        if (mbar_try(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (i >= 16) __nanosleep(256);
+    }
+    *abort_flag = 1;
+    atomicCAS(&g_tc_error, 0, (int)MOE_ERR_TIMEOUT);
+    return false;
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+                 ::"r"(dst), "l"(map), "r"(c0), "r"(c1), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+                 ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0),
+                 "r"(0)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+                 "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, "
+                 "%31, %32};"
+                 ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                 "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+                 "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]),
+                 "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]),
+                 "r"(v[31])
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+                 "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
+                 "[%32];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                   "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+                   "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+                   "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+                   "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                 : "r"(taddr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row
+// groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr)
+{
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor: kind::f16, bf16 A and B (K-major), fp32 D, M = 128, N = n.
+__device__ __forceinline__ uint32_t idesc_bf16(int n)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void e2m1x4_to_f16x2(uint32_t w, uint32_t (&f)[4])
+{
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(f[0]), "=r"(f[1]), "=r"(f[2]), "=r"(f[3])
+        : "r"(w));
+}
+
+// f16x2 of E2M1 values -> bf16x2 (value * 2^-112, exact) -> times m2 (scale * 2^112) in bf16, exact.
+__device__ __forceinline__ uint32_t to_bf16x2_scaled(uint32_t f, uint32_t m2)
+{
+    uint32_t b = ((f & 0x7FFF7FFFu) >> 3) | (f & 0x80008000u);
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(b), "r"(m2));
+    return r;
+}
+
+__device__ uint16_t scale_mult(int wfmt, int c)
+{
+    if (wfmt == MOE_W_MXFP4) {
+        int e = c + 112;
+        e = e < 1 ? 1 : (e > 254 ? 254 : e);
+        return (uint16_t)(e << 7);
+    }
+    int s = (c >> 7) & 1, e = (c >> 3) & 15, m = c & 7;
+    float v = (e == 0) ? ldexpf((float)m, -9) : ldexpf((float)(8 + m), e - 10);
+    v = ldexpf(v, 112);
+    return f32_to_bf16_bits(s ? -v : v);
+}
+
+struct Tile {
+    int e, rb, row0, nrows, bn;
+};
+
+__device__ __forceinline__ Tile tile_of(int u, const int* prefix, int E, int RB, const int32_t* offsets)
+{
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= u) lo = mid;
+        else hi = mid - 1;
+    }
+    Tile t;
+    t.e = lo;
+    int local = u - prefix[lo];
+    int tb = local / RB;
+    t.rb = local % RB;
+    int m = offsets[lo + 1] - offsets[lo];
+    int nblk = (m + BN_MAX - 1) / BN_MAX;
+    int bs = (((m + nblk - 1) / nblk) + 15) & ~15;
+    t.row0 = offsets[lo] + tb * bs;
+    t.nrows = max(0, min(bs, m - tb * bs));
+    t.bn = max(16, (t.nrows + 15) & ~15);
+    return t;
+}
+
+template <int WFMT, int PHASE>
+__global__ void __launch_bounds__(THREADS, 1)
+    ffn_tc_kernel(TcArgs a, const __grid_constant__ CUtensorMap tmap_in)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* sB = smem;                                   // SB x 32 KB, 1024-aligned
+    unsigned char* sA = sB + SB * B_STAGE_BYTES;                // SA x 4 KB
+    unsigned char* sS = sA + SA * A_STAGE_BYTES;                // SA x 512 B
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sS + SA * S_STAGE_BYTES);
+    uint64_t* full_a = bars;
+    uint64_t* empty_a = full_a + SA;
+    uint64_t* full_b = empty_a + SA;
+    uint64_t* empty_b = full_b + SB;
+    uint64_t* a_ready = empty_b + SB;
+    uint64_t* a_free = a_ready + NABUF;
+    uint64_t* d_full = a_free + NABUF;
+    uint64_t* d_empty = d_full + 1;
+    uint64_t* fin = d_empty + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+    int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+    uint16_t* s_mult = reinterpret_cast<uint16_t*>(abort_flag + 1);   // [256]
+    int* prefix = reinterpret_cast<int*>(s_mult + 256);              // [E+1]
+    __shared__ int s_warp[THREADS / 32];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int E = a.E, RB = a.R / BM, KT = a.K / BK;
+    constexpr int STILE = (WFMT == MOE_W_MXFP4) ? 32 : 64;
+
+    // ---- set-up: tables, barriers, tensor memory
+    for (int c = tid; c < 256; c += THREADS) s_mult[c] = scale_mult(WFMT, c);
+    {
+        const int EPT = (E + THREADS - 1) / THREADS;
+        int loc = 0;
+        for (int e = tid * EPT; e < tid * EPT + EPT && e < E; e++) {
+            int m = a.offsets[e + 1] - a.offsets[e];
+            int sl = a.slot_of[e];
+            bool ok = m > 0 && sl >= 0 && sl < a.pool_slots && a.offsets[e] >= 0 && a.offsets[e + 1] <= a.rows;
+            int u = ok ? RB * ((m + BN_MAX - 1) / BN_MAX) : 0;
+            prefix[e] = u;
+            loc += u;
+        }
+        int inc = loc;
+        for (int off = 1; off < 32; off <<= 1) {
+            int o = __shfl_up_sync(0xffffffffu, inc, off);
+            if (lane >= off) inc += o;
+        }
+        if (lane == 31) s_warp[warp] = inc;
+        __syncthreads();
+        int run = inc - loc;
+        for (int w = 0; w < warp; w++) run += s_warp[w];
+        for (int e = tid * EPT; e < tid * EPT + EPT && e < E; e++) {
+            int u = prefix[e];
+            prefix[e] = run;
+            run += u;
+        }
+        if (tid == THREADS - 1) prefix[E] = run;
+    }
+    if (tid == 0) {
+        for (int i = 0; i < SA; i++) {
+            mbar_init(smem_u32(&full_a[i]), 1);
+            mbar_init(smem_u32(&empty_a[i]), 4);
+        }
+        for (int i = 0; i < SB; i++) {
+            mbar_init(smem_u32(&full_b[i]), 1);
+            mbar_init(smem_u32(&empty_b[i]), 1);
+        }
+        for (int i = 0; i < NABUF; i++) {
+            mbar_init(smem_u32(&a_ready[i]), 128);
+            mbar_init(smem_u32(&a_free[i]), 1);
+        }
+        mbar_init(smem_u32(d_full), 1);
+        mbar_init(smem_u32(d_empty), 128);
+        mbar_init(smem_u32(fin), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int total = prefix[E];
+    volatile int* abort_v = abort_flag;
+
+    if (warp == 0) {
+        // ================= copy issue (one thread) =================
+        if (lane == 0) {
+            int sa = 0, sb = 0;
+            uint32_t pa = 0, pb = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+                Tile t = tile_of(u, prefix, E, RB, a.offsets);
+                const char* blob = a.pool + (size_t)a.slot_of[t.e] * a.slot_bytes;
+                const char* wt = blob + a.w_off + (size_t)(8 * t.rb) * KT * 512;
+                const char* st = blob + a.s_off + (size_t)(8 * t.rb) * KT * STILE;
+                for (int c = 0; c < KT && ok; c++) {
+                    ok = mbar_wait(smem_u32(&empty_a[sa]), pa ^ 1, abort_v);
+                    if (!ok) break;
+                    uint32_t fa = smem_u32(&full_a[sa]);
+                    mbar_expect_tx(fa, A_STAGE_BYTES + 8 * STILE);
+                    for (int i = 0; i < 8; i++) {
+                        bulk_g2s(smem_u32(sA + sa * A_STAGE_BYTES + i * 512), wt + ((size_t)i * KT + c) * 512, 512, fa);
+                        bulk_g2s(smem_u32(sS + sa * S_STAGE_BYTES + i * STILE), st + ((size_t)i * KT + c) * STILE,
+                                 STILE, fa);
+                    }
+                    if (++sa == SA) { sa = 0; pa ^= 1; }
+                    ok = mbar_wait(smem_u32(&empty_b[sb]), pb ^ 1, abort_v);
+                    if (!ok) break;
+                    uint32_t fb = smem_u32(&full_b[sb]);
+                    const int nbox = t.bn / 16;
+                    mbar_expect_tx(fb, (uint32_t)nbox * 16 * 128);
+                    for (int j = 0; j < nbox; j++)
+                        tma_load_2d(smem_u32(sB + sb * B_STAGE_BYTES + j * 2048), &tmap_in, c * BK, t.row0 + 16 * j, fb);
+                    if (++sb == SB) { sb = 0; pb ^= 1; }
+                }
+            }
+            // drain: every stage's most recent fill must land before the CTA exits
+            // (stage i was last filled in the current round if i < next stage, else in the
+            // previous one; a stage never filled reads as complete for the previous parity)
+            for (int i = 0; i < SA; i++) mbar_wait(smem_u32(&full_a[i]), (i < sa) ? pa : (pa ^ 1), abort_v);
+            for (int i = 0; i < SB; i++) mbar_wait(smem_u32(&full_b[i]), (i < sb) ? pb : (pb ^ 1), abort_v);
+        }
+    } else if (warp == 1) {
+        // ================= MMA issue (one thread) =================
+        if (lane == 0) {
+            int sb = 0, ab = 0, it = 0;
+            uint32_t pb = 0, pab = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < total && ok; u += gridDim.x, it++) {
+                Tile t = tile_of(u, prefix, E, RB, a.offsets);
+                if (it > 0) {
+                    ok = mbar_wait(smem_u32(d_empty), (it - 1) & 1, abort_v);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                const uint32_t idesc = idesc_bf16(t.bn);
+                for (int c = 0; c < KT && ok; c++) {
+                    ok = mbar_wait(smem_u32(&a_ready[ab]), pab, abort_v) &&
+                         mbar_wait(smem_u32(&full_b[sb]), pb, abort_v);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t bbase = smem_u32(sB + sb * B_STAGE_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; k++)
+                        tc_mma_ts(tmem + D_COL, tmem + A_COL + 32 * ab + 8 * k, smem_desc_sw128(bbase + 32 * k), idesc,
+                                  (c | k) != 0);
+                    tc_commit(smem_u32(&empty_b[sb]));
+                    tc_commit(smem_u32(&a_free[ab]));
+                    if (++sb == SB) { sb = 0; pb ^= 1; }
+                    if (++ab == NABUF) { ab = 0; pab ^= 1; }
+                }
+                if (ok) tc_commit(smem_u32(d_full));
+            }
+            // every MMA issued by this thread completes before tensor memory is released
+            tc_commit(smem_u32(fin));
+            mbar_wait(smem_u32(fin), 0, abort_v);
+        }
+    } else {
+        // ================= expand FP4 -> tensor memory, epilogue =================
+        const int q = warp & 3;                 // tensor-memory lane quarter of this warp
+        const int r = 32 * q + lane;            // weight row inside the 128-row block
+        const int rtl = r >> 4, rr = r & 15, g = rr & 7, half = rr >> 3;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        int sa = 0, ab = 0, it = 0;
+        uint32_t pa = 0, pab = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < total && ok; u += gridDim.x, it++) {
+            Tile t = tile_of(u, prefix, E, RB, a.offsets);
+            for (int c = 0; c < KT && ok; c++) {
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full_a[sa]), pa, abort_v));
+                if (!ok) break;
+                const unsigned char* arow = sA + sa * A_STAGE_BYTES + rtl * 512 + 64 * g + 8 * half;
+                const unsigned char* srow = sS + sa * S_STAGE_BYTES + rtl * STILE;
+                uint2 q4[4];
+#pragma unroll
+                for (int tt = 0; tt < 4; tt++) q4[tt] = *reinterpret_cast<const uint2*>(arow + 16 * tt);
+                uint32_t mult[4];
+                if (WFMT == MOE_W_MXFP4) {
+                    uint32_t m0 = s_mult[srow[4 * g + 2 * half + 0]], m1 = s_mult[srow[4 * g + 2 * half + 1]];
+                    mult[0] = mult[1] = m0 | (m0 << 16);
+                    mult[2] = mult[3] = m1 | (m1 << 16);
+                } else {
+#pragma unroll
+                    for (int b = 0; b < 4; b++) {
+                        uint32_t m = s_mult[srow[8 * g + 4 * half + b]];
+                        mult[b] = m | (m << 16);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&empty_a[sa]));
+                if (++sa == SA) { sa = 0; pa ^= 1; }
+                uint32_t v[32];
+#pragma unroll
+                for (int tt = 0; tt < 4; tt++) {
+                    uint32_t f[4];
+                    e2m1x4_to_f16x2(q4[tt].x, f);
+#pragma unroll
+                    for (int b = 0; b < 4; b++) v[8 * tt + b] = to_bf16x2_scaled(f[b], mult[tt]);
+                    e2m1x4_to_f16x2(q4[tt].y, f);
+#pragma unroll
+                    for (int b = 0; b < 4; b++) v[8 * tt + 4 + b] = to_bf16x2_scaled(f[b], mult[tt]);
+                }
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&a_free[ab]), pab ^ 1, abort_v));
+                if (!ok) break;
+                tc_fence_after();
+                tmem_st32(tmem + lane_base + A_COL + 32 * ab, v);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&a_ready[ab]));
+                if (++ab == NABUF) { ab = 0; pab ^= 1; }
+            }
+            if (!ok) break;
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(d_full), it & 1, abort_v));
+            if (!ok) break;
+            tc_fence_after();
+            const char* blob = a.pool + (size_t)a.slot_of[t.e] * a.slot_bytes;
+            float tsc = 1.0f;
+            if (WFMT == MOE_W_NVFP4) tsc = reinterpret_cast<const float*>(blob + a.ts_off)[PHASE - 1];
+            for (int c0 = 0; c0 < t.bn; c0 += 32) {
+                uint32_t d[32];
+                tmem_ld32(tmem + lane_base + D_COL + c0, d);
+                tmem_wait_ld();
+                if (PHASE == 1) {
+                    const int F = a.R / 2;
+                    const int f = 64 * t.rb + 8 * rtl + g;
+#pragma unroll
+                    for (int j = 0; j < 32; j++) {
+                        float x = __uint_as_float(d[j]) * tsc;
+                        float up = __shfl_down_sync(0xffffffffu, x, 8);
+                        const int n = c0 + j;
+                        if (half == 0 && n < t.nrows) {
+                            float h = x / (1.0f + expf(-x)) * up;
+                            a.out[(size_t)(t.row0 + n) * F + f] = f32_to_bf16_bits(h);
+                        }
+                    }
+                } else {
+                    const int Ho = a.R;
+                    const int o = BM * t.rb + r;
+#pragma unroll
+                    for (int j = 0; j < 32; j++) {
+                        const int n = c0 + j;
+                        if (n < t.nrows) a.out[(size_t)(t.row0 + n) * Ho + o] = f32_to_bf16_bits(__uint_as_float(d[j]) * tsc);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(d_empty));
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// [rows][cols] bf16, boxes of 16 rows x 64 columns, 128-byte swizzle.
+int make_rows_map(CUtensorMap* m, const void* base, int rows, int cols)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return MOE_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64, 16};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+size_t tc_smem_bytes(int E)
+{
+    return 1024 + SB * B_STAGE_BYTES + SA * A_STAGE_BYTES + SA * S_STAGE_BYTES + 8 * (2 * SA + 2 * SB + 2 * NABUF + 3) +
+           8 + 2 * 256 + 4 * (size_t)(E + 1) + 64;
+}
+
+template <int WFMT, int PHASE>
+int launch_one(const TcArgs& a, const CUtensorMap& map, int rows, int sms, cudaStream_t st)
+{
+    size_t smem = tc_smem_bytes(a.E);
+    static bool attr = false;
+    if (!attr) {
+        MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_tc_kernel<WFMT, PHASE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)smem));
+        attr = true;
+    }
+    long RB = a.R / BM;
+    long active = rows < a.E ? rows : a.E;
+    long bound = RB * (active + rows / BN_MAX + 1);
+    int grid = (int)(bound < sms ? bound : sms);
+    if (grid < 1) grid = 1;
+    ffn_tc_kernel<WFMT, PHASE><<<grid, THREADS, smem, st>>>(a, map);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+}  // namespace
+
+bool ffn_tc_supported(const moe_shape* s)
+{
+    return (s->wfmt == MOE_W_MXFP4 || s->wfmt == MOE_W_NVFP4) && (2 * s->ffn) % BM == 0 && s->hidden % BM == 0 &&
+           tc_smem_bytes(s->experts) <= 227 * 1024;
+}
+
+int launch_ffn_tc(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
+                  const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, uint16_t* h,
+                  cudaStream_t st)
+{
+    BlobLayout bl = blob_layout(s);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    CUtensorMap mx, mh;
+    int rc;
+    if ((rc = make_rows_map(&mx, x_perm, rows, s->hidden))) return rc;
+    if ((rc = make_rows_map(&mh, h, rows, s->ffn))) return rc;
+    TcArgs a1{};
+    a1.pool = static_cast<const char*>(pool);
+    a1.slot_bytes = slot_bytes;
+    a1.w_off = bl.w13;
+    a1.s_off = bl.s13;
+    a1.ts_off = bl.ts;
+    a1.R = 2 * s->ffn;
+    a1.K = s->hidden;
+    a1.E = s->experts;
+    a1.slot_of = slot_of;
+    a1.offsets = offsets;
+    a1.pool_slots = pool_slots;
+    a1.rows = rows;
+    a1.out = h;
+    TcArgs a2 = a1;
+    a2.w_off = bl.w2;
+    a2.s_off = bl.s2;
+    a2.R = s->hidden;
+    a2.K = s->ffn;
+    a2.out = y_perm;
+    if (s->wfmt == MOE_W_MXFP4) {
+        if ((rc = launch_one<MOE_W_MXFP4, 1>(a1, mx, rows, sms, st))) return rc;
+        return launch_one<MOE_W_MXFP4, 2>(a2, mh, rows, sms, st);
+    }
+    if ((rc = launch_one<MOE_W_NVFP4, 1>(a1, mx, rows, sms, st))) return rc;
+    return launch_one<MOE_W_NVFP4, 2>(a2, mh, rows, sms, st);
+}
+
+}  // namespace moe
+
+extern "C" int moe_get_device_error(int clear)
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, moe::g_tc_error, sizeof v) != cudaSuccess) return MOE_ERR_CUDA;
+    if (clear && v) {
+        int z = 0;
+        if (cudaMemcpyToSymbol(moe::g_tc_error, &z, sizeof z) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    return v;
+}

@@ -326,6 +326,13 @@ int moe_profile_enable(int timing);
  * counters afterwards.  Synchronous. */
 int moe_profile_read(moe_prof_entry* h_out, int count, int reset);
 
+/*
+ * First error recorded by a device-side bounded wait since the last clear
+ * (MOE_ERR_TIMEOUT when a kernel gave up waiting and drained instead of
+ * hanging), 0 if none; clear != 0 resets it.  Synchronous.
+ */
+int moe_get_device_error(int clear);
+
 #ifdef __cplusplus
 }
 #endif
