@@ -1,26 +1,34 @@
 // Grouped SwiGLU expert FFN over permuted rows, weights streamed from the
-// expert slots.  "A cache hit runs on the GPU" ("FreeToken quantization",
-// section "Como se desplazan los pesos MoE cuantizados por la memoria").
+// expert slots: the decode path.  "A cache hit runs on the GPU"
+// ("FreeToken quantization", section "Como se desplazan los pesos MoE
+// cuantizados por la memoria").
 //
-// Weight-streaming design (decode is bound by HBM: each touched expert's
-// weights are read once per pass):
-//  - the unit of work is one warp x one 16-row tile of W13 (or W2) x up to
-//    32 rows (tokens) of one expert; units run in a persistent grid;
-//  - A (weights) is the mma.sync m16n8k16 row operand, fed straight from
+// Decode is bound by HBM: each touched expert's weights are read once per
+// pass and every token row is reused across all of them.  Design:
+//  - work unit = one warp x one 16-row tile of W13 (or W2) x up to 16 rows
+//    (tokens) of one expert, over the whole K; a persistent grid walks the
+//    units, consecutive warps take consecutive row tiles of the same expert;
+//  - weights are the mma.sync m16n8k16 row operand, straight from
 //    registers: each lane's 16-byte load of a packed tile holds exactly its
-//    fragment elements (rows g and g+8, 16 consecutive k); E2M1 codes become
-//    f16 with cvt.rn.f16x2.e2m1x2, are re-biased into bf16 (x 2^-112, exact)
-//    and multiplied by (block scale x 2^112) in bf16, which is exact because
-//    e2m1 x scale has at most 6 significant bits;
-//  - B (tokens) is bf16 from x_perm (phase 1) or h (phase 2); the k order
-//    inside each 64-column tile is permuted identically for A and B, so a
-//    lane's B data is 16 consecutive elements (two 16-byte loads);
+//    fragment bytes for four k16 steps; E2M1 pairs become f16 pairs with one
+//    cvt.rn.f16x2.e2m1x2 (exact);
+//  - the activations (x_perm, then h) are first rewritten once per call into
+//    a "B-operand" copy: f16 scaled by a power of two per row (so the row's
+//    largest magnitude is in [2^14, 2^15): exact for bf16 inputs, 11-bit
+//    rounding for fp32 h) and permuted inside each 64-column block so that a
+//    lane's fragment data for four k16 steps is 32 contiguous bytes;
+//  - block scales are applied to fp32 partial sums: the MMA accumulates one
+//    scale block (32 columns MXFP4, 16 NVFP4) from zero, then one FFMA per
+//    accumulator element folds it in with the row's scale; the activation
+//    row's power of two and the NVFP4 tensor scale come off in the epilogue;
 //  - phase 1 tiles pair 8 gate rows with the 8 matching up rows, so the
-//    SwiGLU epilogue is lane-local: h = silu(gate) * up, rounded to bf16;
-//  - phase 2 writes y rows in bf16; the NVFP4 tensor scales multiply the
-//    fp32 accumulators.
+//    SwiGLU epilogue is lane-local: h = silu(gate) * up in fp32;
+//  - weights are prefetched eight tiles ahead, activations two tiles ahead.
+// BF16 weights use the same units with bf16 fragments and a bf16 B copy.
 #include <stdlib.h>
 #include <string.h>
+
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 
@@ -28,26 +36,172 @@ namespace moe {
 namespace {
 
 constexpr int kFfnThreads = 128;
-constexpr int kRowsPerUnit = 32;   // 4 n-tiles of 8 tokens
+constexpr int kRowsPerUnit = 16;   // 2 n-tiles of 8 tokens
+constexpr int kPrepThreads = 256;
 
+// ------------------------------------------------------------------ workspace
+struct FfnWs {
+    uint16_t* xb;     // [rows][H] B-operand copy of x_perm (f16 scaled, or bf16)
+    int32_t* xe;      // [rows] row exponent of xb
+    float* h32;       // [rows][F] h in fp32
+    uint16_t* hb;     // [rows][F] B-operand copy of h
+    int32_t* he;      // [rows]
+    int32_t* groups;  // [E+1] exclusive prefix of token groups per expert
+    uint16_t* h16;    // [rows][F] bf16 h of the tensor-core path (aliases h32)
+};
+
+size_t ffn_ws_layout(const moe_shape* s, int rows, void* base, FfnWs* w)
+{
+    size_t o = 0;
+    auto take = [&](size_t b) { size_t at = o; o = align_up(o + b, 256); return at; };
+    const size_t R = rows > 0 ? rows : 1;
+    size_t oxb = take(2 * R * s->hidden);
+    size_t oxe = take(4 * R);
+    size_t oh = take(4 * R * s->ffn);
+    size_t ohb = take(2 * R * s->ffn);
+    size_t ohe = take(4 * R);
+    size_t og = take(4 * (size_t)(s->experts + 1));
+    if (w) {
+        char* b = static_cast<char*>(base);
+        w->xb = reinterpret_cast<uint16_t*>(b + oxb);
+        w->xe = reinterpret_cast<int32_t*>(b + oxe);
+        w->h32 = reinterpret_cast<float*>(b + oh);
+        w->hb = reinterpret_cast<uint16_t*>(b + ohb);
+        w->he = reinterpret_cast<int32_t*>(b + ohe);
+        w->groups = reinterpret_cast<int32_t*>(b + og);
+        w->h16 = reinterpret_cast<uint16_t*>(b + oh);
+    }
+    return o;
+}
+
+// Position inside a 64-column block of column kk in the B-operand copy:
+// quad lane t reads positions 16t..16t+15; k16 step j's two pairs sit at
+// 16t+4j (columns 16j+2t, +1) and 16t+4j+2 (columns 16j+8+2t, +1).
+__device__ __forceinline__ int b_perm(int kk)
+{
+    const int j = kk >> 4, rem = kk & 15;
+    const int t = (rem & 7) >> 1, q = (rem & 1) | ((rem >> 3) << 1);
+    return 16 * t + 4 * j + q;
+}
+
+// ------------------------------------------------------------------ prep
+// One warp per row: B-operand copy (+ row exponent) of a bf16 or fp32 row.
+// With `groups` set, the last CTA writes the per-expert token-group prefix.
+template <bool IN_F32, bool OUT_F16>
+__global__ void __launch_bounds__(kPrepThreads) ffn_prep_kernel(const void* __restrict__ in, int rows, int K,
+                                                                uint16_t* __restrict__ out, int32_t* __restrict__ ex,
+                                                                const int32_t* __restrict__ offsets,
+                                                                const int32_t* __restrict__ slot_of, int E,
+                                                                int pool_slots, int32_t* __restrict__ groups)
+{
+    const int lane = threadIdx.x & 31;
+    if (groups && blockIdx.x == gridDim.x - 1) {
+        __shared__ int s_warp[kPrepThreads / 32];
+        const int EPT = (E + kPrepThreads - 1) / kPrepThreads;   // <= 16 for E <= 4096
+        int loc = 0, cnts[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            int e = threadIdx.x * EPT + i, gcount = 0;
+            if (i < EPT && e < E) {
+                int m = offsets[e + 1] - offsets[e];
+                int sl = slot_of[e];
+                bool ok = m > 0 && sl >= 0 && sl < pool_slots && offsets[e] >= 0 && offsets[e + 1] <= rows;
+                gcount = ok ? (m + kRowsPerUnit - 1) / kRowsPerUnit : 0;
+            }
+            cnts[i] = gcount;
+            loc += gcount;
+        }
+        int inc = loc;
+        for (int off = 1; off < 32; off <<= 1) {
+            int o = __shfl_up_sync(0xffffffffu, inc, off);
+            if (lane >= off) inc += o;
+        }
+        if (lane == 31) s_warp[threadIdx.x >> 5] = inc;
+        __syncthreads();
+        int run = inc - loc;
+        for (int w = 0; w < (int)(threadIdx.x >> 5); w++) run += s_warp[w];
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            int e = threadIdx.x * EPT + i;
+            if (i < EPT && e < E) groups[e] = run;
+            run += cnts[i];
+        }
+        if (threadIdx.x == kPrepThreads - 1) groups[E] = run;
+        return;
+    }
+    const int nblocks = gridDim.x - (groups ? 1 : 0);
+    const int warps_total = nblocks * (kPrepThreads / 32);
+    for (int r = blockIdx.x * (kPrepThreads / 32) + (threadIdx.x >> 5); r < rows; r += warps_total) {
+        int p = 0;
+        if (OUT_F16) {
+            float mx = 0.0f;
+            for (int c = lane; c < K / 4; c += 32) {
+                float v[4];
+                if (IN_F32) {
+                    float4 q = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(in) + (size_t)r * K) + c);
+                    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+                } else {
+                    uint2 q = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(in) + (size_t)r * K) + c);
+                    v[0] = bf16_bits_to_f32(q.x & 0xFFFF); v[1] = bf16_bits_to_f32(q.x >> 16);
+                    v[2] = bf16_bits_to_f32(q.y & 0xFFFF); v[3] = bf16_bits_to_f32(q.y >> 16);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; i++) mx = fmaxf(mx, fabsf(v[i]));
+            }
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            if (mx > 0.0f && mx <= 3.4e38f) {
+                int e2;
+                frexpf(mx, &e2);          // mx = m * 2^e2, m in [0.5, 1)
+                p = 15 - e2;              // mx * 2^p in [2^14, 2^15)
+                p = p < -100 ? -100 : (p > 100 ? 100 : p);
+            }
+            if (lane == 0) ex[r] = p;
+        }
+        const float sc = ldexpf(1.0f, p);
+        for (int c = lane; c < K / 4; c += 32) {
+            float v[4];
+            if (IN_F32) {
+                float4 q = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(in) + (size_t)r * K) + c);
+                v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+            } else {
+                uint2 q = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(in) + (size_t)r * K) + c);
+                v[0] = bf16_bits_to_f32(q.x & 0xFFFF); v[1] = bf16_bits_to_f32(q.x >> 16);
+                v[2] = bf16_bits_to_f32(q.y & 0xFFFF); v[3] = bf16_bits_to_f32(q.y >> 16);
+            }
+            const int k0 = 4 * c, blk = k0 & ~63;
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                uint16_t o;
+                if (OUT_F16) {
+                    __half hv = __float2half_rn(v[i] * sc);
+                    o = *reinterpret_cast<uint16_t*>(&hv);
+                } else {
+                    o = f32_to_bf16_bits(v[i]);
+                }
+                out[(size_t)r * K + blk + b_perm((k0 + i) & 63)] = o;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ GEMM units
 struct FfnArgs {
     const char* pool;
     size_t slot_bytes;
-    size_t w_off;      // tile base of the matrix inside the blob
-    size_t s_off;      // scale-tile base
-    size_t ts_off;     // NVFP4 tensor scales
-    int R, K;          // matrix rows / columns (2F x H for phase 1, H x F for phase 2)
-    int E;
+    size_t w_off, s_off, ts_off;
+    int R, K, E;
     const int32_t* slot_of;
     const int32_t* offsets;
-    int pool_slots;    // slots >= pool_slots (or < 0) are skipped
-    int rows;          // rows of in/out; row ranges are clipped to it
-    const uint16_t* in;    // [rows][K] bf16
-    uint16_t* out;         // [rows][R/2] (phase 1, h) or [rows][R] (phase 2, y)
+    const int32_t* groups;
+    int rows;
+    const uint16_t* in;     // [rows][K] B-operand copy
+    const int32_t* in_ex;   // [rows] its exponents (FP4 formats)
+    float* out_h;           // phase 1: h [rows][R/2] fp32
+    uint16_t* out_y;        // phase 2: y [rows][R] bf16
 };
 
-__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t& f0, uint32_t& f1, uint32_t& f2,
-                                                uint32_t& f3)
+__device__ __forceinline__ void e2m1x4_to_f16x2(uint32_t w, uint32_t& f0, uint32_t& f1, uint32_t& f2, uint32_t& f3)
 {
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
         "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
@@ -59,41 +213,31 @@ __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t& f0, uint32
         : "r"(w));
 }
 
-// f16x2 holding E2M1 values -> bf16x2 of (value * 2^-112), exact, then
-// times the bf16x2 multiplier m2 = (scale * 2^112, scale * 2^112).
-__device__ __forceinline__ uint32_t f16x2_e2m1_to_bf16x2(uint32_t f, uint32_t m2)
-{
-    uint32_t b = ((f & 0x7FFF7FFFu) >> 3) | (f & 0x80008000u);
-    uint32_t r;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(b), "r"(m2));
-    return r;
-}
-
-__device__ __forceinline__ void mma_bf16(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+template <bool F16>
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1)
 {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    if (F16)
+        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                     "{%0,%1,%2,%3};"
+                     : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                     : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    else
+        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                     "{%0,%1,%2,%3};"
+                     : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                     : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// bf16 bits of value(code) * 2^112 for the block-scale codes of the format.
-__device__ uint16_t scale_mult_bits(int wfmt, int c)
+// E8M0 code -> 2^(c-127) (codes 2..142 only reach the kernels)
+__device__ __forceinline__ float mx_scale(uint32_t c) { return __uint_as_float(c << 23); }
+
+// E4M3 code -> value (subnormals m * 2^-9; NaN codes are rejected at packing)
+__device__ __forceinline__ float e4m3_value(uint32_t c)
 {
-    if (wfmt == MOE_W_MXFP4) {
-        int e = c + 112;             // 2^(c-127) * 2^112 = 2^(c-15); codes outside [2,142] rejected at pack
-        if (e < 1) e = 1;
-        if (e > 254) e = 254;
-        return (uint16_t)(e << 7);
-    }
-    // E4M3: sign, 4-bit exponent (bias 7), 3-bit mantissa; subnormals m*2^-9
-    int s = (c >> 7) & 1, e = (c >> 3) & 15, m = c & 7;
-    float v = (e == 0) ? ldexpf((float)m, -9) : ldexpf((float)(8 + m), e - 10);
-    v = ldexpf(v, 112);
-    if (s) v = -v;
-    return f32_to_bf16_bits(v);
+    const uint32_t s = (c >> 7) & 1, e = (c >> 3) & 15, m = c & 7;
+    float v = (e == 0) ? (float)m * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+    return s ? -v : v;
 }
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
@@ -101,93 +245,78 @@ __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 template <int WFMT, int PHASE>
 __global__ void __launch_bounds__(kFfnThreads) ffn_kernel(FfnArgs a)
 {
-    extern __shared__ int s_prefix[];          // [E+1] unit prefix per expert
-    __shared__ uint16_t s_mult[256];
-    __shared__ int s_warp[kFfnThreads / 32];
+    extern __shared__ int s_groups[];          // [E+1]
     const int tid = threadIdx.x, lane = tid & 31, g = lane >> 2, t = lane & 3;
     const int RT = a.R / 16, KT = a.K / 64;
     const int E = a.E;
-
-    if (WFMT != MOE_W_BF16)
-        for (int c = tid; c < 256; c += kFfnThreads) s_mult[c] = scale_mult_bits(WFMT, c);
-    // per-expert unit counts -> exclusive prefix (contiguous experts per thread)
-    const int EPT = (E + kFfnThreads - 1) / kFfnThreads;
-    int loc = 0;
-    for (int e = tid * EPT; e < tid * EPT + EPT && e < E; e++) {
-        int cnt = a.offsets[e + 1] - a.offsets[e];
-        int sl = a.slot_of[e];
-        int u = (cnt > 0 && sl >= 0 && sl < a.pool_slots) ? ((cnt + kRowsPerUnit - 1) / kRowsPerUnit) * RT : 0;
-        s_prefix[e] = u;
-        loc += u;
-    }
-    {
-        int inc = loc;
-        for (int off = 1; off < 32; off <<= 1) {
-            int o = __shfl_up_sync(0xffffffffu, inc, off);
-            if (lane >= off) inc += o;
-        }
-        if (lane == 31) s_warp[tid >> 5] = inc;
-        __syncthreads();
-        int wbase = 0;
-        for (int w = 0; w < (tid >> 5); w++) wbase += s_warp[w];
-        int run = wbase + inc - loc;
-        for (int e = tid * EPT; e < tid * EPT + EPT && e < E; e++) {
-            int u = s_prefix[e];
-            s_prefix[e] = run;
-            run += u;
-        }
-        if (tid == kFfnThreads - 1) s_prefix[E] = run;
-    }
+    constexpr bool FP4 = WFMT != MOE_W_BF16;
+    for (int i = tid; i <= E; i += kFfnThreads) s_groups[i] = a.groups[i];
     __syncthreads();
-    const int total = s_prefix[E];
+    const int total = s_groups[E] * RT;
     const int warps_total = gridDim.x * (kFfnThreads / 32);
 
+    constexpr int PF = FP4 ? 8 : 2;          // weight tiles in flight
+    constexpr int TILE = FP4 ? 512 : 2048;
+    constexpr int STILE = (WFMT == MOE_W_MXFP4) ? 32 : 64;
+    constexpr int NV = FP4 ? 1 : 4;          // uint4 per lane per tile
+    constexpr int XPF = 2;                   // activation tiles in flight (PF is a multiple)
+
     for (int u = blockIdx.x * (kFfnThreads / 32) + (tid >> 5); u < total; u += warps_total) {
-        // expert of unit u: largest e with s_prefix[e] <= u
+        const int gi = u / RT, rt = u % RT;
         int lo = 0, hi = E - 1;
         while (lo < hi) {
             int mid = (lo + hi + 1) >> 1;
-            if (s_prefix[mid] <= u) lo = mid;
+            if (s_groups[mid] <= gi) lo = mid;
             else hi = mid - 1;
         }
         const int e = lo;
-        const int local = u - s_prefix[e];
-        const int tg = local / RT, rt = local % RT;
-        const int row0 = a.offsets[e] + tg * kRowsPerUnit;
+        const int row0 = a.offsets[e] + (gi - s_groups[e]) * kRowsPerUnit;
         const int row_end = min(min(a.offsets[e + 1], row0 + kRowsPerUnit), a.rows);
-        if (row0 < 0 || row0 >= row_end) continue;
         const int nq = (row_end - row0 + 7) >> 3;
         const char* blob = a.pool + (size_t)a.slot_of[e] * a.slot_bytes;
-        float tsc = 1.0f;
-        if (WFMT == MOE_W_NVFP4) tsc = reinterpret_cast<const float*>(blob + a.ts_off)[PHASE - 1];
-
-        float acc[4][4];
-#pragma unroll
-        for (int q = 0; q < 4; q++)
-#pragma unroll
-            for (int i = 0; i < 4; i++) acc[q][i] = 0.0f;
-
-        constexpr int PF = (WFMT == MOE_W_BF16) ? 2 : 8;      // tiles in flight
-        constexpr int TILE = (WFMT == MOE_W_BF16) ? 2048 : 512;
-        constexpr int STILE = (WFMT == MOE_W_MXFP4) ? 32 : 64;
-        constexpr int NV = (WFMT == MOE_W_BF16) ? 4 : 1;     // uint4 per lane per tile
         const char* wt = blob + a.w_off + (size_t)rt * KT * TILE;
         const char* st = blob + a.s_off + (size_t)rt * KT * STILE;
 
+        // activation row of this lane (token g of each n-tile), -1 for padding
+        int xr[2];
+#pragma unroll
+        for (int q = 0; q < 2; q++) xr[q] = (row0 + 8 * q + g < row_end) ? row0 + 8 * q + g : -1;
+
+        float acc[2][4];
+#pragma unroll
+        for (int q = 0; q < 2; q++)
+#pragma unroll
+            for (int i = 0; i < 4; i++) acc[q][i] = 0.0f;
+
         uint4 abuf[PF][NV];
         uint2 sbuf[PF];
+        uint4 xbuf[XPF][2][2];
+        auto load_a = [&](int i, int kt) {
 #pragma unroll
-        for (int i = 0; i < PF; i++) {
-            if (i < KT) {
+            for (int v = 0; v < NV; v++)
+                abuf[i][v] = __ldg(reinterpret_cast<const uint4*>(wt + (size_t)kt * TILE + v * 512 + 16 * lane));
+            if (WFMT == MOE_W_MXFP4) sbuf[i].x = __ldg(reinterpret_cast<const uint32_t*>(st + (size_t)kt * STILE + 4 * g));
+            if (WFMT == MOE_W_NVFP4) sbuf[i] = __ldg(reinterpret_cast<const uint2*>(st + (size_t)kt * STILE + 8 * g));
+        };
+        auto load_x = [&](int i, int kt) {
 #pragma unroll
-                for (int v = 0; v < NV; v++)
-                    abuf[i][v] = __ldg(reinterpret_cast<const uint4*>(wt + (size_t)i * TILE + v * 512 + 16 * lane));
-                if (WFMT == MOE_W_MXFP4)
-                    sbuf[i].x = __ldg(reinterpret_cast<const uint32_t*>(st + (size_t)i * STILE + 4 * g));
-                if (WFMT == MOE_W_NVFP4)
-                    sbuf[i] = __ldg(reinterpret_cast<const uint2*>(st + (size_t)i * STILE + 8 * g));
+            for (int q = 0; q < 2; q++) {
+                if (xr[q] >= 0) {
+                    const uint4* p = reinterpret_cast<const uint4*>(a.in + (size_t)xr[q] * a.K + kt * 64 + 16 * t);
+                    xbuf[i][q][0] = __ldg(p);
+                    xbuf[i][q][1] = __ldg(p + 1);
+                } else {
+                    xbuf[i][q][0] = xbuf[i][q][1] = make_uint4(0, 0, 0, 0);
+                }
             }
-        }
+        };
+#pragma unroll
+        for (int i = 0; i < PF; i++)
+            if (i < KT) load_a(i, i);
+#pragma unroll
+        for (int i = 0; i < XPF; i++)
+            if (i < KT) load_x(i, i);
+
         for (int kt0 = 0; kt0 < KT; kt0 += PF) {
 #pragma unroll
             for (int i = 0; i < PF; i++) {
@@ -196,100 +325,101 @@ __global__ void __launch_bounds__(kFfnThreads) ffn_kernel(FfnArgs a)
                 uint4 cur[NV];
 #pragma unroll
                 for (int v = 0; v < NV; v++) cur[v] = abuf[i][v];
-                uint2 cs = sbuf[i];
-                if (kt + PF < KT) {
+                const uint2 cs = sbuf[i];
+                if (kt + PF < KT) load_a(i, kt + PF);
+                const int xi = i % XPF;   // static once the loop is unrolled
+                uint4 xc[2][2];
 #pragma unroll
-                    for (int v = 0; v < NV; v++)
-                        abuf[i][v] = __ldg(reinterpret_cast<const uint4*>(wt + (size_t)(kt + PF) * TILE + v * 512 +
-                                                                          16 * lane));
-                    if (WFMT == MOE_W_MXFP4)
-                        sbuf[i].x = __ldg(reinterpret_cast<const uint32_t*>(st + (size_t)(kt + PF) * STILE + 4 * g));
-                    if (WFMT == MOE_W_NVFP4)
-                        sbuf[i] = __ldg(reinterpret_cast<const uint2*>(st + (size_t)(kt + PF) * STILE + 8 * g));
+                for (int q = 0; q < 2; q++) {
+                    xc[q][0] = xbuf[xi][q][0];
+                    xc[q][1] = xbuf[xi][q][1];
                 }
-                // A fragments for the 4 k16 steps of this tile: A[j][0..3] = a0,a1,a2,a3
-                uint32_t A[4][4];
-                if (WFMT == MOE_W_BF16) {
+                if (kt + XPF < KT) load_x(xi, kt + XPF);
+                if (!FP4) {
+                    // bf16 fragments: cur[j] = {a0, a2, a1, a3} of step j
 #pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        A[j][0] = cur[j].x;  // row g   k 16t+4j, +1
-                        A[j][2] = cur[j].y;  // row g   k 16t+4j+2, +3
-                        A[j][1] = cur[j].z;  // row g+8
-                        A[j][3] = cur[j].w;
+                    for (int q = 0; q < 2; q++) {
+                        if (q >= nq) break;
+                        const uint32_t X[8] = {xc[q][0].x, xc[q][0].y, xc[q][0].z, xc[q][0].w,
+                                               xc[q][1].x, xc[q][1].y, xc[q][1].z, xc[q][1].w};
+#pragma unroll
+                        for (int j = 0; j < 4; j++)
+                            mma16816<false>(acc[q], cur[j].x, cur[j].z, cur[j].y, cur[j].w, X[2 * j], X[2 * j + 1]);
                     }
                 } else {
-                    uint32_t sg, sg8;
+                    // f16 fragments from E2M1 bytes: row g bytes in .x/.y, row g+8 in .z/.w;
+                    // byte 2j -> a0 (a1) of step j, byte 2j+1 -> a2 (a3)
+                    uint32_t A[4][4];
+                    uint32_t f0, f1, f2, f3;
+                    e2m1x4_to_f16x2(cur[0].x, f0, f1, f2, f3);
+                    A[0][0] = f0; A[0][2] = f1; A[1][0] = f2; A[1][2] = f3;
+                    e2m1x4_to_f16x2(cur[0].y, f0, f1, f2, f3);
+                    A[2][0] = f0; A[2][2] = f1; A[3][0] = f2; A[3][2] = f3;
+                    e2m1x4_to_f16x2(cur[0].z, f0, f1, f2, f3);
+                    A[0][1] = f0; A[0][3] = f1; A[1][1] = f2; A[1][3] = f3;
+                    e2m1x4_to_f16x2(cur[0].w, f0, f1, f2, f3);
+                    A[2][1] = f0; A[2][3] = f1; A[3][1] = f2; A[3][3] = f3;
+                    float sg[4], s8[4];   // scale of k16 steps 0..3 for rows g and g+8
                     if (WFMT == MOE_W_MXFP4) {
-                        sg = (cs.x >> (8 * (t >> 1))) & 0xFF;
-                        sg8 = (cs.x >> (8 * (2 + (t >> 1)))) & 0xFF;
+                        sg[0] = sg[1] = mx_scale(cs.x & 0xFF);
+                        sg[2] = sg[3] = mx_scale((cs.x >> 8) & 0xFF);
+                        s8[0] = s8[1] = mx_scale((cs.x >> 16) & 0xFF);
+                        s8[2] = s8[3] = mx_scale(cs.x >> 24);
                     } else {
-                        sg = (cs.x >> (8 * t)) & 0xFF;
-                        sg8 = (cs.y >> (8 * t)) & 0xFF;
-                    }
-                    uint32_t mg = s_mult[sg], mg8 = s_mult[sg8];
-                    mg |= mg << 16;
-                    mg8 |= mg8 << 16;
-                    uint32_t f[4];
-                    // row g: bytes 0..7 -> steps (byte 2j -> a0, byte 2j+1 -> a2)
-                    e2m1x8_to_f16x2(cur[0].x, f[0], f[1], f[2], f[3]);
-                    A[0][0] = f16x2_e2m1_to_bf16x2(f[0], mg);
-                    A[0][2] = f16x2_e2m1_to_bf16x2(f[1], mg);
-                    A[1][0] = f16x2_e2m1_to_bf16x2(f[2], mg);
-                    A[1][2] = f16x2_e2m1_to_bf16x2(f[3], mg);
-                    e2m1x8_to_f16x2(cur[0].y, f[0], f[1], f[2], f[3]);
-                    A[2][0] = f16x2_e2m1_to_bf16x2(f[0], mg);
-                    A[2][2] = f16x2_e2m1_to_bf16x2(f[1], mg);
-                    A[3][0] = f16x2_e2m1_to_bf16x2(f[2], mg);
-                    A[3][2] = f16x2_e2m1_to_bf16x2(f[3], mg);
-                    e2m1x8_to_f16x2(cur[0].z, f[0], f[1], f[2], f[3]);
-                    A[0][1] = f16x2_e2m1_to_bf16x2(f[0], mg8);
-                    A[0][3] = f16x2_e2m1_to_bf16x2(f[1], mg8);
-                    A[1][1] = f16x2_e2m1_to_bf16x2(f[2], mg8);
-                    A[1][3] = f16x2_e2m1_to_bf16x2(f[3], mg8);
-                    e2m1x8_to_f16x2(cur[0].w, f[0], f[1], f[2], f[3]);
-                    A[2][1] = f16x2_e2m1_to_bf16x2(f[0], mg8);
-                    A[2][3] = f16x2_e2m1_to_bf16x2(f[1], mg8);
-                    A[3][1] = f16x2_e2m1_to_bf16x2(f[2], mg8);
-                    A[3][3] = f16x2_e2m1_to_bf16x2(f[3], mg8);
-                }
 #pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    if (q >= nq) break;
-                    const int r = row0 + q * 8 + g;
-                    uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
-                    if (r < row_end) {
-                        const uint4* xp = reinterpret_cast<const uint4*>(a.in + (size_t)r * a.K + kt * 64 + 16 * t);
-                        x0 = __ldg(xp);
-                        x1 = __ldg(xp + 1);
+                        for (int j = 0; j < 4; j++) {
+                            sg[j] = e4m3_value((cs.x >> (8 * j)) & 0xFF);
+                            s8[j] = e4m3_value((cs.y >> (8 * j)) & 0xFF);
+                        }
                     }
-                    mma_bf16(acc[q], A[0][0], A[0][1], A[0][2], A[0][3], x0.x, x0.y);
-                    mma_bf16(acc[q], A[1][0], A[1][1], A[1][2], A[1][3], x0.z, x0.w);
-                    mma_bf16(acc[q], A[2][0], A[2][1], A[2][2], A[2][3], x1.x, x1.y);
-                    mma_bf16(acc[q], A[3][0], A[3][1], A[3][2], A[3][3], x1.z, x1.w);
+                    constexpr int SPB = (WFMT == MOE_W_MXFP4) ? 2 : 1;   // k16 steps per scale block
+#pragma unroll
+                    for (int q = 0; q < 2; q++) {
+                        if (q >= nq) break;
+                        const uint32_t X[8] = {xc[q][0].x, xc[q][0].y, xc[q][0].z, xc[q][0].w,
+                                               xc[q][1].x, xc[q][1].y, xc[q][1].z, xc[q][1].w};
+#pragma unroll
+                        for (int j0 = 0; j0 < 4; j0 += SPB) {
+                            float tmp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                            for (int j = j0; j < j0 + SPB; j++)
+                                mma16816<true>(tmp, A[j][0], A[j][1], A[j][2], A[j][3], X[2 * j], X[2 * j + 1]);
+                            acc[q][0] = __fmaf_rn(tmp[0], sg[j0], acc[q][0]);
+                            acc[q][1] = __fmaf_rn(tmp[1], sg[j0], acc[q][1]);
+                            acc[q][2] = __fmaf_rn(tmp[2], s8[j0], acc[q][2]);
+                            acc[q][3] = __fmaf_rn(tmp[3], s8[j0], acc[q][3]);
+                        }
+                    }
                 }
             }
         }
-        // epilogue
+        // epilogue: undo the activation row exponents, apply the NVFP4 tensor scale
+        float tsc = 1.0f;
+        if (WFMT == MOE_W_NVFP4) tsc = reinterpret_cast<const float*>(blob + a.ts_off)[PHASE - 1];
 #pragma unroll
-        for (int q = 0; q < 4; q++) {
+        for (int q = 0; q < 2; q++) {
             if (q >= nq) break;
             const int r0 = row0 + q * 8 + 2 * t, r1 = r0 + 1;
+            float u0 = tsc, u1 = tsc;
+            if (FP4) {
+                if (r0 < row_end) u0 = ldexpf(tsc, -__ldg(a.in_ex + r0));
+                if (r1 < row_end) u1 = ldexpf(tsc, -__ldg(a.in_ex + r1));
+            }
             if (PHASE == 1) {
                 const int F = a.R / 2;
                 const int f = 8 * rt + g;
-                float g0 = acc[q][0] * tsc, g1 = acc[q][1] * tsc, u0 = acc[q][2] * tsc, u1 = acc[q][3] * tsc;
-                if (r0 < row_end) a.out[(size_t)r0 * F + f] = f32_to_bf16_bits(silu(g0) * u0);
-                if (r1 < row_end) a.out[(size_t)r1 * F + f] = f32_to_bf16_bits(silu(g1) * u1);
+                if (r0 < row_end) a.out_h[(size_t)r0 * F + f] = silu(acc[q][0] * u0) * (acc[q][2] * u0);
+                if (r1 < row_end) a.out_h[(size_t)r1 * F + f] = silu(acc[q][1] * u1) * (acc[q][3] * u1);
             } else {
                 const int Ho = a.R;
                 const int o = 16 * rt + g;
                 if (r0 < row_end) {
-                    a.out[(size_t)r0 * Ho + o] = f32_to_bf16_bits(acc[q][0] * tsc);
-                    a.out[(size_t)r0 * Ho + o + 8] = f32_to_bf16_bits(acc[q][2] * tsc);
+                    a.out_y[(size_t)r0 * Ho + o] = f32_to_bf16_bits(acc[q][0] * u0);
+                    a.out_y[(size_t)r0 * Ho + o + 8] = f32_to_bf16_bits(acc[q][2] * u0);
                 }
                 if (r1 < row_end) {
-                    a.out[(size_t)r1 * Ho + o] = f32_to_bf16_bits(acc[q][1] * tsc);
-                    a.out[(size_t)r1 * Ho + o + 8] = f32_to_bf16_bits(acc[q][3] * tsc);
+                    a.out_y[(size_t)r1 * Ho + o] = f32_to_bf16_bits(acc[q][1] * u1);
+                    a.out_y[(size_t)r1 * Ho + o + 8] = f32_to_bf16_bits(acc[q][3] * u1);
                 }
             }
         }
@@ -297,31 +427,72 @@ __global__ void __launch_bounds__(kFfnThreads) ffn_kernel(FfnArgs a)
 }
 
 template <int WFMT>
-int launch_ffn_fmt(const moe_shape* s, const BlobLayout& bl, FfnArgs a1, FfnArgs a2, int rows, int sms,
-                   cudaStream_t st)
+int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, size_t slot_bytes, int pool_slots,
+                  const int32_t* slot_of, const int32_t* offsets, const uint16_t* x_perm, int rows,
+                  uint16_t* y_perm, const FfnWs& w, int sms, cudaStream_t st)
 {
-    const int E = s->experts;
-    size_t smem = sizeof(int) * (E + 1);
-    auto grid_for = [&](int R) {
+    constexpr bool FP4 = WFMT != MOE_W_BF16;
+    const int E = s->experts, H = s->hidden, F = s->ffn;
+    const int wpb = kPrepThreads / 32;
+    int prep_blocks = (rows + wpb - 1) / wpb;
+    if (prep_blocks > sms * 4) prep_blocks = sms * 4;
+    ffn_prep_kernel<false, FP4><<<prep_blocks + 1, kPrepThreads, 0, st>>>(x_perm, rows, H, w.xb, w.xe, offsets,
+                                                                           slot_of, E, pool_slots, w.groups);
+    MOE_LAUNCH_CHECK();
+    FfnArgs a{};
+    a.pool = static_cast<const char*>(pool);
+    a.slot_bytes = slot_bytes;
+    a.ts_off = bl.ts;
+    a.E = E;
+    a.slot_of = slot_of;
+    a.offsets = offsets;
+    a.groups = w.groups;
+    a.rows = rows;
+    const size_t smem = sizeof(int) * (E + 1);
+    // persistent grid: as many CTAs as fit at once (registers bound residency)
+    static int resident[2] = {0, 0};
+    if (!resident[0]) {
+        MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident[0], ffn_kernel<WFMT, 1>, kFfnThreads, smem));
+        MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident[1], ffn_kernel<WFMT, 2>, kFfnThreads, smem));
+        if (resident[0] < 1) resident[0] = 1;
+        if (resident[1] < 1) resident[1] = 1;
+    }
+    auto grid_for = [&](int R, int phase) {
         long max_units = (long)((rows + kRowsPerUnit - 1) / kRowsPerUnit + (rows < E ? rows : E)) * (R / 16);
-        long g = (max_units + 3) / 4;
-        long cap = (long)sms * 8;
-        return (int)(g < 1 ? 1 : (g > cap ? cap : g));
+        long gsz = (max_units + 3) / 4;
+        long cap = (long)sms * resident[phase - 1];
+        return (int)(gsz < 1 ? 1 : (gsz > cap ? cap : gsz));
     };
-    ffn_kernel<WFMT, 1><<<grid_for(a1.R), kFfnThreads, smem, st>>>(a1);
+    a.w_off = bl.w13;
+    a.s_off = bl.s13;
+    a.R = 2 * F;
+    a.K = H;
+    a.in = w.xb;
+    a.in_ex = w.xe;
+    a.out_h = w.h32;
+    ffn_kernel<WFMT, 1><<<grid_for(a.R, 1), kFfnThreads, smem, st>>>(a);
     MOE_LAUNCH_CHECK();
-    ffn_kernel<WFMT, 2><<<grid_for(a2.R), kFfnThreads, smem, st>>>(a2);
+    ffn_prep_kernel<true, FP4><<<prep_blocks, kPrepThreads, 0, st>>>(w.h32, rows, F, w.hb, w.he, nullptr, nullptr,
+                                                                     E, 0, nullptr);
     MOE_LAUNCH_CHECK();
-    (void)bl;
+    FfnArgs b = a;
+    b.w_off = bl.w2;
+    b.s_off = bl.s2;
+    b.R = H;
+    b.K = F;
+    b.in = w.hb;
+    b.in_ex = w.he;
+    b.out_h = nullptr;
+    b.out_y = y_perm;
+    ffn_kernel<WFMT, 2><<<grid_for(b.R, 2), kFfnThreads, smem, st>>>(b);
+    MOE_LAUNCH_CHECK();
     return MOE_OK;
 }
 
-}  // namespace
-
 // Grouped GEMM on tcgen05 when groups are large (prefill: rows >= 4 per
 // expert on average) and the weights are FP4; the weight-streaming mma.sync
-// kernel otherwise.  MOE_FFN_PATH=mma|tc overrides the choice.
-static bool use_tc_path(const moe_shape* s, int rows)
+// kernels otherwise.  MOE_FFN_PATH=mma|tc overrides the choice.
+bool use_tc_path(const moe_shape* s, int rows)
 {
     if (!ffn_tc_supported(s)) return false;
     const char* force = getenv("MOE_FFN_PATH");
@@ -330,7 +501,9 @@ static bool use_tc_path(const moe_shape* s, int rows)
     return rows >= 4 * s->experts;
 }
 
-size_t ffn_ws_bytes(const moe_shape* s, int rows) { return align_up((size_t)rows * s->ffn * 2, 256) + 256; }
+}  // namespace
+
+size_t ffn_ws_bytes(const moe_shape* s, int rows) { return ffn_ws_layout(s, rows, nullptr, nullptr) + 256; }
 
 int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
                const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,
@@ -338,40 +511,27 @@ int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool
 {
     if (rows == 0) return MOE_OK;
     ProfScope ps(MOE_PROF_FFN, st);
-    prof_count(MOE_PROF_FFN, 2);
+    FfnWs w;
+    ffn_ws_layout(s, rows, ws, &w);
+    if (use_tc_path(s, rows)) {
+        prof_count(MOE_PROF_FFN, 2);
+        return launch_ffn_tc(s, pool, slot_bytes, pool_slots, slot_of, offsets, x_perm, rows, y_perm, w.h16, st);
+    }
+    prof_count(MOE_PROF_FFN, 4);
     BlobLayout bl = blob_layout(s);
-    uint16_t* h = static_cast<uint16_t*>(ws);
-    FfnArgs a1{};
-    a1.pool = static_cast<const char*>(pool);
-    a1.slot_bytes = slot_bytes;
-    a1.w_off = bl.w13;
-    a1.s_off = bl.s13;
-    a1.ts_off = bl.ts;
-    a1.R = 2 * s->ffn;
-    a1.K = s->hidden;
-    a1.E = s->experts;
-    a1.slot_of = slot_of;
-    a1.offsets = offsets;
-    a1.pool_slots = pool_slots;
-    a1.rows = rows;
-    a1.in = x_perm;
-    a1.out = h;
-    FfnArgs a2 = a1;
-    a2.w_off = bl.w2;
-    a2.s_off = bl.s2;
-    a2.R = s->hidden;
-    a2.K = s->ffn;
-    a2.in = h;
-    a2.out = y_perm;
-    if (use_tc_path(s, rows))
-        return launch_ffn_tc(s, pool, slot_bytes, pool_slots, slot_of, offsets, x_perm, rows, y_perm, h, st);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     switch (s->wfmt) {
-    case MOE_W_BF16: return launch_ffn_fmt<MOE_W_BF16>(s, bl, a1, a2, rows, sms, st);
-    case MOE_W_MXFP4: return launch_ffn_fmt<MOE_W_MXFP4>(s, bl, a1, a2, rows, sms, st);
-    case MOE_W_NVFP4: return launch_ffn_fmt<MOE_W_NVFP4>(s, bl, a1, a2, rows, sms, st);
+    case MOE_W_BF16:
+        return launch_decode<MOE_W_BF16>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, x_perm, rows, y_perm,
+                                         w, sms, st);
+    case MOE_W_MXFP4:
+        return launch_decode<MOE_W_MXFP4>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, x_perm, rows,
+                                          y_perm, w, sms, st);
+    case MOE_W_NVFP4:
+        return launch_decode<MOE_W_NVFP4>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, x_perm, rows,
+                                          y_perm, w, sms, st);
     }
     return MOE_ERR_INVALID_ARG;
 }

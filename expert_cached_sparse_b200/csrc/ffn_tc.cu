@@ -35,17 +35,18 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN_MAX = 256;
 constexpr int BK = 64;
-constexpr int SA = 4;              // FP4 A stages
+constexpr int SA = 8;              // FP4 A stages
 constexpr int SB = 4;              // token (B) stages
-constexpr int NABUF = 2;           // tensor-memory A buffers
-constexpr int THREADS = 192;       // warp 0 copies, warp 1 MMA, warps 2..5 expand + epilogue
+constexpr int NABUF = 4;           // tensor-memory A buffers
+constexpr int NXW = 8;             // expanding warps: two per tensor-memory lane quarter
+constexpr int THREADS = 32 * (2 + NXW);   // warp 0 copies, warp 1 MMA, warps 2.. expand + epilogue
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t D_COL = 0;      // accumulator columns [0, 256)
-constexpr uint32_t A_COL = 256;    // A buffers: 32 columns each
+constexpr uint32_t A_COL = 256;    // A buffers: 32 columns each (4 buffers: 256..383)
 constexpr uint32_t B_STAGE_BYTES = BN_MAX * 128;
 constexpr uint32_t A_STAGE_BYTES = 8 * 512;
 constexpr uint32_t S_STAGE_BYTES = 8 * 64;
-constexpr unsigned long long WAIT_LIMIT = 1ull << 22;   // tries (each >= ~0.5 us) before giving up
+constexpr long long WAIT_CYCLES = 4000000000ll;   // ~2 s at 2 GHz before a wait gives up
 
 struct TcArgs {
     const char* pool;
@@ -87,13 +88,17 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait; on timeout records MOE_ERR_TIMEOUT and raises the CTA's abort flag.
+// Bounded wait: spins on try_wait (which itself suspends briefly in hardware),
+// gives up after WAIT_CYCLES, records MOE_ERR_TIMEOUT and raises the CTA's
+// abort flag so the other roles drain too.
 __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag)
 {
-    for (unsigned long long i = 0; i < WAIT_LIMIT; i++) {
+    if (mbar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (;;) {
         if (mbar_try(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (i >= 16) __nanosleep(256);
+        if (clock64() - t0 > WAIT_CYCLES) break;
     }
     *abort_flag = 1;
     atomicCAS(&g_tc_error, 0, (int)MOE_ERR_TIMEOUT);
@@ -131,16 +136,13 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
                  : "memory");
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32])
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16])
 {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-                 "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, "
-                 "%31, %32};"
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+                 "%12, %13, %14, %15, %16};"
                  ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
                  "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
-                 "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]),
-                 "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]),
-                 "r"(v[31])
+                 "r"(v[15])
                  : "memory");
 }
 
@@ -293,18 +295,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (tid == 0) {
         for (int i = 0; i < SA; i++) {
             mbar_init(smem_u32(&full_a[i]), 1);
-            mbar_init(smem_u32(&empty_a[i]), 4);
+            mbar_init(smem_u32(&empty_a[i]), NXW);
         }
         for (int i = 0; i < SB; i++) {
             mbar_init(smem_u32(&full_b[i]), 1);
             mbar_init(smem_u32(&empty_b[i]), 1);
         }
         for (int i = 0; i < NABUF; i++) {
-            mbar_init(smem_u32(&a_ready[i]), 128);
+            mbar_init(smem_u32(&a_ready[i]), 32 * NXW);
             mbar_init(smem_u32(&a_free[i]), 1);
         }
         mbar_init(smem_u32(d_full), 1);
-        mbar_init(smem_u32(d_empty), 128);
+        mbar_init(smem_u32(d_empty), 32 * NXW);
         mbar_init(smem_u32(fin), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -397,7 +399,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else {
         // ================= expand FP4 -> tensor memory, epilogue =================
+        // Two warps per tensor-memory lane quarter: set 0 expands bytes 0..3 of
+        // each lane segment (columns 0..15 of the chunk), set 1 bytes 4..7
+        // (columns 16..31); in the epilogue the sets take alternate 32-column
+        // groups of the accumulator.
         const int q = warp & 3;                 // tensor-memory lane quarter of this warp
+        const int set = (warp - 2) >> 2;        // 0 or 1
         const int r = 32 * q + lane;            // weight row inside the 128-row block
         const int rtl = r >> 4, rr = r & 15, g = rr & 7, half = rr >> 3;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
@@ -409,41 +416,38 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int c = 0; c < KT && ok; c++) {
                 ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full_a[sa]), pa, abort_v));
                 if (!ok) break;
-                const unsigned char* arow = sA + sa * A_STAGE_BYTES + rtl * 512 + 64 * g + 8 * half;
+                const unsigned char* arow = sA + sa * A_STAGE_BYTES + rtl * 512 + 64 * g + 8 * half + 4 * set;
                 const unsigned char* srow = sS + sa * S_STAGE_BYTES + rtl * STILE;
-                uint2 q4[4];
+                uint32_t q4[4];
 #pragma unroll
-                for (int tt = 0; tt < 4; tt++) q4[tt] = *reinterpret_cast<const uint2*>(arow + 16 * tt);
-                uint32_t mult[4];
+                for (int tt = 0; tt < 4; tt++) q4[tt] = *reinterpret_cast<const uint32_t*>(arow + 16 * tt);
+                // byte p of lane segment tt is the row's byte 4p+tt (tensor-memory column 4p+tt):
+                // MXFP4 block = column/16 (= set), NVFP4 block = column/8 (= 2*set + p/2)
+                uint32_t m0, m1;
                 if (WFMT == MOE_W_MXFP4) {
-                    uint32_t m0 = s_mult[srow[4 * g + 2 * half + 0]], m1 = s_mult[srow[4 * g + 2 * half + 1]];
-                    mult[0] = mult[1] = m0 | (m0 << 16);
-                    mult[2] = mult[3] = m1 | (m1 << 16);
+                    m0 = s_mult[srow[4 * g + 2 * half + set]];
+                    m1 = m0;
                 } else {
-#pragma unroll
-                    for (int b = 0; b < 4; b++) {
-                        uint32_t m = s_mult[srow[8 * g + 4 * half + b]];
-                        mult[b] = m | (m << 16);
-                    }
+                    m0 = s_mult[srow[8 * g + 4 * half + 2 * set]];
+                    m1 = s_mult[srow[8 * g + 4 * half + 2 * set + 1]];
                 }
+                m0 |= m0 << 16;
+                m1 |= m1 << 16;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&empty_a[sa]));
                 if (++sa == SA) { sa = 0; pa ^= 1; }
-                uint32_t v[32];
+                uint32_t v[16];
 #pragma unroll
                 for (int tt = 0; tt < 4; tt++) {
                     uint32_t f[4];
-                    e2m1x4_to_f16x2(q4[tt].x, f);
+                    e2m1x4_to_f16x2(q4[tt], f);
 #pragma unroll
-                    for (int b = 0; b < 4; b++) v[8 * tt + b] = to_bf16x2_scaled(f[b], mult[tt]);
-                    e2m1x4_to_f16x2(q4[tt].y, f);
-#pragma unroll
-                    for (int b = 0; b < 4; b++) v[8 * tt + 4 + b] = to_bf16x2_scaled(f[b], mult[tt]);
+                    for (int b = 0; b < 4; b++) v[4 * b + tt] = to_bf16x2_scaled(f[b], b < 2 ? m0 : m1);
                 }
                 ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&a_free[ab]), pab ^ 1, abort_v));
                 if (!ok) break;
                 tc_fence_after();
-                tmem_st32(tmem + lane_base + A_COL + 32 * ab, v);
+                tmem_st16(tmem + lane_base + A_COL + 32 * ab + 16 * set, v);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(smem_u32(&a_ready[ab]));
@@ -456,7 +460,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const char* blob = a.pool + (size_t)a.slot_of[t.e] * a.slot_bytes;
             float tsc = 1.0f;
             if (WFMT == MOE_W_NVFP4) tsc = reinterpret_cast<const float*>(blob + a.ts_off)[PHASE - 1];
-            for (int c0 = 0; c0 < t.bn; c0 += 32) {
+            for (int c0 = 32 * set; c0 < t.bn; c0 += 64) {
                 uint32_t d[32];
                 tmem_ld32(tmem + lane_base + D_COL + c0, d);
                 tmem_wait_ld();

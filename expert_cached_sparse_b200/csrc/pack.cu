@@ -21,6 +21,9 @@ inline int w13_canon_row(int p, int F)
     return r < 8 ? f : F + f;
 }
 
+// FP4 tile: lane L = 4g+t holds 8 bytes of row g then 8 of row g+8; its byte
+// p is the row's byte 4p+t of this 64-column block (columns 8p+2t, +1), i.e.
+// bytes 2j and 2j+1 are the mma.sync A-fragment pairs of k16 step j.
 void pack_fp4_matrix(const uint8_t* q, int R, int K, bool w13, int F, uint8_t* out)
 {
     const int KT = K / 64;
@@ -32,8 +35,8 @@ void pack_fp4_matrix(const uint8_t* q, int R, int K, bool w13, int F, uint8_t* o
                 for (int half = 0; half < 2; half++) {
                     int p = 16 * rt + g + 8 * half;
                     int cr = w13 ? w13_canon_row(p, F) : p;
-                    const uint8_t* src = q + (size_t)cr * (K / 2) + (64 * kt + 16 * t) / 2;
-                    memcpy(tile + 16 * L + 8 * half, src, 8);
+                    const uint8_t* src = q + (size_t)cr * (K / 2) + 32 * kt;
+                    for (int b = 0; b < 8; b++) tile[16 * L + 8 * half + b] = src[4 * b + t];
                 }
             }
         }
@@ -55,6 +58,8 @@ void pack_fp4_scales(const uint8_t* sc, int R, int K, bool w13, int F, bool mx, 
         }
 }
 
+// BF16 tile: for k16 step j, lane L = 4g+t holds 16 bytes
+// {a0, a2, a1, a3}: rows g / g+8, column pairs (16j+2t, +1) and (16j+8+2t, +1).
 void pack_bf16_matrix(const uint16_t* w, int R, int K, bool w13, int F, uint8_t* out)
 {
     const int KT = K / 64;
@@ -67,8 +72,10 @@ void pack_bf16_matrix(const uint16_t* w, int R, int K, bool w13, int F, uint8_t*
                     for (int half = 0; half < 2; half++) {
                         int p = 16 * rt + g + 8 * half;
                         int cr = w13 ? w13_canon_row(p, F) : p;
-                        const uint16_t* src = w + (size_t)cr * K + 64 * kt + 16 * t + 4 * j;
-                        memcpy(tile + 512 * j + 16 * L + 8 * half, src, 8);
+                        const uint16_t* src = w + (size_t)cr * K + 64 * kt + 16 * j + 2 * t;
+                        uint8_t* dst = tile + 512 * j + 16 * L;
+                        memcpy(dst + 8 * half, src, 4);          // a0 / a1
+                        memcpy(dst + 8 * half + 4, src + 8, 4);  // a2 / a3
                     }
                 }
         }

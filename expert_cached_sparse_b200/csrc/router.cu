@@ -32,8 +32,11 @@ __device__ __forceinline__ void load_x8(const void* xrow, int c, float v[8])
     }
 }
 
-// Warp per (token, group of EB experts).  TB tokens share each gate-row load.
-template <bool XF32, int TB, int EB>
+// Warp per (token group of TB, expert group of EB).  TB tokens share each
+// gate-row load, EB experts each activation load.  U chunks of every lane
+// are loaded before their multiply-adds, so U loads per operand are in
+// flight; the multiply-adds still run in the lane's ascending chunk order.
+template <bool XF32, int TB, int EB, int U>
 __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restrict__ x,
                                                             const uint16_t* __restrict__ wg,
                                                             const float* __restrict__ bias, int n,
@@ -53,32 +56,46 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restri
         for (int a = 0; a < TB; a++)
 #pragma unroll
             for (int b = 0; b < EB; b++) acc[a][b] = 0.0f;
-        for (int c = lane; c < chunks; c += 32) {
-            float xv[TB][8];
+        for (int c0 = lane; c0 < chunks; c0 += 32 * U) {
+            float xv[U][TB][8];
+            uint4 wq[U][EB];
 #pragma unroll
-            for (int a = 0; a < TB; a++) {
-                int t = tg * TB + a;
-                if (t < n) load_x8<XF32>(static_cast<const char*>(x) + (size_t)t * xrow_bytes, c, xv[a]);
-                else
+            for (int uu = 0; uu < U; uu++) {
+                const int c = c0 + 32 * uu;
 #pragma unroll
-                    for (int i = 0; i < 8; i++) xv[a][i] = 0.0f;
-            }
+                for (int a = 0; a < TB; a++) {
+                    int t = tg * TB + a;
+                    if (c < chunks && t < n)
+                        load_x8<XF32>(static_cast<const char*>(x) + (size_t)t * xrow_bytes, c, xv[uu][a]);
+                    else
 #pragma unroll
-            for (int b = 0; b < EB; b++) {
-                int e = eg * EB + b;
-                if (e >= E) break;
-                uint4 q = __ldg(reinterpret_cast<const uint4*>(wg + (size_t)e * H + 8 * c));
-                uint32_t w4[4] = {q.x, q.y, q.z, q.w};
-                float wv[8];
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    wv[2 * i] = __uint_as_float(w4[i] << 16);
-                    wv[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+                        for (int i = 0; i < 8; i++) xv[uu][a][i] = 0.0f;
                 }
 #pragma unroll
-                for (int a = 0; a < TB; a++)
+                for (int b = 0; b < EB; b++) {
+                    int e = eg * EB + b;
+                    wq[uu][b] = (c < chunks && e < E)
+                                    ? __ldg(reinterpret_cast<const uint4*>(wg + (size_t)e * H + 8 * c))
+                                    : make_uint4(0, 0, 0, 0);
+                }
+            }
 #pragma unroll
-                    for (int i = 0; i < 8; i++) acc[a][b] = __fmaf_rn(xv[a][i], wv[i], acc[a][b]);
+            for (int uu = 0; uu < U; uu++) {
+                if (c0 + 32 * uu >= chunks) break;
+#pragma unroll
+                for (int b = 0; b < EB; b++) {
+                    const uint32_t w4[4] = {wq[uu][b].x, wq[uu][b].y, wq[uu][b].z, wq[uu][b].w};
+                    float wv[8];
+#pragma unroll
+                    for (int i = 0; i < 4; i++) {
+                        wv[2 * i] = __uint_as_float(w4[i] << 16);
+                        wv[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+                    }
+#pragma unroll
+                    for (int a = 0; a < TB; a++)
+#pragma unroll
+                        for (int i = 0; i < 8; i++) acc[a][b] = __fmaf_rn(xv[uu][a][i], wv[i], acc[a][b]);
+                }
             }
         }
 #pragma unroll
@@ -171,13 +188,13 @@ int launch_logits(const void* x, const uint16_t* wg, const float* bias, int n, i
         long units = (long)((E + EB - 1) / EB) * ((n + TB - 1) / TB);
         int grid = (int)((units + wpb - 1) / wpb);
         if (grid > sms * 8) grid = sms * 8;
-        router_logits_kernel<XF32, TB, EB><<<grid, threads, 0, st>>>(x, wg, bias, n, H, E, logits);
+        router_logits_kernel<XF32, TB, EB, 1><<<grid, threads, 0, st>>>(x, wg, bias, n, H, E, logits);
     } else {
         constexpr int TB = 1, EB = 1;
         long units = (long)E * n;
         int grid = (int)((units + wpb - 1) / wpb);
         if (grid > sms * 8) grid = sms * 8;
-        router_logits_kernel<XF32, TB, EB><<<grid, threads, 0, st>>>(x, wg, bias, n, H, E, logits);
+        router_logits_kernel<XF32, TB, EB, 8><<<grid, threads, 0, st>>>(x, wg, bias, n, H, E, logits);
     }
     MOE_LAUNCH_CHECK();
     return MOE_OK;
