@@ -118,6 +118,23 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+# ------------------------------------------------------------------ multi-rank plumbing
+def max_over_ranks(ms: float, device=None) -> float:
+    """The largest per-rank device time (a no-op on one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(world: int, steps: int, tokens_per_step: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every replica's tokens over the slowest replica's time."""
+    return world * steps * tokens_per_step / (ms_max / 1000.0)
+
+
 # ------------------------------------------------------------------ setup
 def build_layer(cfg, seed):
     """Pinned host blobs of every expert, router matrix and bias (seed-fixed weights)."""
@@ -286,11 +303,8 @@ def run_ours(args, cfg, world, rank, local_rank):
     prof = A.moe_profile_read(reset=True)
     A.moe_profile_enable(False)
     st1 = ds.cache.stats()
-    t = torch.tensor([ms], dtype=torch.float64, device=device)
-    if dist_ok:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
-    value = world * K * n / (ms_max / 1000.0)
+    ms_max = max_over_ranks(ms, device)
+    value = throughput(world, K, n, ms_max)
     idx_steps = ds.idx[Wm:Wm + K].cpu().numpy()
     ffn_bytes = ffn_algorithmic_bytes(idx_steps, cfg, slot_bytes)
     ffn_ms = prof["ffn"]["ms"]
@@ -336,10 +350,8 @@ def run_ours(args, cfg, world, rank, local_rank):
         e_.record(ds.stream)
         torch.cuda.synchronize()
         barrier()
-        t = torch.tensor([s_.elapsed_time(e_)], dtype=torch.float64, device=device)
-        if dist_ok:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        line["e2e"] = {"value": world * K * n / (float(t.item()) / 1000.0), "unit": "tokens/s",
+        e2e_ms = max_over_ranks(s_.elapsed_time(e_), device)
+        line["e2e"] = {"value": throughput(world, K, n, e2e_ms), "unit": "tokens/s",
                        "h2d_bytes_per_step": n * cfg.hidden * 2, "d2h_bytes_per_step": n * cfg.hidden * 2,
                        "note": "no L2 flush; expert fills (misses) are part of the step, not input bytes"}
     ds.cache.close()

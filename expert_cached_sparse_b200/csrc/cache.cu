@@ -136,26 +136,52 @@ __device__ __forceinline__ void put_rec(moe_trace_rec* tr, int cap, long pos, ui
 
 constexpr int kLookupThreads = 1024;
 
-// One CTA.  The whole lookup: request set, capacity check, hits, free slots
-// and victims, installs, trace, outputs.  Slots per thread: C <= 8192.
+// Shared memory of one lookup: the layer's slot-table row, every slot's key
+// and stamp, request flags, the miss list and its slots, victim flags.
+static size_t lookup_smem_bytes(int E, int C)
+{
+    return align_up(sizeof(int) * E, 16) + align_up(sizeof(int) * C, 16) + align_up(8 * (size_t)C, 16) +
+           align_up(E, 16) + align_up(sizeof(int) * E, 16) + align_up(sizeof(int) * E, 16) + align_up(C, 16);
+}
+
+// One CTA.  All state the call needs is read into shared memory in one
+// parallel phase (one memory round trip), the decisions are made there,
+// and only the entries that change are written back.
 __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int layer,
                                                                 const int32_t* __restrict__ idx,
                                                                 int count, int E, int C, int trace_cap,
                                                                 int32_t* __restrict__ slot_user)
 {
-    extern __shared__ unsigned char smem[];
-    unsigned char* req = smem;                                        // [E]
-    int* s_list = reinterpret_cast<int*>(smem + align_up(E, 16));     // [E] miss experts, ascending
-    int* s_slot = s_list + E;                                         // [E] slot for miss i
-    unsigned char* s_cand = reinterpret_cast<unsigned char*>(s_slot + E);  // [C] victim candidate
+    extern __shared__ __align__(16) unsigned char smem[];
+    unsigned char* p = smem;
+    int* s_row = reinterpret_cast<int*>(p);                     p += align_up(sizeof(int) * E, 16);
+    int* s_key = reinterpret_cast<int*>(p);                     p += align_up(sizeof(int) * C, 16);
+    unsigned long long* s_stamp = reinterpret_cast<unsigned long long*>(p); p += align_up(8 * (size_t)C, 16);
+    unsigned char* req = p;                                      p += align_up(E, 16);
+    int* s_list = reinterpret_cast<int*>(p);                    p += align_up(sizeof(int) * E, 16);
+    int* s_slot = reinterpret_cast<int*>(p);                    p += align_up(sizeof(int) * E, 16);
+    unsigned char* s_cand = p;
     __shared__ int s_warp[32];
     __shared__ int s_tot, s_bad;
+    __shared__ unsigned int s_base, s_clock;
     __shared__ unsigned long long s_wmin[32];
     const int tid = threadIdx.x;
     constexpr int NT = kLookupThreads;
 
-    for (int e = tid; e < E; e += NT) req[e] = 0;
-    if (tid == 0) s_bad = 0;
+    // ---- phase 0: everything in, in parallel
+    for (int e = tid; e < E; e += NT) {
+        req[e] = 0;
+        s_row[e] = m.slot_table[layer * E + e];
+    }
+    for (int s = tid; s < C; s += NT) {
+        s_key[s] = m.key_of[s];
+        s_stamp[s] = m.stamp[s];
+    }
+    if (tid == 0) {
+        s_bad = 0;
+        s_base = *m.trace_count;
+        s_clock = m.hdr->clock;
+    }
     __syncthreads();
     for (int i = tid; i < count; i += NT) {
         int v = idx[i];
@@ -176,19 +202,18 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int 
         }
         return;
     }
-    // classify each expert: 0 none, 1 hit, 2 miss; ranks by ascending id
-    const int EPT = (E + NT - 1) / NT;            // experts per thread (contiguous)
+    // ---- classify: ranks of hits and misses in ascending expert id
+    const int EPT = (E + NT - 1) / NT;
     const int e0 = tid * EPT;
     int nreq_loc = 0, nhit_loc = 0, nmiss_loc = 0;
     for (int e = e0; e < e0 + EPT && e < E; e++) {
         if (!req[e]) continue;
         nreq_loc++;
-        if (m.slot_table[layer * E + e] >= 0) nhit_loc++;
+        if (s_row[e] >= 0) nhit_loc++;
         else nmiss_loc++;
     }
-    int nreq_tot, nhit_tot, nmiss_tot;
     block_exclusive_scan(nreq_loc, s_warp, &s_tot);
-    nreq_tot = s_tot;
+    const int nreq_tot = s_tot;
     __syncthreads();
     if (nreq_tot > C) {
         if (tid == 0) {
@@ -202,17 +227,16 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int 
         }
         return;
     }
-    int hit_base = block_exclusive_scan(nhit_loc, s_warp, &s_tot);
-    nhit_tot = s_tot;
+    const int hit_base = block_exclusive_scan(nhit_loc, s_warp, &s_tot);
+    const int nhit_tot = s_tot;
     __syncthreads();
-    int miss_base = block_exclusive_scan(nmiss_loc, s_warp, &s_tot);
-    nmiss_tot = s_tot;
+    const int miss_base = block_exclusive_scan(nmiss_loc, s_warp, &s_tot);
+    const int nmiss_tot = s_tot;
     __syncthreads();
+    const unsigned long long T = (unsigned long long)s_clock + 1ull;
+    const uint32_t base = s_base;
 
-    const unsigned long long T = (unsigned long long)hdr->clock + 1ull;
-    const uint32_t base = *m.trace_count;
-
-    // hits (records in ascending expert order); misses listed in ascending order
+    // ---- hits: refresh stamps, records; list the misses
     {
         int hr = hit_base, mr = miss_base;
         for (int e = e0; e < e0 + EPT && e < E; e++) {
@@ -221,11 +245,11 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int 
                 if (slot_user) slot_user[e] = -1;
                 continue;
             }
-            int key = layer * E + e;
-            int s = m.slot_table[key];
+            const int s = s_row[e];
             if (s >= 0) {
+                s_stamp[s] = T;
                 m.stamp[s] = T;
-                put_rec(m.trace, trace_cap, (long)base + hr, (uint32_t)T, s, key, E, MOE_EV_HIT);
+                put_rec(m.trace, trace_cap, (long)base + hr, (uint32_t)T, s, layer * E + e, E, MOE_EV_HIT);
                 hr++;
                 m.slot_all[e] = m.slot_hit[e] = s;
                 m.slot_miss[e] = -1;
@@ -235,41 +259,41 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int 
             }
         }
     }
-    // free slots in ascending order; victim candidates = resident keys not requested
+    // ---- free slots (ascending), victim candidates = resident keys not requested
     const int SPT = (C + NT - 1) / NT;
     const int s0 = tid * SPT;
     int nfree_loc = 0;
     for (int s = s0; s < s0 + SPT && s < C; s++) {
-        int k2 = m.key_of[s];
-        bool isfree = k2 < 0;
+        const int k2 = s_key[s];
+        const bool isfree = k2 < 0;
         nfree_loc += isfree;
-        bool in_r = !isfree && (k2 / E == layer) && req[k2 % E];
+        const bool in_r = !isfree && (k2 / E == layer) && req[k2 % E];
         s_cand[s] = (!isfree && !in_r) ? 1 : 0;
     }
-    int free_base = block_exclusive_scan(nfree_loc, s_warp, &s_tot);
+    const int free_base = block_exclusive_scan(nfree_loc, s_warp, &s_tot);
     const int nfree = s_tot;
     __syncthreads();
     {
         int fr = free_base;
         for (int s = s0; s < s0 + SPT && s < C; s++) {
-            if (m.key_of[s] < 0) {
+            if (s_key[s] < 0) {
                 if (fr < nmiss_tot) s_slot[fr] = s;
                 fr++;
             }
         }
     }
-    // victims: smallest (stamp, slot) among candidates, one round per victim
+    // ---- victims: smallest (stamp, slot) among candidates, one block reduction each
     const int nvict = nmiss_tot > nfree ? nmiss_tot - nfree : 0;
     for (int r = 0; r < nvict; r++) {
         unsigned long long best = ~0ull;
         for (int s = s0; s < s0 + SPT && s < C; s++)
             if (s_cand[s]) {
-                unsigned long long key = (m.stamp[s] << 14) | (unsigned long long)s;
+                const unsigned long long key = (s_stamp[s] << 14) | (unsigned long long)s;
                 best = key < best ? key : best;
             }
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) {
-            unsigned long long o = __shfl_xor_sync(0xffffffffu, best, off);
+            const unsigned long long o = __shfl_xor_sync(0xffffffffu, best, off);
             best = o < best ? o : best;
         }
         if ((tid & 31) == 0) s_wmin[tid >> 5] = best;
@@ -278,7 +302,7 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int 
             unsigned long long b = (tid < (NT >> 5)) ? s_wmin[tid] : ~0ull;
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) {
-                unsigned long long o = __shfl_xor_sync(0xffffffffu, b, off);
+                const unsigned long long o = __shfl_xor_sync(0xffffffffu, b, off);
                 b = o < b ? o : b;
             }
             if (tid == 0) {
@@ -293,17 +317,16 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int 
         __syncthreads();
     }
     __syncthreads();
-    // installs: miss i takes s_slot[i]
-    int nevict_tot = nvict;
+    // ---- installs: miss i takes s_slot[i]
     for (int i = tid; i < nmiss_tot; i += NT) {
-        int e = s_list[i];
-        int key = layer * E + e;
-        int s = s_slot[i];
+        const int e = s_list[i];
+        const int key = layer * E + e;
+        const int s = s_slot[i];
         long pos = (long)base + nhit_tot + i + (i > nfree ? i - nfree : 0);
         int old = -1;
         if (i >= nfree) {
-            old = m.key_of[s];
-            m.slot_table[old] = -1;
+            old = s_key[s];
+            if (old >= 0) m.slot_table[old] = -1;
             put_rec(m.trace, trace_cap, pos, (uint32_t)T, s, old, E, MOE_EV_EVICT);
             pos++;
         }
@@ -314,12 +337,6 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int 
         me.old_key = old;
         me.pad = 0;
         m.miss[i] = me;
-    }
-    __syncthreads();
-    for (int i = tid; i < nmiss_tot; i += NT) {
-        int e = s_list[i];
-        int key = layer * E + e;
-        int s = s_slot[i];
         m.slot_table[key] = s;
         m.key_of[s] = key;
         m.stamp[s] = T;
@@ -328,10 +345,10 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int 
         if (slot_user) slot_user[e] = s;
     }
     if (tid == 0) {
-        long total = (long)nhit_tot + nmiss_tot + nevict_tot;
+        const long total = (long)nhit_tot + nmiss_tot + nvict;
         long end = (long)base + total;
         if (end > trace_cap) {
-            m.stats->trace_dropped += (unsigned long long)(end - (base > (uint32_t)trace_cap ? base : trace_cap));
+            m.stats->trace_dropped += (unsigned long long)(end - ((long)base > (long)trace_cap ? (long)base : (long)trace_cap));
             end = trace_cap;
         }
         *m.trace_count = (uint32_t)(end > (long)base ? end : (long)base);
@@ -340,12 +357,12 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int 
         hdr->n_req = nreq_tot;
         hdr->n_hit = nhit_tot;
         hdr->n_miss = nmiss_tot;
-        hdr->n_evict = nevict_tot;
+        hdr->n_evict = nvict;
         hdr->n_free = nfree;
         m.stats->lookups += 1;
         m.stats->hits += nhit_tot;
         m.stats->misses += nmiss_tot;
-        m.stats->evictions += nevict_tot;
+        m.stats->evictions += nvict;
     }
 }
 
@@ -385,10 +402,6 @@ struct moe_cache {
 
 namespace moe {
 
-static int lookup_smem_bytes(int E, int C)
-{
-    return (int)(align_up(E, 16) + sizeof(int) * 2 * (size_t)E + (size_t)C);
-}
 
 // Enqueue the lookup kernel for `layer`.
 int cache_launch_lookup(moe_cache* c, int layer, const int32_t* idx, int count, int32_t* slot_user,
@@ -504,7 +517,7 @@ extern "C" int moe_cache_create(const moe_shape* shape, void* d_meta, size_t met
     c->blobs.assign(h_blobs, h_blobs + nkeys);
     c->resident.assign(shape->layers, 0);
     c->hbuf.resize(sizeof(LookupHdr) + sizeof(MissEnt) * (size_t)shape->experts);
-    c->lookup_smem = lookup_smem_bytes(shape->experts, capacity);
+    c->lookup_smem = (int)lookup_smem_bytes(shape->experts, capacity);
     if (const char* fi = getenv("MOE_FAULT_INJECT")) {
         if (!strncmp(fi, "fill_fail:", 10)) c->fault_fill_at = atol(fi + 10);
     }
@@ -701,7 +714,7 @@ extern "C" int moe_cache_resize(moe_cache* c, void* d_meta_new, size_t meta_byte
     c->ml = nl;
     c->m = nm;
     c->pool = static_cast<char*>(d_pool_new);
-    c->lookup_smem = lookup_smem_bytes(E, new_capacity);
+    c->lookup_smem = (int)lookup_smem_bytes(E, new_capacity);
     if (c->lookup_smem > 48 * 1024)
         MOE_CUDA_TRY(cudaFuncSetAttribute(lookup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, c->lookup_smem));
     return MOE_OK;

@@ -39,7 +39,7 @@ static inline bool shape_ok(const moe_shape* s)
 
 // ---------------------------------------------------------------- blob layout
 // One packed expert (= one slot).  Matrices are cut into tiles of 16 rows x
-// 64 columns; tile (rt, kt) of a [R][K] matrix sits at index rt*(K/64)+kt.
+// 64 columns; tile (rt, kt) of a [R][K] matrix sits at tile_index(rt, kt).
 // Inside a tile, lane L = 4g+t of a warp owns rows g and g+8, columns
 // [16t, 16t+16): FP4 tiles store for each lane 8 bytes of row g then 8
 // bytes of row g+8 (512 B per tile), BF16 tiles 32 bytes of row g then 32
@@ -49,6 +49,17 @@ static inline bool shape_ok(const moe_shape* s)
 // [g][(g,b0),(g,b1),(g+8,b0),(g+8,b1)], NVFP4 64 B
 // [g][(g,b0..b3),(g+8,b0..b3)] with b the 32- or 16-column block inside
 // the tile.  NVFP4 ends with the two fp32 tensor scales.
+// Tiles are stored in row groups of 8 row tiles (128 rows): for row group G
+// and column block kt the group's tiles are contiguous, so one 128 x 64
+// block is one contiguous copy.  Index of tile (rt, kt) of a matrix with RT
+// row tiles and KT column blocks (the last group may hold fewer than 8):
+__host__ __device__ static inline size_t tile_index(int rt, int kt, int RT, int KT)
+{
+    const int G = rt >> 3, w = rt & 7;
+    const int ng = (RT - 8 * G) < 8 ? (RT - 8 * G) : 8;
+    return (size_t)8 * G * KT + (size_t)kt * ng + w;
+}
+
 struct BlobLayout {
     size_t w13, w2, s13, s2, ts, bytes;
     int tile_bytes;    // 512 (FP4) or 2048 (BF16)
@@ -126,9 +137,19 @@ int launch_permute(const int32_t* idx, int n, int E, int k, const void* x, int x
                    int32_t* offsets, int32_t* row_of, int32_t* assign_of, uint16_t* x_perm, void* ws,
                    cudaStream_t st);
 size_t ffn_ws_bytes(const moe_shape* s, int rows);
+// Source of the grouped FFN's input rows when x_perm is not materialised:
+// row r is token assign_of[r] / k of x (x_dtype).
+struct RowSource {
+    const void* x;
+    int x_dtype;
+    const int32_t* assign_of;
+    int k;
+};
+bool ffn_uses_tc(const moe_shape* s, int rows);
+int ffn_device_error(int clear);   // decode FFN's device error word (0: none)
 int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
                const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,
-               cudaStream_t st);
+               cudaStream_t st, const RowSource* gather = nullptr);
 bool ffn_tc_supported(const moe_shape* s);
 int launch_ffn_tc(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
                   const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, uint16_t* h,

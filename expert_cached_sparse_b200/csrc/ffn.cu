@@ -8,23 +8,27 @@
 //  - work unit = one warp x one 16-row tile of W13 (or W2) x up to 16 rows
 //    (tokens) of one expert, over the whole K; a persistent grid walks the
 //    units, consecutive warps take consecutive row tiles of the same expert;
-//  - weights are the mma.sync m16n8k16 row operand, straight from
-//    registers: each lane's 16-byte load of a packed tile holds exactly its
-//    fragment bytes for four k16 steps; E2M1 pairs become f16 pairs with one
-//    cvt.rn.f16x2.e2m1x2 (exact);
-//  - the activations (x_perm, then h) are first rewritten once per call into
-//    a "B-operand" copy: f16 scaled by a power of two per row (so the row's
-//    largest magnitude is in [2^14, 2^15): exact for bf16 inputs, 11-bit
-//    rounding for fp32 h) and permuted inside each 64-column block so that a
-//    lane's fragment data for four k16 steps is 32 contiguous bytes;
+//  - each warp streams its tiles through its own shared-memory rings with
+//    1-D bulk copies (TMA engine) issued by one lane and completed on
+//    mbarriers: 16 weight tiles (8 KB) and 8 activation tiles in flight per
+//    warp, running ahead across unit boundaries, no registers held;
+//  - weights are the mma.sync m16n8k16 row operand: a lane's 16 bytes of a
+//    packed tile are exactly its fragment bytes for four k16 steps; E2M1
+//    pairs become f16 pairs with one cvt.rn.f16x2.e2m1x2 (exact);
+//  - the activations (x gathered by token, then h) are first rewritten once
+//    per call into an operand copy: f16 scaled by a power of two per row (the
+//    row's largest magnitude lands in [2^14, 2^15): exact for bf16 rows,
+//    11-bit for fp32 h), stored column-block-major ([64-column block][row])
+//    so any 8 consecutive rows of a block are one contiguous 1 KB copy, and
+//    permuted / swizzled inside each 128-byte row so a lane's fragment data
+//    for four k16 steps is two conflict-free 16-byte reads;
 //  - block scales are applied to fp32 partial sums: the MMA accumulates one
 //    scale block (32 columns MXFP4, 16 NVFP4) from zero, then one FFMA per
 //    accumulator element folds it in with the row's scale; the activation
 //    row's power of two and the NVFP4 tensor scale come off in the epilogue;
 //  - phase 1 tiles pair 8 gate rows with the 8 matching up rows, so the
-//    SwiGLU epilogue is lane-local: h = silu(gate) * up in fp32;
-//  - weights are prefetched eight tiles ahead, activations two tiles ahead.
-// BF16 weights use the same units with bf16 fragments and a bf16 B copy.
+//    SwiGLU epilogue is lane-local: h = silu(gate) * up in fp32.
+// BF16 weights use the same units with bf16 fragments and a bf16 operand copy.
 #include <stdlib.h>
 #include <string.h>
 
@@ -33,18 +37,23 @@
 #include "common.cuh"
 
 namespace moe {
+
+__device__ int g_ffn_error;   // first device-side error of the decode FFN (0: none)
+
 namespace {
 
 constexpr int kFfnThreads = 128;
 constexpr int kRowsPerUnit = 16;   // 2 n-tiles of 8 tokens
 constexpr int kPrepThreads = 256;
+constexpr int kRowPad = 16;        // operand copies carry 16 spare rows (whole 8-row reads past the end)
+constexpr long long kWaitCycles = 4000000000ll;   // ~2 s before a wait gives up
 
 // ------------------------------------------------------------------ workspace
 struct FfnWs {
-    uint16_t* xb;     // [rows][H] B-operand copy of x_perm (f16 scaled, or bf16)
+    uint16_t* xb;     // [H/64][rows+16][64] operand copy of the input rows
     int32_t* xe;      // [rows] row exponent of xb
     float* h32;       // [rows][F] h in fp32
-    uint16_t* hb;     // [rows][F] B-operand copy of h
+    uint16_t* hb;     // [F/64][rows+16][64] operand copy of h
     int32_t* he;      // [rows]
     int32_t* groups;  // [E+1] exclusive prefix of token groups per expert
     uint16_t* h16;    // [rows][F] bf16 h of the tensor-core path (aliases h32)
@@ -54,11 +63,11 @@ size_t ffn_ws_layout(const moe_shape* s, int rows, void* base, FfnWs* w)
 {
     size_t o = 0;
     auto take = [&](size_t b) { size_t at = o; o = align_up(o + b, 256); return at; };
-    const size_t R = rows > 0 ? rows : 1;
-    size_t oxb = take(2 * R * s->hidden);
+    const size_t R = rows > 0 ? rows : 1, RP = R + kRowPad;
+    size_t oxb = take(2 * RP * s->hidden);
     size_t oxe = take(4 * R);
     size_t oh = take(4 * R * s->ffn);
-    size_t ohb = take(2 * R * s->ffn);
+    size_t ohb = take(2 * RP * s->ffn);
     size_t ohe = take(4 * R);
     size_t og = take(4 * (size_t)(s->experts + 1));
     if (w) {
@@ -74,9 +83,9 @@ size_t ffn_ws_layout(const moe_shape* s, int rows, void* base, FfnWs* w)
     return o;
 }
 
-// Position inside a 64-column block of column kk in the B-operand copy:
-// quad lane t reads positions 16t..16t+15; k16 step j's two pairs sit at
-// 16t+4j (columns 16j+2t, +1) and 16t+4j+2 (columns 16j+8+2t, +1).
+// Position inside a 64-column block of column kk in the operand copy: quad
+// lane t reads positions 16t..16t+15; k16 step j's two pairs sit at 16t+4j
+// (columns 16j+2t, +1) and 16t+4j+2 (columns 16j+8+2t, +1).
 __device__ __forceinline__ int b_perm(int kk)
 {
     const int j = kk >> 4, rem = kk & 15;
@@ -84,15 +93,26 @@ __device__ __forceinline__ int b_perm(int kk)
     return 16 * t + 4 * j + q;
 }
 
+// Element offset of (row r, column k) in an operand copy with RP rows: block
+// kt = k/64 is [RP][64]; the 16-byte chunks of row r are XOR-swizzled by r&7.
+__device__ __forceinline__ size_t b_index(int r, int k, int RP)
+{
+    const int kt = k >> 6, p = b_perm(k & 63);
+    const int c = (p >> 3) ^ (r & 7);
+    return ((size_t)kt * RP + r) * 64 + c * 8 + (p & 7);
+}
+
 // ------------------------------------------------------------------ prep
-// One warp per row: B-operand copy (+ row exponent) of a bf16 or fp32 row.
-// With `groups` set, the last CTA writes the per-expert token-group prefix.
+// One warp per row: operand copy (+ row exponent) of a bf16 or fp32 row
+// (read directly, or token gather[r]/gk of the source).  With `groups` set,
+// the last CTA writes the per-expert token-group prefix.
 template <bool IN_F32, bool OUT_F16>
 __global__ void __launch_bounds__(kPrepThreads) ffn_prep_kernel(const void* __restrict__ in, int rows, int K,
                                                                 uint16_t* __restrict__ out, int32_t* __restrict__ ex,
                                                                 const int32_t* __restrict__ offsets,
                                                                 const int32_t* __restrict__ slot_of, int E,
-                                                                int pool_slots, int32_t* __restrict__ groups)
+                                                                int pool_slots, int32_t* __restrict__ groups,
+                                                                const int32_t* __restrict__ gather, int gk)
 {
     const int lane = threadIdx.x & 31;
     if (groups && blockIdx.x == gridDim.x - 1) {
@@ -129,22 +149,27 @@ __global__ void __launch_bounds__(kPrepThreads) ffn_prep_kernel(const void* __re
         if (threadIdx.x == kPrepThreads - 1) groups[E] = run;
         return;
     }
+    const int RP = rows + kRowPad;
     const int nblocks = gridDim.x - (groups ? 1 : 0);
     const int warps_total = nblocks * (kPrepThreads / 32);
     for (int r = blockIdx.x * (kPrepThreads / 32) + (threadIdx.x >> 5); r < rows; r += warps_total) {
+        const size_t sr = gather ? (size_t)(__ldg(gather + r) / gk) : (size_t)r;   // source row
+        auto load4 = [&](int c, float (&v)[4]) {
+            if (IN_F32) {
+                float4 q = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(in) + sr * K) + c);
+                v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+            } else {
+                uint2 q = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(in) + sr * K) + c);
+                v[0] = bf16_bits_to_f32(q.x & 0xFFFF); v[1] = bf16_bits_to_f32(q.x >> 16);
+                v[2] = bf16_bits_to_f32(q.y & 0xFFFF); v[3] = bf16_bits_to_f32(q.y >> 16);
+            }
+        };
         int p = 0;
         if (OUT_F16) {
             float mx = 0.0f;
             for (int c = lane; c < K / 4; c += 32) {
                 float v[4];
-                if (IN_F32) {
-                    float4 q = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(in) + (size_t)r * K) + c);
-                    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-                } else {
-                    uint2 q = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(in) + (size_t)r * K) + c);
-                    v[0] = bf16_bits_to_f32(q.x & 0xFFFF); v[1] = bf16_bits_to_f32(q.x >> 16);
-                    v[2] = bf16_bits_to_f32(q.y & 0xFFFF); v[3] = bf16_bits_to_f32(q.y >> 16);
-                }
+                load4(c, v);
 #pragma unroll
                 for (int i = 0; i < 4; i++) mx = fmaxf(mx, fabsf(v[i]));
             }
@@ -161,15 +186,7 @@ __global__ void __launch_bounds__(kPrepThreads) ffn_prep_kernel(const void* __re
         const float sc = ldexpf(1.0f, p);
         for (int c = lane; c < K / 4; c += 32) {
             float v[4];
-            if (IN_F32) {
-                float4 q = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(in) + (size_t)r * K) + c);
-                v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-            } else {
-                uint2 q = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(in) + (size_t)r * K) + c);
-                v[0] = bf16_bits_to_f32(q.x & 0xFFFF); v[1] = bf16_bits_to_f32(q.x >> 16);
-                v[2] = bf16_bits_to_f32(q.y & 0xFFFF); v[3] = bf16_bits_to_f32(q.y >> 16);
-            }
-            const int k0 = 4 * c, blk = k0 & ~63;
+            load4(c, v);
 #pragma unroll
             for (int i = 0; i < 4; i++) {
                 uint16_t o;
@@ -179,7 +196,7 @@ __global__ void __launch_bounds__(kPrepThreads) ffn_prep_kernel(const void* __re
                 } else {
                     o = f32_to_bf16_bits(v[i]);
                 }
-                out[(size_t)r * K + blk + b_perm((k0 + i) & 63)] = o;
+                out[b_index(r, 4 * c + i, RP)] = o;
             }
         }
     }
@@ -195,11 +212,40 @@ struct FfnArgs {
     const int32_t* offsets;
     const int32_t* groups;
     int rows;
-    const uint16_t* in;     // [rows][K] B-operand copy
+    const uint16_t* in;     // operand copy [K/64][rows+16][64]
     const int32_t* in_ex;   // [rows] its exponents (FP4 formats)
     float* out_h;           // phase 1: h [rows][R/2] fp32
     uint16_t* out_y;        // phase 2: y [rows][R] bf16
 };
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+// Bounded wait (about 2 s of clock), false on timeout.
+__device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
+{
+    if (mbar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try(bar, parity))
+        if (clock64() - t0 > kWaitCycles) return false;
+    return true;
+}
+
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
 
 __device__ __forceinline__ void e2m1x4_to_f16x2(uint32_t w, uint32_t& f0, uint32_t& f1, uint32_t& f2, uint32_t& f3)
 {
@@ -242,202 +288,278 @@ __device__ __forceinline__ float e4m3_value(uint32_t c)
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 
+template <int WFMT>
+struct StreamCfg {
+    static constexpr bool FP4 = WFMT != MOE_W_BF16;
+    static constexpr int TILE = FP4 ? 512 : 2048;                 // weight tile bytes
+    static constexpr int STILE = (WFMT == MOE_W_MXFP4) ? 32 : (WFMT == MOE_W_NVFP4 ? 64 : 0);
+    static constexpr int DA = FP4 ? 16 : 4;                       // weight tiles in flight per warp
+    static constexpr int DX = 8;                                  // activation tiles in flight per warp
+    static constexpr int XSTAGE = 2 * 1024;                       // two 8-row blocks
+    static constexpr int WARP_BYTES = DA * (TILE + STILE) + DX * XSTAGE + 8 * (DA + DX);
+};
+
+template <int WFMT>
+size_t stream_smem_bytes(int E)
+{
+    return 128 + (size_t)(kFfnThreads / 32) * StreamCfg<WFMT>::WARP_BYTES + 4 * (size_t)(E + 1);
+}
+
+struct Unit {
+    int e, rt, row0, row_end, nq;
+    const char* blob;
+};
+
+__device__ __forceinline__ Unit unit_of(const FfnArgs& a, const int* s_groups, int u, int RT)
+{
+    Unit U;
+    const int gi = u / RT;
+    U.rt = u % RT;
+    int lo = 0, hi = a.E - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (s_groups[mid] <= gi) lo = mid;
+        else hi = mid - 1;
+    }
+    U.e = lo;
+    U.row0 = a.offsets[lo] + (gi - s_groups[lo]) * kRowsPerUnit;
+    U.row_end = min(min(a.offsets[lo + 1], U.row0 + kRowsPerUnit), a.rows);
+    U.nq = (U.row_end - U.row0 + 7) >> 3;
+    U.blob = a.pool + (size_t)a.slot_of[lo] * a.slot_bytes;
+    return U;
+}
+
 template <int WFMT, int PHASE>
 __global__ void __launch_bounds__(kFfnThreads) ffn_kernel(FfnArgs a)
 {
-    extern __shared__ int s_groups[];          // [E+1]
-    const int tid = threadIdx.x, lane = tid & 31, g = lane >> 2, t = lane & 3;
-    const int RT = a.R / 16, KT = a.K / 64;
-    const int E = a.E;
-    constexpr bool FP4 = WFMT != MOE_W_BF16;
-    for (int i = tid; i <= E; i += kFfnThreads) s_groups[i] = a.groups[i];
+    using CFG = StreamCfg<WFMT>;
+    constexpr bool FP4 = CFG::FP4;
+    constexpr int TILE = CFG::TILE, STILE = CFG::STILE, DA = CFG::DA, DX = CFG::DX, XSTAGE = CFG::XSTAGE;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int tid = threadIdx.x, lane = tid & 31, wib = tid >> 5, g = lane >> 2, t = lane & 3;
+    const int RT = a.R / 16, KT = a.K / 64, RP = a.rows + kRowPad;
+    unsigned char* wbase = smem + 128 + (size_t)wib * CFG::WARP_BYTES;
+    unsigned char* sA = wbase;                                    // DA x TILE
+    unsigned char* sS = sA + DA * TILE;                           // DA x STILE
+    unsigned char* sX = sS + DA * STILE;                          // DX x XSTAGE
+    uint64_t* barA = reinterpret_cast<uint64_t*>(sX + DX * XSTAGE);
+    uint64_t* barX = barA + DA;
+    int* s_groups = reinterpret_cast<int*>(smem + 128 + (size_t)(kFfnThreads / 32) * CFG::WARP_BYTES);
+    for (int i = tid; i <= a.E; i += kFfnThreads) s_groups[i] = a.groups[i];
+    if (lane == 0) {
+        for (int i = 0; i < DA; i++)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&barA[i])) : "memory");
+        for (int i = 0; i < DX; i++)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&barX[i])) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
     __syncthreads();
-    const int total = s_groups[E] * RT;
+    const int total_units = s_groups[a.E] * RT;
     const int warps_total = gridDim.x * (kFfnThreads / 32);
+    const int wg = blockIdx.x * (kFfnThreads / 32) + wib;
+    const int n_units = wg < total_units ? (total_units - 1 - wg) / warps_total + 1 : 0;
+    const long n_tiles = (long)n_units * KT;
 
-    constexpr int PF = FP4 ? 8 : 2;          // weight tiles in flight
-    constexpr int TILE = FP4 ? 512 : 2048;
-    constexpr int STILE = (WFMT == MOE_W_MXFP4) ? 32 : 64;
-    constexpr int NV = FP4 ? 1 : 4;          // uint4 per lane per tile
-    constexpr int XPF = 2;                   // activation tiles in flight (PF is a multiple)
-
-    for (int u = blockIdx.x * (kFfnThreads / 32) + (tid >> 5); u < total; u += warps_total) {
-        const int gi = u / RT, rt = u % RT;
-        int lo = 0, hi = E - 1;
-        while (lo < hi) {
-            int mid = (lo + hi + 1) >> 1;
-            if (s_groups[mid] <= gi) lo = mid;
-            else hi = mid - 1;
+    // producer (lane 0): issues tile n of this warp's stream into its ring stages
+    Unit pa, px;             // unit of the weight / activation stream head
+    int pa_idx = -1, px_idx = -1;
+    auto issue_a = [&](long n) {
+        const int ui = (int)(n / KT), kt = (int)(n % KT);
+        if (ui != pa_idx) {
+            pa = unit_of(a, s_groups, wg + ui * warps_total, RT);
+            pa_idx = ui;
         }
-        const int e = lo;
-        const int row0 = a.offsets[e] + (gi - s_groups[e]) * kRowsPerUnit;
-        const int row_end = min(min(a.offsets[e + 1], row0 + kRowsPerUnit), a.rows);
-        const int nq = (row_end - row0 + 7) >> 3;
-        const char* blob = a.pool + (size_t)a.slot_of[e] * a.slot_bytes;
-        const char* wt = blob + a.w_off + (size_t)rt * KT * TILE;
-        const char* st = blob + a.s_off + (size_t)rt * KT * STILE;
-
-        // activation row of this lane (token g of each n-tile), -1 for padding
-        int xr[2];
-#pragma unroll
-        for (int q = 0; q < 2; q++) xr[q] = (row0 + 8 * q + g < row_end) ? row0 + 8 * q + g : -1;
-
-        float acc[2][4];
-#pragma unroll
-        for (int q = 0; q < 2; q++)
-#pragma unroll
-            for (int i = 0; i < 4; i++) acc[q][i] = 0.0f;
-
-        uint4 abuf[PF][NV];
-        uint2 sbuf[PF];
-        uint4 xbuf[XPF][2][2];
-        auto load_a = [&](int i, int kt) {
-#pragma unroll
-            for (int v = 0; v < NV; v++)
-                abuf[i][v] = __ldg(reinterpret_cast<const uint4*>(wt + (size_t)kt * TILE + v * 512 + 16 * lane));
-            if (WFMT == MOE_W_MXFP4) sbuf[i].x = __ldg(reinterpret_cast<const uint32_t*>(st + (size_t)kt * STILE + 4 * g));
-            if (WFMT == MOE_W_NVFP4) sbuf[i] = __ldg(reinterpret_cast<const uint2*>(st + (size_t)kt * STILE + 8 * g));
-        };
-        auto load_x = [&](int i, int kt) {
-#pragma unroll
-            for (int q = 0; q < 2; q++) {
-                if (xr[q] >= 0) {
-                    const uint4* p = reinterpret_cast<const uint4*>(a.in + (size_t)xr[q] * a.K + kt * 64 + 16 * t);
-                    xbuf[i][q][0] = __ldg(p);
-                    xbuf[i][q][1] = __ldg(p + 1);
-                } else {
-                    xbuf[i][q][0] = xbuf[i][q][1] = make_uint4(0, 0, 0, 0);
-                }
-            }
-        };
-#pragma unroll
-        for (int i = 0; i < PF; i++)
-            if (i < KT) load_a(i, i);
-#pragma unroll
-        for (int i = 0; i < XPF; i++)
-            if (i < KT) load_x(i, i);
-
-        for (int kt0 = 0; kt0 < KT; kt0 += PF) {
-#pragma unroll
-            for (int i = 0; i < PF; i++) {
-                const int kt = kt0 + i;
-                if (kt >= KT) break;
-                uint4 cur[NV];
-#pragma unroll
-                for (int v = 0; v < NV; v++) cur[v] = abuf[i][v];
-                const uint2 cs = sbuf[i];
-                if (kt + PF < KT) load_a(i, kt + PF);
-                const int xi = i % XPF;   // static once the loop is unrolled
-                uint4 xc[2][2];
-#pragma unroll
-                for (int q = 0; q < 2; q++) {
-                    xc[q][0] = xbuf[xi][q][0];
-                    xc[q][1] = xbuf[xi][q][1];
-                }
-                if (kt + XPF < KT) load_x(xi, kt + XPF);
-                if (!FP4) {
-                    // bf16 fragments: cur[j] = {a0, a2, a1, a3} of step j
-#pragma unroll
-                    for (int q = 0; q < 2; q++) {
-                        if (q >= nq) break;
-                        const uint32_t X[8] = {xc[q][0].x, xc[q][0].y, xc[q][0].z, xc[q][0].w,
-                                               xc[q][1].x, xc[q][1].y, xc[q][1].z, xc[q][1].w};
-#pragma unroll
-                        for (int j = 0; j < 4; j++)
-                            mma16816<false>(acc[q], cur[j].x, cur[j].z, cur[j].y, cur[j].w, X[2 * j], X[2 * j + 1]);
-                    }
-                } else {
-                    // f16 fragments from E2M1 bytes: row g bytes in .x/.y, row g+8 in .z/.w;
-                    // byte 2j -> a0 (a1) of step j, byte 2j+1 -> a2 (a3)
-                    uint32_t A[4][4];
-                    uint32_t f0, f1, f2, f3;
-                    e2m1x4_to_f16x2(cur[0].x, f0, f1, f2, f3);
-                    A[0][0] = f0; A[0][2] = f1; A[1][0] = f2; A[1][2] = f3;
-                    e2m1x4_to_f16x2(cur[0].y, f0, f1, f2, f3);
-                    A[2][0] = f0; A[2][2] = f1; A[3][0] = f2; A[3][2] = f3;
-                    e2m1x4_to_f16x2(cur[0].z, f0, f1, f2, f3);
-                    A[0][1] = f0; A[0][3] = f1; A[1][1] = f2; A[1][3] = f3;
-                    e2m1x4_to_f16x2(cur[0].w, f0, f1, f2, f3);
-                    A[2][1] = f0; A[2][3] = f1; A[3][1] = f2; A[3][3] = f3;
-                    float sg[4], s8[4];   // scale of k16 steps 0..3 for rows g and g+8
-                    if (WFMT == MOE_W_MXFP4) {
-                        sg[0] = sg[1] = mx_scale(cs.x & 0xFF);
-                        sg[2] = sg[3] = mx_scale((cs.x >> 8) & 0xFF);
-                        s8[0] = s8[1] = mx_scale((cs.x >> 16) & 0xFF);
-                        s8[2] = s8[3] = mx_scale(cs.x >> 24);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 4; j++) {
-                            sg[j] = e4m3_value((cs.x >> (8 * j)) & 0xFF);
-                            s8[j] = e4m3_value((cs.y >> (8 * j)) & 0xFF);
-                        }
-                    }
-                    constexpr int SPB = (WFMT == MOE_W_MXFP4) ? 2 : 1;   // k16 steps per scale block
-#pragma unroll
-                    for (int q = 0; q < 2; q++) {
-                        if (q >= nq) break;
-                        const uint32_t X[8] = {xc[q][0].x, xc[q][0].y, xc[q][0].z, xc[q][0].w,
-                                               xc[q][1].x, xc[q][1].y, xc[q][1].z, xc[q][1].w};
-#pragma unroll
-                        for (int j0 = 0; j0 < 4; j0 += SPB) {
-                            float tmp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-                            for (int j = j0; j < j0 + SPB; j++)
-                                mma16816<true>(tmp, A[j][0], A[j][1], A[j][2], A[j][3], X[2 * j], X[2 * j + 1]);
-                            acc[q][0] = __fmaf_rn(tmp[0], sg[j0], acc[q][0]);
-                            acc[q][1] = __fmaf_rn(tmp[1], sg[j0], acc[q][1]);
-                            acc[q][2] = __fmaf_rn(tmp[2], s8[j0], acc[q][2]);
-                            acc[q][3] = __fmaf_rn(tmp[3], s8[j0], acc[q][3]);
-                        }
-                    }
-                }
-            }
+        const Unit& pu = pa;
+        const int st = (int)(n % DA);
+        const uint32_t bar = smem_u32(&barA[st]);
+        const size_t ti = tile_index(pu.rt, kt, RT, KT);
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(TILE + STILE) : "memory");
+        bulk_copy(smem_u32(sA + st * TILE), pu.blob + a.w_off + ti * TILE, TILE, bar);
+        if (STILE) bulk_copy(smem_u32(sS + st * STILE), pu.blob + a.s_off + ti * STILE, STILE, bar);
+    };
+    auto issue_x = [&](long n) {
+        const int ui = (int)(n / KT), kt = (int)(n % KT);
+        if (ui != px_idx) {
+            px = unit_of(a, s_groups, wg + ui * warps_total, RT);
+            px_idx = ui;
         }
-        // epilogue: undo the activation row exponents, apply the NVFP4 tensor scale
-        float tsc = 1.0f;
-        if (WFMT == MOE_W_NVFP4) tsc = reinterpret_cast<const float*>(blob + a.ts_off)[PHASE - 1];
+        const Unit& pu = px;
+        const int st = (int)(n % DX);
+        const uint32_t bar = smem_u32(&barX[st]);
+        const uint32_t bytes = (uint32_t)pu.nq * 1024;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+        bulk_copy(smem_u32(sX + st * XSTAGE), a.in + ((size_t)kt * RP + pu.row0) * 64, bytes, bar);
+    };
+    long na = 0, nx = 0;   // tiles issued (lane 0 only)
+    if (lane == 0) {
+        for (; na < DA && na < n_tiles; na++) issue_a(na);
+        for (; nx < DX && nx < n_tiles; nx++) issue_x(nx);
+    }
+
+    bool ok = true;
+    long n = 0;
+    Unit cu;
+    float acc[2][4];
+    for (; n < n_tiles; n++) {
+        const int kt = (int)(n % KT);
+        if (kt == 0) {
+            cu = unit_of(a, s_groups, wg + (int)(n / KT) * warps_total, RT);
+#pragma unroll
+            for (int q = 0; q < 2; q++)
+#pragma unroll
+                for (int i = 0; i < 4; i++) acc[q][i] = 0.0f;
+        }
+        const int sa = (int)(n % DA), sx = (int)(n % DX);
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&barA[sa]), (uint32_t)((n / DA) & 1)) &&
+                                          mbar_wait_bounded(smem_u32(&barX[sx]), (uint32_t)((n / DX) & 1)));
+        if (!ok) break;
+        // operands from shared memory
+        uint4 cur[FP4 ? 1 : 4];
+#pragma unroll
+        for (int v = 0; v < (FP4 ? 1 : 4); v++) cur[v] = *reinterpret_cast<const uint4*>(sA + sa * TILE + v * 512 + 16 * lane);
+        uint2 cs = make_uint2(0, 0);
+        if (WFMT == MOE_W_MXFP4) cs.x = *reinterpret_cast<const uint32_t*>(sS + sa * STILE + 4 * g);
+        if (WFMT == MOE_W_NVFP4) cs = *reinterpret_cast<const uint2*>(sS + sa * STILE + 8 * g);
+        const int sw = (cu.row0 + g) & 7;
+        uint4 xc[2][2];
 #pragma unroll
         for (int q = 0; q < 2; q++) {
-            if (q >= nq) break;
-            const int r0 = row0 + q * 8 + 2 * t, r1 = r0 + 1;
-            float u0 = tsc, u1 = tsc;
-            if (FP4) {
-                if (r0 < row_end) u0 = ldexpf(tsc, -__ldg(a.in_ex + r0));
-                if (r1 < row_end) u1 = ldexpf(tsc, -__ldg(a.in_ex + r1));
-            }
-            if (PHASE == 1) {
-                const int F = a.R / 2;
-                const int f = 8 * rt + g;
-                if (r0 < row_end) a.out_h[(size_t)r0 * F + f] = silu(acc[q][0] * u0) * (acc[q][2] * u0);
-                if (r1 < row_end) a.out_h[(size_t)r1 * F + f] = silu(acc[q][1] * u1) * (acc[q][3] * u1);
+            if (q < cu.nq) {
+                const unsigned char* xrow = sX + sx * XSTAGE + q * 1024 + g * 128;
+                xc[q][0] = *reinterpret_cast<const uint4*>(xrow + (((2 * t) ^ sw) << 4));
+                xc[q][1] = *reinterpret_cast<const uint4*>(xrow + (((2 * t + 1) ^ sw) << 4));
             } else {
-                const int Ho = a.R;
-                const int o = 16 * rt + g;
-                if (r0 < row_end) {
-                    a.out_y[(size_t)r0 * Ho + o] = f32_to_bf16_bits(acc[q][0] * u0);
-                    a.out_y[(size_t)r0 * Ho + o + 8] = f32_to_bf16_bits(acc[q][2] * u0);
+                xc[q][0] = xc[q][1] = make_uint4(0, 0, 0, 0);
+            }
+        }
+        // stages consumed: refill them with the tiles DA / DX ahead
+        __syncwarp();
+        if (lane == 0) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            if (na < n_tiles) issue_a(na++);
+            if (nx < n_tiles) issue_x(nx++);
+        }
+        if (!FP4) {
+            // bf16 fragments: cur[j] = {a0, a2, a1, a3} of step j
+#pragma unroll
+            for (int q = 0; q < 2; q++) {
+                if (q >= cu.nq) break;
+                const uint32_t X[8] = {xc[q][0].x, xc[q][0].y, xc[q][0].z, xc[q][0].w,
+                                       xc[q][1].x, xc[q][1].y, xc[q][1].z, xc[q][1].w};
+#pragma unroll
+                for (int j = 0; j < 4; j++)
+                    mma16816<false>(acc[q], cur[j].x, cur[j].z, cur[j].y, cur[j].w, X[2 * j], X[2 * j + 1]);
+            }
+        } else {
+            // f16 fragments from E2M1 bytes: row g bytes in .x/.y, row g+8 in .z/.w;
+            // byte 2j -> a0 (a1) of step j, byte 2j+1 -> a2 (a3)
+            uint32_t A[4][4];
+            uint32_t f0, f1, f2, f3;
+            e2m1x4_to_f16x2(cur[0].x, f0, f1, f2, f3);
+            A[0][0] = f0; A[0][2] = f1; A[1][0] = f2; A[1][2] = f3;
+            e2m1x4_to_f16x2(cur[0].y, f0, f1, f2, f3);
+            A[2][0] = f0; A[2][2] = f1; A[3][0] = f2; A[3][2] = f3;
+            e2m1x4_to_f16x2(cur[0].z, f0, f1, f2, f3);
+            A[0][1] = f0; A[0][3] = f1; A[1][1] = f2; A[1][3] = f3;
+            e2m1x4_to_f16x2(cur[0].w, f0, f1, f2, f3);
+            A[2][1] = f0; A[2][3] = f1; A[3][1] = f2; A[3][3] = f3;
+            float sg[4], s8[4];   // scale of k16 steps 0..3 for rows g and g+8
+            if (WFMT == MOE_W_MXFP4) {
+                sg[0] = sg[1] = mx_scale(cs.x & 0xFF);
+                sg[2] = sg[3] = mx_scale((cs.x >> 8) & 0xFF);
+                s8[0] = s8[1] = mx_scale((cs.x >> 16) & 0xFF);
+                s8[2] = s8[3] = mx_scale(cs.x >> 24);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    sg[j] = e4m3_value((cs.x >> (8 * j)) & 0xFF);
+                    s8[j] = e4m3_value((cs.y >> (8 * j)) & 0xFF);
                 }
-                if (r1 < row_end) {
-                    a.out_y[(size_t)r1 * Ho + o] = f32_to_bf16_bits(acc[q][1] * u1);
-                    a.out_y[(size_t)r1 * Ho + o + 8] = f32_to_bf16_bits(acc[q][3] * u1);
+            }
+            constexpr int SPB = (WFMT == MOE_W_MXFP4) ? 2 : 1;   // k16 steps per scale block
+#pragma unroll
+            for (int q = 0; q < 2; q++) {
+                if (q >= cu.nq) break;
+                const uint32_t X[8] = {xc[q][0].x, xc[q][0].y, xc[q][0].z, xc[q][0].w,
+                                       xc[q][1].x, xc[q][1].y, xc[q][1].z, xc[q][1].w};
+#pragma unroll
+                for (int j0 = 0; j0 < 4; j0 += SPB) {
+                    float tmp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                    for (int j = j0; j < j0 + SPB; j++)
+                        mma16816<true>(tmp, A[j][0], A[j][1], A[j][2], A[j][3], X[2 * j], X[2 * j + 1]);
+                    acc[q][0] = __fmaf_rn(tmp[0], sg[j0], acc[q][0]);
+                    acc[q][1] = __fmaf_rn(tmp[1], sg[j0], acc[q][1]);
+                    acc[q][2] = __fmaf_rn(tmp[2], s8[j0], acc[q][2]);
+                    acc[q][3] = __fmaf_rn(tmp[3], s8[j0], acc[q][3]);
                 }
             }
         }
+        if (kt == KT - 1) {
+            // epilogue: undo the activation row exponents, apply the NVFP4 tensor scale
+            float tsc = 1.0f;
+            if (WFMT == MOE_W_NVFP4) tsc = reinterpret_cast<const float*>(cu.blob + a.ts_off)[PHASE - 1];
+#pragma unroll
+            for (int q = 0; q < 2; q++) {
+                if (q >= cu.nq) break;
+                const int r0 = cu.row0 + q * 8 + 2 * t, r1 = r0 + 1;
+                float u0 = tsc, u1 = tsc;
+                if (FP4) {
+                    if (r0 < cu.row_end) u0 = ldexpf(tsc, -__ldg(a.in_ex + r0));
+                    if (r1 < cu.row_end) u1 = ldexpf(tsc, -__ldg(a.in_ex + r1));
+                }
+                if (PHASE == 1) {
+                    const int F = a.R / 2;
+                    const int f = 8 * cu.rt + g;
+                    if (r0 < cu.row_end) a.out_h[(size_t)r0 * F + f] = silu(acc[q][0] * u0) * (acc[q][2] * u0);
+                    if (r1 < cu.row_end) a.out_h[(size_t)r1 * F + f] = silu(acc[q][1] * u1) * (acc[q][3] * u1);
+                } else {
+                    const int Ho = a.R;
+                    const int o = 16 * cu.rt + g;
+                    if (r0 < cu.row_end) {
+                        a.out_y[(size_t)r0 * Ho + o] = f32_to_bf16_bits(acc[q][0] * u0);
+                        a.out_y[(size_t)r0 * Ho + o + 8] = f32_to_bf16_bits(acc[q][2] * u0);
+                    }
+                    if (r1 < cu.row_end) {
+                        a.out_y[(size_t)r1 * Ho + o] = f32_to_bf16_bits(acc[q][1] * u1);
+                        a.out_y[(size_t)r1 * Ho + o + 8] = f32_to_bf16_bits(acc[q][3] * u1);
+                    }
+                }
+            }
+        }
+    }
+    if (!ok) {
+        // a wait ran out: record it, then let every copy still in flight land
+        if (lane == 0) {
+            atomicCAS(&g_ffn_error, 0, (int)MOE_ERR_TIMEOUT);
+            for (long m = n; m < na; m++) mbar_wait_bounded(smem_u32(&barA[m % DA]), (uint32_t)((m / DA) & 1));
+            for (long m = n; m < nx; m++) mbar_wait_bounded(smem_u32(&barX[m % DX]), (uint32_t)((m / DX) & 1));
+        }
+        __syncwarp();
     }
 }
 
 template <int WFMT>
 int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, size_t slot_bytes, int pool_slots,
                   const int32_t* slot_of, const int32_t* offsets, const uint16_t* x_perm, int rows,
-                  uint16_t* y_perm, const FfnWs& w, int sms, cudaStream_t st)
+                  uint16_t* y_perm, const FfnWs& w, int sms, cudaStream_t st, const RowSource* gather)
 {
     constexpr bool FP4 = WFMT != MOE_W_BF16;
     const int E = s->experts, H = s->hidden, F = s->ffn;
     const int wpb = kPrepThreads / 32;
     int prep_blocks = (rows + wpb - 1) / wpb;
     if (prep_blocks > sms * 4) prep_blocks = sms * 4;
-    ffn_prep_kernel<false, FP4><<<prep_blocks + 1, kPrepThreads, 0, st>>>(x_perm, rows, H, w.xb, w.xe, offsets,
-                                                                           slot_of, E, pool_slots, w.groups);
+    if (gather && gather->x_dtype == MOE_DT_F32)
+        ffn_prep_kernel<true, FP4><<<prep_blocks + 1, kPrepThreads, 0, st>>>(
+            gather->x, rows, H, w.xb, w.xe, offsets, slot_of, E, pool_slots, w.groups, gather->assign_of, gather->k);
+    else if (gather)
+        ffn_prep_kernel<false, FP4><<<prep_blocks + 1, kPrepThreads, 0, st>>>(
+            gather->x, rows, H, w.xb, w.xe, offsets, slot_of, E, pool_slots, w.groups, gather->assign_of, gather->k);
+    else
+        ffn_prep_kernel<false, FP4><<<prep_blocks + 1, kPrepThreads, 0, st>>>(x_perm, rows, H, w.xb, w.xe, offsets,
+                                                                               slot_of, E, pool_slots, w.groups,
+                                                                               nullptr, 1);
     MOE_LAUNCH_CHECK();
     FfnArgs a{};
     a.pool = static_cast<const char*>(pool);
@@ -448,10 +570,12 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     a.offsets = offsets;
     a.groups = w.groups;
     a.rows = rows;
-    const size_t smem = sizeof(int) * (E + 1);
-    // persistent grid: as many CTAs as fit at once (registers bound residency)
+    const size_t smem = stream_smem_bytes<WFMT>(E);
+    // persistent grid: as many CTAs as fit at once
     static int resident[2] = {0, 0};
     if (!resident[0]) {
+        MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_kernel<WFMT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_kernel<WFMT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
         MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident[0], ffn_kernel<WFMT, 1>, kFfnThreads, smem));
         MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident[1], ffn_kernel<WFMT, 2>, kFfnThreads, smem));
         if (resident[0] < 1) resident[0] = 1;
@@ -473,7 +597,7 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     ffn_kernel<WFMT, 1><<<grid_for(a.R, 1), kFfnThreads, smem, st>>>(a);
     MOE_LAUNCH_CHECK();
     ffn_prep_kernel<true, FP4><<<prep_blocks, kPrepThreads, 0, st>>>(w.h32, rows, F, w.hb, w.he, nullptr, nullptr,
-                                                                     E, 0, nullptr);
+                                                                     E, 0, nullptr, nullptr, 1);
     MOE_LAUNCH_CHECK();
     FfnArgs b = a;
     b.w_off = bl.w2;
@@ -505,9 +629,22 @@ bool use_tc_path(const moe_shape* s, int rows)
 
 size_t ffn_ws_bytes(const moe_shape* s, int rows) { return ffn_ws_layout(s, rows, nullptr, nullptr) + 256; }
 
+bool ffn_uses_tc(const moe_shape* s, int rows) { return use_tc_path(s, rows); }
+
+int ffn_device_error(int clear)
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_ffn_error, sizeof v) != cudaSuccess) return MOE_ERR_CUDA;
+    if (clear && v) {
+        int z = 0;
+        if (cudaMemcpyToSymbol(g_ffn_error, &z, sizeof z) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    return v;
+}
+
 int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
                const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,
-               cudaStream_t st)
+               cudaStream_t st, const RowSource* gather)
 {
     if (rows == 0) return MOE_OK;
     ProfScope ps(MOE_PROF_FFN, st);
@@ -525,13 +662,13 @@ int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool
     switch (s->wfmt) {
     case MOE_W_BF16:
         return launch_decode<MOE_W_BF16>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, x_perm, rows, y_perm,
-                                         w, sms, st);
+                                         w, sms, st, gather);
     case MOE_W_MXFP4:
         return launch_decode<MOE_W_MXFP4>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, x_perm, rows,
-                                          y_perm, w, sms, st);
+                                          y_perm, w, sms, st, gather);
     case MOE_W_NVFP4:
         return launch_decode<MOE_W_NVFP4>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, x_perm, rows,
-                                          y_perm, w, sms, st);
+                                          y_perm, w, sms, st, gather);
     }
     return MOE_ERR_INVALID_ARG;
 }

@@ -234,9 +234,15 @@ __device__ __forceinline__ Tile tile_of(int u, const int* prefix, int E, int RB,
     return t;
 }
 
+// Token-row tensor maps with boxes of 16, 32, 64 and 128 rows (64 columns):
+// a block of bn rows is loaded with at most four boxes.
+struct RowMaps {
+    CUtensorMap m[4];
+};
+
 template <int WFMT, int PHASE>
 __global__ void __launch_bounds__(THREADS, 1)
-    ffn_tc_kernel(TcArgs a, const __grid_constant__ CUtensorMap tmap_in)
+    ffn_tc_kernel(TcArgs a, const __grid_constant__ RowMaps maps)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -333,26 +339,29 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                 Tile t = tile_of(u, prefix, E, RB, a.offsets);
                 const char* blob = a.pool + (size_t)a.slot_of[t.e] * a.slot_bytes;
-                const char* wt = blob + a.w_off + (size_t)(8 * t.rb) * KT * 512;
-                const char* st = blob + a.s_off + (size_t)(8 * t.rb) * KT * STILE;
+                const int RT = a.R / 16;
                 for (int c = 0; c < KT && ok; c++) {
                     ok = mbar_wait(smem_u32(&empty_a[sa]), pa ^ 1, abort_v);
                     if (!ok) break;
-                    uint32_t fa = smem_u32(&full_a[sa]);
+                    const uint32_t fa = smem_u32(&full_a[sa]);
+                    const size_t ti = tile_index(8 * t.rb, c, RT, KT);   // 8 contiguous row tiles
                     mbar_expect_tx(fa, A_STAGE_BYTES + 8 * STILE);
-                    for (int i = 0; i < 8; i++) {
-                        bulk_g2s(smem_u32(sA + sa * A_STAGE_BYTES + i * 512), wt + ((size_t)i * KT + c) * 512, 512, fa);
-                        bulk_g2s(smem_u32(sS + sa * S_STAGE_BYTES + i * STILE), st + ((size_t)i * KT + c) * STILE,
-                                 STILE, fa);
-                    }
+                    bulk_g2s(smem_u32(sA + sa * A_STAGE_BYTES), blob + a.w_off + ti * 512, A_STAGE_BYTES, fa);
+                    bulk_g2s(smem_u32(sS + sa * S_STAGE_BYTES), blob + a.s_off + ti * STILE, 8 * STILE, fa);
                     if (++sa == SA) { sa = 0; pa ^= 1; }
                     ok = mbar_wait(smem_u32(&empty_b[sb]), pb ^ 1, abort_v);
                     if (!ok) break;
-                    uint32_t fb = smem_u32(&full_b[sb]);
-                    const int nbox = t.bn / 16;
-                    mbar_expect_tx(fb, (uint32_t)nbox * 16 * 128);
-                    for (int j = 0; j < nbox; j++)
-                        tma_load_2d(smem_u32(sB + sb * B_STAGE_BYTES + j * 2048), &tmap_in, c * BK, t.row0 + 16 * j, fb);
+                    const uint32_t fb = smem_u32(&full_b[sb]);
+                    mbar_expect_tx(fb, (uint32_t)t.bn * 128);
+                    int done = 0;
+#pragma unroll
+                    for (int mi = 3; mi >= 0; mi--) {
+                        const int box = 16 << mi;
+                        while (t.bn - done >= box) {
+                            tma_load_2d(smem_u32(sB + sb * B_STAGE_BYTES + done * 128), &maps.m[mi], c * BK, t.row0 + done, fb);
+                            done += box;
+                        }
+                    }
                     if (++sb == SB) { sb = 0; pb ^= 1; }
                 }
             }
@@ -516,19 +525,28 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// [rows][cols] bf16, boxes of 16 rows x 64 columns, 128-byte swizzle.
-int make_rows_map(CUtensorMap* m, const void* base, int rows, int cols)
+// [rows][cols] bf16, boxes of box_rows rows x 64 columns, 128-byte swizzle.
+int make_rows_map(CUtensorMap* m, const void* base, int rows, int cols, int box_rows)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return MOE_ERR_CUDA;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
     cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {64, 16};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int make_row_maps(RowMaps* rm, const void* base, int rows, int cols)
+{
+    for (int i = 0; i < 4; i++) {
+        int rc = make_rows_map(&rm->m[i], base, rows, cols, 16 << i);
+        if (rc) return rc;
+    }
+    return MOE_OK;
 }
 
 size_t tc_smem_bytes(int E)
@@ -538,7 +556,7 @@ size_t tc_smem_bytes(int E)
 }
 
 template <int WFMT, int PHASE>
-int launch_one(const TcArgs& a, const CUtensorMap& map, int rows, int sms, cudaStream_t st)
+int launch_one(const TcArgs& a, const RowMaps& map, int rows, int sms, cudaStream_t st)
 {
     size_t smem = tc_smem_bytes(a.E);
     static bool attr = false;
@@ -573,10 +591,10 @@ int launch_ffn_tc(const moe_shape* s, const void* pool, size_t slot_bytes, int p
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    CUtensorMap mx, mh;
+    RowMaps mx, mh;
     int rc;
-    if ((rc = make_rows_map(&mx, x_perm, rows, s->hidden))) return rc;
-    if ((rc = make_rows_map(&mh, h, rows, s->ffn))) return rc;
+    if ((rc = make_row_maps(&mx, x_perm, rows, s->hidden))) return rc;
+    if ((rc = make_row_maps(&mh, h, rows, s->ffn))) return rc;
     TcArgs a1{};
     a1.pool = static_cast<const char*>(pool);
     a1.slot_bytes = slot_bytes;
@@ -615,5 +633,6 @@ extern "C" int moe_get_device_error(int clear)
         int z = 0;
         if (cudaMemcpyToSymbol(moe::g_tc_error, &z, sizeof z) != cudaSuccess) return MOE_ERR_CUDA;
     }
-    return v;
+    const int d = moe::ffn_device_error(clear);
+    return v ? v : d;
 }

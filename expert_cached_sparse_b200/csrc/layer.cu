@@ -100,24 +100,30 @@ extern "C" int moe_layer_forward(moe_cache* c, int32_t layer, const void* d_x, i
     int rc;
     if ((rc = launch_router(d_x, x_dtype, d_wg, d_bias, n, H, E, k, L.logits, idx, w, st))) return rc;
     if ((rc = cache_launch_lookup(c, layer, idx, A, nullptr, st))) return rc;
-    if ((rc = launch_permute(idx, n, E, k, d_x, x_dtype, H, L.offsets, L.row_of, L.assign_of, L.x_perm, L.perm_ws,
-                             st)))
+    // The tensor-core path reads x_perm through TMA, so it is materialised; the
+    // decode path gathers token rows straight into its own operand copy.
+    const bool tc = ffn_uses_tc(s, A);
+    uint16_t* xp = tc ? L.x_perm : nullptr;
+    if ((rc = launch_permute(idx, n, E, k, d_x, x_dtype, H, L.offsets, L.row_of, L.assign_of, xp, L.perm_ws, st)))
         return rc;
+    const RowSource src{d_x, x_dtype, L.assign_of, k};
+    const RowSource* gather = tc ? nullptr : &src;
     const char* pool = cache_pool(c);
     const size_t sb = cache_slot_bytes(c);
+    const int C = cache_capacity_int(c);
     if (cache_layer_resident(c, layer)) {
         // every expert of this layer is resident: no miss is possible, nothing is read back
-        if ((rc = launch_ffn(s, pool, sb, cache_capacity_int(c), cache_slot_all(c), L.offsets, L.x_perm, A, L.y_perm, L.ffn_ws, st)))
+        if ((rc = launch_ffn(s, pool, sb, C, cache_slot_all(c), L.offsets, xp, A, L.y_perm, L.ffn_ws, st, gather)))
             return rc;
     } else {
         // hits first, while the host learns the miss list and issues the fills
-        if ((rc = launch_ffn(s, pool, sb, cache_capacity_int(c), cache_slot_hit(c), L.offsets, L.x_perm, A, L.y_perm, L.ffn_ws, st)))
+        if ((rc = launch_ffn(s, pool, sb, C, cache_slot_hit(c), L.offsets, xp, A, L.y_perm, L.ffn_ws, st, gather)))
             return rc;
         int nm = 0;
         if ((rc = cache_read_and_fill(c, layer, st, cp, &nm))) return rc;
         if (nm > 0) {
             MOE_CUDA_TRY(cudaStreamWaitEvent(st, cache_fill_event(c), 0));
-            if ((rc = launch_ffn(s, pool, sb, cache_capacity_int(c), cache_slot_miss(c), L.offsets, L.x_perm, A, L.y_perm, L.ffn_ws, st)))
+            if ((rc = launch_ffn(s, pool, sb, C, cache_slot_miss(c), L.offsets, xp, A, L.y_perm, L.ffn_ws, st, gather)))
                 return rc;
         }
     }

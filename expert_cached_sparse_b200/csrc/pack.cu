@@ -29,7 +29,7 @@ void pack_fp4_matrix(const uint8_t* q, int R, int K, bool w13, int F, uint8_t* o
     const int KT = K / 64;
     for (int rt = 0; rt < R / 16; rt++)
         for (int kt = 0; kt < KT; kt++) {
-            uint8_t* tile = out + ((size_t)rt * KT + kt) * 512;
+            uint8_t* tile = out + moe::tile_index(rt, kt, R / 16, KT) * 512;
             for (int L = 0; L < 32; L++) {
                 int g = L >> 2, t = L & 3;
                 for (int half = 0; half < 2; half++) {
@@ -47,7 +47,7 @@ void pack_fp4_scales(const uint8_t* sc, int R, int K, bool w13, int F, bool mx, 
     const int KT = K / 64, per = mx ? 32 : 16, nb = K / per, bpt = 64 / per, stile = mx ? 32 : 64;
     for (int rt = 0; rt < R / 16; rt++)
         for (int kt = 0; kt < KT; kt++) {
-            uint8_t* tile = out + ((size_t)rt * KT + kt) * stile;
+            uint8_t* tile = out + moe::tile_index(rt, kt, R / 16, KT) * stile;
             for (int g = 0; g < 8; g++)
                 for (int half = 0; half < 2; half++) {
                     int p = 16 * rt + g + 8 * half;
@@ -65,7 +65,7 @@ void pack_bf16_matrix(const uint16_t* w, int R, int K, bool w13, int F, uint8_t*
     const int KT = K / 64;
     for (int rt = 0; rt < R / 16; rt++)
         for (int kt = 0; kt < KT; kt++) {
-            uint8_t* tile = out + ((size_t)rt * KT + kt) * 2048;
+            uint8_t* tile = out + moe::tile_index(rt, kt, R / 16, KT) * 2048;
             for (int j = 0; j < 4; j++)
                 for (int L = 0; L < 32; L++) {
                     int g = L >> 2, t = L & 3;

@@ -146,8 +146,105 @@ __global__ void perm_scatter_gather_kernel(const int32_t* __restrict__ idx, int 
             row_of[a] = row;
             assign_of[row] = a;
         }
+        if (!x_perm) continue;
         const int t = a / k;
         uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)row * H);
+        if (XF32) {
+            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + (size_t)t * H);
+            for (int c = lane; c < H / 8; c += 32) {
+                float4 p = __ldg(src + 2 * c), q = __ldg(src + 2 * c + 1);
+                uint4 o;
+                o.x = (uint32_t)f32_to_bf16_bits(p.x) | ((uint32_t)f32_to_bf16_bits(p.y) << 16);
+                o.y = (uint32_t)f32_to_bf16_bits(p.z) | ((uint32_t)f32_to_bf16_bits(p.w) << 16);
+                o.z = (uint32_t)f32_to_bf16_bits(q.x) | ((uint32_t)f32_to_bf16_bits(q.y) << 16);
+                o.w = (uint32_t)f32_to_bf16_bits(q.z) | ((uint32_t)f32_to_bf16_bits(q.w) << 16);
+                dst[c] = o;
+            }
+        } else {
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + (size_t)t * H);
+            for (int c = lane; c < H / 8; c += 32) dst[c] = __ldg(src + c);
+        }
+    }
+}
+
+// Small calls (decode): one CTA does the whole index work.  Per-expert
+// counts, an exclusive block scan for the offsets, and for every assignment
+// its rank among earlier assignments to the same expert (a scan over the
+// call's indices held in shared memory).
+constexpr int kSmallA = 1024;
+constexpr int kSmallE = 1024;
+
+__global__ void __launch_bounds__(1024) perm_small_kernel(const int32_t* __restrict__ idx, int A, int E,
+                                                          int32_t* __restrict__ offsets, int32_t* __restrict__ row_of,
+                                                          int32_t* __restrict__ assign_of)
+{
+    __shared__ int s_idx[kSmallA];
+    __shared__ int s_cnt[kSmallE];
+    __shared__ int s_warp[32];
+    __shared__ int s_tot;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
+    __syncthreads();
+    for (int a = tid; a < A; a += blockDim.x) {
+        int e = idx[a];
+        if (e < 0 || e >= E) e = -1;          // out-of-range experts get no row
+        s_idx[a] = e;
+        if (e >= 0) atomicAdd(&s_cnt[e], 1);  // integer counts: order-independent
+    }
+    __syncthreads();
+    // offsets: exclusive scan of the counts (E <= blockDim.x)
+    const int v = (tid < E) ? s_cnt[tid] : 0;
+    int inc = v;
+    for (int off = 1; off < 32; off <<= 1) {
+        int o = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += o;
+    }
+    if (lane == 31) s_warp[w] = inc;
+    __syncthreads();
+    if (w == 0) {
+        int x = (lane < (int)(blockDim.x >> 5)) ? s_warp[lane] : 0;
+        int xi = x;
+        for (int off = 1; off < 32; off <<= 1) {
+            int o = __shfl_up_sync(0xffffffffu, xi, off);
+            if (lane >= off) xi += o;
+        }
+        s_warp[lane] = xi - x;
+        if (lane == 31) s_tot = xi;
+    }
+    __syncthreads();
+    const int excl = s_warp[w] + inc - v;
+    __syncthreads();
+    if (tid < E) {
+        offsets[tid] = excl;
+        s_cnt[tid] = excl;                    // reuse as the base row of each expert
+    }
+    if (tid == 0) offsets[E] = s_tot;
+    __syncthreads();
+    for (int a = tid; a < A; a += blockDim.x) {
+        const int e = s_idx[a];
+        if (e < 0) {
+            row_of[a] = -1;
+            continue;
+        }
+        int rank = 0;
+        for (int b = 0; b < a; b++) rank += (s_idx[b] == e);
+        const int row = s_cnt[e] + rank;
+        row_of[a] = row;
+        assign_of[row] = a;
+    }
+}
+
+// x_perm[row] = bf16(x[assign_of[row] / k]): one warp per row.
+template <bool XF32>
+__global__ void perm_gather_kernel(const int32_t* __restrict__ assign_of, const int32_t* __restrict__ offsets, int E,
+                                   int k, const void* __restrict__ x, int H, uint16_t* __restrict__ x_perm)
+{
+    const int lane = threadIdx.x & 31;
+    const int rows = offsets[E];
+    const int warps_total = gridDim.x * (blockDim.x >> 5);
+    for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps_total) {
+        const int t = assign_of[r] / k;
+        uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * H);
         if (XF32) {
             const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + (size_t)t * H);
             for (int c = lane; c < H / 8; c += 32) {
@@ -180,6 +277,23 @@ int launch_permute(const int32_t* idx, int n, int E, int k, const void* x, int x
         return MOE_OK;
     }
     ProfScope ps(MOE_PROF_PERMUTE, st);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (A <= kSmallA && E <= kSmallE) {
+        perm_small_kernel<<<1, 1024, 0, st>>>(idx, A, E, offsets, row_of, assign_of);
+        MOE_LAUNCH_CHECK();
+        prof_count(MOE_PROF_PERMUTE, x_perm ? 2 : 1);
+        if (!x_perm) return MOE_OK;
+        int grid = (A + 7) / 8;
+        if (grid > sms * 8) grid = sms * 8;
+        if (x_dtype == MOE_DT_F32)
+            perm_gather_kernel<true><<<grid, 256, 0, st>>>(assign_of, offsets, E, k, x, H, x_perm);
+        else
+            perm_gather_kernel<false><<<grid, 256, 0, st>>>(assign_of, offsets, E, k, x, H, x_perm);
+        MOE_LAUNCH_CHECK();
+        return MOE_OK;
+    }
     prof_count(MOE_PROF_PERMUTE, 3);
     PermWs p;
     ws_layout(A, E, &p, ws);
@@ -189,9 +303,6 @@ int launch_permute(const int32_t* idx, int n, int E, int k, const void* x, int x
     MOE_LAUNCH_CHECK();
     perm_scan_kernel<<<1, kPermThreads, 0, st>>>(p.chunk_hist, chunks, E, offsets);
     MOE_LAUNCH_CHECK();
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int grid = (A + 7) / 8;
     if (grid > sms * 8) grid = sms * 8;
     if (x_dtype == MOE_DT_F32)
