@@ -45,6 +45,8 @@ def parse():
     p.add_argument("--no-extras", action="store_true", help="skip the resident / prefill / batch-sweep legs")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--leg", choices=["all", "resident", "prefill"], default="all",
+                   help="resident / prefill: run only that context leg (profiling); prints its own JSON line")
     return p.parse_args()
 
 
@@ -281,6 +283,11 @@ def run_ours(args, cfg, world, rank, local_rank):
     slot_bytes = A.moe_slot_bytes(shape)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     hbm_peak, peak_kind = measured_peaks()
+    if args.leg != "all":
+        res = extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=(args.leg,))
+        if rank == 0:
+            print(json.dumps({"leg": args.leg, "steps": K, "warmup": Wm, "results": res}), flush=True)
+        return
 
     # ---- headline: 64-slot decode stream
     ds = DecodeStream(cfg, shape, blobs, wg, bias, n, 2 * K + Wm, cfg.capacity, rank, device)
@@ -371,9 +378,9 @@ def run_ours(args, cfg, world, rank, local_rank):
         print(json.dumps(line), flush=True)
 
 
-def extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak):
-    """Context legs: the same layer with every expert resident (HBM-bound decode),
-    the 4096-token prefill, and the decode stream at batch 1 and 4."""
+def extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=("resident", "prefill")):
+    """Context legs: the same layer with every expert resident (HBM-bound decode)
+    at batch 1, 4 and 16, and the 4096-token prefill."""
     import torch
 
     from expert_cached_sparse_b200 import api as A
@@ -381,7 +388,7 @@ def extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak):
     out = {}
     slot_bytes = A.moe_slot_bytes(shape)
     # resident decode (256 slots, all experts preloaded)
-    for n in (1, 4, 16):
+    for n in ((1, 4, 16) if "resident" in legs else ()):
         ds = DecodeStream(cfg, shape, blobs, wg, bias, n, K + Wm, cfg.experts, 0, device, tag="resident")
         ds.cache.lookup_update(0, torch.arange(cfg.experts, dtype=torch.int32, device=device))
         torch.cuda.synchronize()
@@ -404,6 +411,8 @@ def extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak):
             "step_ms_breakdown": {k: prof[k]["ms"] / K for k in prof}}
         ds.cache.close()
         del ds
+    if "prefill" not in legs:
+        return out
     # prefill: 4096 tokens, Zipf(0.8), all experts resident
     pcfg = W.DS_PREFILL
     pbias = W.gen_bias(pcfg, 0, 0)

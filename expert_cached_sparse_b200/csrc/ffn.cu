@@ -167,11 +167,16 @@ __global__ void __launch_bounds__(kPrepThreads) ffn_prep_kernel(const void* __re
         int p = 0;
         if (OUT_F16) {
             float mx = 0.0f;
-            for (int c = lane; c < K / 4; c += 32) {
-                float v[4];
-                load4(c, v);
+            for (int c0 = lane; c0 < K / 4; c0 += 32 * 8) {
+                float v[8][4];
 #pragma unroll
-                for (int i = 0; i < 4; i++) mx = fmaxf(mx, fabsf(v[i]));
+                for (int u = 0; u < 8; u++)
+                    if (c0 + 32 * u < K / 4) load4(c0 + 32 * u, v[u]);
+#pragma unroll
+                for (int u = 0; u < 8; u++)
+                    if (c0 + 32 * u < K / 4)
+#pragma unroll
+                        for (int i = 0; i < 4; i++) mx = fmaxf(mx, fabsf(v[u][i]));
             }
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -184,19 +189,26 @@ __global__ void __launch_bounds__(kPrepThreads) ffn_prep_kernel(const void* __re
             if (lane == 0) ex[r] = p;
         }
         const float sc = ldexpf(1.0f, p);
-        for (int c = lane; c < K / 4; c += 32) {
-            float v[4];
-            load4(c, v);
+        for (int c0 = lane; c0 < K / 4; c0 += 32 * 8) {
+            float v[8][4];
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                uint16_t o;
-                if (OUT_F16) {
-                    __half hv = __float2half_rn(v[i] * sc);
-                    o = *reinterpret_cast<uint16_t*>(&hv);
-                } else {
-                    o = f32_to_bf16_bits(v[i]);
+            for (int u = 0; u < 8; u++)
+                if (c0 + 32 * u < K / 4) load4(c0 + 32 * u, v[u]);
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const int c = c0 + 32 * u;
+                if (c >= K / 4) break;
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    uint16_t o;
+                    if (OUT_F16) {
+                        __half hv = __float2half_rn(v[u][i] * sc);
+                        o = *reinterpret_cast<uint16_t*>(&hv);
+                    } else {
+                        o = f32_to_bf16_bits(v[u][i]);
+                    }
+                    out[b_index(r, 4 * c + i, RP)] = o;
                 }
-                out[b_index(r, 4 * c + i, RP)] = o;
             }
         }
     }
@@ -433,10 +445,10 @@ __global__ void __launch_bounds__(kFfnThreads) ffn_kernel(FfnArgs a)
                 xc[q][0] = xc[q][1] = make_uint4(0, 0, 0, 0);
             }
         }
-        // stages consumed: refill them with the tiles DA / DX ahead
+        // stages consumed (their values are in registers): refill them with the
+        // tiles DA / DX ahead
         __syncwarp();
         if (lane == 0) {
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             if (na < n_tiles) issue_a(na++);
             if (nx < n_tiles) issue_x(nx++);
         }
@@ -571,15 +583,21 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     a.groups = w.groups;
     a.rows = rows;
     const size_t smem = stream_smem_bytes<WFMT>(E);
-    // persistent grid: as many CTAs as fit at once
-    static int resident[2] = {0, 0};
-    if (!resident[0]) {
+    // persistent grid: as many CTAs as fit at once (recomputed when the
+    // shared-memory size, which grows with E, changes)
+    static size_t attr_smem = 0, occ_smem = 0;
+    static int resident[2] = {1, 1};
+    if (smem > attr_smem) {
         MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_kernel<WFMT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
         MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_kernel<WFMT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        attr_smem = smem;
+    }
+    if (smem != occ_smem) {
         MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident[0], ffn_kernel<WFMT, 1>, kFfnThreads, smem));
         MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident[1], ffn_kernel<WFMT, 2>, kFfnThreads, smem));
         if (resident[0] < 1) resident[0] = 1;
         if (resident[1] < 1) resident[1] = 1;
+        occ_smem = smem;
     }
     auto grid_for = [&](int R, int phase) {
         long max_units = (long)((rows + kRowsPerUnit - 1) / kRowsPerUnit + (rows < E ? rows : E)) * (R / 16);

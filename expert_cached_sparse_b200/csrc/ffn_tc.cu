@@ -559,11 +559,11 @@ template <int WFMT, int PHASE>
 int launch_one(const TcArgs& a, const RowMaps& map, int rows, int sms, cudaStream_t st)
 {
     size_t smem = tc_smem_bytes(a.E);
-    static bool attr = false;
-    if (!attr) {
+    static size_t attr_smem = 0;
+    if (smem > attr_smem) {
         MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_tc_kernel<WFMT, PHASE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)smem));
-        attr = true;
+        attr_smem = smem;
     }
     long RB = a.R / BM;
     long active = rows < a.E ? rows : a.E;
