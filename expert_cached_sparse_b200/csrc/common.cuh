@@ -100,6 +100,9 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f)
     return *reinterpret_cast<uint16_t*>(&h);
 }
 
+// 2^p for |p| <= 126 (the operand-copy exponents stay within +-100)
+__device__ __forceinline__ float pow2i(int p) { return __int_as_float((127 + p) << 23); }
+
 __device__ __forceinline__ uint32_t lane_id()
 {
     uint32_t l;
@@ -151,9 +154,21 @@ int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool
                const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,
                cudaStream_t st, const RowSource* gather = nullptr);
 bool ffn_tc_supported(const moe_shape* s);
+// Operands of the tensor-core path: f16 row copies of x and h with per-row
+// power-of-two exponents, and the fp32 h the first GEMM writes.
+struct TcOperands {
+    const uint16_t* x16;
+    const int32_t* xe;
+    float* h32;
+    const uint16_t* h16;
+    const int32_t* he;
+};
+}  // namespace moe
+#include <functional>
+namespace moe {
 int launch_ffn_tc(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
-                  const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, uint16_t* h,
-                  cudaStream_t st);
+                  const int32_t* offsets, int rows, uint16_t* y_perm, const TcOperands& op, cudaStream_t st,
+                  const std::function<int()>& between);
 int launch_combine(const uint16_t* y_perm, const int32_t* row_of, const float* w, int n, int k, int H,
                    void* out, int out_dtype, cudaStream_t st);
 }  // namespace moe

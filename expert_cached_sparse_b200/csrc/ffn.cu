@@ -105,8 +105,10 @@ __device__ __forceinline__ size_t b_index(int r, int k, int RP)
 // ------------------------------------------------------------------ prep
 // One warp per row: operand copy (+ row exponent) of a bf16 or fp32 row
 // (read directly, or token gather[r]/gk of the source).  With `groups` set,
-// the last CTA writes the per-expert token-group prefix.
-template <bool IN_F32, bool OUT_F16>
+// the last CTA writes the per-expert token-group prefix.  ROWMAJOR writes a
+// plain [rows][K] f16 copy (the tensor-core path's TMA source) instead of the
+// column-block-major fragment layout.
+template <bool IN_F32, bool OUT_F16, bool ROWMAJOR = false>
 __global__ void __launch_bounds__(kPrepThreads) ffn_prep_kernel(const void* __restrict__ in, int rows, int K,
                                                                 uint16_t* __restrict__ out, int32_t* __restrict__ ex,
                                                                 const int32_t* __restrict__ offsets,
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kPrepThreads) ffn_prep_kernel(const void* __re
                     } else {
                         o = f32_to_bf16_bits(v[u][i]);
                     }
-                    out[b_index(r, 4 * c + i, RP)] = o;
+                    out[ROWMAJOR ? (size_t)r * K + 4 * c + i : b_index(r, 4 * c + i, RP)] = o;
                 }
             }
         }
@@ -371,60 +373,68 @@ __global__ void __launch_bounds__(kFfnThreads) ffn_kernel(FfnArgs a)
     const int warps_total = gridDim.x * (kFfnThreads / 32);
     const int wg = blockIdx.x * (kFfnThreads / 32) + wib;
     const int n_units = wg < total_units ? (total_units - 1 - wg) / warps_total + 1 : 0;
-    const long n_tiles = (long)n_units * KT;
 
-    // producer (lane 0): issues tile n of this warp's stream into its ring stages
-    Unit pa, px;             // unit of the weight / activation stream head
-    int pa_idx = -1, px_idx = -1;
-    auto issue_a = [&](long n) {
-        const int ui = (int)(n / KT), kt = (int)(n % KT);
-        if (ui != pa_idx) {
-            pa = unit_of(a, s_groups, wg + ui * warps_total, RT);
-            pa_idx = ui;
+    // Tile stream of this warp: units wg, wg + warps_total, ... each KT tiles.
+    // All positions advance incrementally (no division in the loop).
+    // Producer state (lane 0): the next weight / activation tile to issue.
+    struct Cursor {
+        int ui, kt, stage;
+        uint32_t unused;
+    };
+    Cursor ca{0, 0, 0, 0}, cx{0, 0, 0, 0};
+    Unit pa, px;
+    pa.e = px.e = -1;
+    int pa_ui = -1, px_ui = -1;
+    int issued_a = 0, issued_x = 0;           // tiles issued per stream
+    const int n_tiles = n_units * KT;         // < 2^31 for any supported shape
+    auto issue_a = [&]() {
+        if (ca.ui != pa_ui) {
+            pa = unit_of(a, s_groups, wg + ca.ui * warps_total, RT);
+            pa_ui = ca.ui;
         }
-        const Unit& pu = pa;
-        const int st = (int)(n % DA);
-        const uint32_t bar = smem_u32(&barA[st]);
-        const size_t ti = tile_index(pu.rt, kt, RT, KT);
+        const uint32_t bar = smem_u32(&barA[ca.stage]);
+        const size_t ti = tile_index(pa.rt, ca.kt, RT, KT);
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(TILE + STILE) : "memory");
-        bulk_copy(smem_u32(sA + st * TILE), pu.blob + a.w_off + ti * TILE, TILE, bar);
-        if (STILE) bulk_copy(smem_u32(sS + st * STILE), pu.blob + a.s_off + ti * STILE, STILE, bar);
+        bulk_copy(smem_u32(sA + ca.stage * TILE), pa.blob + a.w_off + ti * TILE, TILE, bar);
+        if (STILE) bulk_copy(smem_u32(sS + ca.stage * STILE), pa.blob + a.s_off + ti * STILE, STILE, bar);
+        issued_a++;
+        if (++ca.kt == KT) { ca.kt = 0; ca.ui++; }
+        if (++ca.stage == DA) ca.stage = 0;
     };
-    auto issue_x = [&](long n) {
-        const int ui = (int)(n / KT), kt = (int)(n % KT);
-        if (ui != px_idx) {
-            px = unit_of(a, s_groups, wg + ui * warps_total, RT);
-            px_idx = ui;
+    auto issue_x = [&]() {
+        if (cx.ui != px_ui) {
+            px = unit_of(a, s_groups, wg + cx.ui * warps_total, RT);
+            px_ui = cx.ui;
         }
-        const Unit& pu = px;
-        const int st = (int)(n % DX);
-        const uint32_t bar = smem_u32(&barX[st]);
-        const uint32_t bytes = (uint32_t)pu.nq * 1024;
+        const uint32_t bar = smem_u32(&barX[cx.stage]);
+        const uint32_t bytes = (uint32_t)px.nq * 1024;
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-        bulk_copy(smem_u32(sX + st * XSTAGE), a.in + ((size_t)kt * RP + pu.row0) * 64, bytes, bar);
+        bulk_copy(smem_u32(sX + cx.stage * XSTAGE), a.in + ((size_t)cx.kt * RP + px.row0) * 64, bytes, bar);
+        issued_x++;
+        if (++cx.kt == KT) { cx.kt = 0; cx.ui++; }
+        if (++cx.stage == DX) cx.stage = 0;
     };
-    long na = 0, nx = 0;   // tiles issued (lane 0 only)
     if (lane == 0) {
-        for (; na < DA && na < n_tiles; na++) issue_a(na);
-        for (; nx < DX && nx < n_tiles; nx++) issue_x(nx);
+        while (issued_a < DA && issued_a < n_tiles) issue_a();
+        while (issued_x < DX && issued_x < n_tiles) issue_x();
     }
 
     bool ok = true;
-    long n = 0;
+    int n = 0, kt = 0, ui = 0, sa = 0, sx = 0;
+    uint32_t pha = 0, phx = 0;               // parity of the current pass over each ring
     Unit cu;
+    cu.e = -1;
     float acc[2][4];
     for (; n < n_tiles; n++) {
-        const int kt = (int)(n % KT);
         if (kt == 0) {
-            cu = unit_of(a, s_groups, wg + (int)(n / KT) * warps_total, RT);
+            cu = unit_of(a, s_groups, wg + ui * warps_total, RT);
 #pragma unroll
             for (int q = 0; q < 2; q++)
 #pragma unroll
                 for (int i = 0; i < 4; i++) acc[q][i] = 0.0f;
         }
-        const int sa = (int)(n % DA), sx = (int)(n % DX);
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&barA[sa]), (uint32_t)((n / DA) & 1)) &&
-                                          mbar_wait_bounded(smem_u32(&barX[sx]), (uint32_t)((n / DX) & 1)));
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&barA[sa]), pha) &&
+                                          mbar_wait_bounded(smem_u32(&barX[sx]), phx));
         if (!ok) break;
         // operands from shared memory
         uint4 cur[FP4 ? 1 : 4];
@@ -445,12 +455,14 @@ __global__ void __launch_bounds__(kFfnThreads) ffn_kernel(FfnArgs a)
                 xc[q][0] = xc[q][1] = make_uint4(0, 0, 0, 0);
             }
         }
+        if (++sa == DA) { sa = 0; pha ^= 1; }
+        if (++sx == DX) { sx = 0; phx ^= 1; }
         // stages consumed (their values are in registers): refill them with the
         // tiles DA / DX ahead
         __syncwarp();
         if (lane == 0) {
-            if (na < n_tiles) issue_a(na++);
-            if (nx < n_tiles) issue_x(nx++);
+            if (issued_a < n_tiles) issue_a();
+            if (issued_x < n_tiles) issue_x();
         }
         if (!FP4) {
             // bf16 fragments: cur[j] = {a0, a2, a1, a3} of step j
@@ -518,8 +530,8 @@ __global__ void __launch_bounds__(kFfnThreads) ffn_kernel(FfnArgs a)
                 const int r0 = cu.row0 + q * 8 + 2 * t, r1 = r0 + 1;
                 float u0 = tsc, u1 = tsc;
                 if (FP4) {
-                    if (r0 < cu.row_end) u0 = ldexpf(tsc, -__ldg(a.in_ex + r0));
-                    if (r1 < cu.row_end) u1 = ldexpf(tsc, -__ldg(a.in_ex + r1));
+                    if (r0 < cu.row_end) u0 = tsc * pow2i(-__ldg(a.in_ex + r0));
+                    if (r1 < cu.row_end) u1 = tsc * pow2i(-__ldg(a.in_ex + r1));
                 }
                 if (PHASE == 1) {
                     const int F = a.R / 2;
@@ -540,13 +552,15 @@ __global__ void __launch_bounds__(kFfnThreads) ffn_kernel(FfnArgs a)
                 }
             }
         }
+        if (++kt == KT) { kt = 0; ui++; }
     }
     if (!ok) {
         // a wait ran out: record it, then let every copy still in flight land
+        // (tile m sits in stage m % D with parity (m / D) & 1)
         if (lane == 0) {
             atomicCAS(&g_ffn_error, 0, (int)MOE_ERR_TIMEOUT);
-            for (long m = n; m < na; m++) mbar_wait_bounded(smem_u32(&barA[m % DA]), (uint32_t)((m / DA) & 1));
-            for (long m = n; m < nx; m++) mbar_wait_bounded(smem_u32(&barX[m % DX]), (uint32_t)((m / DX) & 1));
+            for (int m = n; m < issued_a; m++) mbar_wait_bounded(smem_u32(&barA[m % DA]), (uint32_t)((m / DA) & 1));
+            for (int m = n; m < issued_x; m++) mbar_wait_bounded(smem_u32(&barX[m % DX]), (uint32_t)((m / DX) & 1));
         }
         __syncwarp();
     }
@@ -668,15 +682,29 @@ int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool
     ProfScope ps(MOE_PROF_FFN, st);
     FfnWs w;
     ffn_ws_layout(s, rows, ws, &w);
+    int dev0 = 0, sms0 = 148;
+    cudaGetDevice(&dev0);
+    cudaDeviceGetAttribute(&sms0, cudaDevAttrMultiProcessorCount, dev0);
     if (use_tc_path(s, rows)) {
-        prof_count(MOE_PROF_FFN, 2);
-        return launch_ffn_tc(s, pool, slot_bytes, pool_slots, slot_of, offsets, x_perm, rows, y_perm, w.h16, st);
+        // tensor-core path: f16 operand rows (x, then h), each scaled by a power of two
+        prof_count(MOE_PROF_FFN, 4);
+        const int wpb = kPrepThreads / 32;
+        int pb = (rows + wpb - 1) / wpb;
+        if (pb > sms0 * 8) pb = sms0 * 8;
+        ffn_prep_kernel<false, true, true><<<pb, kPrepThreads, 0, st>>>(x_perm, rows, s->hidden, w.xb, w.xe, nullptr,
+                                                                         nullptr, s->experts, 0, nullptr, nullptr, 1);
+        MOE_LAUNCH_CHECK();
+        TcOperands op{w.xb, w.xe, w.h32, w.hb, w.he};
+        return launch_ffn_tc(s, pool, slot_bytes, pool_slots, slot_of, offsets, rows, y_perm, op, st, [&]() -> int {
+            ffn_prep_kernel<true, true, true><<<pb, kPrepThreads, 0, st>>>(w.h32, rows, s->ffn, w.hb, w.he, nullptr,
+                                                                            nullptr, s->experts, 0, nullptr, nullptr, 1);
+            MOE_LAUNCH_CHECK();
+            return MOE_OK;
+        });
     }
     prof_count(MOE_PROF_FFN, 4);
     BlobLayout bl = blob_layout(s);
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = sms0;
     switch (s->wfmt) {
     case MOE_W_BF16:
         return launch_decode<MOE_W_BF16>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, x_perm, rows, y_perm,

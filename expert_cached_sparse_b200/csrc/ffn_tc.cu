@@ -23,6 +23,7 @@
 //    chain the roles; every wait is bounded and a timeout sets an error word
 //    and drains the CTA instead of hanging.
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 
@@ -56,7 +57,9 @@ struct TcArgs {
     const int32_t* slot_of;
     const int32_t* offsets;
     int pool_slots, rows;
-    uint16_t* out;
+    const int32_t* in_ex;   // power-of-two exponent of each B row (token)
+    float* out_h;           // phase 1: h [rows][R/2] fp32
+    uint16_t* out_y;        // phase 2: y [rows][R] bf16
 };
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -88,15 +91,18 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait: spins on try_wait (which itself suspends briefly in hardware),
-// gives up after WAIT_CYCLES, records MOE_ERR_TIMEOUT and raises the CTA's
-// abort flag so the other roles drain too.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag)
+// Bounded wait: try_wait (which suspends briefly in hardware) in a tight
+// loop; every 32 tries it checks the CTA's abort flag and the clock, and after
+// WAIT_CYCLES it records MOE_ERR_TIMEOUT and raises the abort flag so the
+// other roles drain too.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag)
 {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
-        if (mbar_try(bar, parity)) return true;
+#pragma unroll 1
+        for (int i = 0; i < 32; i++)
+            if (mbar_try(bar, parity)) return true;
         if (*abort_flag) return false;
         if (clock64() - t0 > WAIT_CYCLES) break;
     }
@@ -171,10 +177,10 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr)
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// Instruction descriptor: kind::f16, bf16 A and B (K-major), fp32 D, M = 128, N = n.
-__device__ __forceinline__ uint32_t idesc_bf16(int n)
+// Instruction descriptor: kind::f16, f16 A and B (K-major), fp32 D, M = 128, N = n.
+__device__ __forceinline__ uint32_t idesc_f16(int n)
 {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
 __device__ __forceinline__ void e2m1x4_to_f16x2(uint32_t w, uint32_t (&f)[4])
@@ -186,26 +192,28 @@ __device__ __forceinline__ void e2m1x4_to_f16x2(uint32_t w, uint32_t (&f)[4])
         : "r"(w));
 }
 
-// f16x2 of E2M1 values -> bf16x2 (value * 2^-112, exact) -> times m2 (scale * 2^112) in bf16, exact.
-__device__ __forceinline__ uint32_t to_bf16x2_scaled(uint32_t f, uint32_t m2)
+// f16x2 of E2M1 values times the f16x2 block scale m2: exact, since E2M1 x
+// scale has at most 6 significant bits and stays in the f16 normal range
+// (MXFP4 scale codes 114..140, any finite E4M3 scale).
+__device__ __forceinline__ uint32_t to_f16x2_scaled(uint32_t f, uint32_t m2)
 {
-    uint32_t b = ((f & 0x7FFF7FFFu) >> 3) | (f & 0x80008000u);
     uint32_t r;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(b), "r"(m2));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(f), "r"(m2));
     return r;
 }
 
+// f16 bits of the block scale of code c.
 __device__ uint16_t scale_mult(int wfmt, int c)
 {
     if (wfmt == MOE_W_MXFP4) {
-        int e = c + 112;
-        e = e < 1 ? 1 : (e > 254 ? 254 : e);
-        return (uint16_t)(e << 7);
+        int e = c - 112;                       // 2^(c-127) as f16: exponent field c-127+15
+        e = e < 1 ? 1 : (e > 30 ? 30 : e);     // codes outside 114..140 are rejected at packing
+        return (uint16_t)(e << 10);
     }
     int s = (c >> 7) & 1, e = (c >> 3) & 15, m = c & 7;
     float v = (e == 0) ? ldexpf((float)m, -9) : ldexpf((float)(8 + m), e - 10);
-    v = ldexpf(v, 112);
-    return f32_to_bf16_bits(s ? -v : v);
+    __half h = __float2half_rn(s ? -v : v);
+    return *reinterpret_cast<uint16_t*>(&h);
 }
 
 struct Tile {
@@ -384,7 +392,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (!ok) break;
                     tc_fence_after();
                 }
-                const uint32_t idesc = idesc_bf16(t.bn);
+                const uint32_t idesc = idesc_f16(t.bn);
                 for (int c = 0; c < KT && ok; c++) {
                     ok = mbar_wait(smem_u32(&a_ready[ab]), pab, abort_v) &&
                          mbar_wait(smem_u32(&full_b[sb]), pb, abort_v);
@@ -451,7 +459,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     uint32_t f[4];
                     e2m1x4_to_f16x2(q4[tt], f);
 #pragma unroll
-                    for (int b = 0; b < 4; b++) v[4 * b + tt] = to_bf16x2_scaled(f[b], b < 2 ? m0 : m1);
+                    for (int b = 0; b < 4; b++) v[4 * b + tt] = to_f16x2_scaled(f[b], b < 2 ? m0 : m1);
                 }
                 ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&a_free[ab]), pab ^ 1, abort_v));
                 if (!ok) break;
@@ -478,13 +486,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const int f = 64 * t.rb + 8 * rtl + g;
 #pragma unroll
                     for (int j = 0; j < 32; j++) {
-                        float x = __uint_as_float(d[j]) * tsc;
-                        float up = __shfl_down_sync(0xffffffffu, x, 8);
                         const int n = c0 + j;
-                        if (half == 0 && n < t.nrows) {
-                            float h = x / (1.0f + expf(-x)) * up;
-                            a.out[(size_t)(t.row0 + n) * F + f] = f32_to_bf16_bits(h);
-                        }
+                        const float u = (n < t.nrows) ? tsc * pow2i(-__ldg(a.in_ex + t.row0 + n)) : 0.0f;
+                        const float x = __uint_as_float(d[j]) * u;
+                        const float up = __shfl_down_sync(0xffffffffu, x, 8);
+                        if (half == 0 && n < t.nrows)
+                            a.out_h[(size_t)(t.row0 + n) * F + f] = x / (1.0f + expf(-x)) * up;
                     }
                 } else {
                     const int Ho = a.R;
@@ -492,7 +499,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 32; j++) {
                         const int n = c0 + j;
-                        if (n < t.nrows) a.out[(size_t)(t.row0 + n) * Ho + o] = f32_to_bf16_bits(__uint_as_float(d[j]) * tsc);
+                        if (n < t.nrows) {
+                            const float u = tsc * pow2i(-__ldg(a.in_ex + t.row0 + n));
+                            a.out_y[(size_t)(t.row0 + n) * Ho + o] = f32_to_bf16_bits(__uint_as_float(d[j]) * u);
+                        }
                     }
                 }
             }
@@ -525,7 +535,7 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// [rows][cols] bf16, boxes of box_rows rows x 64 columns, 128-byte swizzle.
+// [rows][cols] f16, boxes of box_rows rows x 64 columns, 128-byte swizzle.
 int make_rows_map(CUtensorMap* m, const void* base, int rows, int cols, int box_rows)
 {
     EncodeTiledFn fn = encode_fn();
@@ -534,7 +544,7 @@ int make_rows_map(CUtensorMap* m, const void* base, int rows, int cols, int box_
     cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
     cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
@@ -584,8 +594,8 @@ bool ffn_tc_supported(const moe_shape* s)
 }
 
 int launch_ffn_tc(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
-                  const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, uint16_t* h,
-                  cudaStream_t st)
+                  const int32_t* offsets, int rows, uint16_t* y_perm, const TcOperands& op, cudaStream_t st,
+                  const std::function<int()>& between)
 {
     BlobLayout bl = blob_layout(s);
     int dev = 0, sms = 148;
@@ -593,8 +603,8 @@ int launch_ffn_tc(const moe_shape* s, const void* pool, size_t slot_bytes, int p
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     RowMaps mx, mh;
     int rc;
-    if ((rc = make_row_maps(&mx, x_perm, rows, s->hidden))) return rc;
-    if ((rc = make_row_maps(&mh, h, rows, s->ffn))) return rc;
+    if ((rc = make_row_maps(&mx, op.x16, rows, s->hidden))) return rc;
+    if ((rc = make_row_maps(&mh, op.h16, rows, s->ffn))) return rc;
     TcArgs a1{};
     a1.pool = static_cast<const char*>(pool);
     a1.slot_bytes = slot_bytes;
@@ -608,18 +618,23 @@ int launch_ffn_tc(const moe_shape* s, const void* pool, size_t slot_bytes, int p
     a1.offsets = offsets;
     a1.pool_slots = pool_slots;
     a1.rows = rows;
-    a1.out = h;
+    a1.in_ex = op.xe;
+    a1.out_h = op.h32;
     TcArgs a2 = a1;
     a2.w_off = bl.w2;
     a2.s_off = bl.s2;
     a2.R = s->hidden;
     a2.K = s->ffn;
-    a2.out = y_perm;
+    a2.in_ex = op.he;
+    a2.out_h = nullptr;
+    a2.out_y = y_perm;
     if (s->wfmt == MOE_W_MXFP4) {
         if ((rc = launch_one<MOE_W_MXFP4, 1>(a1, mx, rows, sms, st))) return rc;
+        if ((rc = between())) return rc;
         return launch_one<MOE_W_MXFP4, 2>(a2, mh, rows, sms, st);
     }
     if ((rc = launch_one<MOE_W_NVFP4, 1>(a1, mx, rows, sms, st))) return rc;
+    if ((rc = between())) return rc;
     return launch_one<MOE_W_NVFP4, 2>(a2, mh, rows, sms, st);
 }
 

@@ -81,10 +81,12 @@ void pack_bf16_matrix(const uint16_t* w, int R, int K, bool w13, int F, uint8_t*
         }
 }
 
+// E8M0 block scales 2^-13 .. 2^13: E2M1 x scale is then exact in f16 (the
+// tensor-core operand type) as well as in bf16.
 bool mx_codes_ok(const uint8_t* sc, size_t n)
 {
     for (size_t i = 0; i < n; i++)
-        if (sc[i] < 2 || sc[i] > 142) return false;
+        if (sc[i] < 114 || sc[i] > 140) return false;
     return true;
 }
 

@@ -121,6 +121,118 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restri
     }
 }
 
+// Many tokens (prefill): a CTA computes a 32-token x 16-expert block of logits
+// with both operand slices staged in shared memory as fp32.  K is walked in
+// slices of 256 elements = 32 chunks of 8, so lane l of every warp owns chunk
+// l of each slice: the per-(token, expert) order is the same fixed order as
+// above (lane chunks ascending, then the xor butterfly).  Warp w owns tokens
+// 4w..4w+3 and all 16 experts (64 accumulators per lane).
+constexpr int RT_TOK = 32, RT_EXP = 16, RT_K = 256;
+
+template <bool XF32>
+__global__ void __launch_bounds__(256) router_logits_tiled_kernel(const void* __restrict__ x,
+                                                                  const uint16_t* __restrict__ wg,
+                                                                  const float* __restrict__ bias, int n, int H,
+                                                                  int E, float* __restrict__ logits)
+{
+    __shared__ __align__(16) float xs[RT_TOK][RT_K];
+    __shared__ __align__(16) float ws[RT_EXP][RT_K];
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int t0 = blockIdx.x * RT_TOK, e0 = blockIdx.y * RT_EXP;
+    float acc[4][RT_EXP];
+#pragma unroll
+    for (int a = 0; a < 4; a++)
+#pragma unroll
+        for (int b = 0; b < RT_EXP; b++) acc[a][b] = 0.0f;
+    for (int k0 = 0; k0 < H; k0 += RT_K) {
+        // stage: x slice (32 x 256) and gate slice (16 x 256) as fp32
+        for (int i = tid; i < RT_TOK * RT_K / 8; i += 256) {
+            const int r = i / (RT_K / 8), c = i % (RT_K / 8);
+            const int t = t0 + r, k = k0 + 8 * c;
+            float v[8];
+            if (t < n && k < H) {
+                if (XF32) {
+                    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + (size_t)t * H + k);
+                    float4 a = __ldg(p), b = __ldg(p + 1);
+                    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+                } else {
+                    uint4 q = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + (size_t)t * H + k));
+                    const uint32_t u4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        v[2 * j] = __uint_as_float(u4[j] << 16);
+                        v[2 * j + 1] = __uint_as_float(u4[j] & 0xFFFF0000u);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; j++) v[j] = 0.0f;
+            }
+            float4* d = reinterpret_cast<float4*>(&xs[r][8 * c]);
+            d[0] = make_float4(v[0], v[1], v[2], v[3]);
+            d[1] = make_float4(v[4], v[5], v[6], v[7]);
+        }
+        for (int i = tid; i < RT_EXP * RT_K / 8; i += 256) {
+            const int r = i / (RT_K / 8), c = i % (RT_K / 8);
+            const int e = e0 + r, k = k0 + 8 * c;
+            float v[8];
+            if (e < E && k < H) {
+                uint4 q = __ldg(reinterpret_cast<const uint4*>(wg + (size_t)e * H + k));
+                const uint32_t u4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    v[2 * j] = __uint_as_float(u4[j] << 16);
+                    v[2 * j + 1] = __uint_as_float(u4[j] & 0xFFFF0000u);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; j++) v[j] = 0.0f;
+            }
+            float4* d = reinterpret_cast<float4*>(&ws[r][8 * c]);
+            d[0] = make_float4(v[0], v[1], v[2], v[3]);
+            d[1] = make_float4(v[4], v[5], v[6], v[7]);
+        }
+        __syncthreads();
+        if (k0 + 8 * lane < H) {   // lane's chunk exists in this slice
+            float xv[4][8];
+#pragma unroll
+            for (int a = 0; a < 4; a++) {
+                const float4* p = reinterpret_cast<const float4*>(&xs[4 * w + a][8 * lane]);
+                float4 q0 = p[0], q1 = p[1];
+                xv[a][0] = q0.x; xv[a][1] = q0.y; xv[a][2] = q0.z; xv[a][3] = q0.w;
+                xv[a][4] = q1.x; xv[a][5] = q1.y; xv[a][6] = q1.z; xv[a][7] = q1.w;
+            }
+#pragma unroll
+            for (int b = 0; b < RT_EXP; b++) {
+                const float4* p = reinterpret_cast<const float4*>(&ws[b][8 * lane]);
+                float4 q0 = p[0], q1 = p[1];
+                const float wv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                for (int a = 0; a < 4; a++)
+#pragma unroll
+                    for (int i = 0; i < 8; i++) acc[a][b] = __fmaf_rn(xv[a][i], wv[i], acc[a][b]);
+            }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int a = 0; a < 4; a++)
+#pragma unroll
+        for (int b = 0; b < RT_EXP; b++)
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1)
+                acc[a][b] = __fadd_rn(acc[a][b], __shfl_xor_sync(0xffffffffu, acc[a][b], off));
+    // lane b of the warp writes expert e0+b for the warp's 4 tokens
+#pragma unroll
+    for (int a = 0; a < 4; a++) {
+        const int t = t0 + 4 * w + a;
+#pragma unroll
+        for (int b = 0; b < RT_EXP; b++)
+            if (lane == b && t < n && e0 + b < E)
+                logits[(size_t)t * E + e0 + b] = bias ? __fadd_rn(acc[a][b], __ldg(bias + e0 + b)) : acc[a][b];
+    }
+}
+
 // a ranks above b: larger logit; ties -> lower index; NaN below everything.
 __device__ __forceinline__ bool ranks_above(float a, int ia, float b, int ib)
 {
@@ -184,11 +296,8 @@ int launch_logits(const void* x, const uint16_t* wg, const float* bias, int n, i
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int threads = 256, wpb = threads / 32;
     if (n >= 64) {
-        constexpr int TB = 4, EB = 8;
-        long units = (long)((E + EB - 1) / EB) * ((n + TB - 1) / TB);
-        int grid = (int)((units + wpb - 1) / wpb);
-        if (grid > sms * 8) grid = sms * 8;
-        router_logits_kernel<XF32, TB, EB, 1><<<grid, threads, 0, st>>>(x, wg, bias, n, H, E, logits);
+        dim3 grid((n + RT_TOK - 1) / RT_TOK, (E + RT_EXP - 1) / RT_EXP);
+        router_logits_tiled_kernel<XF32><<<grid, 256, 0, st>>>(x, wg, bias, n, H, E, logits);
     } else {
         constexpr int TB = 1, EB = 1;
         long units = (long)E * n;

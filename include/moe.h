@@ -159,8 +159,9 @@ size_t moe_layer_workspace_bytes(const moe_shape* shape, int32_t n);
  *   NULL).  BF16: w13/w2 are uint16 bit patterns, scales NULL.
  * blob_out: moe_slot_bytes(shape) bytes.
  * Errors: MOE_ERR_UNSUPPORTED for NaN scale codes, MXFP4 scale codes
- * outside [2, 142] (block scales 2^-125 .. 2^15) or non-finite NVFP4 tensor
- * scales.
+ * outside [114, 140] (block scales 2^-13 .. 2^13, the range in which every
+ * E2M1 x scale product is an exact f16 and bf16 number) or non-finite NVFP4
+ * tensor scales.
  */
 int moe_pack_expert(const moe_shape* shape, const void* h_w13, const uint8_t* h_w13_scales,
                     const void* h_w2, const uint8_t* h_w2_scales, const float* h_tensor_scales,
