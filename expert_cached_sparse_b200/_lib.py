@@ -34,6 +34,7 @@ EXPORTS = [
     "moe_cache_read_trace", "moe_cache_get_stats", "moe_cache_snapshot", "moe_cache_capacity",
     "moe_cache_destroy", "moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine",
     "moe_layer_forward", "moe_profile_enable", "moe_profile_read", "moe_get_device_error",
+    "moe_permute_noalloc",
 ]
 PROF_KINDS = ["router", "lookup", "permute", "ffn", "combine", "fill"]
 
@@ -86,6 +87,7 @@ def _load():
         "moe_cache_destroy": (C.c_int, [P]),
         "moe_router_topk": (C.c_int, [P, I32, P, P, I32, I32, I32, I32, P, P, P, P]),
         "moe_permute": (C.c_int, [P, I32, I32, I32, P, I32, I32, P, P, P, P, P, SZ, P]),
+        "moe_permute_noalloc": (C.c_int, [P, I32, I32, I32, P, I32, I32, P, P, P, P, P]),
         "moe_grouped_ffn": (C.c_int, [SP, P, I32, P, P, P, I32, P, P, SZ, P]),
         "moe_combine": (C.c_int, [P, P, P, I32, I32, I32, P, I32, P]),
         "moe_layer_forward": (C.c_int, [P, I32, P, I32, P, P, I32, P, P, SZ, P, P, P, P]),

@@ -86,6 +86,13 @@ def moe_permute(topk_idx, n, experts, k, x, hidden, offsets, row_of, assign_of, 
     check("moe_permute", rc)
 
 
+def moe_permute_noalloc(topk_idx, n, experts, k, x, hidden, offsets, row_of, assign_of, x_perm, stream=None):
+    """moe_permute with the library's static scratch instead of a workspace (see include/moe.h)."""
+    rc = L.lib.moe_permute_noalloc(ptr(topk_idx), n, experts, k, ptr(x), _dt(x), hidden, ptr(offsets), ptr(row_of),
+                                   ptr(assign_of), ptr(x_perm), stream_handle(stream))
+    check("moe_permute_noalloc", rc)
+
+
 def moe_grouped_ffn(shape, pool, pool_slots, slot_of, offsets, x_perm, rows, y_perm, ws, stream=None):
     rc = L.lib.moe_grouped_ffn(C.byref(shape), ptr(pool), pool_slots, ptr(slot_of), ptr(offsets), ptr(x_perm), rows,
                                ptr(y_perm), ptr(ws), ws.numel() * ws.element_size(), stream_handle(stream))

@@ -339,3 +339,58 @@ extern "C" int moe_permute(const int32_t* d_topk_idx, int32_t n, int32_t experts
     return moe::launch_permute(d_topk_idx, n, experts, k, d_x, x_dtype, hidden, d_expert_offsets, d_row_of,
                                d_assign_of, d_x_perm, d_ws, moe::as_stream(stream));
 }
+
+// ---------------------------------------------------------------------------
+// moe_permute_noalloc: the same permutation for callers that must not
+// allocate device memory themselves (see include/moe.h).  Its scratch lives
+// in one file-scope device array that every GPU loading this library holds
+// until the process exits.  Host code cannot pass the array's name to a
+// kernel (on the host it is only a stand-in symbol), so the device address is
+// looked up with cudaGetSymbolAddress once per device, with that device
+// current, on the first call made on it.
+#include <mutex>
+
+namespace {
+
+constexpr size_t kPermuteStaticScratch = MOE_PERMUTE_NOALLOC_MAX_SCRATCH;
+static __device__ __align__(256) unsigned char g_permute_scratch[kPermuteStaticScratch];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices];   // device address of g_permute_scratch per device
+
+// Device address of the static scratch on the current device (nullptr on failure).
+void* permute_static_scratch()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
+        g_scratch_addr[dev] = p;
+    }
+    return g_scratch_addr[dev];
+}
+
+}  // namespace
+
+extern "C" int moe_permute_noalloc(const int32_t* d_topk_idx, int32_t n, int32_t experts, int32_t k,
+                                   const void* d_x, int32_t x_dtype, int32_t hidden, int32_t* d_expert_offsets,
+                                   int32_t* d_row_of, int32_t* d_assign_of, uint16_t* d_x_perm, void* stream)
+{
+    if (n < 0 || experts <= 0 || experts > moe::kMaxExperts || k <= 0 || hidden <= 0 || hidden % 8)
+        return MOE_ERR_INVALID_ARG;
+    if (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
+    if (!d_expert_offsets) return MOE_ERR_INVALID_ARG;
+    if (n > 0 && (!d_topk_idx || !d_x || !d_row_of || !d_assign_of || !d_x_perm)) return MOE_ERR_INVALID_ARG;
+    if (((uintptr_t)d_x | (uintptr_t)d_x_perm) & 15) return MOE_ERR_INVALID_ARG;
+    if ((long long)n * k > (1ll << 30)) return MOE_ERR_UNSUPPORTED;
+    if (moe::permute_ws_bytes(n, experts, k) > kPermuteStaticScratch) return MOE_ERR_UNSUPPORTED;
+    void* scratch = permute_static_scratch();
+    if (!scratch) return MOE_ERR_CUDA;
+    // Every scratch entry the kernels read is written earlier in the same call,
+    // so the previous call's contents need no clearing.
+    return moe::launch_permute(d_topk_idx, n, experts, k, d_x, x_dtype, hidden, d_expert_offsets, d_row_of,
+                               d_assign_of, d_x_perm, scratch, moe::as_stream(stream));
+}

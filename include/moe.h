@@ -269,6 +269,31 @@ int moe_permute(const int32_t* d_topk_idx, int32_t n, int32_t experts, int32_t k
                 void* stream);
 
 /*
+ * moe_permute without a caller-provided workspace.  No counterpart on the
+ * FreeToken pages: this is a convenience for callers that cannot allocate
+ * device memory of their own -- for example code running inside a host
+ * framework whose allocator owns all GPU memory and forbids foreign
+ * cudaMalloc calls, or a latency-critical serving loop that must never enter
+ * the CUDA allocator (cudaMalloc / cudaFree may synchronise the device).
+ * Arguments, outputs and ordering are those of moe_permute.
+ * The scratch is one static device array of MOE_PERMUTE_NOALLOC_MAX_SCRATCH
+ * bytes inside libmoe.so, present on every GPU that loads the library for the
+ * life of the process.  The first call on a device looks the array's device
+ * address up (with that device current); make that first call before any
+ * stream capture.  Allocates nothing: no cudaMalloc, cudaFree or other
+ * allocating routine.  Nothing in the array has to start at zero: every
+ * entry a call reads is written earlier in that same call, so leftovers of a
+ * previous call are harmless.  Sizes whose moe_permute_workspace_bytes() exceed the
+ * array return MOE_ERR_UNSUPPORTED before anything is enqueued.  All calls on
+ * a device share the one array: calls that may overlap on the GPU (different
+ * streams, or other host threads) race and must be serialised by the caller.
+ */
+#define MOE_PERMUTE_NOALLOC_MAX_SCRATCH (1u << 20)
+int moe_permute_noalloc(const int32_t* d_topk_idx, int32_t n, int32_t experts, int32_t k, const void* d_x,
+                        int32_t x_dtype, int32_t hidden, int32_t* d_expert_offsets, int32_t* d_row_of,
+                        int32_t* d_assign_of, uint16_t* d_x_perm, void* stream);
+
+/*
  * Grouped SwiGLU expert FFN over the permuted rows.  d_slot_pool holds
  * pool_slots packed blobs of moe_slot_bytes() each.  For every expert e
  * with rows [offsets[e], offsets[e+1]) (clipped to [0, rows)) and
