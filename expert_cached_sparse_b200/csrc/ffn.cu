@@ -42,7 +42,6 @@ __device__ int g_ffn_error;   // first device-side error of the decode FFN (0: n
 
 namespace {
 
-constexpr int kFfnThreads = 128;
 constexpr int kRowsPerUnit = 16;   // 2 n-tiles of 8 tokens
 constexpr int kPrepThreads = 256;
 constexpr int kRowPad = 16;        // operand copies carry 16 spare rows (whole 8-row reads past the end)
@@ -56,7 +55,7 @@ struct FfnWs {
     uint16_t* hb;     // [F/64][rows+16][64] operand copy of h
     int32_t* he;      // [rows]
     int32_t* groups;  // [E+1] exclusive prefix of token groups per expert
-    uint16_t* h16;    // [rows][F] bf16 h of the tensor-core path (aliases h32)
+    float* part;      // K-slice partial sums, at most 1024 x max(2F, H) fp32
 };
 
 size_t ffn_ws_layout(const moe_shape* s, int rows, void* base, FfnWs* w)
@@ -70,6 +69,8 @@ size_t ffn_ws_layout(const moe_shape* s, int rows, void* base, FfnWs* w)
     size_t ohb = take(2 * RP * s->ffn);
     size_t ohe = take(4 * R);
     size_t og = take(4 * (size_t)(s->experts + 1));
+    const size_t prow = (size_t)(8 * R < 1024 ? 8 * R : 1024);
+    size_t op = take(4 * prow * (size_t)(2 * s->ffn > s->hidden ? 2 * s->ffn : s->hidden));
     if (w) {
         char* b = static_cast<char*>(base);
         w->xb = reinterpret_cast<uint16_t*>(b + oxb);
@@ -78,7 +79,7 @@ size_t ffn_ws_layout(const moe_shape* s, int rows, void* base, FfnWs* w)
         w->hb = reinterpret_cast<uint16_t*>(b + ohb);
         w->he = reinterpret_cast<int32_t*>(b + ohe);
         w->groups = reinterpret_cast<int32_t*>(b + og);
-        w->h16 = reinterpret_cast<uint16_t*>(b + oh);
+        w->part = reinterpret_cast<float*>(b + op);
     }
     return o;
 }
@@ -230,6 +231,8 @@ struct FfnArgs {
     const int32_t* in_ex;   // [rows] its exponents (FP4 formats)
     float* out_h;           // phase 1: h [rows][R/2] fp32
     uint16_t* out_y;        // phase 2: y [rows][R] bf16
+    int S;                  // K split: each unit covers 1/S of the column blocks
+    float* part;            // S > 1: partial sums [S][rows][R] fp32
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -246,13 +249,21 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
 }
 
 // Bounded wait (about 2 s of clock), false on timeout.
-__device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
 {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try(bar, parity))
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 16; i++)
+            if (mbar_try(bar, parity)) return true;
         if (clock64() - t0 > kWaitCycles) return false;
-    return true;
+    }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
@@ -302,33 +313,46 @@ __device__ __forceinline__ float e4m3_value(uint32_t c)
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 
+// ---- CTA-cooperative weight streaming -------------------------------------
+// A CTA owns units (token group, 128-row block of W, slice of K).  Warp 8
+// (one lane) issues per 64-column chunk three bulk copies into a ring
+// stage: the block's eight 512-byte FP4 tiles (contiguous in the slot), their
+// scales, and the token group's 8 or 16 activation rows of that chunk.
+// Warps 0..7 each consume one 16-row tile of the stage and release it on an
+// mbarrier as soon as their operands are in registers.
+constexpr int kCW = 8;                        // compute warps
+constexpr int kDecThreads = 32 * (kCW + 1);   // + one copy-issue warp
+
 template <int WFMT>
-struct StreamCfg {
+struct DecCfg {
     static constexpr bool FP4 = WFMT != MOE_W_BF16;
-    static constexpr int TILE = FP4 ? 512 : 2048;                 // weight tile bytes
+    static constexpr int TILE = FP4 ? 512 : 2048;
     static constexpr int STILE = (WFMT == MOE_W_MXFP4) ? 32 : (WFMT == MOE_W_NVFP4 ? 64 : 0);
-    static constexpr int DA = FP4 ? 16 : 4;                       // weight tiles in flight per warp
-    static constexpr int DX = 8;                                  // activation tiles in flight per warp
-    static constexpr int XSTAGE = 2 * 1024;                       // two 8-row blocks
-    static constexpr int WARP_BYTES = DA * (TILE + STILE) + DX * XSTAGE + 8 * (DA + DX);
+    static constexpr int D = FP4 ? 8 : 4;                        // ring stages
+    static constexpr int A_BYTES = kCW * TILE;
+    static constexpr int S_BYTES = kCW * STILE;
+    static constexpr int X_BYTES = 2 * 1024;                     // up to 16 rows x 128 bytes
+    static constexpr int STAGE = A_BYTES + S_BYTES + X_BYTES;
 };
 
 template <int WFMT>
-size_t stream_smem_bytes(int E)
+size_t dec_smem_bytes(int E)
 {
-    return 128 + (size_t)(kFfnThreads / 32) * StreamCfg<WFMT>::WARP_BYTES + 4 * (size_t)(E + 1);
+    return 1024 + (size_t)DecCfg<WFMT>::D * DecCfg<WFMT>::STAGE + 4 * (size_t)(E + 1);
 }
 
-struct Unit {
-    int e, rt, row0, row_end, nq;
+struct DecUnit {
+    int e, G, ng, row0, row_end, nq, k0, k1, s;
     const char* blob;
 };
 
-__device__ __forceinline__ Unit unit_of(const FfnArgs& a, const int* s_groups, int u, int RT)
+__device__ __forceinline__ DecUnit dec_unit(const FfnArgs& a, const int* s_groups, int u, int RT, int RB, int KT)
 {
-    Unit U;
-    const int gi = u / RT;
-    U.rt = u % RT;
+    DecUnit U;
+    U.s = u % a.S;
+    const int rest = u / a.S;
+    U.G = rest % RB;
+    const int gi = rest / RB;
     int lo = 0, hi = a.E - 1;
     while (lo < hi) {
         int mid = (lo + hi + 1) >> 1;
@@ -339,232 +363,259 @@ __device__ __forceinline__ Unit unit_of(const FfnArgs& a, const int* s_groups, i
     U.row0 = a.offsets[lo] + (gi - s_groups[lo]) * kRowsPerUnit;
     U.row_end = min(min(a.offsets[lo + 1], U.row0 + kRowsPerUnit), a.rows);
     U.nq = (U.row_end - U.row0 + 7) >> 3;
+    U.ng = min(8, RT - 8 * U.G);
+    U.k0 = (int)((long)KT * U.s / a.S);
+    U.k1 = (int)((long)KT * (U.s + 1) / a.S);
     U.blob = a.pool + (size_t)a.slot_of[lo] * a.slot_bytes;
     return U;
 }
 
 template <int WFMT, int PHASE>
-__global__ void __launch_bounds__(kFfnThreads) ffn_kernel(FfnArgs a)
+__global__ void __launch_bounds__(kDecThreads) ffn_kernel(FfnArgs a)
 {
-    using CFG = StreamCfg<WFMT>;
+    using CFG = DecCfg<WFMT>;
     constexpr bool FP4 = CFG::FP4;
-    constexpr int TILE = CFG::TILE, STILE = CFG::STILE, DA = CFG::DA, DX = CFG::DX, XSTAGE = CFG::XSTAGE;
-    extern __shared__ __align__(128) unsigned char smem[];
-    const int tid = threadIdx.x, lane = tid & 31, wib = tid >> 5, g = lane >> 2, t = lane & 3;
-    const int RT = a.R / 16, KT = a.K / 64, RP = a.rows + kRowPad;
-    unsigned char* wbase = smem + 128 + (size_t)wib * CFG::WARP_BYTES;
-    unsigned char* sA = wbase;                                    // DA x TILE
-    unsigned char* sS = sA + DA * TILE;                           // DA x STILE
-    unsigned char* sX = sS + DA * STILE;                          // DX x XSTAGE
-    uint64_t* barA = reinterpret_cast<uint64_t*>(sX + DX * XSTAGE);
-    uint64_t* barX = barA + DA;
-    int* s_groups = reinterpret_cast<int*>(smem + 128 + (size_t)(kFfnThreads / 32) * CFG::WARP_BYTES);
-    for (int i = tid; i <= a.E; i += kFfnThreads) s_groups[i] = a.groups[i];
-    if (lane == 0) {
-        for (int i = 0; i < DA; i++)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&barA[i])) : "memory");
-        for (int i = 0; i < DX; i++)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&barX[i])) : "memory");
+    constexpr int TILE = CFG::TILE, STILE = CFG::STILE, D = CFG::D, STAGE = CFG::STAGE;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);            // [D]
+    uint64_t* empty = full + D;                                     // [D]
+    unsigned char* ring = smem + 1024;
+    int* s_groups = reinterpret_cast<int*>(ring + (size_t)D * STAGE);
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, t = lane & 3;
+    const int RT = a.R / 16, RB = (RT + 7) / 8, KT = a.K / 64, RP = a.rows + kRowPad;
+    for (int i = tid; i <= a.E; i += kDecThreads) s_groups[i] = a.groups[i];
+    if (tid == 0) {
+        for (int i = 0; i < D; i++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&full[i])) : "memory");
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&empty[i])), "r"(kCW) : "memory");
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     __syncthreads();
-    const int total_units = s_groups[a.E] * RT;
-    const int warps_total = gridDim.x * (kFfnThreads / 32);
-    const int wg = blockIdx.x * (kFfnThreads / 32) + wib;
-    const int n_units = wg < total_units ? (total_units - 1 - wg) / warps_total + 1 : 0;
+    const int total = s_groups[a.E] * RB * a.S;
 
-    // Tile stream of this warp: units wg, wg + warps_total, ... each KT tiles.
-    // All positions advance incrementally (no division in the loop).
-    // Producer state (lane 0): the next weight / activation tile to issue.
-    struct Cursor {
-        int ui, kt, stage;
-        uint32_t unused;
-    };
-    Cursor ca{0, 0, 0, 0}, cx{0, 0, 0, 0};
-    Unit pa, px;
-    pa.e = px.e = -1;
-    int pa_ui = -1, px_ui = -1;
-    int issued_a = 0, issued_x = 0;           // tiles issued per stream
-    const int n_tiles = n_units * KT;         // < 2^31 for any supported shape
-    auto issue_a = [&]() {
-        if (ca.ui != pa_ui) {
-            pa = unit_of(a, s_groups, wg + ca.ui * warps_total, RT);
-            pa_ui = ca.ui;
+    if (w == kCW) {
+        // ------------------------------------------------ copy issue (one lane)
+        if (lane == 0) {
+            int st = 0;
+            uint32_t ph = 0;
+            long issued = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+                const DecUnit U = dec_unit(a, s_groups, u, RT, RB, KT);
+                const uint32_t bytes = U.ng * (TILE + STILE) + U.nq * 1024;
+                for (int kt = U.k0; kt < U.k1; kt++) {
+                    if (!(ok = mbar_wait_bounded(smem_u32(&empty[st]), ph ^ 1))) break;
+                    const uint32_t bar = smem_u32(&full[st]);
+                    unsigned char* sg = ring + (size_t)st * STAGE;
+                    const size_t ti = tile_index(8 * U.G, kt, RT, KT);
+                    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                                 : "memory");
+                    bulk_copy(smem_u32(sg), U.blob + a.w_off + ti * TILE, U.ng * TILE, bar);
+                    if (STILE) bulk_copy(smem_u32(sg + CFG::A_BYTES), U.blob + a.s_off + ti * STILE, U.ng * STILE, bar);
+                    bulk_copy(smem_u32(sg + CFG::A_BYTES + CFG::S_BYTES), a.in + ((size_t)kt * RP + U.row0) * 64,
+                              U.nq * 1024, bar);
+                    issued++;
+                    if (++st == D) { st = 0; ph ^= 1; }
+                }
+            }
+            if (!ok) atomicCAS(&g_ffn_error, 0, (int)MOE_ERR_TIMEOUT);
+            // let the last copies land before the CTA exits (stage i was last
+            // filled in this pass if i < st, else in the previous one)
+            for (int i = 0; i < D && i < issued; i++)
+                mbar_wait_bounded(smem_u32(&full[i]), i < st ? ph : (ph ^ 1));
         }
-        const uint32_t bar = smem_u32(&barA[ca.stage]);
-        const size_t ti = tile_index(pa.rt, ca.kt, RT, KT);
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(TILE + STILE) : "memory");
-        bulk_copy(smem_u32(sA + ca.stage * TILE), pa.blob + a.w_off + ti * TILE, TILE, bar);
-        if (STILE) bulk_copy(smem_u32(sS + ca.stage * STILE), pa.blob + a.s_off + ti * STILE, STILE, bar);
-        issued_a++;
-        if (++ca.kt == KT) { ca.kt = 0; ca.ui++; }
-        if (++ca.stage == DA) ca.stage = 0;
-    };
-    auto issue_x = [&]() {
-        if (cx.ui != px_ui) {
-            px = unit_of(a, s_groups, wg + cx.ui * warps_total, RT);
-            px_ui = cx.ui;
-        }
-        const uint32_t bar = smem_u32(&barX[cx.stage]);
-        const uint32_t bytes = (uint32_t)px.nq * 1024;
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-        bulk_copy(smem_u32(sX + cx.stage * XSTAGE), a.in + ((size_t)cx.kt * RP + px.row0) * 64, bytes, bar);
-        issued_x++;
-        if (++cx.kt == KT) { cx.kt = 0; cx.ui++; }
-        if (++cx.stage == DX) cx.stage = 0;
-    };
-    if (lane == 0) {
-        while (issued_a < DA && issued_a < n_tiles) issue_a();
-        while (issued_x < DX && issued_x < n_tiles) issue_x();
+        return;
     }
 
+    // ------------------------------------------------ compute warps
+    int st = 0;
+    uint32_t ph = 0;
     bool ok = true;
-    int n = 0, kt = 0, ui = 0, sa = 0, sx = 0;
-    uint32_t pha = 0, phx = 0;               // parity of the current pass over each ring
-    Unit cu;
-    cu.e = -1;
-    float acc[2][4];
-    for (; n < n_tiles; n++) {
-        if (kt == 0) {
-            cu = unit_of(a, s_groups, wg + ui * warps_total, RT);
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        const DecUnit U = dec_unit(a, s_groups, u, RT, RB, KT);
+        const bool act = w < U.ng;          // this warp has a row tile in the block
+        const int rt = 8 * U.G + w;
+        const int sw = (U.row0 + g) & 7;
+        float acc[2][4];
 #pragma unroll
-            for (int q = 0; q < 2; q++)
+        for (int q = 0; q < 2; q++)
 #pragma unroll
-                for (int i = 0; i < 4; i++) acc[q][i] = 0.0f;
+            for (int i = 0; i < 4; i++) acc[q][i] = 0.0f;
+        for (int kt = U.k0; kt < U.k1; kt++) {
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&full[st]), ph));
+            if (!ok) break;
+            const unsigned char* sg = ring + (size_t)st * STAGE;
+            uint4 cur[FP4 ? 1 : 4];
+            uint2 cs = make_uint2(0, 0);
+            uint4 xc[2][2];
+            if (act) {
+#pragma unroll
+                for (int v = 0; v < (FP4 ? 1 : 4); v++)
+                    cur[v] = *reinterpret_cast<const uint4*>(sg + w * TILE + v * 512 + 16 * lane);
+                if (WFMT == MOE_W_MXFP4) cs.x = *reinterpret_cast<const uint32_t*>(sg + CFG::A_BYTES + w * STILE + 4 * g);
+                if (WFMT == MOE_W_NVFP4) cs = *reinterpret_cast<const uint2*>(sg + CFG::A_BYTES + w * STILE + 8 * g);
+#pragma unroll
+                for (int q = 0; q < 2; q++) {
+                    if (q < U.nq) {
+                        const unsigned char* xrow = sg + CFG::A_BYTES + CFG::S_BYTES + q * 1024 + g * 128;
+                        xc[q][0] = *reinterpret_cast<const uint4*>(xrow + (((2 * t) ^ sw) << 4));
+                        xc[q][1] = *reinterpret_cast<const uint4*>(xrow + (((2 * t + 1) ^ sw) << 4));
+                    } else {
+                        xc[q][0] = xc[q][1] = make_uint4(0, 0, 0, 0);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&empty[st]));   // operands are in registers
+            if (++st == D) { st = 0; ph ^= 1; }
+            if (!act) continue;
+            if (!FP4) {
+                // bf16 fragments: cur[j] = {a0, a2, a1, a3} of step j
+#pragma unroll
+                for (int q = 0; q < 2; q++) {
+                    if (q >= U.nq) break;
+                    const uint32_t X[8] = {xc[q][0].x, xc[q][0].y, xc[q][0].z, xc[q][0].w,
+                                           xc[q][1].x, xc[q][1].y, xc[q][1].z, xc[q][1].w};
+#pragma unroll
+                    for (int j = 0; j < 4; j++)
+                        mma16816<false>(acc[q], cur[j].x, cur[j].z, cur[j].y, cur[j].w, X[2 * j], X[2 * j + 1]);
+                }
+            } else {
+                // f16 fragments from E2M1 bytes: row g bytes in .x/.y, row g+8 in .z/.w;
+                // byte 2j -> a0 (a1) of step j, byte 2j+1 -> a2 (a3)
+                uint32_t A[4][4];
+                uint32_t f0, f1, f2, f3;
+                e2m1x4_to_f16x2(cur[0].x, f0, f1, f2, f3);
+                A[0][0] = f0; A[0][2] = f1; A[1][0] = f2; A[1][2] = f3;
+                e2m1x4_to_f16x2(cur[0].y, f0, f1, f2, f3);
+                A[2][0] = f0; A[2][2] = f1; A[3][0] = f2; A[3][2] = f3;
+                e2m1x4_to_f16x2(cur[0].z, f0, f1, f2, f3);
+                A[0][1] = f0; A[0][3] = f1; A[1][1] = f2; A[1][3] = f3;
+                e2m1x4_to_f16x2(cur[0].w, f0, f1, f2, f3);
+                A[2][1] = f0; A[2][3] = f1; A[3][1] = f2; A[3][3] = f3;
+                float sg4[4], s84[4];   // scale of k16 steps 0..3 for rows g and g+8
+                if (WFMT == MOE_W_MXFP4) {
+                    sg4[0] = sg4[1] = mx_scale(cs.x & 0xFF);
+                    sg4[2] = sg4[3] = mx_scale((cs.x >> 8) & 0xFF);
+                    s84[0] = s84[1] = mx_scale((cs.x >> 16) & 0xFF);
+                    s84[2] = s84[3] = mx_scale(cs.x >> 24);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        sg4[j] = e4m3_value((cs.x >> (8 * j)) & 0xFF);
+                        s84[j] = e4m3_value((cs.y >> (8 * j)) & 0xFF);
+                    }
+                }
+                constexpr int SPB = (WFMT == MOE_W_MXFP4) ? 2 : 1;   // k16 steps per scale block
+#pragma unroll
+                for (int q = 0; q < 2; q++) {
+                    if (q >= U.nq) break;
+                    const uint32_t X[8] = {xc[q][0].x, xc[q][0].y, xc[q][0].z, xc[q][0].w,
+                                           xc[q][1].x, xc[q][1].y, xc[q][1].z, xc[q][1].w};
+#pragma unroll
+                    for (int j0 = 0; j0 < 4; j0 += SPB) {
+                        float tmp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                        for (int j = j0; j < j0 + SPB; j++)
+                            mma16816<true>(tmp, A[j][0], A[j][1], A[j][2], A[j][3], X[2 * j], X[2 * j + 1]);
+                        acc[q][0] = __fmaf_rn(tmp[0], sg4[j0], acc[q][0]);
+                        acc[q][1] = __fmaf_rn(tmp[1], sg4[j0], acc[q][1]);
+                        acc[q][2] = __fmaf_rn(tmp[2], s84[j0], acc[q][2]);
+                        acc[q][3] = __fmaf_rn(tmp[3], s84[j0], acc[q][3]);
+                    }
+                }
+            }
         }
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&barA[sa]), pha) &&
-                                          mbar_wait_bounded(smem_u32(&barX[sx]), phx));
-        if (!ok) break;
-        // operands from shared memory
-        uint4 cur[FP4 ? 1 : 4];
-#pragma unroll
-        for (int v = 0; v < (FP4 ? 1 : 4); v++) cur[v] = *reinterpret_cast<const uint4*>(sA + sa * TILE + v * 512 + 16 * lane);
-        uint2 cs = make_uint2(0, 0);
-        if (WFMT == MOE_W_MXFP4) cs.x = *reinterpret_cast<const uint32_t*>(sS + sa * STILE + 4 * g);
-        if (WFMT == MOE_W_NVFP4) cs = *reinterpret_cast<const uint2*>(sS + sa * STILE + 8 * g);
-        const int sw = (cu.row0 + g) & 7;
-        uint4 xc[2][2];
+        if (!ok || !act) continue;
+        // epilogue: undo the activation row exponents, apply the NVFP4 tensor scale;
+        // a K slice of a split unit writes fp32 partial sums instead
+        float tsc = 1.0f;
+        if (WFMT == MOE_W_NVFP4) tsc = reinterpret_cast<const float*>(U.blob + a.ts_off)[PHASE - 1];
 #pragma unroll
         for (int q = 0; q < 2; q++) {
-            if (q < cu.nq) {
-                const unsigned char* xrow = sX + sx * XSTAGE + q * 1024 + g * 128;
-                xc[q][0] = *reinterpret_cast<const uint4*>(xrow + (((2 * t) ^ sw) << 4));
-                xc[q][1] = *reinterpret_cast<const uint4*>(xrow + (((2 * t + 1) ^ sw) << 4));
+            if (q >= U.nq) break;
+            const int r0 = U.row0 + q * 8 + 2 * t, r1 = r0 + 1;
+            float u0 = tsc, u1 = tsc;
+            if (FP4) {
+                if (r0 < U.row_end) u0 = tsc * pow2i(-__ldg(a.in_ex + r0));
+                if (r1 < U.row_end) u1 = tsc * pow2i(-__ldg(a.in_ex + r1));
+            }
+            if (a.S > 1) {
+                // rows 16 rt + g and 16 rt + g + 8 of the packed matrix
+                float* pb = a.part + (size_t)U.s * a.rows * a.R;
+                const int c0 = 16 * rt + g;
+                if (r0 < U.row_end) {
+                    pb[(size_t)r0 * a.R + c0] = acc[q][0] * u0;
+                    pb[(size_t)r0 * a.R + c0 + 8] = acc[q][2] * u0;
+                }
+                if (r1 < U.row_end) {
+                    pb[(size_t)r1 * a.R + c0] = acc[q][1] * u1;
+                    pb[(size_t)r1 * a.R + c0 + 8] = acc[q][3] * u1;
+                }
+            } else if (PHASE == 1) {
+                const int F = a.R / 2;
+                const int f = 8 * rt + g;
+                if (r0 < U.row_end) a.out_h[(size_t)r0 * F + f] = silu(acc[q][0] * u0) * (acc[q][2] * u0);
+                if (r1 < U.row_end) a.out_h[(size_t)r1 * F + f] = silu(acc[q][1] * u1) * (acc[q][3] * u1);
             } else {
-                xc[q][0] = xc[q][1] = make_uint4(0, 0, 0, 0);
-            }
-        }
-        if (++sa == DA) { sa = 0; pha ^= 1; }
-        if (++sx == DX) { sx = 0; phx ^= 1; }
-        // stages consumed (their values are in registers): refill them with the
-        // tiles DA / DX ahead
-        __syncwarp();
-        if (lane == 0) {
-            if (issued_a < n_tiles) issue_a();
-            if (issued_x < n_tiles) issue_x();
-        }
-        if (!FP4) {
-            // bf16 fragments: cur[j] = {a0, a2, a1, a3} of step j
-#pragma unroll
-            for (int q = 0; q < 2; q++) {
-                if (q >= cu.nq) break;
-                const uint32_t X[8] = {xc[q][0].x, xc[q][0].y, xc[q][0].z, xc[q][0].w,
-                                       xc[q][1].x, xc[q][1].y, xc[q][1].z, xc[q][1].w};
-#pragma unroll
-                for (int j = 0; j < 4; j++)
-                    mma16816<false>(acc[q], cur[j].x, cur[j].z, cur[j].y, cur[j].w, X[2 * j], X[2 * j + 1]);
-            }
-        } else {
-            // f16 fragments from E2M1 bytes: row g bytes in .x/.y, row g+8 in .z/.w;
-            // byte 2j -> a0 (a1) of step j, byte 2j+1 -> a2 (a3)
-            uint32_t A[4][4];
-            uint32_t f0, f1, f2, f3;
-            e2m1x4_to_f16x2(cur[0].x, f0, f1, f2, f3);
-            A[0][0] = f0; A[0][2] = f1; A[1][0] = f2; A[1][2] = f3;
-            e2m1x4_to_f16x2(cur[0].y, f0, f1, f2, f3);
-            A[2][0] = f0; A[2][2] = f1; A[3][0] = f2; A[3][2] = f3;
-            e2m1x4_to_f16x2(cur[0].z, f0, f1, f2, f3);
-            A[0][1] = f0; A[0][3] = f1; A[1][1] = f2; A[1][3] = f3;
-            e2m1x4_to_f16x2(cur[0].w, f0, f1, f2, f3);
-            A[2][1] = f0; A[2][3] = f1; A[3][1] = f2; A[3][3] = f3;
-            float sg[4], s8[4];   // scale of k16 steps 0..3 for rows g and g+8
-            if (WFMT == MOE_W_MXFP4) {
-                sg[0] = sg[1] = mx_scale(cs.x & 0xFF);
-                sg[2] = sg[3] = mx_scale((cs.x >> 8) & 0xFF);
-                s8[0] = s8[1] = mx_scale((cs.x >> 16) & 0xFF);
-                s8[2] = s8[3] = mx_scale(cs.x >> 24);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    sg[j] = e4m3_value((cs.x >> (8 * j)) & 0xFF);
-                    s8[j] = e4m3_value((cs.y >> (8 * j)) & 0xFF);
+                const int Ho = a.R;
+                const int o = 16 * rt + g;
+                if (r0 < U.row_end) {
+                    a.out_y[(size_t)r0 * Ho + o] = f32_to_bf16_bits(acc[q][0] * u0);
+                    a.out_y[(size_t)r0 * Ho + o + 8] = f32_to_bf16_bits(acc[q][2] * u0);
                 }
-            }
-            constexpr int SPB = (WFMT == MOE_W_MXFP4) ? 2 : 1;   // k16 steps per scale block
-#pragma unroll
-            for (int q = 0; q < 2; q++) {
-                if (q >= cu.nq) break;
-                const uint32_t X[8] = {xc[q][0].x, xc[q][0].y, xc[q][0].z, xc[q][0].w,
-                                       xc[q][1].x, xc[q][1].y, xc[q][1].z, xc[q][1].w};
-#pragma unroll
-                for (int j0 = 0; j0 < 4; j0 += SPB) {
-                    float tmp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-                    for (int j = j0; j < j0 + SPB; j++)
-                        mma16816<true>(tmp, A[j][0], A[j][1], A[j][2], A[j][3], X[2 * j], X[2 * j + 1]);
-                    acc[q][0] = __fmaf_rn(tmp[0], sg[j0], acc[q][0]);
-                    acc[q][1] = __fmaf_rn(tmp[1], sg[j0], acc[q][1]);
-                    acc[q][2] = __fmaf_rn(tmp[2], s8[j0], acc[q][2]);
-                    acc[q][3] = __fmaf_rn(tmp[3], s8[j0], acc[q][3]);
+                if (r1 < U.row_end) {
+                    a.out_y[(size_t)r1 * Ho + o] = f32_to_bf16_bits(acc[q][1] * u1);
+                    a.out_y[(size_t)r1 * Ho + o + 8] = f32_to_bf16_bits(acc[q][3] * u1);
                 }
             }
         }
-        if (kt == KT - 1) {
-            // epilogue: undo the activation row exponents, apply the NVFP4 tensor scale
-            float tsc = 1.0f;
-            if (WFMT == MOE_W_NVFP4) tsc = reinterpret_cast<const float*>(cu.blob + a.ts_off)[PHASE - 1];
-#pragma unroll
-            for (int q = 0; q < 2; q++) {
-                if (q >= cu.nq) break;
-                const int r0 = cu.row0 + q * 8 + 2 * t, r1 = r0 + 1;
-                float u0 = tsc, u1 = tsc;
-                if (FP4) {
-                    if (r0 < cu.row_end) u0 = tsc * pow2i(-__ldg(a.in_ex + r0));
-                    if (r1 < cu.row_end) u1 = tsc * pow2i(-__ldg(a.in_ex + r1));
-                }
-                if (PHASE == 1) {
-                    const int F = a.R / 2;
-                    const int f = 8 * cu.rt + g;
-                    if (r0 < cu.row_end) a.out_h[(size_t)r0 * F + f] = silu(acc[q][0] * u0) * (acc[q][2] * u0);
-                    if (r1 < cu.row_end) a.out_h[(size_t)r1 * F + f] = silu(acc[q][1] * u1) * (acc[q][3] * u1);
-                } else {
-                    const int Ho = a.R;
-                    const int o = 16 * cu.rt + g;
-                    if (r0 < cu.row_end) {
-                        a.out_y[(size_t)r0 * Ho + o] = f32_to_bf16_bits(acc[q][0] * u0);
-                        a.out_y[(size_t)r0 * Ho + o + 8] = f32_to_bf16_bits(acc[q][2] * u0);
-                    }
-                    if (r1 < cu.row_end) {
-                        a.out_y[(size_t)r1 * Ho + o] = f32_to_bf16_bits(acc[q][1] * u1);
-                        a.out_y[(size_t)r1 * Ho + o + 8] = f32_to_bf16_bits(acc[q][3] * u1);
-                    }
-                }
-            }
-        }
-        if (++kt == KT) { kt = 0; ui++; }
     }
-    if (!ok) {
-        // a wait ran out: record it, then let every copy still in flight land
-        // (tile m sits in stage m % D with parity (m / D) & 1)
-        if (lane == 0) {
-            atomicCAS(&g_ffn_error, 0, (int)MOE_ERR_TIMEOUT);
-            for (int m = n; m < issued_a; m++) mbar_wait_bounded(smem_u32(&barA[m % DA]), (uint32_t)((m / DA) & 1));
-            for (int m = n; m < issued_x; m++) mbar_wait_bounded(smem_u32(&barX[m % DX]), (uint32_t)((m / DX) & 1));
+    if (!ok && lane == 0) atomicCAS(&g_ffn_error, 0, (int)MOE_ERR_TIMEOUT);
+}
+
+// Sum of the K-slice partials (ascending slice order), one CTA per row; rows
+// of an expert that the FFN skipped (no slot, out of range) are left as they
+// are.  Phase 1: h = silu(gate) * up from the packed gate / up rows; phase 2:
+// y in bf16.
+template <int PHASE>
+__global__ void __launch_bounds__(256) ffn_reduce_kernel(const float* __restrict__ part, int S, int rows, int R,
+                                                         const int32_t* __restrict__ offsets,
+                                                         const int32_t* __restrict__ slot_of, int E, int pool_slots,
+                                                         float* __restrict__ h, uint16_t* __restrict__ y)
+{
+    const int r = blockIdx.x;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (__ldg(offsets + mid) <= r) lo = mid;
+        else hi = mid - 1;
+    }
+    const int o0 = __ldg(offsets + lo), o1 = __ldg(offsets + lo + 1), sl = __ldg(slot_of + lo);
+    if (!(o0 >= 0 && o0 <= r && r < o1 && o1 <= rows && sl >= 0 && sl < pool_slots)) return;
+    const int outw = PHASE == 1 ? R / 2 : R;
+    for (int c = threadIdx.x; c < outw; c += blockDim.x) {
+        if (PHASE == 1) {
+            const int pg = 16 * (c >> 3) + (c & 7);      // packed row of gate feature c; up is 8 rows on
+            float gs = 0.0f, us = 0.0f;
+            for (int s = 0; s < S; s++) {
+                const float* pr = part + ((size_t)s * rows + r) * R;
+                gs += pr[pg];
+                us += pr[pg + 8];
+            }
+            h[(size_t)r * outw + c] = silu(gs) * us;
+        } else {
+            float ys = 0.0f;
+            for (int s = 0; s < S; s++) ys += part[((size_t)s * rows + r) * R + c];
+            y[(size_t)r * outw + c] = f32_to_bf16_bits(ys);
         }
-        __syncwarp();
     }
 }
+
+// Row-major activations larger than this never split K (partials stay small).
+constexpr int kSplitRowsCap = 1024;
 
 template <int WFMT>
 int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, size_t slot_bytes, int pool_slots,
@@ -596,29 +647,41 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     a.offsets = offsets;
     a.groups = w.groups;
     a.rows = rows;
-    const size_t smem = stream_smem_bytes<WFMT>(E);
+    a.part = w.part;
+    const size_t smem = dec_smem_bytes<WFMT>(E);
     // persistent grid: as many CTAs as fit at once (recomputed when the
     // shared-memory size, which grows with E, changes)
     static size_t attr_smem = 0, occ_smem = 0;
-    static int resident[2] = {1, 1};
+    static int resident = 1;
     if (smem > attr_smem) {
         MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_kernel<WFMT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
         MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_kernel<WFMT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
         attr_smem = smem;
     }
     if (smem != occ_smem) {
-        MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident[0], ffn_kernel<WFMT, 1>, kFfnThreads, smem));
-        MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident[1], ffn_kernel<WFMT, 2>, kFfnThreads, smem));
-        if (resident[0] < 1) resident[0] = 1;
-        if (resident[1] < 1) resident[1] = 1;
+        MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, ffn_kernel<WFMT, 1>, kDecThreads, smem));
+        if (resident < 1) resident = 1;
         occ_smem = smem;
     }
-    auto grid_for = [&](int R, int phase) {
-        long max_units = (long)((rows + kRowsPerUnit - 1) / kRowsPerUnit + (rows < E ? rows : E)) * (R / 16);
-        long gsz = (max_units + 3) / 4;
-        long cap = (long)sms * resident[phase - 1];
-        return (int)(gsz < 1 ? 1 : (gsz > cap ? cap : gsz));
+    const long slots = (long)sms * resident;
+    // K split so that the (estimated) number of units covers the grid twice
+    auto plan = [&](int R, int K, int& S, int& grid) {
+        const long RB = (R / 16 + 7) / 8;
+        const long groups_est = (rows < E ? rows : E);
+        const long base = groups_est * RB;
+        long Sx = base > 0 ? (2 * slots + base - 1) / base : 1;
+        const long kmax = (K / 64) / 4;
+        if (Sx > kmax) Sx = kmax;
+        if (Sx > 8) Sx = 8;
+        if ((long)rows * Sx > kSplitRowsCap) Sx = kSplitRowsCap / (rows > 0 ? rows : 1);
+        if (Sx < 1) Sx = 1;
+        S = (int)Sx;
+        const long units_max = ((long)(rows + kRowsPerUnit - 1) / kRowsPerUnit + (rows < E ? rows : E)) * RB * S;
+        grid = (int)(units_max < slots ? (units_max < 1 ? 1 : units_max) : slots);
     };
+    int S1, g1, S2, g2;
+    plan(2 * F, H, S1, g1);
+    plan(H, F, S2, g2);
     a.w_off = bl.w13;
     a.s_off = bl.s13;
     a.R = 2 * F;
@@ -626,8 +689,14 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     a.in = w.xb;
     a.in_ex = w.xe;
     a.out_h = w.h32;
-    ffn_kernel<WFMT, 1><<<grid_for(a.R, 1), kFfnThreads, smem, st>>>(a);
+    a.S = S1;
+    ffn_kernel<WFMT, 1><<<g1, kDecThreads, smem, st>>>(a);
     MOE_LAUNCH_CHECK();
+    if (S1 > 1) {
+        ffn_reduce_kernel<1><<<rows, 256, 0, st>>>(w.part, S1, rows, 2 * F, offsets, slot_of, E, pool_slots, w.h32,
+                                                   nullptr);
+        MOE_LAUNCH_CHECK();
+    }
     ffn_prep_kernel<true, FP4><<<prep_blocks, kPrepThreads, 0, st>>>(w.h32, rows, F, w.hb, w.he, nullptr, nullptr,
                                                                      E, 0, nullptr, nullptr, 1);
     MOE_LAUNCH_CHECK();
@@ -640,8 +709,14 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     b.in_ex = w.he;
     b.out_h = nullptr;
     b.out_y = y_perm;
-    ffn_kernel<WFMT, 2><<<grid_for(b.R, 2), kFfnThreads, smem, st>>>(b);
+    b.S = S2;
+    ffn_kernel<WFMT, 2><<<g2, kDecThreads, smem, st>>>(b);
     MOE_LAUNCH_CHECK();
+    if (S2 > 1) {
+        ffn_reduce_kernel<2><<<rows, 256, 0, st>>>(w.part, S2, rows, H, offsets, slot_of, E, pool_slots, nullptr,
+                                                   y_perm);
+        MOE_LAUNCH_CHECK();
+    }
     return MOE_OK;
 }
 

@@ -177,3 +177,36 @@ def test_trace40_nvfp4(orc):
         assert trace_rows(R.cache.read_trace()) == expect, s
     st = R.cache.stats()
     assert st["lookups"] == 48 * 40
+
+
+def test_resident_layer_replays_from_a_cuda_graph(orc):
+    """With every expert of the layer resident, moe_layer_forward reads
+    nothing back to the host, so a whole layer step can be captured in a CUDA
+    graph and replayed; replays with fresh inputs match eager calls exactly."""
+    cfg = W.scaled(W.DS_DECODE, experts=16, hidden=256, ffn=128, top_k=4, capacity=16)
+    R = Runner(cfg)
+    preload(R.cache, cfg)
+    wg, bias = R.router(0)
+    wgd, bd = dev(wg), dev(bias)
+    n = 8
+    xs = [W.gen_x(cfg, 0, n, "graph", i) for i in range(3)]
+    eager = []
+    for x in xs:
+        out, idx, _ = R.forward(0, x)
+        eager.append((out, idx))
+    xin = dev(xs[0]).clone()
+    out = torch.empty_like(xin)
+    idx = torch.empty(n, cfg.top_k, dtype=torch.int32, device="cuda")
+    ws = torch.empty(A.moe_layer_workspace_bytes(R.L.shape, n), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        A.moe_layer_forward(R.cache, 0, xin, wgd, bd, out, ws, stream=s, copy_stream=R.copy, topk_idx_out=idx)
+    for x, (o_ref, i_ref) in zip(xs, eager):
+        xin.copy_(dev(x))
+        g.replay()
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(host(idx), i_ref)
+        np.testing.assert_array_equal(host(out), o_ref)
+    del g

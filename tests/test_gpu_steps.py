@@ -165,6 +165,21 @@ def test_grouped_ffn_full_size(orc, base):
     assert worst < ALARM_REL_L2, worst
 
 
+@pytest.mark.parametrize("base", [W.DS_DECODE, W.TRACE40, W.QWEN_BF16], ids=["mxfp4", "nvfp4", "bf16"])
+@pytest.mark.parametrize("passes", [1, 2])
+def test_grouped_ffn_split_k(orc, base, passes, monkeypatch):
+    """Full expert shapes with few token groups: the streaming kernels split K
+    across CTAs and reduce the partial sums; rows of a skipped expert stay
+    untouched, and a second pass over the other experts keeps the first's."""
+    monkeypatch.setenv("MOE_FFN_PATH", "mma")
+    cfg = W.scaled(base, experts=6, top_k=2, layers=1)
+    counts = [1, 3, 2, 9, 0, 1]
+    slots = [4, -1, 0, 2, 5, 3]
+    worst = _ffn_case(orc, cfg, counts, slots, pool_slots=6, seed=5, passes=passes)
+    assert worst < ALARM_REL_L2, worst
+    assert A.L.lib.moe_get_device_error(1) == 0
+
+
 def test_grouped_ffn_slot_out_of_range_is_skipped(orc):
     cfg = W.scaled(W.DS_DECODE, **SMALL)
     counts = [2, 2, 0, 0, 0, 0, 0, 1]
