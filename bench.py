@@ -45,6 +45,7 @@ def parse():
     p.add_argument("--no-extras", action="store_true", help="skip the resident / prefill / batch-sweep legs")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--resident-batch", default="1,4,16", help="batch sizes of the resident decode leg")
     p.add_argument("--leg", choices=["all", "resident", "prefill"], default="all",
                    help="resident / prefill: run only that context leg (profiling); prints its own JSON line")
     return p.parse_args()
@@ -284,7 +285,8 @@ def run_ours(args, cfg, world, rank, local_rank):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     hbm_peak, peak_kind = measured_peaks()
     if args.leg != "all":
-        res = extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=(args.leg,))
+        res = extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=(args.leg,),
+                     batches=tuple(int(b) for b in args.resident_batch.split(",")))
         if rank == 0:
             print(json.dumps({"leg": args.leg, "steps": K, "warmup": Wm, "results": res}), flush=True)
         return
@@ -378,7 +380,8 @@ def run_ours(args, cfg, world, rank, local_rank):
         print(json.dumps(line), flush=True)
 
 
-def extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=("resident", "prefill")):
+def extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=("resident", "prefill"),
+           batches=(1, 4, 16)):
     """Context legs: the same layer with every expert resident (HBM-bound decode)
     at batch 1, 4 and 16, and the 4096-token prefill."""
     import torch
@@ -388,7 +391,7 @@ def extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=("r
     out = {}
     slot_bytes = A.moe_slot_bytes(shape)
     # resident decode (256 slots, all experts preloaded)
-    for n in ((1, 4, 16) if "resident" in legs else ()):
+    for n in (batches if "resident" in legs else ()):
         ds = DecodeStream(cfg, shape, blobs, wg, bias, n, K + Wm, cfg.experts, 0, device, tag="resident")
         ds.cache.lookup_update(0, torch.arange(cfg.experts, dtype=torch.int32, device=device))
         torch.cuda.synchronize()

@@ -55,8 +55,24 @@ struct FfnWs {
     uint16_t* hb;     // [F/64][rows+16][64] operand copy of h
     int32_t* he;      // [rows]
     int32_t* groups;  // [E+1] exclusive prefix of token groups per expert
-    float* part;      // K-slice partial sums, at most 1024 x max(2F, H) fp32
+    int32_t* cnt;     // [ncnt] pieces finished per unit of a unit split across CTAs
+    int ncnt;
+    float* pieces;    // [kMaxDecCtas][2][kPieceFloats] partial sums of split units
 };
+
+constexpr int kCW = 8;                               // compute warps of the streaming kernel
+constexpr int kMaxDecCtas = 1024;                    // CTAs of one streaming launch, at most
+constexpr int kPieceFloats = kCW * 2 * 32 * 4;       // one CTA's partial tile set [warp][q][lane][4]
+
+// Units (token group x 128-row block) of a layer call, at most: token groups
+// number at most rows/16 + (experts with rows) per expert, blocks max(2F, H)/128.
+long dec_units_max(const moe_shape* s, int rows)
+{
+    const long R = 2 * s->ffn > s->hidden ? 2 * s->ffn : s->hidden;
+    const long RB = (R / 16 + 7) / 8;
+    const long groups = (rows + kRowsPerUnit - 1) / kRowsPerUnit + (rows < s->experts ? rows : s->experts);
+    return groups * RB;
+}
 
 size_t ffn_ws_layout(const moe_shape* s, int rows, void* base, FfnWs* w)
 {
@@ -69,8 +85,9 @@ size_t ffn_ws_layout(const moe_shape* s, int rows, void* base, FfnWs* w)
     size_t ohb = take(2 * RP * s->ffn);
     size_t ohe = take(4 * R);
     size_t og = take(4 * (size_t)(s->experts + 1));
-    const size_t prow = (size_t)(8 * R < 1024 ? 8 * R : 1024);
-    size_t op = take(4 * prow * (size_t)(2 * s->ffn > s->hidden ? 2 * s->ffn : s->hidden));
+    const long ncnt = dec_units_max(s, (int)R);
+    size_t oc = take(4 * (size_t)ncnt);
+    size_t op = take(4 * (size_t)kMaxDecCtas * 2 * kPieceFloats);
     if (w) {
         char* b = static_cast<char*>(base);
         w->xb = reinterpret_cast<uint16_t*>(b + oxb);
@@ -79,7 +96,9 @@ size_t ffn_ws_layout(const moe_shape* s, int rows, void* base, FfnWs* w)
         w->hb = reinterpret_cast<uint16_t*>(b + ohb);
         w->he = reinterpret_cast<int32_t*>(b + ohe);
         w->groups = reinterpret_cast<int32_t*>(b + og);
-        w->part = reinterpret_cast<float*>(b + op);
+        w->cnt = reinterpret_cast<int32_t*>(b + oc);
+        w->ncnt = (int)ncnt;
+        w->pieces = reinterpret_cast<float*>(b + op);
     }
     return o;
 }
@@ -106,7 +125,7 @@ __device__ __forceinline__ size_t b_index(int r, int k, int RP)
 // ------------------------------------------------------------------ prep
 // One warp per row: operand copy (+ row exponent) of a bf16 or fp32 row
 // (read directly, or token gather[r]/gk of the source).  With `groups` set,
-// the last CTA writes the per-expert token-group prefix.  ROWMAJOR writes a
+// the last CTA writes the per-expert token-group prefix and clears `zero`.  ROWMAJOR writes a
 // plain [rows][K] f16 copy (the tensor-core path's TMA source) instead of the
 // column-block-major fragment layout.
 template <bool IN_F32, bool OUT_F16, bool ROWMAJOR = false>
@@ -115,10 +134,12 @@ __global__ void __launch_bounds__(kPrepThreads) ffn_prep_kernel(const void* __re
                                                                 const int32_t* __restrict__ offsets,
                                                                 const int32_t* __restrict__ slot_of, int E,
                                                                 int pool_slots, int32_t* __restrict__ groups,
-                                                                const int32_t* __restrict__ gather, int gk)
+                                                                const int32_t* __restrict__ gather, int gk,
+                                                                int32_t* __restrict__ zero, int nzero)
 {
     const int lane = threadIdx.x & 31;
     if (groups && blockIdx.x == gridDim.x - 1) {
+        for (int i = threadIdx.x; i < nzero; i += kPrepThreads) zero[i] = 0;
         __shared__ int s_warp[kPrepThreads / 32];
         const int EPT = (E + kPrepThreads - 1) / kPrepThreads;   // <= 16 for E <= 4096
         int loc = 0, cnts[16];
@@ -231,8 +252,8 @@ struct FfnArgs {
     const int32_t* in_ex;   // [rows] its exponents (FP4 formats)
     float* out_h;           // phase 1: h [rows][R/2] fp32
     uint16_t* out_y;        // phase 2: y [rows][R] bf16
-    int S;                  // K split: each unit covers 1/S of the column blocks
-    float* part;            // S > 1: partial sums [S][rows][R] fp32
+    int32_t* cnt;           // per unit: pieces finished (units split across CTAs)
+    float* pieces;          // [gridDim.x][2][kPieceFloats]
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -248,8 +269,10 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait (about 2 s of clock), false on timeout.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
+// Bounded wait (about 2 s of clock), false on timeout.  With `abort` set the
+// wait also gives up as soon as another warp of the CTA has raised it, and
+// raises it itself on a timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort = nullptr)
 {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
@@ -257,7 +280,11 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
 #pragma unroll 1
         for (int i = 0; i < 16; i++)
             if (mbar_try(bar, parity)) return true;
-        if (clock64() - t0 > kWaitCycles) return false;
+        if (abort && *abort) return false;
+        if (clock64() - t0 > kWaitCycles) {
+            if (abort) *abort = 1;
+            return false;
+        }
     }
 }
 
@@ -300,7 +327,7 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
                      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// E8M0 code -> 2^(c-127) (codes 2..142 only reach the kernels)
+// E8M0 code -> 2^(c-127) (codes 114..140 only reach the kernels)
 __device__ __forceinline__ float mx_scale(uint32_t c) { return __uint_as_float(c << 23); }
 
 // E4M3 code -> value (subnormals m * 2^-9; NaN codes are rejected at packing)
@@ -314,25 +341,32 @@ __device__ __forceinline__ float e4m3_value(uint32_t c)
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 
 // ---- CTA-cooperative weight streaming -------------------------------------
-// A CTA owns units (token group, 128-row block of W, slice of K).  Warp 8
-// (one lane) issues per 64-column chunk three bulk copies into a ring
-// stage: the block's eight 512-byte FP4 tiles (contiguous in the slot), their
-// scales, and the token group's 8 or 16 activation rows of that chunk.
-// Warps 0..7 each consume one 16-row tile of the stage and release it on an
-// mbarrier as soon as their operands are in registers.
-constexpr int kCW = 8;                        // compute warps
+// Work is a list of units (token group of one expert, 128-row block of W),
+// each KP = ceil(K/128) stages of two 64-column chunks long.  With at least
+// as many units as CTAs, CTAs take whole units round-robin.  Otherwise the
+// concatenated stage list is cut into equal ranges over the CTAs (stream-K):
+// a CTA runs whole units where its range covers them and pieces of the units
+// at its range ends.  A piece's partial sums go to a per-CTA buffer; the CTA that
+// finishes a unit's last piece adds all pieces in CTA order (deterministic)
+// and writes the result.
+// Inside a CTA, warp 8 (one lane) fills a ring stage with bulk copies: the
+// block's FP4 (or bf16) tiles of both chunks (contiguous in the slot), their
+// scales, and the token group's 8 or 16 activation rows of each chunk.
+// Warps 0..7 each multiply the 16-row tile they own in both chunks and then
+// release the stage on an mbarrier.
 constexpr int kDecThreads = 32 * (kCW + 1);   // + one copy-issue warp
+constexpr int kKC = 2;                        // 64-column chunks per stage
 
 template <int WFMT>
 struct DecCfg {
     static constexpr bool FP4 = WFMT != MOE_W_BF16;
     static constexpr int TILE = FP4 ? 512 : 2048;
     static constexpr int STILE = (WFMT == MOE_W_MXFP4) ? 32 : (WFMT == MOE_W_NVFP4 ? 64 : 0);
-    static constexpr int D = FP4 ? 8 : 4;                        // ring stages
-    static constexpr int A_BYTES = kCW * TILE;
-    static constexpr int S_BYTES = kCW * STILE;
-    static constexpr int X_BYTES = 2 * 1024;                     // up to 16 rows x 128 bytes
-    static constexpr int STAGE = A_BYTES + S_BYTES + X_BYTES;
+    static constexpr int D = FP4 ? 4 : 2;                        // ring stages
+    static constexpr int A_BYTES = kKC * kCW * TILE;
+    static constexpr int S_BYTES = kKC * kCW * STILE;
+    static constexpr int X_CHUNK = 2 * 1024;                     // up to 16 rows x 128 bytes
+    static constexpr int STAGE = A_BYTES + S_BYTES + kKC * X_CHUNK;
 };
 
 template <int WFMT>
@@ -342,17 +376,17 @@ size_t dec_smem_bytes(int E)
 }
 
 struct DecUnit {
-    int e, G, ng, row0, row_end, nq, k0, k1, s;
+    int e, G, ng, row0, row_end, nq, k0, k1;
     const char* blob;
 };
 
-__device__ __forceinline__ DecUnit dec_unit(const FfnArgs& a, const int* s_groups, int u, int RT, int RB, int KT)
+// Unit u, column chunks [k0, k1).
+__device__ __forceinline__ DecUnit dec_unit(const FfnArgs& a, const int* s_groups, int u, int RT, int RB, int k0,
+                                            int k1)
 {
     DecUnit U;
-    U.s = u % a.S;
-    const int rest = u / a.S;
-    U.G = rest % RB;
-    const int gi = rest / RB;
+    U.G = u % RB;
+    const int gi = u / RB;
     int lo = 0, hi = a.E - 1;
     while (lo < hi) {
         int mid = (lo + hi + 1) >> 1;
@@ -364,36 +398,252 @@ __device__ __forceinline__ DecUnit dec_unit(const FfnArgs& a, const int* s_group
     U.row_end = min(min(a.offsets[lo + 1], U.row0 + kRowsPerUnit), a.rows);
     U.nq = (U.row_end - U.row0 + 7) >> 3;
     U.ng = min(8, RT - 8 * U.G);
-    U.k0 = (int)((long)KT * U.s / a.S);
-    U.k1 = (int)((long)KT * (U.s + 1) / a.S);
+    U.k0 = k0;
+    U.k1 = k1;
     U.blob = a.pool + (size_t)a.slot_of[lo] * a.slot_bytes;
     return U;
 }
 
-template <int WFMT, int PHASE>
-__global__ void __launch_bounds__(kDecThreads) ffn_kernel(FfnArgs a)
+// Stage-list ranges: CTA c owns [bound(c), bound(c+1)).
+__device__ __forceinline__ long dec_bound(long W, int c, int grid) { return W * c / grid; }
+
+__device__ __forceinline__ int dec_cta_of(long W, long idx, int grid)
+{
+    int c = (int)(idx * grid / W);
+    while (c + 1 < grid && dec_bound(W, c + 1, grid) <= idx) c++;
+    while (c > 0 && dec_bound(W, c, grid) > idx) c--;
+    return c;
+}
+
+// Operands of one 16-row x 64-column tile in registers.
+template <int WFMT, int NQ>
+struct TileRegs {
+    uint4 w[WFMT == MOE_W_BF16 ? 4 : 1];
+    uint2 sc;
+    uint4 x[NQ][2];
+};
+
+template <int WFMT, int NQ>
+__device__ __forceinline__ void load_tile(TileRegs<WFMT, NQ>& T, const unsigned char* sg, int c, int ng, int w,
+                                          int lane, int g, int t, int sw)
 {
     using CFG = DecCfg<WFMT>;
-    constexpr bool FP4 = CFG::FP4;
+    const unsigned char* wt = sg + (c * ng + w) * CFG::TILE + 16 * lane;
+#pragma unroll
+    for (int v = 0; v < (CFG::FP4 ? 1 : 4); v++) T.w[v] = *reinterpret_cast<const uint4*>(wt + v * 512);
+    const unsigned char* st = sg + CFG::A_BYTES + (c * ng + w) * CFG::STILE;
+    if (WFMT == MOE_W_MXFP4) T.sc.x = *reinterpret_cast<const uint32_t*>(st + 4 * g);
+    if (WFMT == MOE_W_NVFP4) T.sc = *reinterpret_cast<const uint2*>(st + 8 * g);
+#pragma unroll
+    for (int q = 0; q < NQ; q++) {
+        const unsigned char* xrow = sg + CFG::A_BYTES + CFG::S_BYTES + c * CFG::X_CHUNK + q * 1024 + g * 128;
+        T.x[q][0] = *reinterpret_cast<const uint4*>(xrow + (((2 * t) ^ sw) << 4));
+        T.x[q][1] = *reinterpret_cast<const uint4*>(xrow + (((2 * t + 1) ^ sw) << 4));
+    }
+}
+
+// Multiply-accumulate of one tile.  FP4: the MMAs of one scale block sum
+// into a zeroed fp32 block result that is then scaled into the accumulator
+// (two independent chains per tile for MXFP4, four for NVFP4).
+template <int WFMT, int NQ>
+__device__ __forceinline__ void mma_tile(float (&acc)[2][4], const TileRegs<WFMT, NQ>& T)
+{
+    if (WFMT == MOE_W_BF16) {
+        // bf16 fragments: w[j] = {a0, a2, a1, a3} of step j
+#pragma unroll
+        for (int q = 0; q < NQ; q++) {
+            const uint32_t X[8] = {T.x[q][0].x, T.x[q][0].y, T.x[q][0].z, T.x[q][0].w,
+                                   T.x[q][1].x, T.x[q][1].y, T.x[q][1].z, T.x[q][1].w};
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                mma16816<false>(acc[q], T.w[j].x, T.w[j].z, T.w[j].y, T.w[j].w, X[2 * j], X[2 * j + 1]);
+        }
+        return;
+    }
+    // f16 fragments from E2M1 bytes: row g bytes in .x/.y, row g+8 in .z/.w;
+    // byte 2j -> a0 (a1) of step j, byte 2j+1 -> a2 (a3)
+    uint32_t A[4][4];
+    uint32_t f0, f1, f2, f3;
+    e2m1x4_to_f16x2(T.w[0].x, f0, f1, f2, f3);
+    A[0][0] = f0; A[0][2] = f1; A[1][0] = f2; A[1][2] = f3;
+    e2m1x4_to_f16x2(T.w[0].y, f0, f1, f2, f3);
+    A[2][0] = f0; A[2][2] = f1; A[3][0] = f2; A[3][2] = f3;
+    e2m1x4_to_f16x2(T.w[0].z, f0, f1, f2, f3);
+    A[0][1] = f0; A[0][3] = f1; A[1][1] = f2; A[1][3] = f3;
+    e2m1x4_to_f16x2(T.w[0].w, f0, f1, f2, f3);
+    A[2][1] = f0; A[2][3] = f1; A[3][1] = f2; A[3][3] = f3;
+    float sg4[4], s84[4];   // scale of k16 steps 0..3 for rows g and g+8
+    if (WFMT == MOE_W_MXFP4) {
+        sg4[0] = sg4[1] = mx_scale(T.sc.x & 0xFF);
+        sg4[2] = sg4[3] = mx_scale((T.sc.x >> 8) & 0xFF);
+        s84[0] = s84[1] = mx_scale((T.sc.x >> 16) & 0xFF);
+        s84[2] = s84[3] = mx_scale(T.sc.x >> 24);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            sg4[j] = e4m3_value((T.sc.x >> (8 * j)) & 0xFF);
+            s84[j] = e4m3_value((T.sc.y >> (8 * j)) & 0xFF);
+        }
+    }
+    constexpr int SPB = (WFMT == MOE_W_MXFP4) ? 2 : 1;   // k16 steps per scale block
+#pragma unroll
+    for (int q = 0; q < NQ; q++) {
+        const uint32_t X[8] = {T.x[q][0].x, T.x[q][0].y, T.x[q][0].z, T.x[q][0].w,
+                               T.x[q][1].x, T.x[q][1].y, T.x[q][1].z, T.x[q][1].w};
+#pragma unroll
+        for (int j0 = 0; j0 < 4; j0 += SPB) {
+            float tmp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int j = j0; j < j0 + SPB; j++)
+                mma16816<true>(tmp, A[j][0], A[j][1], A[j][2], A[j][3], X[2 * j], X[2 * j + 1]);
+            acc[q][0] = __fmaf_rn(tmp[0], sg4[j0], acc[q][0]);
+            acc[q][1] = __fmaf_rn(tmp[1], sg4[j0], acc[q][1]);
+            acc[q][2] = __fmaf_rn(tmp[2], s84[j0], acc[q][2]);
+            acc[q][3] = __fmaf_rn(tmp[3], s84[j0], acc[q][3]);
+        }
+    }
+}
+
+// Ring position shared by the compute warps.
+struct Ring {
+    int st;
+    uint32_t ph;
+    __device__ __forceinline__ void next(int D)
+    {
+        if (++st == D) { st = 0; ph ^= 1; }
+    }
+};
+
+// One unit's stages for a compute warp: wait, multiply its tile of both
+// chunks, release.  Returns false when a wait gave up.
+template <int WFMT, int NQ>
+__device__ __forceinline__ bool run_unit(float (&acc)[2][4], const DecUnit& U, bool act, Ring& R,
+                                         unsigned char* ring, uint64_t* full, uint64_t* empty, int w, int lane,
+                                         volatile int* abort)
+{
+    using CFG = DecCfg<WFMT>;
+    const int g = lane >> 2, t = lane & 3, sw = (U.row0 + g) & 7;
+    for (int kt = U.k0; kt < U.k1; kt += kKC) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&full[R.st]), R.ph, abort))) return false;
+        const unsigned char* sg = ring + (size_t)R.st * CFG::STAGE;
+        if (act) {
+            // one tile's operands live at a time; the stage is released after both
+            TileRegs<WFMT, NQ> T;
+            load_tile<WFMT, NQ>(T, sg, 0, U.ng, w, lane, g, t, sw);
+            mma_tile<WFMT, NQ>(acc, T);
+            if (kt + 1 < U.k1) {
+                load_tile<WFMT, NQ>(T, sg, 1, U.ng, w, lane, g, t, sw);
+                mma_tile<WFMT, NQ>(acc, T);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty[R.st]));
+        R.next(CFG::D);
+    }
+    return true;
+}
+
+// Final values of a warp's tile: undo the activation row exponents, apply
+// the NVFP4 tensor scale, then h = silu(gate) * up (phase 1) or y in bf16.
+template <int WFMT, int PHASE>
+__device__ __forceinline__ void write_tile(const FfnArgs& a, const DecUnit& U, int rt, const float (&acc)[2][4],
+                                           int g, int t)
+{
+    float tsc = 1.0f;
+    if (WFMT == MOE_W_NVFP4) tsc = reinterpret_cast<const float*>(U.blob + a.ts_off)[PHASE - 1];
+#pragma unroll
+    for (int q = 0; q < 2; q++) {
+        if (q >= U.nq) break;
+        const int r0 = U.row0 + q * 8 + 2 * t, r1 = r0 + 1;
+        float u0 = tsc, u1 = tsc;
+        if (WFMT != MOE_W_BF16) {
+            if (r0 < U.row_end) u0 = tsc * pow2i(-__ldg(a.in_ex + r0));
+            if (r1 < U.row_end) u1 = tsc * pow2i(-__ldg(a.in_ex + r1));
+        }
+        if (PHASE == 1) {
+            const int F = a.R / 2;
+            const int f = 8 * rt + g;
+            if (r0 < U.row_end) a.out_h[(size_t)r0 * F + f] = silu(acc[q][0] * u0) * (acc[q][2] * u0);
+            if (r1 < U.row_end) a.out_h[(size_t)r1 * F + f] = silu(acc[q][1] * u1) * (acc[q][3] * u1);
+        } else {
+            const int Ho = a.R;
+            const int o = 16 * rt + g;
+            if (r0 < U.row_end) {
+                a.out_y[(size_t)r0 * Ho + o] = f32_to_bf16_bits(acc[q][0] * u0);
+                a.out_y[(size_t)r0 * Ho + o + 8] = f32_to_bf16_bits(acc[q][2] * u0);
+            }
+            if (r1 < U.row_end) {
+                a.out_y[(size_t)r1 * Ho + o] = f32_to_bf16_bits(acc[q][1] * u1);
+                a.out_y[(size_t)r1 * Ho + o + 8] = f32_to_bf16_bits(acc[q][3] * u1);
+            }
+        }
+    }
+}
+
+// Segments of one CTA: whole units u = blockIdx.x + i * gridDim.x, or the
+// stream-K pieces of its stage range [pos, end): unit u, pairs [p0, p1).
+struct Seg {
+    long pos;     // next unit (whole) or next stage (stream-K)
+    long start;   // first stage of the current segment (stream-K)
+    int u, p0, p1;
+    __device__ __forceinline__ bool next(bool whole, int NU, int KP, long end)
+    {
+        if (whole) {
+            if (pos >= NU) return false;
+            u = (int)pos;
+            p0 = 0;
+            p1 = KP;
+            pos += gridDim.x;
+            return true;
+        }
+        if (pos >= end) return false;
+        start = pos;
+        u = (int)(pos / KP);
+        p0 = (int)(pos % KP);
+        p1 = (int)min((long)KP, p0 + (end - pos));
+        pos += p1 - p0;
+        return true;
+    }
+};
+
+__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kCW) : "memory"); }
+
+template <int WFMT, int PHASE>
+__global__ void __launch_bounds__(kDecThreads, 3) ffn_kernel(FfnArgs a)
+{
+    using CFG = DecCfg<WFMT>;
     constexpr int TILE = CFG::TILE, STILE = CFG::STILE, D = CFG::D, STAGE = CFG::STAGE;
     extern __shared__ __align__(1024) unsigned char smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);            // [D]
     uint64_t* empty = full + D;                                     // [D]
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + 512);
+    volatile int* s_last = reinterpret_cast<volatile int*>(smem + 516);
     unsigned char* ring = smem + 1024;
     int* s_groups = reinterpret_cast<int*>(ring + (size_t)D * STAGE);
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, t = lane & 3;
-    const int RT = a.R / 16, RB = (RT + 7) / 8, KT = a.K / 64, RP = a.rows + kRowPad;
+    const int RT = a.R / 16, RB = (RT + 7) / 8, KT = a.K / 64, KP = (KT + kKC - 1) / kKC, RP = a.rows + kRowPad;
     for (int i = tid; i <= a.E; i += kDecThreads) s_groups[i] = a.groups[i];
     if (tid == 0) {
         for (int i = 0; i < D; i++) {
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&full[i])) : "memory");
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&empty[i])), "r"(kCW) : "memory");
         }
+        *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     __syncthreads();
-    const int total = s_groups[a.E] * RB * a.S;
+    // With at least one unit per CTA, whole units go round-robin (an SM's
+    // CTAs share its issue slots, so uneven unit counts per CTA even out per
+    // SM); with fewer units than CTAs, the units' stages are cut into equal
+    // ranges over the CTAs (stream-K).
+    const int NU = s_groups[a.E] * RB;
+    const bool whole = NU >= (int)gridDim.x;
+    const long W = whole ? 0 : (long)NU * KP;     // stream-K stages
+    // CTAs in the stream-K part: no more than stages, so that no range is empty
+    const int grid = (int)(W < (long)gridDim.x ? W : (long)gridDim.x);
+    const bool in_use = (int)blockIdx.x < grid;
+    const long b0 = in_use ? dec_bound(W, blockIdx.x, grid) : 0, b1 = in_use ? dec_bound(W, blockIdx.x + 1, grid) : 0;
 
     if (w == kCW) {
         // ------------------------------------------------ copy issue (one lane)
@@ -402,24 +652,29 @@ __global__ void __launch_bounds__(kDecThreads) ffn_kernel(FfnArgs a)
             uint32_t ph = 0;
             long issued = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-                const DecUnit U = dec_unit(a, s_groups, u, RT, RB, KT);
-                const uint32_t bytes = U.ng * (TILE + STILE) + U.nq * 1024;
-                for (int kt = U.k0; kt < U.k1; kt++) {
-                    if (!(ok = mbar_wait_bounded(smem_u32(&empty[st]), ph ^ 1))) break;
+            auto issue = [&](const DecUnit& U) {
+                for (int kt = U.k0; kt < U.k1 && ok; kt += kKC) {
+                    const int nc = min(kKC, U.k1 - kt);
+                    if (!(ok = mbar_wait_bounded(smem_u32(&empty[st]), ph ^ 1, s_abort))) break;
                     const uint32_t bar = smem_u32(&full[st]);
                     unsigned char* sg = ring + (size_t)st * STAGE;
-                    const size_t ti = tile_index(8 * U.G, kt, RT, KT);
+                    const size_t ti = tile_index(8 * U.G, kt, RT, KT);   // chunks kt, kt+1 are adjacent
+                    const uint32_t bytes = nc * (U.ng * (TILE + STILE) + U.nq * 1024);
                     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                                  : "memory");
-                    bulk_copy(smem_u32(sg), U.blob + a.w_off + ti * TILE, U.ng * TILE, bar);
-                    if (STILE) bulk_copy(smem_u32(sg + CFG::A_BYTES), U.blob + a.s_off + ti * STILE, U.ng * STILE, bar);
-                    bulk_copy(smem_u32(sg + CFG::A_BYTES + CFG::S_BYTES), a.in + ((size_t)kt * RP + U.row0) * 64,
-                              U.nq * 1024, bar);
+                    bulk_copy(smem_u32(sg), U.blob + a.w_off + ti * TILE, nc * U.ng * TILE, bar);
+                    if (STILE)
+                        bulk_copy(smem_u32(sg + CFG::A_BYTES), U.blob + a.s_off + ti * STILE, nc * U.ng * STILE, bar);
+                    for (int c = 0; c < nc; c++)
+                        bulk_copy(smem_u32(sg + CFG::A_BYTES + CFG::S_BYTES + c * CFG::X_CHUNK),
+                                  a.in + ((size_t)(kt + c) * RP + U.row0) * 64, U.nq * 1024, bar);
                     issued++;
                     if (++st == D) { st = 0; ph ^= 1; }
                 }
-            }
+            };
+            Seg sg{whole ? (long)blockIdx.x : b0};
+            while (ok && sg.next(whole, NU, KP, b1))
+                issue(dec_unit(a, s_groups, sg.u, RT, RB, kKC * sg.p0, min(KT, kKC * sg.p1)));
             if (!ok) atomicCAS(&g_ffn_error, 0, (int)MOE_ERR_TIMEOUT);
             // let the last copies land before the CTA exits (stage i was last
             // filled in this pass if i < st, else in the previous one)
@@ -430,192 +685,77 @@ __global__ void __launch_bounds__(kDecThreads) ffn_kernel(FfnArgs a)
     }
 
     // ------------------------------------------------ compute warps
-    int st = 0;
-    uint32_t ph = 0;
+    // Every compute warp walks the same segments and meets the same named
+    // barriers; after a failed wait a warp keeps walking without waiting.
+    Ring R{0, 0};
     bool ok = true;
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-        const DecUnit U = dec_unit(a, s_groups, u, RT, RB, KT);
-        const bool act = w < U.ng;          // this warp has a row tile in the block
-        const int rt = 8 * U.G + w;
-        const int sw = (U.row0 + g) & 7;
-        float acc[2][4];
+    auto multiply = [&](const DecUnit& U, float (&acc)[2][4]) {
 #pragma unroll
         for (int q = 0; q < 2; q++)
 #pragma unroll
             for (int i = 0; i < 4; i++) acc[q][i] = 0.0f;
-        for (int kt = U.k0; kt < U.k1; kt++) {
-            ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&full[st]), ph));
-            if (!ok) break;
-            const unsigned char* sg = ring + (size_t)st * STAGE;
-            uint4 cur[FP4 ? 1 : 4];
-            uint2 cs = make_uint2(0, 0);
-            uint4 xc[2][2];
-            if (act) {
+        if (ok)
+            ok = U.nq == 1 ? run_unit<WFMT, 1>(acc, U, w < U.ng, R, ring, full, empty, w, lane, s_abort)
+                           : run_unit<WFMT, 2>(acc, U, w < U.ng, R, ring, full, empty, w, lane, s_abort);
+    };
+    Seg sg{whole ? (long)blockIdx.x : b0};
+    while (sg.next(whole, NU, KP, b1)) {
+        const int u = sg.u, p0 = sg.p0, p1 = sg.p1;
+        const long idx = sg.start;
+        const DecUnit U = dec_unit(a, s_groups, u, RT, RB, kKC * p0, min(KT, kKC * p1));
+        const bool act = w < U.ng;          // this warp has a row tile in the block
+        const int rt = 8 * U.G + w;
+        float acc[2][4];
+        multiply(U, acc);
+        if (p0 == 0 && p1 == KP) {
+            if (ok && act) write_tile<WFMT, PHASE>(a, U, rt, acc, g, t);
+        } else {
+            // a piece: publish the partial sums, count the piece, and let the
+            // CTA that completes the unit add all pieces up in CTA order
+            const int slot = idx == b0 ? 0 : 1;
+            float* mine = a.pieces + ((size_t)blockIdx.x * 2 + slot) * kPieceFloats;
+            if (ok && act)
 #pragma unroll
-                for (int v = 0; v < (FP4 ? 1 : 4); v++)
-                    cur[v] = *reinterpret_cast<const uint4*>(sg + w * TILE + v * 512 + 16 * lane);
-                if (WFMT == MOE_W_MXFP4) cs.x = *reinterpret_cast<const uint32_t*>(sg + CFG::A_BYTES + w * STILE + 4 * g);
-                if (WFMT == MOE_W_NVFP4) cs = *reinterpret_cast<const uint2*>(sg + CFG::A_BYTES + w * STILE + 8 * g);
-#pragma unroll
-                for (int q = 0; q < 2; q++) {
-                    if (q < U.nq) {
-                        const unsigned char* xrow = sg + CFG::A_BYTES + CFG::S_BYTES + q * 1024 + g * 128;
-                        xc[q][0] = *reinterpret_cast<const uint4*>(xrow + (((2 * t) ^ sw) << 4));
-                        xc[q][1] = *reinterpret_cast<const uint4*>(xrow + (((2 * t + 1) ^ sw) << 4));
-                    } else {
-                        xc[q][0] = xc[q][1] = make_uint4(0, 0, 0, 0);
-                    }
-                }
+                for (int q = 0; q < 2; q++)
+                    if (q < U.nq)
+                        *reinterpret_cast<float4*>(mine + ((w * 2 + q) * 32 + lane) * 4) =
+                            make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]);
+            __threadfence();
+            compute_bar();
+            const long u_lo = (long)u * KP, u_hi = u_lo + KP - 1;
+            const int c_lo = dec_cta_of(W, u_lo, grid), c_hi = dec_cta_of(W, u_hi, grid);
+            if (tid == 0) {
+                int last = 0;
+                if (!*s_abort) last = atomicAdd(a.cnt + u, 1) == c_hi - c_lo;
+                *s_last = last;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&empty[st]));   // operands are in registers
-            if (++st == D) { st = 0; ph ^= 1; }
-            if (!act) continue;
-            if (!FP4) {
-                // bf16 fragments: cur[j] = {a0, a2, a1, a3} of step j
+            compute_bar();
+            if (*s_last) {
+                __threadfence();
+                if (ok && act) {
+                    float sum[2][4];
 #pragma unroll
-                for (int q = 0; q < 2; q++) {
-                    if (q >= U.nq) break;
-                    const uint32_t X[8] = {xc[q][0].x, xc[q][0].y, xc[q][0].z, xc[q][0].w,
-                                           xc[q][1].x, xc[q][1].y, xc[q][1].z, xc[q][1].w};
+                    for (int q = 0; q < 2; q++)
 #pragma unroll
-                    for (int j = 0; j < 4; j++)
-                        mma16816<false>(acc[q], cur[j].x, cur[j].z, cur[j].y, cur[j].w, X[2 * j], X[2 * j + 1]);
-                }
-            } else {
-                // f16 fragments from E2M1 bytes: row g bytes in .x/.y, row g+8 in .z/.w;
-                // byte 2j -> a0 (a1) of step j, byte 2j+1 -> a2 (a3)
-                uint32_t A[4][4];
-                uint32_t f0, f1, f2, f3;
-                e2m1x4_to_f16x2(cur[0].x, f0, f1, f2, f3);
-                A[0][0] = f0; A[0][2] = f1; A[1][0] = f2; A[1][2] = f3;
-                e2m1x4_to_f16x2(cur[0].y, f0, f1, f2, f3);
-                A[2][0] = f0; A[2][2] = f1; A[3][0] = f2; A[3][2] = f3;
-                e2m1x4_to_f16x2(cur[0].z, f0, f1, f2, f3);
-                A[0][1] = f0; A[0][3] = f1; A[1][1] = f2; A[1][3] = f3;
-                e2m1x4_to_f16x2(cur[0].w, f0, f1, f2, f3);
-                A[2][1] = f0; A[2][3] = f1; A[3][1] = f2; A[3][3] = f3;
-                float sg4[4], s84[4];   // scale of k16 steps 0..3 for rows g and g+8
-                if (WFMT == MOE_W_MXFP4) {
-                    sg4[0] = sg4[1] = mx_scale(cs.x & 0xFF);
-                    sg4[2] = sg4[3] = mx_scale((cs.x >> 8) & 0xFF);
-                    s84[0] = s84[1] = mx_scale((cs.x >> 16) & 0xFF);
-                    s84[2] = s84[3] = mx_scale(cs.x >> 24);
-                } else {
+                        for (int i = 0; i < 4; i++) sum[q][i] = 0.0f;
+                    for (int c = c_lo; c <= c_hi; c++) {
+                        const int sl = dec_bound(W, c, grid) >= u_lo ? 0 : 1;
+                        const float* pc = a.pieces + ((size_t)c * 2 + sl) * kPieceFloats;
 #pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        sg4[j] = e4m3_value((cs.x >> (8 * j)) & 0xFF);
-                        s84[j] = e4m3_value((cs.y >> (8 * j)) & 0xFF);
+                        for (int q = 0; q < 2; q++)
+                            if (q < U.nq) {
+                                const float4 v = __ldcg(reinterpret_cast<const float4*>(pc + ((w * 2 + q) * 32 + lane) * 4));
+                                sum[q][0] += v.x; sum[q][1] += v.y; sum[q][2] += v.z; sum[q][3] += v.w;
+                            }
                     }
+                    write_tile<WFMT, PHASE>(a, U, rt, sum, g, t);
                 }
-                constexpr int SPB = (WFMT == MOE_W_MXFP4) ? 2 : 1;   // k16 steps per scale block
-#pragma unroll
-                for (int q = 0; q < 2; q++) {
-                    if (q >= U.nq) break;
-                    const uint32_t X[8] = {xc[q][0].x, xc[q][0].y, xc[q][0].z, xc[q][0].w,
-                                           xc[q][1].x, xc[q][1].y, xc[q][1].z, xc[q][1].w};
-#pragma unroll
-                    for (int j0 = 0; j0 < 4; j0 += SPB) {
-                        float tmp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-                        for (int j = j0; j < j0 + SPB; j++)
-                            mma16816<true>(tmp, A[j][0], A[j][1], A[j][2], A[j][3], X[2 * j], X[2 * j + 1]);
-                        acc[q][0] = __fmaf_rn(tmp[0], sg4[j0], acc[q][0]);
-                        acc[q][1] = __fmaf_rn(tmp[1], sg4[j0], acc[q][1]);
-                        acc[q][2] = __fmaf_rn(tmp[2], s84[j0], acc[q][2]);
-                        acc[q][3] = __fmaf_rn(tmp[3], s84[j0], acc[q][3]);
-                    }
-                }
-            }
-        }
-        if (!ok || !act) continue;
-        // epilogue: undo the activation row exponents, apply the NVFP4 tensor scale;
-        // a K slice of a split unit writes fp32 partial sums instead
-        float tsc = 1.0f;
-        if (WFMT == MOE_W_NVFP4) tsc = reinterpret_cast<const float*>(U.blob + a.ts_off)[PHASE - 1];
-#pragma unroll
-        for (int q = 0; q < 2; q++) {
-            if (q >= U.nq) break;
-            const int r0 = U.row0 + q * 8 + 2 * t, r1 = r0 + 1;
-            float u0 = tsc, u1 = tsc;
-            if (FP4) {
-                if (r0 < U.row_end) u0 = tsc * pow2i(-__ldg(a.in_ex + r0));
-                if (r1 < U.row_end) u1 = tsc * pow2i(-__ldg(a.in_ex + r1));
-            }
-            if (a.S > 1) {
-                // rows 16 rt + g and 16 rt + g + 8 of the packed matrix
-                float* pb = a.part + (size_t)U.s * a.rows * a.R;
-                const int c0 = 16 * rt + g;
-                if (r0 < U.row_end) {
-                    pb[(size_t)r0 * a.R + c0] = acc[q][0] * u0;
-                    pb[(size_t)r0 * a.R + c0 + 8] = acc[q][2] * u0;
-                }
-                if (r1 < U.row_end) {
-                    pb[(size_t)r1 * a.R + c0] = acc[q][1] * u1;
-                    pb[(size_t)r1 * a.R + c0 + 8] = acc[q][3] * u1;
-                }
-            } else if (PHASE == 1) {
-                const int F = a.R / 2;
-                const int f = 8 * rt + g;
-                if (r0 < U.row_end) a.out_h[(size_t)r0 * F + f] = silu(acc[q][0] * u0) * (acc[q][2] * u0);
-                if (r1 < U.row_end) a.out_h[(size_t)r1 * F + f] = silu(acc[q][1] * u1) * (acc[q][3] * u1);
-            } else {
-                const int Ho = a.R;
-                const int o = 16 * rt + g;
-                if (r0 < U.row_end) {
-                    a.out_y[(size_t)r0 * Ho + o] = f32_to_bf16_bits(acc[q][0] * u0);
-                    a.out_y[(size_t)r0 * Ho + o + 8] = f32_to_bf16_bits(acc[q][2] * u0);
-                }
-                if (r1 < U.row_end) {
-                    a.out_y[(size_t)r1 * Ho + o] = f32_to_bf16_bits(acc[q][1] * u1);
-                    a.out_y[(size_t)r1 * Ho + o + 8] = f32_to_bf16_bits(acc[q][3] * u1);
-                }
+                if (tid == 0) a.cnt[u] = 0;
             }
         }
     }
     if (!ok && lane == 0) atomicCAS(&g_ffn_error, 0, (int)MOE_ERR_TIMEOUT);
 }
-
-// Sum of the K-slice partials (ascending slice order), one CTA per row; rows
-// of an expert that the FFN skipped (no slot, out of range) are left as they
-// are.  Phase 1: h = silu(gate) * up from the packed gate / up rows; phase 2:
-// y in bf16.
-template <int PHASE>
-__global__ void __launch_bounds__(256) ffn_reduce_kernel(const float* __restrict__ part, int S, int rows, int R,
-                                                         const int32_t* __restrict__ offsets,
-                                                         const int32_t* __restrict__ slot_of, int E, int pool_slots,
-                                                         float* __restrict__ h, uint16_t* __restrict__ y)
-{
-    const int r = blockIdx.x;
-    int lo = 0, hi = E - 1;
-    while (lo < hi) {
-        int mid = (lo + hi + 1) >> 1;
-        if (__ldg(offsets + mid) <= r) lo = mid;
-        else hi = mid - 1;
-    }
-    const int o0 = __ldg(offsets + lo), o1 = __ldg(offsets + lo + 1), sl = __ldg(slot_of + lo);
-    if (!(o0 >= 0 && o0 <= r && r < o1 && o1 <= rows && sl >= 0 && sl < pool_slots)) return;
-    const int outw = PHASE == 1 ? R / 2 : R;
-    for (int c = threadIdx.x; c < outw; c += blockDim.x) {
-        if (PHASE == 1) {
-            const int pg = 16 * (c >> 3) + (c & 7);      // packed row of gate feature c; up is 8 rows on
-            float gs = 0.0f, us = 0.0f;
-            for (int s = 0; s < S; s++) {
-                const float* pr = part + ((size_t)s * rows + r) * R;
-                gs += pr[pg];
-                us += pr[pg + 8];
-            }
-            h[(size_t)r * outw + c] = silu(gs) * us;
-        } else {
-            float ys = 0.0f;
-            for (int s = 0; s < S; s++) ys += part[((size_t)s * rows + r) * R + c];
-            y[(size_t)r * outw + c] = f32_to_bf16_bits(ys);
-        }
-    }
-}
-
-// Row-major activations larger than this never split K (partials stay small).
-constexpr int kSplitRowsCap = 1024;
 
 template <int WFMT>
 int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, size_t slot_bytes, int pool_slots,
@@ -629,14 +769,15 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     if (prep_blocks > sms * 4) prep_blocks = sms * 4;
     if (gather && gather->x_dtype == MOE_DT_F32)
         ffn_prep_kernel<true, FP4><<<prep_blocks + 1, kPrepThreads, 0, st>>>(
-            gather->x, rows, H, w.xb, w.xe, offsets, slot_of, E, pool_slots, w.groups, gather->assign_of, gather->k);
+            gather->x, rows, H, w.xb, w.xe, offsets, slot_of, E, pool_slots, w.groups, gather->assign_of, gather->k,
+            w.cnt, w.ncnt);
     else if (gather)
         ffn_prep_kernel<false, FP4><<<prep_blocks + 1, kPrepThreads, 0, st>>>(
-            gather->x, rows, H, w.xb, w.xe, offsets, slot_of, E, pool_slots, w.groups, gather->assign_of, gather->k);
+            gather->x, rows, H, w.xb, w.xe, offsets, slot_of, E, pool_slots, w.groups, gather->assign_of, gather->k,
+            w.cnt, w.ncnt);
     else
-        ffn_prep_kernel<false, FP4><<<prep_blocks + 1, kPrepThreads, 0, st>>>(x_perm, rows, H, w.xb, w.xe, offsets,
-                                                                               slot_of, E, pool_slots, w.groups,
-                                                                               nullptr, 1);
+        ffn_prep_kernel<false, FP4><<<prep_blocks + 1, kPrepThreads, 0, st>>>(
+            x_perm, rows, H, w.xb, w.xe, offsets, slot_of, E, pool_slots, w.groups, nullptr, 1, w.cnt, w.ncnt);
     MOE_LAUNCH_CHECK();
     FfnArgs a{};
     a.pool = static_cast<const char*>(pool);
@@ -647,7 +788,8 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     a.offsets = offsets;
     a.groups = w.groups;
     a.rows = rows;
-    a.part = w.part;
+    a.cnt = w.cnt;
+    a.pieces = w.pieces;
     const size_t smem = dec_smem_bytes<WFMT>(E);
     // persistent grid: as many CTAs as fit at once (recomputed when the
     // shared-memory size, which grows with E, changes)
@@ -656,6 +798,9 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     if (smem > attr_smem) {
         MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_kernel<WFMT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
         MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_kernel<WFMT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        // several CTAs share an SM: take the largest shared-memory split
+        MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_kernel<WFMT, 1>, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+        MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_kernel<WFMT, 2>, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
         attr_smem = smem;
     }
     if (smem != occ_smem) {
@@ -663,25 +808,15 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
         if (resident < 1) resident = 1;
         occ_smem = smem;
     }
-    const long slots = (long)sms * resident;
-    // K split so that the (estimated) number of units covers the grid twice
-    auto plan = [&](int R, int K, int& S, int& grid) {
-        const long RB = (R / 16 + 7) / 8;
-        const long groups_est = (rows < E ? rows : E);
-        const long base = groups_est * RB;
-        long Sx = base > 0 ? (2 * slots + base - 1) / base : 1;
-        const long kmax = (K / 64) / 4;
-        if (Sx > kmax) Sx = kmax;
-        if (Sx > 8) Sx = 8;
-        if ((long)rows * Sx > kSplitRowsCap) Sx = kSplitRowsCap / (rows > 0 ? rows : 1);
-        if (Sx < 1) Sx = 1;
-        S = (int)Sx;
-        const long units_max = ((long)(rows + kRowsPerUnit - 1) / kRowsPerUnit + (rows < E ? rows : E)) * RB * S;
-        grid = (int)(units_max < slots ? (units_max < 1 ? 1 : units_max) : slots);
+    long grid = (long)sms * resident;
+    if (grid > kMaxDecCtas) grid = kMaxDecCtas;
+    // no more CTAs than stages (upper bound of the stage count: every unit possible)
+    auto grid_for = [&](int R, int K) {
+        const long RB = (R / 16 + 7) / 8, KP = (K / 64 + kKC - 1) / kKC;
+        const long groups = (rows + kRowsPerUnit - 1) / kRowsPerUnit + (rows < E ? rows : E);
+        const long wmax = groups * RB * KP;
+        return (int)(wmax < grid ? (wmax < 1 ? 1 : wmax) : grid);
     };
-    int S1, g1, S2, g2;
-    plan(2 * F, H, S1, g1);
-    plan(H, F, S2, g2);
     a.w_off = bl.w13;
     a.s_off = bl.s13;
     a.R = 2 * F;
@@ -689,16 +824,10 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     a.in = w.xb;
     a.in_ex = w.xe;
     a.out_h = w.h32;
-    a.S = S1;
-    ffn_kernel<WFMT, 1><<<g1, kDecThreads, smem, st>>>(a);
+    ffn_kernel<WFMT, 1><<<grid_for(2 * F, H), kDecThreads, smem, st>>>(a);
     MOE_LAUNCH_CHECK();
-    if (S1 > 1) {
-        ffn_reduce_kernel<1><<<rows, 256, 0, st>>>(w.part, S1, rows, 2 * F, offsets, slot_of, E, pool_slots, w.h32,
-                                                   nullptr);
-        MOE_LAUNCH_CHECK();
-    }
     ffn_prep_kernel<true, FP4><<<prep_blocks, kPrepThreads, 0, st>>>(w.h32, rows, F, w.hb, w.he, nullptr, nullptr,
-                                                                     E, 0, nullptr, nullptr, 1);
+                                                                     E, 0, nullptr, nullptr, 1, nullptr, 0);
     MOE_LAUNCH_CHECK();
     FfnArgs b = a;
     b.w_off = bl.w2;
@@ -709,14 +838,8 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     b.in_ex = w.he;
     b.out_h = nullptr;
     b.out_y = y_perm;
-    b.S = S2;
-    ffn_kernel<WFMT, 2><<<g2, kDecThreads, smem, st>>>(b);
+    ffn_kernel<WFMT, 2><<<grid_for(H, F), kDecThreads, smem, st>>>(b);
     MOE_LAUNCH_CHECK();
-    if (S2 > 1) {
-        ffn_reduce_kernel<2><<<rows, 256, 0, st>>>(w.part, S2, rows, H, offsets, slot_of, E, pool_slots, nullptr,
-                                                   y_perm);
-        MOE_LAUNCH_CHECK();
-    }
     return MOE_OK;
 }
 
@@ -767,12 +890,14 @@ int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool
         int pb = (rows + wpb - 1) / wpb;
         if (pb > sms0 * 8) pb = sms0 * 8;
         ffn_prep_kernel<false, true, true><<<pb, kPrepThreads, 0, st>>>(x_perm, rows, s->hidden, w.xb, w.xe, nullptr,
-                                                                         nullptr, s->experts, 0, nullptr, nullptr, 1);
+                                                                         nullptr, s->experts, 0, nullptr, nullptr, 1,
+                                                                         nullptr, 0);
         MOE_LAUNCH_CHECK();
         TcOperands op{w.xb, w.xe, w.h32, w.hb, w.he};
         return launch_ffn_tc(s, pool, slot_bytes, pool_slots, slot_of, offsets, rows, y_perm, op, st, [&]() -> int {
             ffn_prep_kernel<true, true, true><<<pb, kPrepThreads, 0, st>>>(w.h32, rows, s->ffn, w.hb, w.he, nullptr,
-                                                                            nullptr, s->experts, 0, nullptr, nullptr, 1);
+                                                                            nullptr, s->experts, 0, nullptr, nullptr, 1,
+                                                                            nullptr, 0);
             MOE_LAUNCH_CHECK();
             return MOE_OK;
         });
