@@ -103,27 +103,14 @@ size_t ffn_ws_layout(const moe_shape* s, int rows, void* base, FfnWs* w)
     return o;
 }
 
-// Position inside a 64-column block of column kk in the operand copy: quad
-// lane t reads positions 16t..16t+15; k16 step j's two pairs sit at 16t+4j
-// (columns 16j+2t, +1) and 16t+4j+2 (columns 16j+8+2t, +1).
-__device__ __forceinline__ int b_perm(int kk)
-{
-    const int j = kk >> 4, rem = kk & 15;
-    const int t = (rem & 7) >> 1, q = (rem & 1) | ((rem >> 3) << 1);
-    return 16 * t + 4 * j + q;
-}
-
-// Element offset of (row r, column k) in an operand copy with RP rows: block
-// kt = k/64 is [RP][64]; the 16-byte chunks of row r are XOR-swizzled by r&7.
-__device__ __forceinline__ size_t b_index(int r, int k, int RP)
-{
-    const int kt = k >> 6, p = b_perm(k & 63);
-    const int c = (p >> 3) ^ (r & 7);
-    return ((size_t)kt * RP + r) * 64 + c * 8 + (p & 7);
-}
+// Operand copy layout (the MMA B fragments of the streaming kernel): block
+// kt = k/64 is [RP][64] elements.  Inside a row's block, quad lane t reads
+// positions 16t..16t+15, where k16 step j's two column pairs sit at 16t+4j
+// (columns 16j+2t, +1) and 16t+4j+2 (columns 16j+8+2t, +1); the eight 16-byte
+// chunks of row r are stored XOR-swizzled by r&7.
 
 // ------------------------------------------------------------------ prep
-// One warp per row: operand copy (+ row exponent) of a bf16 or fp32 row
+// Operand copy (+ row exponent) of a bf16 or fp32 row
 // (read directly, or token gather[r]/gk of the source).  With `groups` set,
 // the last CTA writes the per-expert token-group prefix and clears `zero`.  ROWMAJOR writes a
 // plain [rows][K] f16 copy (the tensor-core path's TMA source) instead of the
@@ -173,68 +160,85 @@ __global__ void __launch_bounds__(kPrepThreads) ffn_prep_kernel(const void* __re
         if (threadIdx.x == kPrepThreads - 1) groups[E] = run;
         return;
     }
+    // one CTA per row: pass 1 finds the row's largest magnitude (f16 copies
+    // are scaled by a power of two), pass 2 writes 16-byte output chunks
+    __shared__ float s_max[kPrepThreads / 32 + 1];
     const int RP = rows + kRowPad;
     const int nblocks = gridDim.x - (groups ? 1 : 0);
-    const int warps_total = nblocks * (kPrepThreads / 32);
-    for (int r = blockIdx.x * (kPrepThreads / 32) + (threadIdx.x >> 5); r < rows; r += warps_total) {
+    const int nch = K / 8;   // 8-element chunks per row
+    const int wid = threadIdx.x >> 5;
+    for (int r = blockIdx.x; r < rows; r += nblocks) {
         const size_t sr = gather ? (size_t)(__ldg(gather + r) / gk) : (size_t)r;   // source row
-        auto load4 = [&](int c, float (&v)[4]) {
-            if (IN_F32) {
-                float4 q = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(in) + sr * K) + c);
-                v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-            } else {
-                uint2 q = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(in) + sr * K) + c);
-                v[0] = bf16_bits_to_f32(q.x & 0xFFFF); v[1] = bf16_bits_to_f32(q.x >> 16);
-                v[2] = bf16_bits_to_f32(q.y & 0xFFFF); v[3] = bf16_bits_to_f32(q.y >> 16);
-            }
-        };
+        const float* inf = static_cast<const float*>(in) + sr * K;
+        const uint16_t* inb = static_cast<const uint16_t*>(in) + sr * K;
         int p = 0;
         if (OUT_F16) {
             float mx = 0.0f;
-            for (int c0 = lane; c0 < K / 4; c0 += 32 * 8) {
-                float v[8][4];
+            for (int c = threadIdx.x; c < nch; c += kPrepThreads) {
+                if (IN_F32) {
+                    const float4 a = __ldg(reinterpret_cast<const float4*>(inf + 8 * c));
+                    const float4 b = __ldg(reinterpret_cast<const float4*>(inf + 8 * c) + 1);
+                    mx = fmaxf(mx, fmaxf(fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))),
+                                         fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w)))));
+                } else {
+                    const uint4 q = __ldg(reinterpret_cast<const uint4*>(inb + 8 * c));
+                    const uint32_t u[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-                for (int u = 0; u < 8; u++)
-                    if (c0 + 32 * u < K / 4) load4(c0 + 32 * u, v[u]);
-#pragma unroll
-                for (int u = 0; u < 8; u++)
-                    if (c0 + 32 * u < K / 4)
-#pragma unroll
-                        for (int i = 0; i < 4; i++) mx = fmaxf(mx, fabsf(v[u][i]));
+                    for (int i = 0; i < 4; i++)
+                        mx = fmaxf(mx, fmaxf(fabsf(bf16_bits_to_f32(u[i] & 0xFFFF)), fabsf(bf16_bits_to_f32(u[i] >> 16))));
+                }
             }
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            if (lane == 0) s_max[wid] = mx;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                float m = 0.0f;
+                for (int i = 0; i < kPrepThreads / 32; i++) m = fmaxf(m, s_max[i]);
+                s_max[kPrepThreads / 32] = m;
+            }
+            __syncthreads();
+            mx = s_max[kPrepThreads / 32];
             if (mx > 0.0f && mx <= 3.4e38f) {
                 int e2;
                 frexpf(mx, &e2);          // mx = m * 2^e2, m in [0.5, 1)
                 p = 15 - e2;              // mx * 2^p in [2^14, 2^15)
                 p = p < -100 ? -100 : (p > 100 ? 100 : p);
             }
-            if (lane == 0) ex[r] = p;
+            if (threadIdx.x == 0) ex[r] = p;
         }
         const float sc = ldexpf(1.0f, p);
-        for (int c0 = lane; c0 < K / 4; c0 += 32 * 8) {
-            float v[8][4];
-#pragma unroll
-            for (int u = 0; u < 8; u++)
-                if (c0 + 32 * u < K / 4) load4(c0 + 32 * u, v[u]);
-#pragma unroll
-            for (int u = 0; u < 8; u++) {
-                const int c = c0 + 32 * u;
-                if (c >= K / 4) break;
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    uint16_t o;
-                    if (OUT_F16) {
-                        __half hv = __float2half_rn(v[u][i] * sc);
-                        o = *reinterpret_cast<uint16_t*>(&hv);
-                    } else {
-                        o = f32_to_bf16_bits(v[u][i]);
-                    }
-                    out[ROWMAJOR ? (size_t)r * K + 4 * c + i : b_index(r, 4 * c + i, RP)] = o;
-                }
+        auto cvt2 = [&](float v0, float v1) -> uint32_t {
+            if (OUT_F16) {
+                const __half2 h = __floats2half2_rn(v0 * sc, v1 * sc);
+                return *reinterpret_cast<const uint32_t*>(&h);
+            }
+            return (uint32_t)f32_to_bf16_bits(v0) | ((uint32_t)f32_to_bf16_bits(v1) << 16);
+        };
+        // two adjacent source columns (col even)
+        auto pair = [&](int col) -> uint32_t {
+            if (IN_F32) {
+                const float2 v = __ldg(reinterpret_cast<const float2*>(inf + col));
+                return cvt2(v.x, v.y);
+            }
+            const uint32_t q = __ldg(reinterpret_cast<const uint32_t*>(inb + col));
+            return cvt2(bf16_bits_to_f32(q & 0xFFFF), bf16_bits_to_f32(q >> 16));
+        };
+        for (int c = threadIdx.x; c < nch; c += kPrepThreads) {
+            uint4 o;
+            if (ROWMAJOR) {
+                o = make_uint4(pair(8 * c), pair(8 * c + 2), pair(8 * c + 4), pair(8 * c + 6));
+                *reinterpret_cast<uint4*>(out + (size_t)r * K + 8 * c) = o;
+            } else {
+                // output chunk cc of 64-column block kt holds, for j = 2(cc&1) + jj
+                // and t = cc/2, the pairs at columns 16j + 8h + 2t (element 4jj + 2h)
+                const int kt = c >> 3, cc = c & 7, t = cc >> 1, jb = 2 * (cc & 1);
+                const int base = 64 * kt + 16 * jb + 2 * t;
+                o = make_uint4(pair(base), pair(base + 8), pair(base + 16), pair(base + 24));
+                *reinterpret_cast<uint4*>(out + ((size_t)kt * RP + r) * 64 + (size_t)((cc ^ (r & 7)) * 8)) = o;
             }
         }
+        if (OUT_F16) __syncthreads();   // s_max is reused by the next row
     }
 }
 
@@ -764,9 +768,7 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
 {
     constexpr bool FP4 = WFMT != MOE_W_BF16;
     const int E = s->experts, H = s->hidden, F = s->ffn;
-    const int wpb = kPrepThreads / 32;
-    int prep_blocks = (rows + wpb - 1) / wpb;
-    if (prep_blocks > sms * 4) prep_blocks = sms * 4;
+    int prep_blocks = rows < sms * 8 ? rows : sms * 8;   // a CTA per row
     if (gather && gather->x_dtype == MOE_DT_F32)
         ffn_prep_kernel<true, FP4><<<prep_blocks + 1, kPrepThreads, 0, st>>>(
             gather->x, rows, H, w.xb, w.xe, offsets, slot_of, E, pool_slots, w.groups, gather->assign_of, gather->k,
@@ -886,9 +888,7 @@ int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool
     if (use_tc_path(s, rows)) {
         // tensor-core path: f16 operand rows (x, then h), each scaled by a power of two
         prof_count(MOE_PROF_FFN, 4);
-        const int wpb = kPrepThreads / 32;
-        int pb = (rows + wpb - 1) / wpb;
-        if (pb > sms0 * 8) pb = sms0 * 8;
+        const int pb = rows < sms0 * 8 ? rows : sms0 * 8;   // a CTA per row
         ffn_prep_kernel<false, true, true><<<pb, kPrepThreads, 0, st>>>(x_perm, rows, s->hidden, w.xb, w.xe, nullptr,
                                                                          nullptr, s->experts, 0, nullptr, nullptr, 1,
                                                                          nullptr, 0);

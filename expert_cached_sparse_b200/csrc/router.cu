@@ -287,6 +287,55 @@ __global__ void __launch_bounds__(128) router_topk_kernel(const float* __restric
     }
 }
 
+// Warp per token with the token's logits in registers (EPL per lane, expert
+// lane + 32 i in slot i): k rounds of arg-max over the experts not yet taken,
+// then the same weights as router_topk_kernel.
+template <int EPL>
+__global__ void __launch_bounds__(128) router_topk_reg_kernel(const float* __restrict__ logits, int n, int E, int k,
+                                                              int32_t* __restrict__ idx, float* __restrict__ w)
+{
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= n) return;
+    const float* lt = logits + (size_t)t * E;
+    float v[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; i++) v[i] = (lane + 32 * i < E) ? __ldg(lt + lane + 32 * i) : 0.0f;
+    uint32_t avail = 0;   // bit i: expert lane + 32 i exists and is not taken
+#pragma unroll
+    for (int i = 0; i < EPL; i++)
+        if (lane + 32 * i < E) avail |= 1u << i;
+    float my_l = 0.0f;
+    int my_i = 0;
+    for (int r = 0; r < k; r++) {
+        float bv = 0.0f;
+        int bi = -1;
+#pragma unroll
+        for (int i = 0; i < EPL; i++)
+            if (((avail >> i) & 1) && (bi < 0 || ranks_above(v[i], lane + 32 * i, bv, bi))) {
+                bv = v[i];
+                bi = lane + 32 * i;
+            }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (oi >= 0 && (bi < 0 || ranks_above(ov, oi, bv, bi))) { bv = ov; bi = oi; }
+        }
+        if ((bi & 31) == lane) avail &= ~(1u << (bi >> 5));
+        if (lane == r) { my_l = bv; my_i = bi; }
+    }
+    const float lmax = __shfl_sync(0xffffffffu, my_l, 0);
+    float p = (lane < k) ? expf(my_l - lmax) : 0.0f;
+    float z = p;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+    if (lane < k) {
+        idx[(size_t)t * k + lane] = my_i;
+        w[(size_t)t * k + lane] = p / z;
+    }
+}
+
 template <bool XF32>
 int launch_logits(const void* x, const uint16_t* wg, const float* bias, int n, int H, int E,
                   float* logits, cudaStream_t st)
@@ -321,8 +370,13 @@ int launch_router(const void* x, int x_dtype, const uint16_t* wg, const float* b
                                      : launch_logits<false>(x, wg, bias, n, H, E, logits, st);
     if (rc) return rc;
     const int wpb = 4;
-    size_t smem = (size_t)wpb * E;
-    router_topk_kernel<<<(n + wpb - 1) / wpb, wpb * 32, smem, st>>>(logits, n, E, k, idx, w);
+    const int blocks = (n + wpb - 1) / wpb;
+    if (E <= 256)
+        router_topk_reg_kernel<8><<<blocks, wpb * 32, 0, st>>>(logits, n, E, k, idx, w);
+    else if (E <= 1024)
+        router_topk_reg_kernel<32><<<blocks, wpb * 32, 0, st>>>(logits, n, E, k, idx, w);
+    else
+        router_topk_kernel<<<blocks, wpb * 32, (size_t)wpb * E, st>>>(logits, n, E, k, idx, w);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }

@@ -26,7 +26,11 @@ def _x_dev(cfg, x):
 # ------------------------------------------------------------------ router
 ROUTER_CASES = [(W.TINY, 64), (W.TINY, 1), (W.DS_DECODE, 1), (W.DS_DECODE, 4), (W.DS_DECODE, 16),
                 (W.DS_DECODE, 37), (W.DS_PREFILL, 300), (W.QWEN_BF16, 512), (W.QWEN_BF16, 8),
-                (W.TRACE40, 1)]
+                (W.TRACE40, 1),
+                # expert counts of the other top-k kernels (more than 256, more than 1024) and k = E
+                (W.scaled(W.DS_DECODE, hidden=256, experts=600, top_k=8), 5),
+                (W.scaled(W.DS_DECODE, hidden=256, experts=2048, top_k=32), 3),
+                (W.scaled(W.DS_DECODE, hidden=256, experts=32, top_k=32), 7)]
 
 
 @pytest.mark.parametrize("cfg,n", ROUTER_CASES, ids=lambda v: getattr(v, "name", str(v)))
