@@ -273,6 +273,22 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread for up to kSuspendNs
+// while the phase is incomplete (it resumes when the phase completes), so
+// waiting warps do not take issue slots from working ones.
+constexpr uint32_t kSuspendNs = 20000;
+
+__device__ __forceinline__ bool mbar_try_suspend(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity), "n"(kSuspendNs)
+                 : "memory");
+    return ok != 0;
+}
+
 // Bounded wait (about 2 s of clock), false on timeout.  With `abort` set the
 // wait also gives up as soon as another warp of the CTA has raised it, and
 // raises it itself on a timeout.
@@ -281,9 +297,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
-#pragma unroll 1
-        for (int i = 0; i < 16; i++)
-            if (mbar_try(bar, parity)) return true;
+        if (mbar_try_suspend(bar, parity)) return true;
         if (abort && *abort) return false;
         if (clock64() - t0 > kWaitCycles) {
             if (abort) *abort = 1;

@@ -12,9 +12,11 @@
 //    bf16 (E2M1 x block scale is exact in bf16) and write it with
 //    tcgen05.st straight into tensor memory, where the MMA reads its A
 //    operand; no bf16 weight tile ever touches shared memory;
-//  - tokens (x_perm, or h for the down projection) arrive by TMA in 16-row
-//    boxes with the 128-byte swizzle the MMA's shared-memory descriptor
-//    expects; rows past the expert's block are loaded but never stored;
+//  - tokens (x_perm, or h for the down projection) arrive by TMA in 16- to
+//    128-row boxes with the 128-byte swizzle the MMA's shared-memory
+//    descriptor expects, as many 64-column chunks per 32 KB stage as fit, so
+//    small token blocks keep more chunks in flight; rows past the expert's
+//    block are loaded but never stored;
 //  - the accumulator lives in tensor memory (128 lanes x N fp32 columns);
 //    the same four warps read it back with tcgen05.ld for the epilogue:
 //    SwiGLU (gate and up rows are 8 lanes apart, one shuffle) into h, or the
@@ -36,14 +38,15 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN_MAX = 256;
 constexpr int BK = 64;
-constexpr int SA = 8;              // FP4 A stages
-constexpr int SB = 4;              // token (B) stages
-constexpr int NABUF = 4;           // tensor-memory A buffers
-constexpr int NXW = 8;             // expanding warps: two per tensor-memory lane quarter
+constexpr int SA = 16;             // FP4 A stages (one 64-column chunk each)
+constexpr int SB = 4;              // token (B) stages: as many 64-column chunks as fit 32 KB
+constexpr int NABUF = 8;           // tensor-memory A buffers
+constexpr int NXG = 1;             // expanding groups: group g expands chunks g, g+NXG, ...
+constexpr int NXW = 8 * NXG;       // expanding warps: two per tensor-memory lane quarter and group
 constexpr int THREADS = 32 * (2 + NXW);   // warp 0 copies, warp 1 MMA, warps 2.. expand + epilogue
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t D_COL = 0;      // accumulator columns [0, 256)
-constexpr uint32_t A_COL = 256;    // A buffers: 32 columns each (4 buffers: 256..383)
+constexpr uint32_t A_COL = 256;    // A buffers: 32 columns each (8 buffers: 256..511)
 constexpr uint32_t B_STAGE_BYTES = BN_MAX * 128;
 constexpr uint32_t A_STAGE_BYTES = 8 * 512;
 constexpr uint32_t S_STAGE_BYTES = 8 * 64;
@@ -91,18 +94,31 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait: try_wait (which suspends briefly in hardware) in a tight
-// loop; every 32 tries it checks the CTA's abort flag and the clock, and after
-// WAIT_CYCLES it records MOE_ERR_TIMEOUT and raises the abort flag so the
-// other roles drain too.
+// try_wait that lets the hardware suspend the thread for up to kSuspendNs
+// while the phase is incomplete (it resumes when the phase completes), so
+// waiting warps do not take issue slots from working ones.
+constexpr uint32_t kSuspendNs = 20000;
+
+__device__ __forceinline__ bool mbar_try_suspend(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity), "n"(kSuspendNs)
+                 : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: suspending try_wait in a loop; after every try it checks the
+// CTA's abort flag and the clock, and after WAIT_CYCLES it records
+// MOE_ERR_TIMEOUT and raises the abort flag so the other roles drain too.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag)
 {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
-#pragma unroll 1
-        for (int i = 0; i < 32; i++)
-            if (mbar_try(bar, parity)) return true;
+        if (mbar_try_suspend(bar, parity)) return true;
         if (*abort_flag) return false;
         if (clock64() - t0 > WAIT_CYCLES) break;
     }
@@ -218,6 +234,7 @@ __device__ uint16_t scale_mult(int wfmt, int c)
 
 struct Tile {
     int e, rb, row0, nrows, bn;
+    int ncps;   // 64-column chunks of the token block per B stage
 };
 
 __device__ __forceinline__ Tile tile_of(int u, const int* prefix, int E, int RB, const int32_t* offsets)
@@ -239,6 +256,7 @@ __device__ __forceinline__ Tile tile_of(int u, const int* prefix, int E, int RB,
     t.row0 = offsets[lo] + tb * bs;
     t.nrows = max(0, min(bs, m - tb * bs));
     t.bn = max(16, (t.nrows + 15) & ~15);
+    t.ncps = min(8, (int)(B_STAGE_BYTES / (t.bn * 128)));
     return t;
 }
 
@@ -309,14 +327,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (tid == 0) {
         for (int i = 0; i < SA; i++) {
             mbar_init(smem_u32(&full_a[i]), 1);
-            mbar_init(smem_u32(&empty_a[i]), NXW);
+            mbar_init(smem_u32(&empty_a[i]), NXW / NXG);
         }
         for (int i = 0; i < SB; i++) {
             mbar_init(smem_u32(&full_b[i]), 1);
             mbar_init(smem_u32(&empty_b[i]), 1);
         }
         for (int i = 0; i < NABUF; i++) {
-            mbar_init(smem_u32(&a_ready[i]), 32 * NXW);
+            mbar_init(smem_u32(&a_ready[i]), 32 * NXW / NXG);
             mbar_init(smem_u32(&a_free[i]), 1);
         }
         mbar_init(smem_u32(d_full), 1);
@@ -357,17 +375,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                     bulk_g2s(smem_u32(sA + sa * A_STAGE_BYTES), blob + a.w_off + ti * 512, A_STAGE_BYTES, fa);
                     bulk_g2s(smem_u32(sS + sa * S_STAGE_BYTES), blob + a.s_off + ti * STILE, 8 * STILE, fa);
                     if (++sa == SA) { sa = 0; pa ^= 1; }
+                    if (c % t.ncps) continue;   // this chunk's tokens came with an earlier B stage
                     ok = mbar_wait(smem_u32(&empty_b[sb]), pb ^ 1, abort_v);
                     if (!ok) break;
                     const uint32_t fb = smem_u32(&full_b[sb]);
-                    mbar_expect_tx(fb, (uint32_t)t.bn * 128);
-                    int done = 0;
+                    const int nch = min(t.ncps, KT - c);
+                    mbar_expect_tx(fb, (uint32_t)(nch * t.bn * 128));
+                    for (int j = 0; j < nch; j++) {
+                        const uint32_t dst = smem_u32(sB + sb * B_STAGE_BYTES + j * t.bn * 128);
+                        int done = 0;
 #pragma unroll
-                    for (int mi = 3; mi >= 0; mi--) {
-                        const int box = 16 << mi;
-                        while (t.bn - done >= box) {
-                            tma_load_2d(smem_u32(sB + sb * B_STAGE_BYTES + done * 128), &maps.m[mi], c * BK, t.row0 + done, fb);
-                            done += box;
+                        for (int mi = 3; mi >= 0; mi--) {
+                            const int box = 16 << mi;
+                            while (t.bn - done >= box) {
+                                tma_load_2d(dst + done * 128, &maps.m[mi], (c + j) * BK, t.row0 + done, fb);
+                                done += box;
+                            }
                         }
                     }
                     if (++sb == SB) { sb = 0; pb ^= 1; }
@@ -394,18 +417,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 const uint32_t idesc = idesc_f16(t.bn);
                 for (int c = 0; c < KT && ok; c++) {
-                    ok = mbar_wait(smem_u32(&a_ready[ab]), pab, abort_v) &&
-                         mbar_wait(smem_u32(&full_b[sb]), pb, abort_v);
+                    const int j = c % t.ncps;   // chunk inside the B stage
+                    if (j == 0) ok = mbar_wait(smem_u32(&full_b[sb]), pb, abort_v);
+                    ok = ok && mbar_wait(smem_u32(&a_ready[ab]), pab, abort_v);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t bbase = smem_u32(sB + sb * B_STAGE_BYTES);
+                    const uint32_t bbase = smem_u32(sB + sb * B_STAGE_BYTES + j * t.bn * 128);
 #pragma unroll
                     for (int k = 0; k < BK / 16; k++)
                         tc_mma_ts(tmem + D_COL, tmem + A_COL + 32 * ab + 8 * k, smem_desc_sw128(bbase + 32 * k), idesc,
                                   (c | k) != 0);
-                    tc_commit(smem_u32(&empty_b[sb]));
                     tc_commit(smem_u32(&a_free[ab]));
-                    if (++sb == SB) { sb = 0; pb ^= 1; }
+                    if (j == t.ncps - 1 || c == KT - 1) {   // the stage's last chunk
+                        tc_commit(smem_u32(&empty_b[sb]));
+                        if (++sb == SB) { sb = 0; pb ^= 1; }
+                    }
                     if (++ab == NABUF) { ab = 0; pab ^= 1; }
                 }
                 if (ok) tc_commit(smem_u32(d_full));
@@ -416,21 +442,28 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else {
         // ================= expand FP4 -> tensor memory, epilogue =================
-        // Two warps per tensor-memory lane quarter: set 0 expands bytes 0..3 of
-        // each lane segment (columns 0..15 of the chunk), set 1 bytes 4..7
-        // (columns 16..31); in the epilogue the sets take alternate 32-column
+        // Per group, two warps per tensor-memory lane quarter: set 0 expands
+        // bytes 0..3 of each lane segment (columns 0..15 of the chunk), set 1
+        // bytes 4..7 (columns 16..31).  Group g takes the chunks whose running
+        // index is g mod NXG, so NXG chunks are expanded at once.  In the
+        // epilogue the 2*NXG warps of a quarter take interleaved 32-column
         // groups of the accumulator.
+        const int xw = warp - 2;
         const int q = warp & 3;                 // tensor-memory lane quarter of this warp
-        const int set = (warp - 2) >> 2;        // 0 or 1
+        const int set = (xw >> 2) & 1;          // 0 or 1
+        const int grp = xw >> 3;                // 0 .. NXG-1
         const int r = 32 * q + lane;            // weight row inside the 128-row block
         const int rtl = r >> 4, rr = r & 15, g = rr & 7, half = rr >> 3;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        int sa = 0, ab = 0, it = 0;
-        uint32_t pa = 0, pab = 0;
+        int it = 0, pend = -1;   // pend: buffer whose tensor-memory store is in flight
+        long ci = 0;             // running chunk index over this CTA's tiles
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x, it++) {
             Tile t = tile_of(u, prefix, E, RB, a.offsets);
-            for (int c = 0; c < KT && ok; c++) {
+            for (int c = 0; c < KT && ok; c++, ci++) {
+                if ((int)(ci % NXG) != grp) continue;
+                const int sa = (int)(ci % SA), ab = (int)(ci % NABUF);
+                const uint32_t pa = (uint32_t)(ci / SA) & 1, pab = (uint32_t)(ci / NABUF) & 1;
                 ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full_a[sa]), pa, abort_v));
                 if (!ok) break;
                 const unsigned char* arow = sA + sa * A_STAGE_BYTES + rtl * 512 + 64 * g + 8 * half + 4 * set;
@@ -452,7 +485,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                 m1 |= m1 << 16;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&empty_a[sa]));
-                if (++sa == SA) { sa = 0; pa ^= 1; }
                 uint32_t v[16];
 #pragma unroll
                 for (int tt = 0; tt < 4; tt++) {
@@ -463,12 +495,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&a_free[ab]), pab ^ 1, abort_v));
                 if (!ok) break;
+                // the previous chunk's store has run while this chunk was expanded:
+                // complete it and hand that buffer to the MMA
+                if (pend >= 0) {
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(smem_u32(&a_ready[pend]));
+                }
                 tc_fence_after();
                 tmem_st16(tmem + lane_base + A_COL + 32 * ab + 16 * set, v);
+                pend = ab;
+            }
+            if (pend >= 0) {   // the tile's last chunk
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(smem_u32(&a_ready[ab]));
-                if (++ab == NABUF) { ab = 0; pab ^= 1; }
+                mbar_arrive(smem_u32(&a_ready[pend]));
+                pend = -1;
             }
             if (!ok) break;
             ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(d_full), it & 1, abort_v));
@@ -477,9 +519,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             const char* blob = a.pool + (size_t)a.slot_of[t.e] * a.slot_bytes;
             float tsc = 1.0f;
             if (WFMT == MOE_W_NVFP4) tsc = reinterpret_cast<const float*>(blob + a.ts_off)[PHASE - 1];
-            for (int c0 = 32 * set; c0 < t.bn; c0 += 64) {
+            for (int c0 = 32 * (set + 2 * grp); c0 < t.bn; c0 += 64 * NXG) {
                 uint32_t d[32];
                 tmem_ld32(tmem + lane_base + D_COL + c0, d);
+                // lane j holds the scale of token column c0 + j (row exponent, NVFP4 tensor scale)
+                const int nl = c0 + lane;
+                const float ul = (nl < t.nrows) ? tsc * pow2i(-__ldg(a.in_ex + t.row0 + nl)) : 0.0f;
                 tmem_wait_ld();
                 if (PHASE == 1) {
                     const int F = a.R / 2;
@@ -487,11 +532,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 32; j++) {
                         const int n = c0 + j;
-                        const float u = (n < t.nrows) ? tsc * pow2i(-__ldg(a.in_ex + t.row0 + n)) : 0.0f;
-                        const float x = __uint_as_float(d[j]) * u;
+                        const float x = __uint_as_float(d[j]) * __shfl_sync(0xffffffffu, ul, j);
                         const float up = __shfl_down_sync(0xffffffffu, x, 8);
                         if (half == 0 && n < t.nrows)
-                            a.out_h[(size_t)(t.row0 + n) * F + f] = x / (1.0f + expf(-x)) * up;
+                            a.out_h[(size_t)(t.row0 + n) * F + f] = x / (1.0f + __expf(-x)) * up;
                     }
                 } else {
                     const int Ho = a.R;
@@ -499,10 +543,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 32; j++) {
                         const int n = c0 + j;
-                        if (n < t.nrows) {
-                            const float u = tsc * pow2i(-__ldg(a.in_ex + t.row0 + n));
+                        const float u = __shfl_sync(0xffffffffu, ul, j);
+                        if (n < t.nrows)
                             a.out_y[(size_t)(t.row0 + n) * Ho + o] = f32_to_bf16_bits(__uint_as_float(d[j]) * u);
-                        }
                     }
                 }
             }
