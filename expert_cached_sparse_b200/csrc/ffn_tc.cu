@@ -36,18 +36,19 @@ __device__ int g_tc_error;   // first device-side error of the tensor-core FFN (
 namespace {
 
 constexpr int BM = 128;
-constexpr int BN_MAX = 256;
+constexpr int BN_MAX = 128;       // token rows per tile (two accumulators fit tensor memory)
 constexpr int BK = 64;
 constexpr int SA = 16;             // FP4 A stages (one 64-column chunk each)
 constexpr int SB = 4;              // token (B) stages: as many 64-column chunks as fit 32 KB
 constexpr int NABUF = 8;           // tensor-memory A buffers
 constexpr int NXG = 1;             // expanding groups: group g expands chunks g, g+NXG, ...
 constexpr int NXW = 8 * NXG;       // expanding warps: two per tensor-memory lane quarter and group
-constexpr int THREADS = 32 * (2 + NXW);   // warp 0 copies, warp 1 MMA, warps 2.. expand + epilogue
+constexpr int NEPI = 4;            // epilogue warps, one per tensor-memory lane quarter
+constexpr int THREADS = 32 * (2 + NXW + NEPI);   // warp 0 copies, warp 1 MMA, then expand, then epilogue
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t D_COL = 0;      // accumulator columns [0, 256)
+constexpr uint32_t D_COL = 0;      // two accumulators: columns [0, 128) and [128, 256)
 constexpr uint32_t A_COL = 256;    // A buffers: 32 columns each (8 buffers: 256..511)
-constexpr uint32_t B_STAGE_BYTES = BN_MAX * 128;
+constexpr uint32_t B_STAGE_BYTES = 32 * 1024;
 constexpr uint32_t A_STAGE_BYTES = 8 * 512;
 constexpr uint32_t S_STAGE_BYTES = 8 * 64;
 constexpr long long WAIT_CYCLES = 4000000000ll;   // ~2 s at 2 GHz before a wait gives up
@@ -282,9 +283,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint64_t* empty_b = full_b + SB;
     uint64_t* a_ready = empty_b + SB;
     uint64_t* a_free = a_ready + NABUF;
-    uint64_t* d_full = a_free + NABUF;
-    uint64_t* d_empty = d_full + 1;
-    uint64_t* fin = d_empty + 1;
+    uint64_t* d_full = a_free + NABUF;   // [2]
+    uint64_t* d_empty = d_full + 2;      // [2]
+    uint64_t* fin = d_empty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
     int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
     uint16_t* s_mult = reinterpret_cast<uint16_t*>(abort_flag + 1);   // [256]
@@ -337,8 +338,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(smem_u32(&a_ready[i]), 32 * NXW / NXG);
             mbar_init(smem_u32(&a_free[i]), 1);
         }
-        mbar_init(smem_u32(d_full), 1);
-        mbar_init(smem_u32(d_empty), 32 * NXW);
+        for (int i = 0; i < 2; i++) {
+            mbar_init(smem_u32(&d_full[i]), 1);
+            mbar_init(smem_u32(&d_empty[i]), 32 * NEPI);
+        }
         mbar_init(smem_u32(fin), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -410,8 +413,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             bool ok = true;
             for (int u = blockIdx.x; u < total && ok; u += gridDim.x, it++) {
                 Tile t = tile_of(u, prefix, E, RB, a.offsets);
-                if (it > 0) {
-                    ok = mbar_wait(smem_u32(d_empty), (it - 1) & 1, abort_v);
+                const int db = it & 1;   // accumulator of this tile
+                if (it >= 2) {           // its previous tile's epilogue is done
+                    ok = mbar_wait(smem_u32(&d_empty[db]), ((it >> 1) - 1) & 1, abort_v);
                     if (!ok) break;
                     tc_fence_after();
                 }
@@ -425,7 +429,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint32_t bbase = smem_u32(sB + sb * B_STAGE_BYTES + j * t.bn * 128);
 #pragma unroll
                     for (int k = 0; k < BK / 16; k++)
-                        tc_mma_ts(tmem + D_COL, tmem + A_COL + 32 * ab + 8 * k, smem_desc_sw128(bbase + 32 * k), idesc,
+                        tc_mma_ts(tmem + D_COL + BN_MAX * db, tmem + A_COL + 32 * ab + 8 * k, smem_desc_sw128(bbase + 32 * k), idesc,
                                   (c | k) != 0);
                     tc_commit(smem_u32(&a_free[ab]));
                     if (j == t.ncps - 1 || c == KT - 1) {   // the stage's last chunk
@@ -434,20 +438,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                     if (++ab == NABUF) { ab = 0; pab ^= 1; }
                 }
-                if (ok) tc_commit(smem_u32(d_full));
+                if (ok) tc_commit(smem_u32(&d_full[db]));
             }
             // every MMA issued by this thread completes before tensor memory is released
             tc_commit(smem_u32(fin));
             mbar_wait(smem_u32(fin), 0, abort_v);
         }
-    } else {
-        // ================= expand FP4 -> tensor memory, epilogue =================
+    } else if (warp < 2 + NXW) {
+        // ================= expand FP4 -> tensor memory =================
         // Per group, two warps per tensor-memory lane quarter: set 0 expands
         // bytes 0..3 of each lane segment (columns 0..15 of the chunk), set 1
         // bytes 4..7 (columns 16..31).  Group g takes the chunks whose running
-        // index is g mod NXG, so NXG chunks are expanded at once.  In the
-        // epilogue the 2*NXG warps of a quarter take interleaved 32-column
-        // groups of the accumulator.
+        // index is g mod NXG.
         const int xw = warp - 2;
         const int q = warp & 3;                 // tensor-memory lane quarter of this warp
         const int set = (xw >> 2) & 1;          // 0 or 1
@@ -455,11 +457,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int r = 32 * q + lane;            // weight row inside the 128-row block
         const int rtl = r >> 4, rr = r & 15, g = rr & 7, half = rr >> 3;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        int it = 0, pend = -1;   // pend: buffer whose tensor-memory store is in flight
+        int pend = -1;           // buffer whose tensor-memory store is in flight
         long ci = 0;             // running chunk index over this CTA's tiles
         bool ok = true;
-        for (int u = blockIdx.x; u < total && ok; u += gridDim.x, it++) {
-            Tile t = tile_of(u, prefix, E, RB, a.offsets);
+        for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
             for (int c = 0; c < KT && ok; c++, ci++) {
                 if ((int)(ci % NXG) != grp) continue;
                 const int sa = (int)(ci % SA), ab = (int)(ci % NABUF);
@@ -512,16 +513,27 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mbar_arrive(smem_u32(&a_ready[pend]));
                 pend = -1;
             }
-            if (!ok) break;
-            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(d_full), it & 1, abort_v));
-            if (!ok) break;
+        }
+    } else {
+        // ================= epilogue: accumulator -> h or y =================
+        // One warp per tensor-memory lane quarter; tile `it` used accumulator
+        // it & 1, so this runs while the next tile is multiplied.
+        const int q = warp & 3;
+        const int r = 32 * q + lane;            // weight row inside the 128-row block
+        const int rtl = r >> 4, rr = r & 15, g = rr & 7, half = rr >> 3;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        int it = 0;
+        for (int u = blockIdx.x; u < total; u += gridDim.x, it++) {
+            const Tile t = tile_of(u, prefix, E, RB, a.offsets);
+            const int db = it & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&d_full[db]), (it >> 1) & 1, abort_v))) break;
             tc_fence_after();
             const char* blob = a.pool + (size_t)a.slot_of[t.e] * a.slot_bytes;
             float tsc = 1.0f;
             if (WFMT == MOE_W_NVFP4) tsc = reinterpret_cast<const float*>(blob + a.ts_off)[PHASE - 1];
-            for (int c0 = 32 * (set + 2 * grp); c0 < t.bn; c0 += 64 * NXG) {
+            for (int c0 = 0; c0 < t.bn; c0 += 32) {
                 uint32_t d[32];
-                tmem_ld32(tmem + lane_base + D_COL + c0, d);
+                tmem_ld32(tmem + lane_base + D_COL + BN_MAX * db + c0, d);
                 // lane j holds the scale of token column c0 + j (row exponent, NVFP4 tensor scale)
                 const int nl = c0 + lane;
                 const float ul = (nl < t.nrows) ? tsc * pow2i(-__ldg(a.in_ex + t.row0 + nl)) : 0.0f;
@@ -550,7 +562,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(smem_u32(d_empty));
+            mbar_arrive(smem_u32(&d_empty[db]));
         }
     }
     __syncthreads();
@@ -604,7 +616,7 @@ int make_row_maps(RowMaps* rm, const void* base, int rows, int cols)
 
 size_t tc_smem_bytes(int E)
 {
-    return 1024 + SB * B_STAGE_BYTES + SA * A_STAGE_BYTES + SA * S_STAGE_BYTES + 8 * (2 * SA + 2 * SB + 2 * NABUF + 3) +
+    return 1024 + SB * B_STAGE_BYTES + SA * A_STAGE_BYTES + SA * S_STAGE_BYTES + 8 * (2 * SA + 2 * SB + 2 * NABUF + 5) +
            8 + 2 * 256 + 4 * (size_t)(E + 1) + 64;
 }
 
