@@ -38,7 +38,7 @@ L2_FLUSH_BYTES = 256 << 20
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--batch", type=int, default=16)
@@ -78,10 +78,14 @@ class Clocks:
             os.close(fd)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + ",".join(self.FIELDS),
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        t0 = time.time()   # the sampler is running once it has written a line
+        while time.time() - t0 < 5 and os.path.getsize(self.path) == 0 and self.proc.poll() is None:
+            time.sleep(0.01)
 
     def stop(self):
         if not self.proc:
@@ -186,6 +190,21 @@ class DecodeStream:
         self.A.moe_layer_forward(self.cache, 0, self.x[s] if x is None else x, self.wg, self.bias,
                                  self.out if out is None else out, self.ws, stream=self.stream,
                                  copy_stream=self.copy, topk_idx_out=self.idx[s])
+
+
+# DRAM bytes (read + write) per grouped-FFN call of the headline decode
+# stream, summed over the call's kernels (operand preps and both projections)
+# and averaged over the calls of an ncu capture of that workload.  Valid only
+# for the FFN source it was measured on: another source reports null.
+FFN_TRAFFIC = {"source_sha1": "1f525af80ef26cd84af8ddbd89d3403c5c5f9406", "bytes_per_call": 206345808}
+
+
+def ffn_traffic():
+    import hashlib
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "expert_cached_sparse_b200", "csrc", "ffn.cu")
+    with open(path, "rb") as f:
+        h = hashlib.sha1(f.read()).hexdigest()
+    return FFN_TRAFFIC["bytes_per_call"] if h == FFN_TRAFFIC["source_sha1"] else None
 
 
 def ffn_algorithmic_bytes(idx_steps, cfg, slot_bytes):
@@ -331,7 +350,7 @@ def run_ours(args, cfg, world, rank, local_rank):
             "dtype": "bf16", "data": "synthetic", "config": workload_config(cfg, n, world)}
     line["roofline"] = {"kernel": "grouped SwiGLU FFN (ffn_kernel gate-up + down, weight streaming)",
                         "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                        "frac": achieved / hbm_peak, "peak_kind": peak_kind, "traffic": None,
+                        "frac": achieved / hbm_peak, "peak_kind": peak_kind, "traffic": ffn_traffic(),
                         "algorithmic_bytes_per_call": ffn_bytes / ffn_calls,
                         "avg_call_ms": ffn_ms / ffn_calls, "calls": ffn_calls}
     line["gpu_launches"] = int(kernels)
