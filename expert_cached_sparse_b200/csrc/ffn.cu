@@ -5,13 +5,15 @@
 //
 // Decode is bound by HBM: each touched expert's weights are read once per
 // pass and every token row is reused across all of them.  Design:
-//  - work unit = one warp x one 16-row tile of W13 (or W2) x up to 16 rows
-//    (tokens) of one expert, over the whole K; a persistent grid walks the
-//    units, consecutive warps take consecutive row tiles of the same expert;
-//  - each warp streams its tiles through its own shared-memory rings with
-//    1-D bulk copies (TMA engine) issued by one lane and completed on
-//    mbarriers: 16 weight tiles (8 KB) and 8 activation tiles in flight per
-//    warp, running ahead across unit boundaries, no registers held;
+//  - work unit = (token group of up to 16 rows of one expert, 128-row block
+//    of W13 or W2), over the whole K; a persistent grid of three CTAs per SM
+//    walks the units (round-robin, or stream-K ranges when there are fewer
+//    units than CTAs, see the kernel);
+//  - per CTA, one lane streams the units through a shared-memory ring with
+//    1-D bulk copies (TMA engine) completed on mbarriers: a stage is four
+//    64-column chunks of the block (one contiguous copy of eight 512-byte
+//    tiles per chunk run), their scales and the group's activation rows;
+//    eight compute warps each own one 16-row tile of the block;
 //  - weights are the mma.sync m16n8k16 row operand: a lane's 16 bytes of a
 //    packed tile are exactly its fragment bytes for four k16 steps; E2M1
 //    pairs become f16 pairs with one cvt.rn.f16x2.e2m1x2 (exact);
@@ -368,23 +370,23 @@ __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 // finishes a unit's last piece adds all pieces in CTA order (deterministic)
 // and writes the result.
 // Inside a CTA, warp 8 (one lane) fills a ring stage with bulk copies: the
-// block's FP4 (or bf16) tiles of both chunks (contiguous in the slot), their
-// scales, and the token group's 8 or 16 activation rows of each chunk.
-// Warps 0..7 each multiply the 16-row tile they own in both chunks and then
-// release the stage on an mbarrier.
+// block's FP4 (or bf16) tiles of KC consecutive chunks (contiguous in the
+// slot), their scales, and the token group's 8 or 16 activation rows of each
+// chunk.  Warps 0..7 each multiply the 16-row tile they own in every chunk of
+// the stage and then release it on an mbarrier.
 constexpr int kDecThreads = 32 * (kCW + 1);   // + one copy-issue warp
-constexpr int kKC = 2;                        // 64-column chunks per stage
 
 template <int WFMT>
 struct DecCfg {
     static constexpr bool FP4 = WFMT != MOE_W_BF16;
     static constexpr int TILE = FP4 ? 512 : 2048;
+    static constexpr int KC = FP4 ? 4 : 1;                       // 64-column chunks per stage
     static constexpr int STILE = (WFMT == MOE_W_MXFP4) ? 32 : (WFMT == MOE_W_NVFP4 ? 64 : 0);
-    static constexpr int D = FP4 ? 4 : 2;                        // ring stages
-    static constexpr int A_BYTES = kKC * kCW * TILE;
-    static constexpr int S_BYTES = kKC * kCW * STILE;
+    static constexpr int D = FP4 ? 2 : 4;                        // ring stages
+    static constexpr int A_BYTES = KC * kCW * TILE;
+    static constexpr int S_BYTES = KC * kCW * STILE;
     static constexpr int X_CHUNK = 2 * 1024;                     // up to 16 rows x 128 bytes
-    static constexpr int STAGE = A_BYTES + S_BYTES + kKC * X_CHUNK;
+    static constexpr int STAGE = A_BYTES + S_BYTES + KC * X_CHUNK;
 };
 
 template <int WFMT>
@@ -541,17 +543,18 @@ __device__ __forceinline__ bool run_unit(float (&acc)[2][4], const DecUnit& U, b
 {
     using CFG = DecCfg<WFMT>;
     const int g = lane >> 2, t = lane & 3, sw = (U.row0 + g) & 7;
-    for (int kt = U.k0; kt < U.k1; kt += kKC) {
+    for (int kt = U.k0; kt < U.k1; kt += CFG::KC) {
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&full[R.st]), R.ph, abort))) return false;
         const unsigned char* sg = ring + (size_t)R.st * CFG::STAGE;
         if (act) {
             // one tile's operands live at a time; the stage is released after both
             TileRegs<WFMT, NQ> T;
-            load_tile<WFMT, NQ>(T, sg, 0, U.ng, w, lane, g, t, sw);
-            mma_tile<WFMT, NQ>(acc, T);
-            if (kt + 1 < U.k1) {
-                load_tile<WFMT, NQ>(T, sg, 1, U.ng, w, lane, g, t, sw);
-                mma_tile<WFMT, NQ>(acc, T);
+#pragma unroll
+            for (int cc = 0; cc < CFG::KC; cc++) {
+                if (kt + cc < U.k1) {
+                    load_tile<WFMT, NQ>(T, sg, cc, U.ng, w, lane, g, t, sw);
+                    mma_tile<WFMT, NQ>(acc, T);
+                }
             }
         }
         __syncwarp();
@@ -599,7 +602,7 @@ __device__ __forceinline__ void write_tile(const FfnArgs& a, const DecUnit& U, i
 }
 
 // Segments of one CTA: whole units u = blockIdx.x + i * gridDim.x, or the
-// stream-K pieces of its stage range [pos, end): unit u, pairs [p0, p1).
+// stream-K pieces of its stage range [pos, end): unit u, stages [p0, p1).
 struct Seg {
     long pos;     // next unit (whole) or next stage (stream-K)
     long start;   // first stage of the current segment (stream-K)
@@ -639,7 +642,7 @@ __global__ void __launch_bounds__(kDecThreads, 3) ffn_kernel(FfnArgs a)
     unsigned char* ring = smem + 1024;
     int* s_groups = reinterpret_cast<int*>(ring + (size_t)D * STAGE);
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, t = lane & 3;
-    const int RT = a.R / 16, RB = (RT + 7) / 8, KT = a.K / 64, KP = (KT + kKC - 1) / kKC, RP = a.rows + kRowPad;
+    const int RT = a.R / 16, RB = (RT + 7) / 8, KT = a.K / 64, KP = (KT + CFG::KC - 1) / CFG::KC, RP = a.rows + kRowPad;
     for (int i = tid; i <= a.E; i += kDecThreads) s_groups[i] = a.groups[i];
     if (tid == 0) {
         for (int i = 0; i < D; i++) {
@@ -671,8 +674,8 @@ __global__ void __launch_bounds__(kDecThreads, 3) ffn_kernel(FfnArgs a)
             long issued = 0;
             bool ok = true;
             auto issue = [&](const DecUnit& U) {
-                for (int kt = U.k0; kt < U.k1 && ok; kt += kKC) {
-                    const int nc = min(kKC, U.k1 - kt);
+                for (int kt = U.k0; kt < U.k1 && ok; kt += CFG::KC) {
+                    const int nc = min(CFG::KC, U.k1 - kt);
                     if (!(ok = mbar_wait_bounded(smem_u32(&empty[st]), ph ^ 1, s_abort))) break;
                     const uint32_t bar = smem_u32(&full[st]);
                     unsigned char* sg = ring + (size_t)st * STAGE;
@@ -692,7 +695,7 @@ __global__ void __launch_bounds__(kDecThreads, 3) ffn_kernel(FfnArgs a)
             };
             Seg sg{whole ? (long)blockIdx.x : b0};
             while (ok && sg.next(whole, NU, KP, b1))
-                issue(dec_unit(a, s_groups, sg.u, RT, RB, kKC * sg.p0, min(KT, kKC * sg.p1)));
+                issue(dec_unit(a, s_groups, sg.u, RT, RB, CFG::KC * sg.p0, min(KT, CFG::KC * sg.p1)));
             if (!ok) atomicCAS(&g_ffn_error, 0, (int)MOE_ERR_TIMEOUT);
             // let the last copies land before the CTA exits (stage i was last
             // filled in this pass if i < st, else in the previous one)
@@ -720,7 +723,7 @@ __global__ void __launch_bounds__(kDecThreads, 3) ffn_kernel(FfnArgs a)
     while (sg.next(whole, NU, KP, b1)) {
         const int u = sg.u, p0 = sg.p0, p1 = sg.p1;
         const long idx = sg.start;
-        const DecUnit U = dec_unit(a, s_groups, u, RT, RB, kKC * p0, min(KT, kKC * p1));
+        const DecUnit U = dec_unit(a, s_groups, u, RT, RB, CFG::KC * p0, min(KT, CFG::KC * p1));
         const bool act = w < U.ng;          // this warp has a row tile in the block
         const int rt = 8 * U.G + w;
         float acc[2][4];
@@ -828,7 +831,7 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     if (grid > kMaxDecCtas) grid = kMaxDecCtas;
     // no more CTAs than stages (upper bound of the stage count: every unit possible)
     auto grid_for = [&](int R, int K) {
-        const long RB = (R / 16 + 7) / 8, KP = (K / 64 + kKC - 1) / kKC;
+        const long RB = (R / 16 + 7) / 8, KP = (K / 64 + DecCfg<WFMT>::KC - 1) / DecCfg<WFMT>::KC;
         const long groups = (rows + kRowsPerUnit - 1) / kRowsPerUnit + (rows < E ? rows : E);
         const long wmax = groups * RB * KP;
         return (int)(wmax < grid ? (wmax < 1 ? 1 : wmax) : grid);
