@@ -49,6 +49,30 @@ constexpr int kPrepThreads = 256;
 constexpr int kRowPad = 16;        // operand copies carry 16 spare rows (whole 8-row reads past the end)
 constexpr long long kWaitCycles = 4000000000ll;   // ~2 s before a wait gives up
 
+// Programmatic dependent launch: the kernels of one FFN call are launched so
+// that each may start while the previous one drains; every kernel waits for
+// its predecessor's results (griddepcontrol.wait, a no-op for a normal
+// launch) before reading them, and lets its successor launch once all its
+// CTAs are running.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ------------------------------------------------------------------ workspace
 struct FfnWs {
     uint16_t* xb;     // [H/64][rows+16][64] operand copy of the input rows
@@ -126,6 +150,8 @@ __global__ void __launch_bounds__(kPrepThreads) ffn_prep_kernel(const void* __re
                                                                 const int32_t* __restrict__ gather, int gk,
                                                                 int32_t* __restrict__ zero, int nzero)
 {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     if (groups && blockIdx.x == gridDim.x - 1) {
         for (int i = threadIdx.x; i < nzero; i += kPrepThreads) zero[i] = 0;
@@ -643,6 +669,7 @@ __global__ void __launch_bounds__(kDecThreads, 3) ffn_kernel(FfnArgs a)
     int* s_groups = reinterpret_cast<int*>(ring + (size_t)D * STAGE);
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, t = lane & 3;
     const int RT = a.R / 16, RB = (RT + 7) / 8, KT = a.K / 64, KP = (KT + CFG::KC - 1) / CFG::KC, RP = a.rows + kRowPad;
+    pdl_wait();
     for (int i = tid; i <= a.E; i += kDecThreads) s_groups[i] = a.groups[i];
     if (tid == 0) {
         for (int i = 0; i < D; i++) {
@@ -654,6 +681,7 @@ __global__ void __launch_bounds__(kDecThreads, 3) ffn_kernel(FfnArgs a)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     __syncthreads();
+    pdl_trigger();
     // With at least one unit per CTA, whole units go round-robin (an SM's
     // CTAs share its issue slots, so uneven unit counts per CTA even out per
     // SM); with fewer units than CTAs, the units' stages are cut into equal
@@ -786,18 +814,15 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     constexpr bool FP4 = WFMT != MOE_W_BF16;
     const int E = s->experts, H = s->hidden, F = s->ffn;
     int prep_blocks = rows < sms * 8 ? rows : sms * 8;   // a CTA per row
+    const void* src = gather ? gather->x : static_cast<const void*>(x_perm);
+    const int32_t* gidx = gather ? gather->assign_of : nullptr;
+    const int gk = gather ? gather->k : 1;
     if (gather && gather->x_dtype == MOE_DT_F32)
-        ffn_prep_kernel<true, FP4><<<prep_blocks + 1, kPrepThreads, 0, st>>>(
-            gather->x, rows, H, w.xb, w.xe, offsets, slot_of, E, pool_slots, w.groups, gather->assign_of, gather->k,
-            w.cnt, w.ncnt);
-    else if (gather)
-        ffn_prep_kernel<false, FP4><<<prep_blocks + 1, kPrepThreads, 0, st>>>(
-            gather->x, rows, H, w.xb, w.xe, offsets, slot_of, E, pool_slots, w.groups, gather->assign_of, gather->k,
-            w.cnt, w.ncnt);
+        MOE_CUDA_TRY(launch_pdl(ffn_prep_kernel<true, FP4>, prep_blocks + 1, kPrepThreads, 0, st, src, rows, H, w.xb,
+                                w.xe, offsets, slot_of, E, pool_slots, w.groups, gidx, gk, w.cnt, w.ncnt));
     else
-        ffn_prep_kernel<false, FP4><<<prep_blocks + 1, kPrepThreads, 0, st>>>(
-            x_perm, rows, H, w.xb, w.xe, offsets, slot_of, E, pool_slots, w.groups, nullptr, 1, w.cnt, w.ncnt);
-    MOE_LAUNCH_CHECK();
+        MOE_CUDA_TRY(launch_pdl(ffn_prep_kernel<false, FP4>, prep_blocks + 1, kPrepThreads, 0, st, src, rows, H, w.xb,
+                                w.xe, offsets, slot_of, E, pool_slots, w.groups, gidx, gk, w.cnt, w.ncnt));
     FfnArgs a{};
     a.pool = static_cast<const char*>(pool);
     a.slot_bytes = slot_bytes;
@@ -843,11 +868,10 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     a.in = w.xb;
     a.in_ex = w.xe;
     a.out_h = w.h32;
-    ffn_kernel<WFMT, 1><<<grid_for(2 * F, H), kDecThreads, smem, st>>>(a);
-    MOE_LAUNCH_CHECK();
-    ffn_prep_kernel<true, FP4><<<prep_blocks, kPrepThreads, 0, st>>>(w.h32, rows, F, w.hb, w.he, nullptr, nullptr,
-                                                                     E, 0, nullptr, nullptr, 1, nullptr, 0);
-    MOE_LAUNCH_CHECK();
+    MOE_CUDA_TRY(launch_pdl(ffn_kernel<WFMT, 1>, grid_for(2 * F, H), kDecThreads, smem, st, a));
+    MOE_CUDA_TRY(launch_pdl(ffn_prep_kernel<true, FP4>, prep_blocks, kPrepThreads, 0, st,
+                            static_cast<const void*>(w.h32), rows, F, w.hb, w.he, nullptr, nullptr, E, 0, nullptr,
+                            nullptr, 1, nullptr, 0));
     FfnArgs b = a;
     b.w_off = bl.w2;
     b.s_off = bl.s2;
@@ -857,8 +881,7 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     b.in_ex = w.he;
     b.out_h = nullptr;
     b.out_y = y_perm;
-    ffn_kernel<WFMT, 2><<<grid_for(H, F), kDecThreads, smem, st>>>(b);
-    MOE_LAUNCH_CHECK();
+    MOE_CUDA_TRY(launch_pdl(ffn_kernel<WFMT, 2>, grid_for(H, F), kDecThreads, smem, st, b));
     return MOE_OK;
 }
 

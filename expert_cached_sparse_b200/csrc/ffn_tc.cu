@@ -6,24 +6,25 @@
 // whole layers; the pages' own design streams the next layer's experts over
 // PCIe, here every expert is already resident).  Design for sm_100a:
 //  - swap-AB: the expert's weight rows are the MMA's M side (128 rows per
-//    tile), tokens the N side (up to 256 per tile), K in chunks of 64;
+//    tile), tokens the N side (up to 128 per tile), K in chunks of 64;
 //  - weights stay packed FP4 in HBM; a bulk copy brings each 128 x 64 FP4
-//    chunk (4 KB + scales) to shared memory, four warps expand it exactly to
-//    bf16 (E2M1 x block scale is exact in bf16) and write it with
-//    tcgen05.st straight into tensor memory, where the MMA reads its A
-//    operand; no bf16 weight tile ever touches shared memory;
+//    chunk (4 KB + scales) to shared memory, eight warps expand it exactly to
+//    f16 (E2M1 x block scale is exact in f16 for the accepted scale codes)
+//    and write it with tcgen05.st straight into tensor memory, where the MMA
+//    reads its A operand; no f16 weight tile ever touches shared memory;
 //  - tokens (x_perm, or h for the down projection) arrive by TMA in 16- to
 //    128-row boxes with the 128-byte swizzle the MMA's shared-memory
 //    descriptor expects, as many 64-column chunks per 32 KB stage as fit, so
 //    small token blocks keep more chunks in flight; rows past the expert's
 //    block are loaded but never stored;
-//  - the accumulator lives in tensor memory (128 lanes x N fp32 columns);
-//    the same four warps read it back with tcgen05.ld for the epilogue:
-//    SwiGLU (gate and up rows are 8 lanes apart, one shuffle) into h, or the
-//    NVFP4 tensor scale into y;
-//  - warp 0 issues copies, warp 1 issues MMAs (one thread each); mbarriers
-//    chain the roles; every wait is bounded and a timeout sets an error word
-//    and drains the CTA instead of hanging.
+//  - two accumulators live in tensor memory (128 lanes x up to 128 fp32
+//    columns each); four epilogue warps read one back with tcgen05.ld while
+//    the MMA fills the other: SwiGLU (gate and up rows are 8 lanes apart, one
+//    shuffle) into h, or the NVFP4 tensor scale into y;
+//  - warp 0 issues the weight copies, the last warp the token copies, warp 1
+//    the MMAs (one thread each); mbarriers chain the roles; every wait is
+//    bounded and a timeout sets an error word and drains the CTA instead of
+//    hanging.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -44,7 +45,8 @@ constexpr int NABUF = 8;           // tensor-memory A buffers
 constexpr int NXG = 1;             // expanding groups: group g expands chunks g, g+NXG, ...
 constexpr int NXW = 8 * NXG;       // expanding warps: two per tensor-memory lane quarter and group
 constexpr int NEPI = 4;            // epilogue warps, one per tensor-memory lane quarter
-constexpr int THREADS = 32 * (2 + NXW + NEPI);   // warp 0 copies, warp 1 MMA, then expand, then epilogue
+constexpr int BWARP = 2 + NXW + NEPI;           // token (B) copy issue
+constexpr int THREADS = 32 * (BWARP + 1);         // warp 0 weight copies, warp 1 MMA, expand, epilogue, B copies
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t D_COL = 0;      // two accumulators: columns [0, 128) and [128, 256)
 constexpr uint32_t A_COL = 256;    // A buffers: 32 columns each (8 buffers: 256..511)
@@ -360,10 +362,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     volatile int* abort_v = abort_flag;
 
     if (warp == 0) {
-        // ================= copy issue (one thread) =================
+        // ================= weight copy issue (one thread) =================
         if (lane == 0) {
-            int sa = 0, sb = 0;
-            uint32_t pa = 0, pb = 0;
+            int sa = 0;
+            uint32_t pa = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                 Tile t = tile_of(u, prefix, E, RB, a.offsets);
@@ -378,7 +380,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                     bulk_g2s(smem_u32(sA + sa * A_STAGE_BYTES), blob + a.w_off + ti * 512, A_STAGE_BYTES, fa);
                     bulk_g2s(smem_u32(sS + sa * S_STAGE_BYTES), blob + a.s_off + ti * STILE, 8 * STILE, fa);
                     if (++sa == SA) { sa = 0; pa ^= 1; }
-                    if (c % t.ncps) continue;   // this chunk's tokens came with an earlier B stage
+                }
+            }
+            // drain: every stage's most recent fill must land before the CTA exits
+            // (stage i was last filled in the current round if i < next stage, else in the
+            // previous one; a stage never filled reads as complete for the previous parity)
+            for (int i = 0; i < SA; i++) mbar_wait(smem_u32(&full_a[i]), (i < sa) ? pa : (pa ^ 1), abort_v);
+        }
+    } else if (warp == BWARP) {
+        // ================= token copy issue (one thread) =================
+        if (lane == 0) {
+            int sb = 0;
+            uint32_t pb = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+                Tile t = tile_of(u, prefix, E, RB, a.offsets);
+                for (int c = 0; c < KT && ok; c += t.ncps) {
                     ok = mbar_wait(smem_u32(&empty_b[sb]), pb ^ 1, abort_v);
                     if (!ok) break;
                     const uint32_t fb = smem_u32(&full_b[sb]);
@@ -399,10 +416,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (++sb == SB) { sb = 0; pb ^= 1; }
                 }
             }
-            // drain: every stage's most recent fill must land before the CTA exits
-            // (stage i was last filled in the current round if i < next stage, else in the
-            // previous one; a stage never filled reads as complete for the previous parity)
-            for (int i = 0; i < SA; i++) mbar_wait(smem_u32(&full_a[i]), (i < sa) ? pa : (pa ^ 1), abort_v);
             for (int i = 0; i < SB; i++) mbar_wait(smem_u32(&full_b[i]), (i < sb) ? pb : (pb ^ 1), abort_v);
         }
     } else if (warp == 1) {
@@ -514,7 +527,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 pend = -1;
             }
         }
-    } else {
+    } else if (warp < BWARP) {
         // ================= epilogue: accumulator -> h or y =================
         // One warp per tensor-memory lane quarter; tile `it` used accumulator
         // it & 1, so this runs while the next tile is multiplied.
