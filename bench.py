@@ -196,7 +196,7 @@ class DecodeStream:
 # stream, summed over the call's kernels (operand preps and both projections)
 # and averaged over the calls of an ncu capture of that workload.  Valid only
 # for the FFN source it was measured on: another source reports null.
-FFN_TRAFFIC = {"source_sha1": "1f525af80ef26cd84af8ddbd89d3403c5c5f9406", "bytes_per_call": 206345808}
+FFN_TRAFFIC = {"source_sha1": "118de52eab62464152f7736fe4617ecc89b163ff", "bytes_per_call": 205504176}
 
 
 def ffn_traffic():
