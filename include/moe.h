@@ -299,13 +299,18 @@ int moe_permute_noalloc(const int32_t* d_topk_idx, int32_t n, int32_t experts, i
  * with rows [offsets[e], offsets[e+1]) (clipped to [0, rows)) and
  * 0 <= d_slot_of_expert[e] < pool_slots, the weights are read from that
  * slot and
- *   h = silu(x W1^T) * (x W3^T)   (fp32 accumulation, h rounded to bf16),
+ *   h = silu(x W1^T) * (x W3^T)   (fp32 accumulation),
  *   y = h W2^T                    (fp32 accumulation, y rounded to bf16)
  * is written to d_y_perm rows.  Rows of experts with any other slot value
  * (-1 in particular) are left untouched, so hits and misses can run as two
- * passes.  d_ws: moe_ffn_workspace_bytes() bytes (holds h).  FP4 weights are
- * expanded exactly to bf16 (E2M1 times its block scale is exact there); the
- * NVFP4 tensor scales are applied in fp32.
+ * passes.  d_ws: moe_ffn_workspace_bytes() bytes (operand copies of x and
+ * h, h itself, and the partial sums of work split across CTAs).  The MMAs
+ * take f16 operands: FP4 weights are expanded exactly (E2M1 times its block
+ * scale is exact in f16 for the accepted scale codes), x and h rows are
+ * scaled by a power of two so their largest magnitude lands in [2^14, 2^15)
+ * (exact for bf16 x, 11 significant bits for h); the row scale and the
+ * NVFP4 tensor scales are undone in fp32.  Results are deterministic: the
+ * same inputs give the same bits on every call.
  */
 int moe_grouped_ffn(const moe_shape* shape, const void* d_slot_pool, int32_t pool_slots,
                     const int32_t* d_slot_of_expert, const int32_t* d_expert_offsets,
