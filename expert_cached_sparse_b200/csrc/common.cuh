@@ -21,6 +21,7 @@ namespace moe {
 constexpr int kMaxExperts = 4096;
 constexpr int kMaxCapacity = 8192;
 constexpr int kMaxTopK = 32;
+constexpr int kMaxDevices = 64;   // device ordinals with per-device launch caches
 
 static inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 

@@ -837,8 +837,15 @@ int launch_decode(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     const size_t smem = dec_smem_bytes<WFMT>(E);
     // persistent grid: as many CTAs as fit at once (recomputed when the
     // shared-memory size, which grows with E, changes)
-    static size_t attr_smem = 0, occ_smem = 0;
-    static int resident = 1;
+    // function attributes and occupancy are per device (context)
+    int dev = 0;
+    MOE_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+    static size_t attr_smem_dev[kMaxDevices], occ_smem_dev[kMaxDevices];
+    static int resident_dev[kMaxDevices];
+    size_t& attr_smem = attr_smem_dev[dev];
+    size_t& occ_smem = occ_smem_dev[dev];
+    int& resident = resident_dev[dev];
     if (smem > attr_smem) {
         MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_kernel<WFMT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
         MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_kernel<WFMT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));

@@ -637,7 +637,11 @@ template <int WFMT, int PHASE>
 int launch_one(const TcArgs& a, const RowMaps& map, int rows, int sms, cudaStream_t st)
 {
     size_t smem = tc_smem_bytes(a.E);
-    static size_t attr_smem = 0;
+    int dev = 0;   // the attribute is per device (context)
+    MOE_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+    static size_t attr_smem_dev[kMaxDevices];
+    size_t& attr_smem = attr_smem_dev[dev];
     if (smem > attr_smem) {
         MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_tc_kernel<WFMT, PHASE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)smem));
