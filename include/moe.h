@@ -179,6 +179,10 @@ int moe_pack_expert(const moe_shape* shape, const void* h_w13, const uint8_t* h_
  *   point to the same blob).
  * All slots start free (cold cache).  Initialises d_meta on `stream` and
  * synchronises it.
+ * Testing hook: with MOE_FAULT_INJECT=fill_fail:<n> in the environment when
+ * the cache is created, the n-th fill (counting from 1, once) reports a failed
+ * copy: the lookup that needed it returns MOE_ERR_FILL before any copy is
+ * issued and its installs are rolled back.
  */
 int moe_cache_create(const moe_shape* shape, void* d_meta, size_t meta_bytes, void* d_slot_pool,
                      int32_t capacity, int32_t trace_capacity, const void* const* h_blobs,
@@ -311,6 +315,10 @@ int moe_permute_noalloc(const int32_t* d_topk_idx, int32_t n, int32_t experts, i
  * (exact for bf16 x, 11 significant bits for h); the row scale and the
  * NVFP4 tensor scales are undone in fp32.  Results are deterministic: the
  * same inputs give the same bits on every call.
+ * Kernel choice: FP4 formats with at least 4 rows per expert on average run
+ * the tcgen05 grouped GEMM, everything else the weight-streaming kernels;
+ * the environment variable MOE_FFN_PATH=mma or =tc forces one of them (read
+ * at every call; intended for testing).
  */
 int moe_grouped_ffn(const moe_shape* shape, const void* d_slot_pool, int32_t pool_slots,
                     const int32_t* d_slot_of_expert, const int32_t* d_expert_offsets,

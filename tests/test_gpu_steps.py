@@ -172,9 +172,10 @@ def test_grouped_ffn_full_size(orc, base):
 @pytest.mark.parametrize("base", [W.DS_DECODE, W.TRACE40, W.QWEN_BF16], ids=["mxfp4", "nvfp4", "bf16"])
 @pytest.mark.parametrize("passes", [1, 2])
 def test_grouped_ffn_split_k(orc, base, passes, monkeypatch):
-    """Full expert shapes with few token groups: the streaming kernels split K
-    across CTAs and reduce the partial sums; rows of a skipped expert stay
-    untouched, and a second pass over the other experts keeps the first's."""
+    """Full expert shapes with fewer work units than CTAs: the streaming
+    kernels cut the units' K stages into equal ranges over the CTAs and add the
+    pieces up; rows of a skipped expert stay untouched, and a second pass over
+    the other experts keeps the first's."""
     monkeypatch.setenv("MOE_FFN_PATH", "mma")
     cfg = W.scaled(base, experts=6, top_k=2, layers=1)
     counts = [1, 3, 2, 9, 0, 1]
