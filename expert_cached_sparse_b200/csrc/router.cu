@@ -126,7 +126,9 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restri
 // slices of 256 elements = 32 chunks of 8, so lane l of every warp owns chunk
 // l of each slice: the per-(token, expert) order is the same fixed order as
 // above (lane chunks ascending, then the xor butterfly).  Warp w owns tokens
-// 4w..4w+3 and all 16 experts (64 accumulators per lane).
+// 4w..4w+3 and all 16 experts (64 accumulators per lane).  A staged row keeps
+// the first four elements of every chunk, then the last four, so a warp's
+// 16-byte reads of one half are 512 contiguous bytes (no bank conflicts).
 constexpr int RT_TOK = 32, RT_EXP = 16, RT_K = 256;
 
 template <bool XF32>
@@ -168,9 +170,8 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(const void* __
 #pragma unroll
                 for (int j = 0; j < 8; j++) v[j] = 0.0f;
             }
-            float4* d = reinterpret_cast<float4*>(&xs[r][8 * c]);
-            d[0] = make_float4(v[0], v[1], v[2], v[3]);
-            d[1] = make_float4(v[4], v[5], v[6], v[7]);
+            *reinterpret_cast<float4*>(&xs[r][4 * c]) = make_float4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<float4*>(&xs[r][RT_K / 2 + 4 * c]) = make_float4(v[4], v[5], v[6], v[7]);
         }
         for (int i = tid; i < RT_EXP * RT_K / 8; i += 256) {
             const int r = i / (RT_K / 8), c = i % (RT_K / 8);
@@ -188,24 +189,23 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(const void* __
 #pragma unroll
                 for (int j = 0; j < 8; j++) v[j] = 0.0f;
             }
-            float4* d = reinterpret_cast<float4*>(&ws[r][8 * c]);
-            d[0] = make_float4(v[0], v[1], v[2], v[3]);
-            d[1] = make_float4(v[4], v[5], v[6], v[7]);
+            *reinterpret_cast<float4*>(&ws[r][4 * c]) = make_float4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<float4*>(&ws[r][RT_K / 2 + 4 * c]) = make_float4(v[4], v[5], v[6], v[7]);
         }
         __syncthreads();
         if (k0 + 8 * lane < H) {   // lane's chunk exists in this slice
             float xv[4][8];
 #pragma unroll
             for (int a = 0; a < 4; a++) {
-                const float4* p = reinterpret_cast<const float4*>(&xs[4 * w + a][8 * lane]);
-                float4 q0 = p[0], q1 = p[1];
+                const float4 q0 = *reinterpret_cast<const float4*>(&xs[4 * w + a][4 * lane]);
+                const float4 q1 = *reinterpret_cast<const float4*>(&xs[4 * w + a][RT_K / 2 + 4 * lane]);
                 xv[a][0] = q0.x; xv[a][1] = q0.y; xv[a][2] = q0.z; xv[a][3] = q0.w;
                 xv[a][4] = q1.x; xv[a][5] = q1.y; xv[a][6] = q1.z; xv[a][7] = q1.w;
             }
 #pragma unroll
             for (int b = 0; b < RT_EXP; b++) {
-                const float4* p = reinterpret_cast<const float4*>(&ws[b][8 * lane]);
-                float4 q0 = p[0], q1 = p[1];
+                const float4 q0 = *reinterpret_cast<const float4*>(&ws[b][4 * lane]);
+                const float4 q1 = *reinterpret_cast<const float4*>(&ws[b][RT_K / 2 + 4 * lane]);
                 const float wv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
                 for (int a = 0; a < 4; a++)
