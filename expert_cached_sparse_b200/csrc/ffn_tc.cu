@@ -6,7 +6,7 @@
 // whole layers; the pages' own design streams the next layer's experts over
 // PCIe, here every expert is already resident).  Design for sm_100a:
 //  - swap-AB: the expert's weight rows are the MMA's M side (128 rows per
-//    tile), tokens the N side (up to 128 per tile), K in chunks of 64;
+//    tile), tokens the N side (up to 192 per tile), K in chunks of 64;
 //  - weights stay packed FP4 in HBM; a bulk copy brings each 128 x 64 FP4
 //    chunk (4 KB + scales) to shared memory, eight warps expand it exactly to
 //    f16 (E2M1 x block scale is exact in f16 for the accepted scale codes)
@@ -17,7 +17,7 @@
 //    descriptor expects, as many 64-column chunks per 32 KB stage as fit, so
 //    small token blocks keep more chunks in flight; rows past the expert's
 //    block are loaded but never stored;
-//  - two accumulators live in tensor memory (128 lanes x up to 128 fp32
+//  - two accumulators live in tensor memory (128 lanes x up to 192 fp32
 //    columns each); four epilogue warps read one back with tcgen05.ld while
 //    the MMA fills the other: SwiGLU (gate and up rows are 8 lanes apart, one
 //    shuffle) into h, or the NVFP4 tensor scale into y;
@@ -37,19 +37,19 @@ __device__ int g_tc_error;   // first device-side error of the tensor-core FFN (
 namespace {
 
 constexpr int BM = 128;
-constexpr int BN_MAX = 128;       // token rows per tile (two accumulators fit tensor memory)
+constexpr int BN_MAX = 192;       // token rows per tile (two accumulators fit tensor memory)
 constexpr int BK = 64;
 constexpr int SA = 16;             // FP4 A stages (one 64-column chunk each)
 constexpr int SB = 4;              // token (B) stages: as many 64-column chunks as fit 32 KB
-constexpr int NABUF = 8;           // tensor-memory A buffers
+constexpr int NABUF = 4;           // tensor-memory A buffers
 constexpr int NXG = 1;             // expanding groups: group g expands chunks g, g+NXG, ...
 constexpr int NXW = 8 * NXG;       // expanding warps: two per tensor-memory lane quarter and group
 constexpr int NEPI = 4;            // epilogue warps, one per tensor-memory lane quarter
 constexpr int BWARP = 2 + NXW + NEPI;           // token (B) copy issue
 constexpr int THREADS = 32 * (BWARP + 1);         // warp 0 weight copies, warp 1 MMA, expand, epilogue, B copies
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t D_COL = 0;      // two accumulators: columns [0, 128) and [128, 256)
-constexpr uint32_t A_COL = 256;    // A buffers: 32 columns each (8 buffers: 256..511)
+constexpr uint32_t D_COL = 0;      // two accumulators: columns [0, 192) and [192, 384)
+constexpr uint32_t A_COL = 384;    // A buffers: 32 columns each (4 buffers: 384..511)
 constexpr uint32_t B_STAGE_BYTES = 32 * 1024;
 constexpr uint32_t A_STAGE_BYTES = 8 * 512;
 constexpr uint32_t S_STAGE_BYTES = 8 * 64;
