@@ -215,14 +215,21 @@ def test_combine_parity(orc, n, k, H, out):
                        o2.view(torch.int16) if o2.dtype == torch.bfloat16 else o2)
 
 
+TC_CASES = {
+    # ragged groups, an expert of 300 rows (two token blocks) and one of 256
+    "ragged": ([0, 1, 17, 300, 33, 70, 3, 256], [3, 9, 0, 4, 5, 2, 7, 1]),
+    # token-block boundaries: one full block, one row over, two full blocks, one over
+    "block_edges": ([192, 193, 384, 385, 16, 15, 1, 0], [1, 0, 3, 2, 5, 4, 7, 6]),
+}
+
+
+@pytest.mark.parametrize("case", sorted(TC_CASES))
 @pytest.mark.parametrize("base", [W.DS_DECODE, W.TRACE40], ids=["mxfp4", "nvfp4"])
-def test_grouped_ffn_tensor_core_path(orc, base, monkeypatch):
-    """The tcgen05 grouped GEMM (prefill path), forced on small shapes: ragged
-    groups including an expert of 300 rows (two token blocks) and one of 256."""
+def test_grouped_ffn_tensor_core_path(orc, base, case, monkeypatch):
+    """The tcgen05 grouped GEMM (prefill path), forced on small shapes."""
     monkeypatch.setenv("MOE_FFN_PATH", "tc")
     cfg = W.scaled(base, hidden=256, ffn=128, experts=8, top_k=2, layers=1)
-    counts = [0, 1, 17, 300, 33, 70, 3, 256]
-    slots = [3, 9, 0, 4, 5, 2, 7, 1]
+    counts, slots = TC_CASES[case]
     worst = _ffn_case(orc, cfg, counts, slots, pool_slots=10, seed=11)
     assert worst < ALARM_REL_L2, worst
     assert A.L.lib.moe_get_device_error(1) == 0
