@@ -196,7 +196,7 @@ class DecodeStream:
 # stream, summed over the call's kernels (operand preps and both projections)
 # and averaged over the calls of an ncu capture of that workload.  Valid only
 # for the FFN source it was measured on: another source reports null.
-FFN_TRAFFIC = {"source_sha1": "0b2d9ab78d50439a0350895bc825c9c2eeedd356", "bytes_per_call": 205321648}
+FFN_TRAFFIC = {"source_sha1": "706ba1c2d9bb3d1f1dd1c3b5a599297608202639", "bytes_per_call": 205387936}
 
 
 def ffn_traffic():

@@ -149,7 +149,6 @@ struct RowSource {
     const int32_t* assign_of;
     int k;
 };
-bool ffn_uses_tc(const moe_shape* s, int rows);
 int ffn_device_error(int clear);   // decode FFN's device error word (0: none)
 int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
                const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,

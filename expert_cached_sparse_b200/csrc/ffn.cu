@@ -908,8 +908,6 @@ bool use_tc_path(const moe_shape* s, int rows)
 
 size_t ffn_ws_bytes(const moe_shape* s, int rows) { return ffn_ws_layout(s, rows, nullptr, nullptr) + 256; }
 
-bool ffn_uses_tc(const moe_shape* s, int rows) { return use_tc_path(s, rows); }
-
 int ffn_device_error(int clear)
 {
     int v = 0;
@@ -936,9 +934,14 @@ int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool
         // tensor-core path: f16 operand rows (x, then h), each scaled by a power of two
         prof_count(MOE_PROF_FFN, 4);
         const int pb = rows < sms0 * 8 ? rows : sms0 * 8;   // a CTA per row
-        ffn_prep_kernel<false, true, true><<<pb, kPrepThreads, 0, st>>>(x_perm, rows, s->hidden, w.xb, w.xe, nullptr,
-                                                                         nullptr, s->experts, 0, nullptr, nullptr, 1,
-                                                                         nullptr, 0);
+        if (gather && gather->x_dtype == MOE_DT_F32)   // token rows gathered straight from x
+            ffn_prep_kernel<true, true, true><<<pb, kPrepThreads, 0, st>>>(gather->x, rows, s->hidden, w.xb, w.xe,
+                                                                            nullptr, nullptr, s->experts, 0, nullptr,
+                                                                            gather->assign_of, gather->k, nullptr, 0);
+        else
+            ffn_prep_kernel<false, true, true><<<pb, kPrepThreads, 0, st>>>(
+                gather ? gather->x : static_cast<const void*>(x_perm), rows, s->hidden, w.xb, w.xe, nullptr, nullptr,
+                s->experts, 0, nullptr, gather ? gather->assign_of : nullptr, gather ? gather->k : 1, nullptr, 0);
         MOE_LAUNCH_CHECK();
         TcOperands op{w.xb, w.xe, w.h32, w.hb, w.he};
         return launch_ffn_tc(s, pool, slot_bytes, pool_slots, slot_of, offsets, rows, y_perm, op, st, [&]() -> int {

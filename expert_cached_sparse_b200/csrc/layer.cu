@@ -30,7 +30,6 @@ struct LayerWs {
     int32_t* offsets;
     int32_t* row_of;
     int32_t* assign_of;
-    uint16_t* x_perm;
     uint16_t* y_perm;
     void* ffn_ws;
     void* perm_ws;
@@ -49,7 +48,6 @@ static LayerWs layer_ws(const moe_shape* s, int n, void* base)
     size_t o_off = take(4 * (E + 1));
     size_t o_row = take(4 * A);
     size_t o_asg = take(4 * A);
-    size_t o_xp = take(2 * A * H);
     size_t o_yp = take(2 * A * H);
     size_t o_ffn = take(ffn_ws_bytes(s, (int)A));
     size_t o_perm = take(permute_ws_bytes(n, s->experts, s->top_k));
@@ -62,7 +60,6 @@ static LayerWs layer_ws(const moe_shape* s, int n, void* base)
         L.offsets = reinterpret_cast<int32_t*>(b + o_off);
         L.row_of = reinterpret_cast<int32_t*>(b + o_row);
         L.assign_of = reinterpret_cast<int32_t*>(b + o_asg);
-        L.x_perm = reinterpret_cast<uint16_t*>(b + o_xp);
         L.y_perm = reinterpret_cast<uint16_t*>(b + o_yp);
         L.ffn_ws = b + o_ffn;
         L.perm_ws = b + o_perm;
@@ -100,14 +97,13 @@ extern "C" int moe_layer_forward(moe_cache* c, int32_t layer, const void* d_x, i
     int rc;
     if ((rc = launch_router(d_x, x_dtype, d_wg, d_bias, n, H, E, k, L.logits, idx, w, st))) return rc;
     if ((rc = cache_launch_lookup(c, layer, idx, A, nullptr, st))) return rc;
-    // The tensor-core path reads x_perm through TMA, so it is materialised; the
-    // decode path gathers token rows straight into its own operand copy.
-    const bool tc = ffn_uses_tc(s, A);
-    uint16_t* xp = tc ? L.x_perm : nullptr;
+    // Both FFN paths gather the token rows straight from x into their own
+    // operand copies, so the permutation writes no x_perm.
+    uint16_t* xp = nullptr;
     if ((rc = launch_permute(idx, n, E, k, d_x, x_dtype, H, L.offsets, L.row_of, L.assign_of, xp, L.perm_ws, st)))
         return rc;
     const RowSource src{d_x, x_dtype, L.assign_of, k};
-    const RowSource* gather = tc ? nullptr : &src;
+    const RowSource* gather = &src;
     const char* pool = cache_pool(c);
     const size_t sb = cache_slot_bytes(c);
     const int C = cache_capacity_int(c);
