@@ -1,7 +1,7 @@
 // Grouped SwiGLU expert FFN over permuted rows, weights streamed from the
-// expert slots: the decode path.  "A cache hit runs on the GPU"
-// ("FreeToken quantization", section "Como se desplazan los pesos MoE
-// cuantizados por la memoria").
+// expert slots: the decode path.  Experts found in the GPU cache are executed
+// on the GPU ("FreeToken quantization", section "Como se desplazan los pesos
+// MoE cuantizados por la memoria").
 //
 // Decode is bound by HBM: each touched expert's weights are read once per
 // pass and every token row is reused across all of them.  Design:

@@ -1,6 +1,6 @@
 // Router: logits in a fixed fp32 order, then top-k and renormalised softmax
-// weights.  "A router activates only a small subset of experts per token"
-// ("FreeToken linux", section "Como gestiona FreeToken la memoria MoE").
+// weights.  Each token goes to a few of the layer's experts ("FreeToken
+// linux", section "Como gestiona FreeToken la memoria MoE").
 //
 // The logit order is part of the contract (it decides integer outputs):
 // for one (token, expert) pair, 32 lanes; lane l owns the 8-element chunks
