@@ -1,11 +1,11 @@
 // Host-side packing of one expert from the canonical layout into the slot
 // blob the kernels stream.  The pages describe a runtime weight format that
 // keeps the expert banks already laid out as the runtime uses them, so
-// start-up needs no tensor discovery or repacking ("FreeToken linux", section "Prepara los pesos del
-// modelo"; "FreeToken 290b model", section "Identifica el modelo y el
-// formato de expertos").  This is that layout for this library; one fill is
-// one contiguous copy of it.  The layout is described in common.cuh
-// (BlobLayout).
+// start-up needs no tensor discovery or repacking ("FreeToken linux",
+// section "Prepara los pesos del modelo"; "FreeToken 290b model", section
+// "Identifica el modelo y el formato de expertos").  This is that layout for
+// this library; one fill is one contiguous copy of it.  The layout is
+// described in common.cuh (BlobLayout).
 #include <math.h>
 #include <string.h>
 
