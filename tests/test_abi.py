@@ -64,7 +64,7 @@ def test_workspace_sizes_grow_with_tokens():
     s = A.shape_of(W.DS_DECODE)
     a, b = A.moe_layer_workspace_bytes(s, 1), A.moe_layer_workspace_bytes(s, 16)
     assert 0 < a < b
-    assert A.moe_layer_workspace_bytes(s, 4096) > 3 * 4096 * 6 * 4096  # x_perm + y_perm + h at least
+    assert A.moe_layer_workspace_bytes(s, 4096) > 3 * 4096 * 6 * 4096  # y_perm + x operand copy + h at least
 
 
 def test_pack_rejects_bad_scale_codes():
@@ -112,3 +112,16 @@ def test_host_argument_errors_need_no_device():
     rc = L.lib.moe_cache_create(C.byref(s), None, 0, None, 8, 16, None, None, C.byref(out))
     assert rc == L.MOE_ERR_INVALID_ARG and not out.value
     assert L.lib.moe_cache_destroy(None) == L.MOE_ERR_INVALID_ARG
+
+
+def test_permute_noalloc_refusals_need_no_device():
+    """Argument errors and inputs too large for the static scratch come back
+    before any device call (dummy 16-byte-aligned addresses are never read)."""
+    fake = C.c_void_p(0x100000)
+    f = L.lib.moe_permute_noalloc
+    assert f(None, -1, 8, 2, fake, 0, 256, fake, fake, fake, fake, None) == L.MOE_ERR_INVALID_ARG
+    assert f(fake, 4, 8, 2, fake, 5, 256, fake, fake, fake, fake, None) == L.MOE_ERR_INVALID_ARG   # dtype
+    assert f(fake, 4, 8, 2, fake, 0, 256, None, fake, fake, fake, None) == L.MOE_ERR_INVALID_ARG   # offsets
+    big = 1 << 20   # tokens whose permute workspace exceeds the 1 MiB scratch
+    assert A.moe_permute_workspace_bytes(big, 256, 8) > (1 << 20)
+    assert f(fake, big, 256, 8, fake, 1, 256, fake, fake, fake, fake, None) == L.MOE_ERR_UNSUPPORTED
