@@ -233,3 +233,46 @@ def test_grouped_ffn_tensor_core_path(orc, base, case, monkeypatch):
     worst = _ffn_case(orc, cfg, counts, slots, pool_slots=10, seed=11)
     assert worst < ALARM_REL_L2, worst
     assert A.L.lib.moe_get_device_error(1) == 0
+
+
+# ------------------------------------------------------------------ self-consistency
+def _ffn_run(cfg, blobs, counts, xb, path, monkeypatch):
+    """y of one moe_grouped_ffn call with expert e in slot e (blobs: host uint8 arrays)."""
+    monkeypatch.setenv("MOE_FFN_PATH", path)
+    shape = A.shape_of(cfg)
+    sb = A.moe_slot_bytes(shape)
+    pool = torch.from_numpy(np.concatenate(blobs)).to("cuda")
+    rows = int(sum(counts))
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    slots = np.arange(cfg.experts, dtype=np.int32)
+    y = torch.empty(rows, cfg.hidden, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(A.moe_ffn_workspace_bytes(shape, rows), dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    A.moe_grouped_ffn(shape, pool, cfg.experts, dev(slots), dev(offsets), dev(xb), rows, y, ws)
+    torch.cuda.synchronize()
+    assert pool.numel() == cfg.experts * sb
+    return y.view(torch.int16).cpu().numpy()
+
+
+@pytest.mark.parametrize("path,counts", [("mma", [1, 3, 2, 9, 0, 1]), ("tc", [40, 3, 200, 9, 0, 70])],
+                         ids=["streaming", "tensor_core"])
+def test_ffn_is_deterministic_and_scale_exact(path, counts, monkeypatch):
+    """Two calls on the same inputs give the same bits (no atomics in any sum),
+    and raising every W2 block-scale code by one doubles y exactly (power-of-two
+    scaling commutes with every rounding step)."""
+    cfg = W.scaled(W.DS_DECODE, experts=6, top_k=2, layers=1)
+    shape = A.shape_of(cfg)
+    experts = [W.gen_expert(cfg, 4, 0, e) for e in range(cfg.experts)]
+    blobs = [A.moe_pack_expert(shape, ew) for ew in experts]
+    rng = np.random.default_rng(9)
+    xb = W.f32_to_bf16_bits(rng.standard_normal((int(sum(counts)), cfg.hidden)).astype(np.float32))
+    y1 = _ffn_run(cfg, blobs, counts, xb, path, monkeypatch)
+    y2 = _ffn_run(cfg, blobs, counts, xb, path, monkeypatch)
+    np.testing.assert_array_equal(y1, y2)
+    for ew in experts:
+        ew.w2_scales = (ew.w2_scales + 1).astype(np.uint8)
+    blobs2 = [A.moe_pack_expert(shape, ew) for ew in experts]
+    y3 = _ffn_run(cfg, blobs2, counts, xb, path, monkeypatch)
+    f1 = W.bf16_bits_to_f32(y1.view(np.uint16))
+    f3 = W.bf16_bits_to_f32(y3.view(np.uint16))
+    np.testing.assert_array_equal(f3, 2 * f1)
