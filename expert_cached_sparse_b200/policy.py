@@ -119,3 +119,56 @@ def replay(policy, trace) -> dict:
         reads += r
         misses += m
     return {"reads": reads, "misses": misses, "miss_rate": misses / reads if reads else 0.0}
+
+
+def belady(trace, capacity: int) -> dict:
+    """Offline optimum for context: on a miss with the cache full, evict the
+    resident key (not requested by the current call) whose next read lies
+    farthest in the future.  Same read and miss counting as `replay`."""
+    calls = [call_keys(layer, experts) for layer, experts in trace]
+    nxt = [dict() for _ in calls]            # per call: key -> index of its next read after this call
+    upcoming: dict[tuple[int, int], int] = {}
+    for t in range(len(calls) - 1, -1, -1):
+        for k in calls[t]:
+            nxt[t][k] = upcoming.get(k, len(calls))
+        for k in calls[t]:
+            upcoming[k] = t
+    resident: dict[tuple[int, int], int] = {}   # key -> its next read
+    heap: list = []                            # (-next read, key), stale entries skipped
+    reads = misses = 0
+    for t, keys in enumerate(calls):
+        if len(keys) > capacity:
+            raise ValueError("call requests more distinct experts than the cache has slots")
+        want = set(keys)
+        for k in keys:
+            reads += 1
+            if k not in resident:
+                misses += 1
+                if len(resident) == capacity:
+                    held = []
+                    while True:
+                        neg, victim = heapq.heappop(heap)
+                        if resident.get(victim) != -neg:
+                            continue            # stale entry
+                        if victim in want:
+                            held.append((neg, victim))
+                            continue
+                        break
+                    for h in held:
+                        heapq.heappush(heap, h)
+                    del resident[victim]
+            resident[k] = nxt[t][k]
+            heapq.heappush(heap, (-nxt[t][k], k))
+    return {"reads": reads, "misses": misses, "miss_rate": misses / reads if reads else 0.0}
+
+
+def balanced_miss_split(misses: float, fill_bw: float, cpu_bw: float) -> float:
+    """Misses to fill over the host link so that filling them takes as long as
+    running the rest on the CPU: q * S / fill_bw = (m - q) * S / cpu_bw gives
+    q = m * fill_bw / (fill_bw + cpu_bw).  The pages print this split garbled
+    (their q exceeds m whenever the link is faster than the CPU path; "FreeToken
+    290b model", section on the miss policy); this is the time-balanced reading.
+    Simulated only: the library fills every miss and runs it on the GPU."""
+    if misses < 0 or fill_bw <= 0 or cpu_bw <= 0:
+        raise ValueError("misses must be >= 0 and bandwidths > 0")
+    return misses * fill_bw / (fill_bw + cpu_bw)

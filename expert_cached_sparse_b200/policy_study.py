@@ -1,5 +1,5 @@
 """Miss rates of the shared LRU, a layer-oriented static split and prefill-time
-hot placement on the 40-layer NVFP4 decode trace (L = 40, E = 256, top-6,
+hot placement (with the offline optimum as a bound) on the 40-layer NVFP4 decode trace (L = 40, E = 256, top-6,
 Zipf(1.0) routing with 10 % of the popularity ranks reshuffled every 32
 steps), at several cache capacities.
 
@@ -77,7 +77,8 @@ def main(argv=None) -> int:
     for c in (int(v) for v in args.capacities.split(",")):
         res = {"shared_lru": P.replay(P.SharedLru(c), decode),
                "static_layer_split": P.replay(P.StaticPlacement(P.layer_split(cfg.layers, cfg.experts, c)), decode),
-               "prefill_hot": P.replay(P.StaticPlacement(P.prefill_hot(prefill, c)), decode)}
+               "prefill_hot": P.replay(P.StaticPlacement(P.prefill_hot(prefill, c)), decode),
+               "belady_bound": P.belady(decode, c)}
         out["capacity"][c] = {k: round(v["miss_rate"], 4) for k, v in res.items()}
         out["reads_per_step"] = res["shared_lru"]["reads"] / args.steps
     print(json.dumps(out), flush=True)

@@ -70,3 +70,28 @@ def test_lru_beats_static_split_on_skewed_routing():
     lru = P.replay(P.SharedLru(cap), trace)["miss_rate"]
     split = P.replay(P.StaticPlacement(P.layer_split(layers, experts, cap)), trace)["miss_rate"]
     assert lru < split
+
+
+def test_belady_is_a_lower_bound_and_optimal_on_a_hand_trace():
+    # one layer, capacity 2, reads a b c a b: optimal evicts c's slot owner with the farthest next use
+    trace = [(0, [0]), (0, [1]), (0, [2]), (0, [0]), (0, [1])]
+    # a, b miss; c misses and evicts b (next read at 4) rather than a (3); a hits; b misses
+    assert P.belady(trace, 2) == {"reads": 5, "misses": 4, "miss_rate": 0.8}
+    rng = np.random.default_rng(3)
+    for cap in (4, 9, 20):
+        trace = [(int(rng.integers(3)), rng.choice(16, size=3, replace=False)) for _ in range(400)]
+        opt = P.belady(trace, cap)["misses"]
+        lru = P.replay(P.SharedLru(cap), trace)["misses"]
+        hot = P.replay(P.StaticPlacement(P.layer_split(3, 16, cap)), trace)["misses"]
+        assert opt <= lru and opt <= hot
+
+
+def test_balanced_miss_split():
+    m, bp, bh = 10.0, 54.0, 18.0
+    q = P.balanced_miss_split(m, bp, bh)
+    assert q == pytest.approx(7.5)
+    assert q / bp == pytest.approx((m - q) / bh)          # both paths take the same time
+    assert 0 <= q <= m
+    assert P.balanced_miss_split(m, 1e9, 1.0) == pytest.approx(m, rel=1e-6)
+    with pytest.raises(ValueError):
+        P.balanced_miss_split(m, 0.0, 1.0)
