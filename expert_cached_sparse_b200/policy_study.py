@@ -1,7 +1,7 @@
 """Miss rates of the shared LRU, a layer-oriented static split and prefill-time
-hot placement (with the offline optimum as a bound) on the 40-layer NVFP4 decode trace (L = 40, E = 256, top-6,
-Zipf(1.0) routing with 10 % of the popularity ranks reshuffled every 32
-steps), at several cache capacities.
+hot placement, with the offline optimum as a bound, on the 40-layer NVFP4
+decode trace (L = 40, E = 256, top-6, Zipf(1.0) routing with 10 % of the
+popularity ranks reshuffled every 32 steps), at several cache capacities.
 
 Routing comes from this library's GPU router (``moe_router_topk``) on the
 seeded synthetic inputs of the trace workload; the policies are replayed on
