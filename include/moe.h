@@ -299,15 +299,17 @@ int moe_permute_noalloc(const int32_t* d_topk_idx, int32_t n, int32_t experts, i
 
 /*
  * Grouped SwiGLU expert FFN over the permuted rows.  d_slot_pool holds
- * pool_slots packed blobs of moe_slot_bytes() each.  For every expert e
- * with rows [offsets[e], offsets[e+1]) (clipped to [0, rows)) and
+ * pool_slots packed blobs of moe_slot_bytes() each.  d_expert_offsets holds
+ * E+1 non-decreasing values with offsets[0] >= 0 and offsets[E] <= rows (the
+ * exclusive prefix sums moe_permute writes); other contents are undefined
+ * behaviour.  For every expert e with rows [offsets[e], offsets[e+1]) and
  * 0 <= d_slot_of_expert[e] < pool_slots, the weights are read from that
  * slot and
  *   h = silu(x W1^T) * (x W3^T)   (fp32 accumulation),
  *   y = h W2^T                    (fp32 accumulation, y rounded to bf16)
  * is written to d_y_perm rows.  Rows of experts with any other slot value
- * (-1 in particular) are left untouched, so hits and misses can run as two
- * passes.  d_ws: moe_ffn_workspace_bytes() bytes (operand copies of x and
+ * (-1 in particular), or whose range does not lie inside [0, rows), are left
+ * untouched, so hits and misses can run as two passes.  d_ws: moe_ffn_workspace_bytes() bytes (operand copies of x and
  * h, h itself, and the partial sums of work split across CTAs).  The MMAs
  * take f16 operands: FP4 weights are expanded exactly (E2M1 times its block
  * scale is exact in f16 for the accepted scale codes), x and h rows are
