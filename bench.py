@@ -125,6 +125,16 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_bf16_tflops():
+    """Dense bf16 tensor peak (burst) and its provenance; the FFN's f16 MMAs run at the same rate."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 # ------------------------------------------------------------------ multi-rank plumbing
 def max_over_ranks(ms: float, device=None) -> float:
     """The largest per-rank device time (a no-op on one rank)."""
@@ -490,8 +500,11 @@ def extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=("r
     A.moe_profile_enable(False)
     idx = ds.idx[1:1 + steps].cpu().numpy()
     flops = steps * n * cfg.top_k * 3 * 2 * cfg.hidden * cfg.ffn
+    tensor_peak, tensor_kind = measured_bf16_tflops()
     out["prefill_4096"] = {"tokens_per_s": steps * n / (ms / 1000), "ms_per_step": ms / steps,
                            "ffn_tflops": flops / (prof["ffn"]["ms"] / 1000) / 1e12,
+                           "ffn_tensor_frac": flops / (prof["ffn"]["ms"] / 1000) / 1e12 / tensor_peak,
+                           "tensor_peak_tflops": tensor_peak, "tensor_peak_kind": tensor_kind,
                            "unique_experts_per_step": float(np.mean([len(np.unique(i)) for i in idx])),
                            "step_ms_breakdown": {k: prof[k]["ms"] / steps for k in prof}}
     ds.cache.close()
