@@ -34,7 +34,7 @@ EXPORTS = [
     "moe_cache_read_trace", "moe_cache_get_stats", "moe_cache_snapshot", "moe_cache_capacity",
     "moe_cache_destroy", "moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine",
     "moe_layer_forward", "moe_profile_enable", "moe_profile_read", "moe_get_device_error",
-    "moe_permute_noalloc",
+    "moe_permute_noalloc", "moe_act_terms",
 ]
 PROF_KINDS = ["router", "lookup", "permute", "ffn", "combine", "fill"]
 
@@ -94,6 +94,7 @@ def _load():
         "moe_profile_enable": (C.c_int, [C.c_int]),
         "moe_profile_read": (C.c_int, [C.POINTER(MoeProf), C.c_int, C.c_int]),
         "moe_get_device_error": (C.c_int, [C.c_int]),
+        "moe_act_terms": (C.c_int, [P, I32, I32, I32, I32, I32, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)

@@ -99,6 +99,14 @@ def moe_grouped_ffn(shape, pool, pool_slots, slot_of, offsets, x_perm, rows, y_p
     check("moe_grouped_ffn", rc)
 
 
+def moe_act_terms(x, rows, K, wfmt, terms, codes, scales, row_exp, stream=None):
+    """E2M1 term encoding of activation rows (the FP4 path's operand encoding):
+    codes uint8 [rows, terms, K], scales uint8 [rows, terms, K/vs], row_exp int32 [rows]."""
+    rc = L.lib.moe_act_terms(ptr(x), _dt(x), rows, K, wfmt, terms, ptr(codes), ptr(scales), ptr(row_exp),
+                             stream_handle(stream))
+    check("moe_act_terms", rc)
+
+
 def moe_combine(y_perm, row_of, topk_w, n, k, hidden, out, stream=None):
     rc = L.lib.moe_combine(ptr(y_perm), ptr(row_of), ptr(topk_w), n, k, hidden, ptr(out), _dt(out),
                            stream_handle(stream))

@@ -35,25 +35,24 @@ static inline bool shape_ok(const moe_shape* s)
     if (s->hidden <= 0 || s->hidden % 64 || s->ffn <= 0 || s->ffn % 64) return false;
     if (s->top_k <= 0 || s->top_k > s->experts || s->top_k > kMaxTopK) return false;
     if (s->wfmt < MOE_W_BF16 || s->wfmt > MOE_W_NVFP4) return false;
+    // FP4 blobs are stored in 128-row x 256-column chunks
+    if (s->wfmt != MOE_W_BF16 && (s->hidden % 256 || s->ffn % 256)) return false;
     return true;
 }
 
 // ---------------------------------------------------------------- blob layout
-// One packed expert (= one slot).  Matrices are cut into tiles of 16 rows x
-// 64 columns; tile (rt, kt) of a [R][K] matrix sits at tile_index(rt, kt).
-// Inside a tile, lane L = 4g+t of a warp owns rows g and g+8, columns
-// [16t, 16t+16): FP4 tiles store for each lane 8 bytes of row g then 8
-// bytes of row g+8 (512 B per tile), BF16 tiles 32 bytes of row g then 32
-// bytes of row g+8 (2048 B per tile).  The W13 rows are reordered so that
-// row tile rt holds gate rows f = 8rt..8rt+7 in its rows 0..7 and the
-// matching up rows in rows 8..15.  FP4 scale tiles: MXFP4 32 B
-// [g][(g,b0),(g,b1),(g+8,b0),(g+8,b1)], NVFP4 64 B
-// [g][(g,b0..b3),(g+8,b0..b3)] with b the 32- or 16-column block inside
-// the tile.  NVFP4 ends with the two fp32 tensor scales.
-// Tiles are stored in row groups of 8 row tiles (128 rows): for row group G
-// and column block kt the group's tiles are contiguous, so one 128 x 64
-// block is one contiguous copy.  Index of tile (rt, kt) of a matrix with RT
-// row tiles and KT column blocks (the last group may hold fewer than 8):
+// One packed expert (= one slot); W13 is [2F][H], W2 is [H][F].
+//
+// BF16 weights: matrices cut into tiles of 16 rows x 64 columns; tile (rt, kt)
+// of a [R][K] matrix sits at tile_index(rt, kt).  Inside a tile, lane L = 4g+t
+// of a warp owns rows g and g+8: for k16 step j its 16 bytes are the
+// mma.sync fragment words {a0, a2, a1, a3} (2048 B per tile).  W13 rows are
+// reordered so row tile rt holds gate rows f = 8rt..8rt+7 in its rows 0..7
+// and the matching up rows in rows 8..15.  Tiles are stored in row groups of
+// 8 row tiles (128 rows): for row group G and column block kt the group's
+// tiles are contiguous, so one 128 x 64 block is one contiguous copy.  Index
+// of tile (rt, kt) of a matrix with RT row tiles and KT column blocks (the
+// last group may hold fewer than 8):
 __host__ __device__ static inline size_t tile_index(int rt, int kt, int RT, int KT)
 {
     const int G = rt >> 3, w = rt & 7;
@@ -61,10 +60,28 @@ __host__ __device__ static inline size_t tile_index(int rt, int kt, int RT, int 
     return (size_t)8 * G * KT + (size_t)kt * ng + w;
 }
 
+// FP4 weights (MXFP4: E8M0 scale per 32 columns; NVFP4: E4M3 scale per 16
+// columns and one fp32 scale per matrix): each matrix is a sequence of
+// chunks, row block G (128 rows) by column chunk c (256 columns), at chunk
+// index G * (K / 256) + c, fp4_chunk_bytes apart.  A chunk is
+//   16384 B: the 128 rows' 128 bytes of E2M1 codes (two per byte, even
+//            column in the low nibble) as the tensor core reads them from
+//            shared memory: row r at 1024 (r / 8) + 128 (r % 8), its
+//            16-byte piece j stored at piece position j ^ (r % 8);
+//   then 256 / 32 / 4 = 2 (MXFP4) or 256 / 16 / 4 = 4 (NVFP4) scale images
+//            of 512 B, image i holding scales 4i..4i+3 of each row: scale s
+//            of row r at byte 16 (r % 32) + 4 (r / 32) + (s % 4).
+// Row r of W2 block G is output row 128 G + r.  Row r of W13 block G, with
+// q = r / 32 and i = r % 32, is gate row f = 64 G + 16 q + (i % 16) when
+// i < 16 and the matching up row (F + f) otherwise.  NVFP4 scales are stored
+// unsigned: a negative block scale is folded into the signs of its 16 codes.
+// The two NVFP4 tensor scales {s13, s2} end the blob.
+__host__ __device__ static inline int fp4_chunk_bytes(int wfmt) { return wfmt == MOE_W_MXFP4 ? 16384 + 1024 : 16384 + 2048; }
+
 struct BlobLayout {
-    size_t w13, w2, s13, s2, ts, bytes;
-    int tile_bytes;    // 512 (FP4) or 2048 (BF16)
-    int stile_bytes;   // 32 (MXFP4), 64 (NVFP4), 0 (BF16)
+    size_t w13, w2, ts, bytes;
+    int tile_bytes;    // BF16: 2048
+    int chunk_bytes;   // FP4: fp4_chunk_bytes
 };
 
 static inline BlobLayout blob_layout(const moe_shape* s)
@@ -73,21 +90,17 @@ static inline BlobLayout blob_layout(const moe_shape* s)
     size_t H = s->hidden, F = s->ffn;
     if (s->wfmt == MOE_W_BF16) {
         b.tile_bytes = 2048;
-        b.stile_bytes = 0;
         b.w13 = 0;
         b.w2 = 2 * F * H * 2;
-        b.s13 = b.s2 = b.ts = b.w2 + H * F * 2;
-        b.bytes = align_up(b.s13, 128);
+        b.ts = b.w2 + H * F * 2;
+        b.bytes = align_up(b.ts, 128);
         return b;
     }
-    size_t per_scale = (s->wfmt == MOE_W_MXFP4) ? 32 : 16;
-    b.tile_bytes = 512;
-    b.stile_bytes = (s->wfmt == MOE_W_MXFP4) ? 32 : 64;
+    const size_t cb = (size_t)fp4_chunk_bytes(s->wfmt);
+    b.chunk_bytes = (int)cb;
     b.w13 = 0;
-    b.w2 = 2 * F * H / 2;
-    b.s13 = b.w2 + H * F / 2;
-    b.s2 = b.s13 + 2 * F * H / per_scale;
-    b.ts = b.s2 + H * F / per_scale;
+    b.w2 = (2 * F / 128) * (H / 256) * cb;
+    b.ts = b.w2 + (H / 128) * (F / 256) * cb;
     b.bytes = align_up(b.ts + (s->wfmt == MOE_W_NVFP4 ? 8 : 0), 128);
     return b;
 }
@@ -149,26 +162,15 @@ struct RowSource {
     const int32_t* assign_of;
     int k;
 };
-int ffn_device_error(int clear);   // decode FFN's device error word (0: none)
+int ffn_device_error(int clear);   // BF16 streaming FFN's device error word (0: none)
+int ffn_fp4_device_error(int clear);   // FP4 FFN's device error word (0: none)
 int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
                const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,
                cudaStream_t st, const RowSource* gather = nullptr);
-bool ffn_tc_supported(const moe_shape* s);
-// Operands of the tensor-core path: f16 row copies of x and h with per-row
-// power-of-two exponents, and the fp32 h the first GEMM writes.
-struct TcOperands {
-    const uint16_t* x16;
-    const int32_t* xe;
-    float* h32;
-    const uint16_t* h16;
-    const int32_t* he;
-};
-}  // namespace moe
-#include <functional>
-namespace moe {
-int launch_ffn_tc(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
-                  const int32_t* offsets, int rows, uint16_t* y_perm, const TcOperands& op, cudaStream_t st,
-                  const std::function<int()>& between);
+size_t ffn_fp4_ws_bytes(const moe_shape* s, int rows);
+int launch_ffn_fp4(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
+                   const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,
+                   cudaStream_t st, const RowSource* gather);
 int launch_combine(const uint16_t* y_perm, const int32_t* row_of, const float* w, int n, int k, int H,
                    void* out, int out_dtype, cudaStream_t st);
 }  // namespace moe

@@ -1,0 +1,1055 @@
+// Grouped SwiGLU expert FFN for FP4 expert weights (MXFP4, NVFP4) on the
+// block-scaled fifth-generation tensor cores: the experts found in the GPU
+// cache execute on the GPU ("FreeToken quantization", section "Como se
+// desplazan los pesos MoE cuantizados por la memoria"; "FreeToken 290b
+// model", section "Como gestiona FreeToken el prellenado y la
+// decodificacion").
+//
+// Design for sm_100a:
+//  - the weights stay E2M1 with their block scales all the way into the
+//    tensor core: tcgen05.mma kind::mxf4 (E8M0 scale per 32 columns, MXFP4)
+//    or kind::mxf4nvf4 block16 (unsigned E4M3 scale per 16 columns, NVFP4)
+//    multiplies them as they sit in shared memory, with the scale factors in
+//    tensor memory.  No SM instruction touches a weight byte;
+//  - the slot blob stores every 128-row x 256-column block of a matrix as the
+//    exact shared-memory image the MMA reads (rows of 128 bytes in the
+//    128-byte swizzle) followed by its scale-factor images (the layout one
+//    tcgen05.cp 32x128b.warpx4 moves to tensor memory), so one bulk copy per
+//    pipeline stage brings weights and scales in (see common.cuh);
+//  - the activations (x rows, then h rows) are rewritten once per call as a
+//    short sum of E2M1 terms, each with its own block scale of the weights'
+//    scale type: term t+1 encodes what terms 0..t left over, so T terms carry
+//    about 3.3 T bits of each block (T = 4 for decode, 3 for prefill: about
+//    2e-4 and 2e-3 relative error).  The terms of a token are consecutive
+//    rows of the MMA's N operand and are summed in the epilogue;
+//  - swap-AB tiles: 128 weight rows are M, (terms x tokens) are N (up to 64
+//    for decode, 192 for prefill), K advances 64 columns per MMA, 256 per
+//    pipeline stage;
+//  - one persistent CTA per SM: warp 0 issues the bulk copies, warp 1 the
+//    scale-factor copies and MMAs (one thread each), warps 2-5 read the
+//    double-buffered accumulator back with tcgen05.ld and apply SwiGLU (gate
+//    and up rows 16 lanes apart) or the NVFP4 tensor scale;
+//  - decode cuts the concatenated K stages of all units into equal ranges
+//    per CTA (stream-K); the CTA finishing a unit sums its pieces in CTA
+//    order, so results are deterministic.  Prefill deals whole units.
+// Every wait is bounded; a timeout records MOE_ERR_TIMEOUT, raises the CTA's
+// abort flag so the other roles drain, and the kernel returns.
+#include <stdlib.h>
+#include <string.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+__device__ int g_fp4_error;   // first device-side error of this file's kernels (0: none)
+
+namespace {
+
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr int kQuantThreads = 128;
+constexpr long long kWaitCycles = 4000000000ll;   // ~2 s before a wait gives up
+constexpr int kMaxCtas = 160;                      // persistent grid: one CTA per SM at most
+constexpr int kSmemBudget = 227 * 1024;
+
+// Tile configurations: decode (few tokens per expert, stream-K) and prefill.
+template <int NMAX_, int T_, bool SPLIT_>
+struct TileCfg {
+    static constexpr int NMAX = NMAX_;   // MMA N per tile (terms x tokens), multiple of 8 T
+    static constexpr int T = T_;         // E2M1 terms per activation value
+    static constexpr int NT = NMAX_ / T_;  // tokens per tile
+    static constexpr bool SPLIT = SPLIT_;
+    static_assert(NMAX_ % (8 * T_) == 0, "token groups of 8 per epilogue step");
+};
+using DecodeCfg = TileCfg<64, 4, true>;
+using PrefillCfg = TileCfg<192, 3, false>;
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+// try_wait that lets the hardware suspend the thread while the phase is
+// incomplete, so waiting warps leave issue slots to working ones.
+__device__ __forceinline__ bool mbar_try_suspend(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity), "n"(20000)
+                 : "memory");
+    return ok != 0;
+}
+// Bounded wait: gives up when another role raised the abort flag, or after
+// kWaitCycles, in which case it records MOE_ERR_TIMEOUT and raises the flag.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag)
+{
+    if (mbar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (;;) {
+        if (mbar_try_suspend(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitCycles) break;
+    }
+    *abort_flag = 1;
+    atomicCAS(&g_fp4_error, 0, (int)MOE_ERR_TIMEOUT);
+    return false;
+}
+
+// Drain wait for this CTA's own asynchronous work (copies, MMAs) before it
+// exits or frees tensor memory: bounded by time only, not by the abort flag.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_suspend(bar, parity))
+        if (clock64() - t0 > kWaitCycles) {
+            atomicCAS(&g_fp4_error, 0, (int)MOE_ERR_TIMEOUT);
+            return;
+        }
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// Shared-memory descriptor of a K-major operand in the 128-byte swizzle:
+// 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr)
+{
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Descriptor of one scale-factor image: 32 rows of 16 bytes, no swizzle.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t addr)
+{
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(128 >> 4) << 32) |
+           ((uint64_t)1 << 46);
+}
+
+// 512-byte scale image -> 4 tensor-memory columns of all 128 lanes (the
+// 32-lane pattern is replicated into the four lane quarters).
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint32_t saddr)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc_sf(saddr)) : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem], E2M1 operands with block scales from tensor memory.
+template <int WFMT>
+__device__ __forceinline__ void tc_mma_fp4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc,
+                                           uint32_t sfa, uint32_t sfb)
+{
+    if (WFMT == MOE_W_MXFP4)
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+                     ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb) : "memory");
+    else
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+                     ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb) : "memory");
+}
+
+// Instruction descriptor (block-scaled kinds): E2M1 A and B, K-major, M = 128,
+// N = n, scale type E8M0 (MXFP4) or E4M3 (NVFP4), scale-factor byte `id`
+// inside each tensor-memory word for A and B.
+template <int WFMT>
+__device__ __forceinline__ uint32_t idesc_fp4(int n, uint32_t id)
+{
+    const uint32_t sfmt = WFMT == MOE_W_MXFP4 ? 1u : 0u;
+    return (id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | (sfmt << 23) | (8u << 24) | (id << 29);
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* v)
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                 : "r"(taddr)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
+
+// E4M3 code -> value (no NaN codes reach here)
+__device__ __forceinline__ float e4m3_value(uint32_t c)
+{
+    const uint32_t e = (c >> 3) & 15, m = c & 7;
+    const float v = (e == 0) ? (float)m * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+    return (c & 0x80) ? -v : v;
+}
+
+// ------------------------------------------------------------------ activation terms
+// Scale of one term of a block whose largest remaining magnitude is m: the
+// smallest scale of the format with m / scale <= 6 (E2M1's largest value).
+template <int WFMT>
+__device__ __forceinline__ uint32_t term_scale(float m, float& sval)
+{
+    if (!(m > 0.0f)) {   // zero block (or NaN): any scale, all codes 0
+        sval = 1.0f;
+        return WFMT == MOE_W_MXFP4 ? 127u : 0x38u;
+    }
+    if (WFMT == MOE_W_MXFP4) {
+        int E;
+        const float f = frexpf(m, &E);            // m = f 2^E, f in [0.5, 1)
+        int code = (f > 0.75f ? E - 2 : E - 3) + 127;   // 6 * 2^(code-127) >= m, minimal
+        code = code < 1 ? 1 : (code > 254 ? 254 : code);
+        sval = __uint_as_float((uint32_t)code << 23);
+        return (uint32_t)code;
+    }
+    const float s = __fdiv_rn(m, 6.0f);
+    uint32_t code;
+    if (s < 0.015625f) {                               // below 2^-6: subnormal steps of 2^-9
+        const float k = ceilf(s * 512.0f);
+        code = (uint32_t)k;                            // 1..8 (8 is 2^-6, the first normal code)
+    } else {
+        const uint32_t b = __float_as_uint(s);
+        int e = (int)(b >> 23) - 127;
+        uint32_t m3 = (b >> 20) & 7;
+        if (b & 0xFFFFF) m3++;                         // round up
+        if (m3 == 8) { m3 = 0; e++; }
+        code = e > 8 ? 0x7Eu : ((uint32_t)(e + 7) << 3) | m3;
+        if (code > 0x7E) code = 0x7E;                  // 448
+    }
+    sval = e4m3_value(code);
+    return code;
+}
+
+// Nearest E2M1 code of x (ties to the even code), |x| <= 6 expected.
+__device__ __forceinline__ uint32_t e2m1_code(float x)
+{
+    const float a = fabsf(x);
+    uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) + (a >= 3.5f) + (a > 5.0f);
+    if (x < 0.0f && c) c |= 8u;
+    return c;
+}
+
+__device__ __forceinline__ float e2m1_val(uint32_t c)
+{
+    const float mag = (c & 7) < 4 ? 0.5f * (float)(c & 7) : (float)(1 << (((c & 7) >> 1) - 1)) * (((c & 1) ? 1.5f : 1.0f));
+    return (c & 8) ? -mag : mag;
+}
+
+// Per-chunk bytes of a token group's operand image with n rows (n multiple of 8).
+__host__ __device__ __forceinline__ int b_chunk_bytes(int n, int nsub)
+{
+    return n * 128 + nsub * ((n + 127) / 128) * 512;
+}
+
+template <int WFMT>
+struct Fmt {
+    static constexpr int VS = WFMT == MOE_W_MXFP4 ? 32 : 16;   // columns per block scale
+    static constexpr int NSUB = 256 / VS / 4;                    // scale images per 256-column chunk
+    static constexpr int CB = 16384 + 512 * NSUB;                // blob bytes per 128 x 256 chunk
+};
+
+// The plan of one call: for every expert e with rows and a slot in the pool,
+// its token groups (of NT rows) are numbered from gpre[e]; the per-chunk
+// bytes of their operand images are summed in boffc (in expert order).
+__global__ void __launch_bounds__(256) fp4_plan_kernel(const int32_t* __restrict__ offsets,
+                                                       const int32_t* __restrict__ slot_of, int E, int rows,
+                                                       int pool_slots, int NT, int T, int nsub,
+                                                       int32_t* __restrict__ gpre, int32_t* __restrict__ boffc,
+                                                       int32_t* __restrict__ zero, int nzero)
+{
+    pdl_wait();
+    for (int i = threadIdx.x; i < nzero; i += 256) zero[i] = 0;
+    __shared__ int s_g[8], s_b[8];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int EPT = (E + 255) / 256;   // <= 16 for E <= 4096
+    int gl = 0, bl = 0, gc[16], bc[16];
+    const int nfull = ((T * NT + 7) / 8) * 8;
+    for (int i = 0; i < 16; i++) {
+        const int e = threadIdx.x * EPT + i;
+        int g = 0, b = 0;
+        if (i < EPT && e < E) {
+            const int m = offsets[e + 1] - offsets[e], sl = slot_of[e];
+            if (m > 0 && sl >= 0 && sl < pool_slots && offsets[e] >= 0 && offsets[e + 1] <= rows) {
+                g = (m + NT - 1) / NT;
+                const int last = m - (g - 1) * NT;
+                b = (g - 1) * b_chunk_bytes(nfull, nsub) + b_chunk_bytes(((T * last + 7) / 8) * 8, nsub);
+            }
+        }
+        gc[i] = g;
+        bc[i] = b;
+        gl += g;
+        bl += b;
+    }
+    int gi = gl, bi = bl;
+    for (int off = 1; off < 32; off <<= 1) {
+        const int go = __shfl_up_sync(0xffffffffu, gi, off), bo = __shfl_up_sync(0xffffffffu, bi, off);
+        if (lane >= off) { gi += go; bi += bo; }
+    }
+    if (lane == 31) { s_g[wid] = gi; s_b[wid] = bi; }
+    __syncthreads();
+    int gr = gi - gl, br = bi - bl;
+    for (int w = 0; w < wid; w++) { gr += s_g[w]; br += s_b[w]; }
+    for (int i = 0; i < 16; i++) {
+        const int e = threadIdx.x * EPT + i;
+        if (i < EPT && e < E) { gpre[e] = gr; boffc[e] = br; }
+        gr += gc[i];
+        br += bc[i];
+    }
+    if (threadIdx.x == 255) { gpre[E] = gr; boffc[E] = br; }
+}
+
+// One CTA per activation row (x gathered by token, or h): writes the row's T
+// E2M1 terms and their block scales into its token group's operand image,
+// and (NVFP4) the power-of-two exponent p the row was scaled by, 2^p times
+// its largest magnitude lying in [2^10, 2^11) so every term scale stays
+// inside the E4M3 range.  Rows of experts without a slot are skipped.
+// CANON: no groups; row r's codes go to ccodes [rows][T][K] (one per byte),
+// its scale codes to cscales [rows][T][K / vs] and p to rex[r].
+template <int WFMT, int T, bool IN_F32, bool CANON = false>
+__global__ void __launch_bounds__(kQuantThreads) fp4_terms_kernel(
+    const void* __restrict__ in, int rows, int K, const int32_t* __restrict__ gather, int gk,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ slot_of, int E, int pool_slots,
+    const int32_t* __restrict__ boffc, int NT, char* __restrict__ bimg, int32_t* __restrict__ rex,
+    uint8_t* __restrict__ ccodes = nullptr, uint8_t* __restrict__ cscales = nullptr)
+{
+    using FM = Fmt<WFMT>;
+    constexpr int VS = FM::VS, NSUB = FM::NSUB, BPC = 256 / VS;   // blocks per chunk
+    pdl_wait();
+    pdl_trigger();
+    __shared__ float s_max[kQuantThreads / 32];
+    const int tid = threadIdx.x, KC = K / 256, nblk = K / VS;
+    const int nfull = ((T * NT + 7) / 8) * 8;
+    for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+        int j = 0, N = 0, nh = 0, BB = 0;
+        char* base = nullptr;
+        if (!CANON) {
+            int lo = 0, hi = E - 1;   // expert of row r: the largest e with offsets[e] <= r
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (offsets[mid] <= r) lo = mid;
+                else hi = mid - 1;
+            }
+            const int e = lo, sl = slot_of[e], m = offsets[e + 1] - offsets[e];
+            if (!(m > 0 && sl >= 0 && sl < pool_slots && offsets[e] >= 0 && offsets[e + 1] <= rows)) continue;
+            const int loc = r - offsets[e], gi = loc / NT, nt = min(NT, m - gi * NT);
+            j = loc % NT;
+            N = ((T * nt + 7) / 8) * 8;
+            nh = (N + 127) / 128;
+            BB = b_chunk_bytes(N, NSUB);
+            base = bimg + (size_t)KC * ((size_t)boffc[e] + (size_t)gi * b_chunk_bytes(nfull, NSUB));
+        }
+        const size_t sr = gather ? (size_t)(__ldg(gather + r) / gk) : (size_t)r;
+        const float* inf = static_cast<const float*>(in) + sr * K;
+        const uint16_t* inb = static_cast<const uint16_t*>(in) + sr * K;
+        int p = 0;
+        if (WFMT == MOE_W_NVFP4) {
+            float mx = 0.0f;
+            for (int k = tid * 8; k < K; k += kQuantThreads * 8) {
+                if (IN_F32) {
+                    const float4 a = __ldg(reinterpret_cast<const float4*>(inf + k));
+                    const float4 b = __ldg(reinterpret_cast<const float4*>(inf + k) + 1);
+                    mx = fmaxf(mx, fmaxf(fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))),
+                                         fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w)))));
+                } else {
+                    const uint4 q = __ldg(reinterpret_cast<const uint4*>(inb + k));
+                    const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                    for (int i = 0; i < 4; i++)
+                        mx = fmaxf(mx, fmaxf(fabsf(bf16_bits_to_f32(u[i] & 0xFFFF)), fabsf(bf16_bits_to_f32(u[i] >> 16))));
+                }
+            }
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            if ((tid & 31) == 0) s_max[tid >> 5] = mx;
+            __syncthreads();
+            mx = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
+            __syncthreads();   // s_max is reused by the next row
+            if (mx > 0.0f && mx <= 3.4e38f) {
+                int e2;
+                frexpf(mx, &e2);          // mx = f 2^e2, f in [0.5, 1)
+                p = 11 - e2;              // mx 2^p in [2^10, 2^11)
+                p = p < -100 ? -100 : (p > 100 ? 100 : p);
+            }
+            if (tid == 0) rex[r] = p;
+        }
+        if (CANON && WFMT == MOE_W_MXFP4 && tid == 0) rex[r] = 0;
+        const float sc = ldexpf(1.0f, p);
+        for (int b = tid; b < nblk; b += kQuantThreads) {
+            float v[VS];
+#pragma unroll
+            for (int i = 0; i < VS; i += 8) {
+                if (IN_F32) {
+                    const float4 a = __ldg(reinterpret_cast<const float4*>(inf + b * VS + i));
+                    const float4 c = __ldg(reinterpret_cast<const float4*>(inf + b * VS + i) + 1);
+                    v[i] = a.x; v[i + 1] = a.y; v[i + 2] = a.z; v[i + 3] = a.w;
+                    v[i + 4] = c.x; v[i + 5] = c.y; v[i + 6] = c.z; v[i + 7] = c.w;
+                } else {
+                    const uint4 q = __ldg(reinterpret_cast<const uint4*>(inb + b * VS + i));
+                    const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                    for (int h = 0; h < 4; h++) {
+                        v[i + 2 * h] = bf16_bits_to_f32(u[h] & 0xFFFF);
+                        v[i + 2 * h + 1] = bf16_bits_to_f32(u[h] >> 16);
+                    }
+                }
+            }
+            if (WFMT == MOE_W_NVFP4)
+#pragma unroll
+                for (int i = 0; i < VS; i++) v[i] = __fmul_rn(v[i], sc);
+            const int c = b / BPC, bc = b % BPC, sub = bc / 4, s4 = bc % 4;
+            const int piece = (bc * VS / 2) / 16, half = (VS == 16) ? (bc & 1) : 0;
+            char* cb = CANON ? nullptr : base + (size_t)c * BB;
+#pragma unroll
+            for (int t = 0; t < T; t++) {
+                const int n = j * T + t;
+                float mx = 0.0f;
+#pragma unroll
+                for (int i = 0; i < VS; i++) mx = fmaxf(mx, fabsf(v[i]));
+                float sval;
+                const uint32_t scode = term_scale<WFMT>(mx, sval);
+                uint32_t packed[VS / 8];
+#pragma unroll
+                for (int w = 0; w < VS / 8; w++) packed[w] = 0;
+#pragma unroll
+                for (int i = 0; i < VS; i++) {
+                    const uint32_t q = e2m1_code(__fdiv_rn(v[i], sval));
+                    packed[i / 8] |= q << (4 * (i % 8));
+                    v[i] = __fsub_rn(v[i], __fmul_rn(e2m1_val(q), sval));
+                }
+                if (CANON) {
+                    uint8_t* cr = ccodes + ((size_t)r * T + t) * K + (size_t)b * VS;
+#pragma unroll
+                    for (int i = 0; i < VS; i++) cr[i] = (uint8_t)((packed[i / 8] >> (4 * (i % 8))) & 15);
+                    cscales[((size_t)r * T + t) * nblk + b] = (uint8_t)scode;
+                    continue;
+                }
+                char* dst = cb + 1024 * (n >> 3) + 128 * (n & 7) + 16 * (piece ^ (n & 7)) + 8 * half;
+                if (VS == 32)
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                else
+                    *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+                cb[N * 128 + 512 * (nh * sub + (n >> 7)) + 16 * (n & 31) + 4 * ((n & 127) >> 5) + s4] = (char)scode;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ grouped GEMM
+struct Fp4Args {
+    const char* pool;
+    size_t slot_bytes;
+    size_t w_off;       // matrix offset inside a blob
+    size_t ts_off;      // NVFP4 tensor scales
+    int R, K, E, rows, pool_slots;
+    const int32_t* slot_of;
+    const int32_t* offsets;
+    const int32_t* gpre;
+    const int32_t* boffc;
+    const char* bimg;       // operand images of this phase's activations
+    const int32_t* rex;     // per-row exponents of the activations (NVFP4), else null
+    float* out_h;           // phase 1: h [rows][R/2] fp32
+    uint16_t* out_y;        // phase 2: y [rows][R] bf16
+    int32_t* cnt;           // per unit: pieces finished (stream-K)
+    float* pieces;          // [gridDim.x][2][128 * NMAX] partial accumulators (stream-K)
+};
+
+template <int WFMT, class CFG>
+struct KCfg {
+    using FM = Fmt<WFMT>;
+    static constexpr int NH = (CFG::NMAX + 127) / 128;
+    static constexpr int A_BYTES = FM::CB;                                // 1024-multiple
+    static constexpr int B_BYTES = CFG::NMAX * 128 + FM::NSUB * NH * 512;  // 1024-multiple
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int D = (kSmemBudget - 2048) / STAGE > 8 ? 8 : (kSmemBudget - 2048) / STAGE;
+    static constexpr int SMEM = 1024 + 1024 + D * STAGE;   // barriers, alignment slack, ring
+    // tensor memory: two accumulators, then two scale-factor sets
+    static constexpr int SF_A = 4 * FM::NSUB, SF_B = 4 * FM::NSUB * NH;
+    static constexpr int SF_COL = 2 * CFG::NMAX;
+    static constexpr int SF_SET = SF_A + SF_B;
+    static constexpr int COLS_USED = SF_COL + 2 * SF_SET;
+    static constexpr uint32_t TMEM_COLS = COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64 : COLS_USED <= 128 ? 128
+                                          : COLS_USED <= 256 ? 256 : 512;
+    static_assert(COLS_USED <= 512, "tensor memory");
+    static_assert(STAGE % 1024 == 0, "1024-byte aligned stages");
+};
+
+// A unit: (token group of one expert, 128-row block of the weight matrix).
+struct Unit {
+    int e, G, row0, nt, n;   // n: MMA N (terms x tokens, multiple of 8)
+    const char* blob;        // the expert's slot
+    const char* a;           // chunk 0 of the weight block
+    const char* b;           // chunk 0 of the token group's operand image
+    int bb;                  // bytes per chunk of that image
+};
+
+template <int WFMT, class CFG>
+__device__ __forceinline__ Unit unit_of(const Fp4Args& a, int u, int RB, int KC)
+{
+    using FM = Fmt<WFMT>;
+    Unit U;
+    U.G = u % RB;
+    const int gi = u / RB;
+    int lo = 0, hi = a.E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(a.gpre + mid) <= gi) lo = mid;
+        else hi = mid - 1;
+    }
+    U.e = lo;
+    const int i = gi - __ldg(a.gpre + lo), m = __ldg(a.offsets + lo + 1) - __ldg(a.offsets + lo);
+    U.row0 = __ldg(a.offsets + lo) + i * CFG::NT;
+    U.nt = min(CFG::NT, m - i * CFG::NT);
+    U.n = ((CFG::T * U.nt + 7) / 8) * 8;
+    U.bb = b_chunk_bytes(U.n, FM::NSUB);
+    U.blob = a.pool + (size_t)__ldg(a.slot_of + lo) * a.slot_bytes;
+    U.a = U.blob + a.w_off + (size_t)U.G * KC * FM::CB;
+    U.b = a.bimg + (size_t)KC * ((size_t)__ldg(a.boffc + lo) + (size_t)i * b_chunk_bytes(CFG::NMAX, FM::NSUB));
+    return U;
+}
+
+// Segments of one CTA: whole units u = blockIdx.x + i * gridDim.x, or the
+// stream-K pieces of its stage range [pos, end): unit u, chunks [p0, p1).
+struct Seg {
+    long pos, start;
+    int u, p0, p1;
+    __device__ __forceinline__ bool next(bool whole, int NU, int KC, long end)
+    {
+        if (whole) {
+            if (pos >= NU) return false;
+            u = (int)pos;
+            p0 = 0;
+            p1 = KC;
+            pos += gridDim.x;
+            return true;
+        }
+        if (pos >= end) return false;
+        start = pos;
+        u = (int)(pos / KC);
+        p0 = (int)(pos % KC);
+        p1 = (int)min((long)KC, p0 + (end - pos));
+        pos += p1 - p0;
+        return true;
+    }
+};
+
+__device__ __forceinline__ long sk_bound(long W, int c, int grid) { return W * c / grid; }
+__device__ __forceinline__ int sk_cta_of(long W, long idx, int grid)
+{
+    int c = (int)(idx * grid / W);
+    while (c + 1 < grid && sk_bound(W, c + 1, grid) <= idx) c++;
+    while (c > 0 && sk_bound(W, c, grid) > idx) c--;
+    return c;
+}
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
+
+// Final values of 8 tokens of a unit from their 8 T accumulator columns d:
+// sum of the terms, the row exponents undone, then SwiGLU into h (phase 1,
+// lanes 0-15 gate rows, 16-31 the matching up rows) or y in bf16.
+template <int WFMT, int PHASE, int T>
+__device__ __forceinline__ void finish8(const Fp4Args& a, const Unit& U, int q, int lane, int ch, const float* d,
+                                        float tsc)
+{
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        const int tok = 8 * ch + j;
+        float v = 0.0f;
+#pragma unroll
+        for (int t = 0; t < T; t++) v += d[j * T + t];
+        const bool live = tok < U.nt;
+        const int row = U.row0 + tok;
+        float u = tsc;
+        if (WFMT == MOE_W_NVFP4 && live) u = tsc * pow2i(-__ldg(a.rex + row));
+        v *= u;
+        if (PHASE == 1) {
+            const float up = __shfl_down_sync(0xffffffffu, v, 16);
+            if (live && lane < 16) {
+                const int F = a.R / 2;
+                a.out_h[(size_t)row * F + 64 * U.G + 16 * q + lane] = silu(v) * up;
+            }
+        } else if (live) {
+            a.out_y[(size_t)row * a.R + 128 * U.G + 32 * q + lane] = f32_to_bf16_bits(v);
+        }
+    }
+}
+
+template <int WFMT, int PHASE, class CFG>
+__global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
+{
+    using FM = Fmt<WFMT>;
+    using KC_ = KCfg<WFMT, CFG>;
+    constexpr int D = KC_::D, STAGE = KC_::STAGE, T = CFG::T;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem =
+        reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // [D]
+    uint64_t* empty = full + D;                           // [D]
+    uint64_t* acc_full = empty + D;                       // [2]
+    uint64_t* acc_empty = acc_full + 2;                   // [2]
+    uint64_t* fin = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+    int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+    int* s_last = abort_flag + 1;
+    unsigned char* ring = smem + 1024;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int RB = a.R / 128, KC = a.K / 256;
+
+    if (tid == 0) {
+        for (int i = 0; i < D; i++) {
+            mbar_init(smem_u32(&full[i]), 1);
+            mbar_init(smem_u32(&empty[i]), 1);
+        }
+        for (int i = 0; i < 2; i++) {
+            mbar_init(smem_u32(&acc_full[i]), 1);
+            mbar_init(smem_u32(&acc_empty[i]), 32 * kEpiWarps);
+        }
+        mbar_init(smem_u32(fin), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(KC_::TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    volatile int* abort_v = abort_flag;
+    pdl_wait();
+    pdl_trigger();
+
+    // work: whole units round-robin (prefill), or the units' K chunks cut into
+    // equal ranges over the CTAs (decode)
+    const int NU = __ldg(a.gpre + a.E) * RB;
+    const bool whole = !CFG::SPLIT;
+    const long W = whole ? 0 : (long)NU * KC;
+    const int grid = whole ? (int)gridDim.x : (int)(W < (long)gridDim.x ? W : (long)gridDim.x);
+    const bool in_use = whole || (int)blockIdx.x < grid;
+    const long b0 = (!whole && in_use) ? sk_bound(W, blockIdx.x, grid) : 0;
+    const long b1 = (!whole && in_use) ? sk_bound(W, blockIdx.x + 1, grid) : 0;
+    const long first = whole ? (long)blockIdx.x : b0;
+
+    if (warp == 0) {
+        // ============ bulk copies: weight chunk image + token group image chunk
+        if (lane == 0 && in_use) {
+            int st = 0;
+            uint32_t ph = 0;
+            long issued = 0;
+            bool ok = true;
+            Seg sg{first};
+            while (ok && sg.next(whole, NU, KC, b1)) {
+                const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC);
+                for (int c = sg.p0; c < sg.p1; c++) {
+                    if (!(ok = mbar_wait(smem_u32(&empty[st]), ph ^ 1, abort_v))) break;
+                    const uint32_t bar = smem_u32(&full[st]);
+                    unsigned char* sp = ring + (size_t)st * STAGE;
+                    mbar_expect_tx(bar, (uint32_t)(FM::CB + U.bb));
+                    bulk_g2s(smem_u32(sp), U.a + (size_t)c * FM::CB, FM::CB, bar);
+                    bulk_g2s(smem_u32(sp + KC_::A_BYTES), U.b + (size_t)c * U.bb, (uint32_t)U.bb, bar);
+                    issued++;
+                    if (++st == D) { st = 0; ph ^= 1; }
+                }
+            }
+            // every issued copy lands before the CTA exits (stage i was last
+            // filled in this pass if i < st, else in the previous one)
+            for (int i = 0; i < D && i < issued; i++) mbar_drain(smem_u32(&full[i]), i < st ? ph : (ph ^ 1));
+        }
+    } else if (warp == 1) {
+        // ============ scale-factor copies and MMAs (one thread)
+        if (lane == 0 && in_use) {
+            int st = 0, it = 0;
+            uint32_t ph = 0;
+            long cc = 0;
+            bool ok = true;
+            Seg sg{first};
+            while (ok && sg.next(whole, NU, KC, b1)) {
+                const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC);
+                const int ab = it & 1, nh = (U.n + 127) / 128;
+                if (it >= 2) {   // the epilogue has read this accumulator's previous unit
+                    if (!(ok = mbar_wait(smem_u32(&acc_empty[ab]), ((it >> 1) - 1) & 1, abort_v))) break;
+                    tc_fence_after();
+                }
+                const uint32_t dcol = tmem + (uint32_t)(ab * CFG::NMAX);
+                for (int c = sg.p0; c < sg.p1; c++, cc++) {
+                    if (!(ok = mbar_wait(smem_u32(&full[st]), ph, abort_v))) break;
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(ring + (size_t)st * STAGE), sb = sa + KC_::A_BYTES;
+                    const uint32_t sfa = tmem + KC_::SF_COL + (uint32_t)((cc & 1) * KC_::SF_SET);
+                    const uint32_t sfb = sfa + KC_::SF_A;
+#pragma unroll
+                    for (int s = 0; s < FM::NSUB; s++) tc_cp_sf(sfa + 4 * s, sa + 16384 + 512 * s);
+                    for (int s = 0; s < FM::NSUB * nh; s++) tc_cp_sf(sfb + 4 * s, sb + U.n * 128 + 512 * s);
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        // MXFP4: two 32-column scales per MMA, bytes 0-1 or 2-3 of a word;
+                        // NVFP4: four 16-column scales per MMA, one image each
+                        const int s = WFMT == MOE_W_MXFP4 ? (k >> 1) : k;
+                        const uint32_t id = WFMT == MOE_W_MXFP4 ? 2u * (k & 1) : 0u;
+                        tc_mma_fp4<WFMT>(dcol, desc_sw128(sa + 32 * k), desc_sw128(sb + 32 * k),
+                                         idesc_fp4<WFMT>(U.n, id), (c > sg.p0 || k > 0) ? 1u : 0u, sfa + 4 * s,
+                                         sfb + 4 * nh * s);
+                    }
+                    tc_commit(smem_u32(&empty[st]));   // the stage is free once these MMAs have read it
+                    if (++st == D) { st = 0; ph ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit(smem_u32(&acc_full[ab]));
+                it++;
+            }
+            // every MMA issued here completes before tensor memory is released
+            tc_commit(smem_u32(fin));
+            mbar_drain(smem_u32(fin), 0);
+        }
+    } else if (in_use) {
+        // ============ epilogue: warps 2..5, tensor-memory lane quarter q.
+        // All four warps walk the same segments and meet the same named
+        // barriers; after a failed wait a warp keeps walking without waiting
+        // or touching tensor memory, so the barriers still match.
+        const int q = warp & 3;
+        const int etid = tid - 64;   // 0..127
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        int it = 0;
+        bool ok = true;
+        Seg sg{first};
+        while (sg.next(whole, NU, KC, b1)) {
+            const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC);
+            const int ab = it & 1;
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[ab]), (it >> 1) & 1, abort_v));
+            if (ok) tc_fence_after();
+            float tsc = 1.0f;
+            if (WFMT == MOE_W_NVFP4) tsc = __ldg(reinterpret_cast<const float*>(U.blob + a.ts_off) + PHASE - 1);
+            const uint32_t dcol = tmem + lane_base + (uint32_t)(ab * CFG::NMAX);
+            const int nch = (U.nt + 7) / 8;
+            if (whole || (sg.p0 == 0 && sg.p1 == KC)) {
+                if (ok) {
+                    for (int ch = 0; ch < nch; ch++) {
+                        uint32_t d[8 * T];
+#pragma unroll
+                        for (int t = 0; t < T; t++) tmem_ld8(dcol + 8 * T * ch + 8 * t, d + 8 * t);
+                        tmem_wait_ld();
+                        finish8<WFMT, PHASE, T>(a, U, q, lane, ch, reinterpret_cast<const float*>(d), tsc);
+                    }
+                    tc_fence_before();
+                    mbar_arrive(smem_u32(&acc_empty[ab]));
+                }
+            } else {
+                // a piece: publish the partial sums, count the piece; the CTA
+                // completing the unit adds all pieces in CTA order
+                const int slot = sg.start == b0 ? 0 : 1;
+                float* mine = a.pieces + ((size_t)blockIdx.x * 2 + slot) * (128 * CFG::NMAX);
+                if (ok) {
+                    for (int ch = 0; ch < nch; ch++) {
+                        uint32_t d[8 * T];
+#pragma unroll
+                        for (int t = 0; t < T; t++) tmem_ld8(dcol + 8 * T * ch + 8 * t, d + 8 * t);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 8 * T; i++)
+                            mine[(size_t)(8 * T * ch + i) * 128 + etid] = __uint_as_float(d[i]);
+                    }
+                    tc_fence_before();
+                    mbar_arrive(smem_u32(&acc_empty[ab]));
+                }
+                __threadfence();
+                epi_bar();
+                const long u_lo = (long)sg.u * KC, u_hi = u_lo + KC - 1;
+                const int c_lo = sk_cta_of(W, u_lo, grid), c_hi = sk_cta_of(W, u_hi, grid);
+                // a warp that failed its wait has raised the abort flag before this barrier
+                if (etid == 0) *s_last = (ok && !*abort_v && atomicAdd(a.cnt + sg.u, 1) == c_hi - c_lo) ? 1 : 0;
+                epi_bar();
+                if (*s_last) {
+                    __threadfence();
+                    for (int ch = 0; ch < nch; ch++) {
+                        float d[8 * T];
+#pragma unroll
+                        for (int i = 0; i < 8 * T; i++) d[i] = 0.0f;
+                        for (int c = c_lo; c <= c_hi; c++) {
+                            const int sl = sk_bound(W, c, grid) >= u_lo ? 0 : 1;
+                            const float* pc = a.pieces + ((size_t)c * 2 + sl) * (128 * CFG::NMAX);
+#pragma unroll
+                            for (int i = 0; i < 8 * T; i++)
+                                d[i] += __ldcg(pc + (size_t)(8 * T * ch + i) * 128 + etid);
+                        }
+                        finish8<WFMT, PHASE, T>(a, U, q, lane, ch, d, tsc);
+                    }
+                    if (etid == 0) a.cnt[sg.u] = 0;
+                }
+                epi_bar();   // s_last is rewritten by the next piece
+            }
+            it++;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(KC_::TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// ------------------------------------------------------------------ host side
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+struct Fp4Ws {
+    int32_t* gpre;
+    int32_t* boffc;
+    int32_t* rex_x;
+    int32_t* rex_h;
+    char* bx;
+    char* bh;
+    float* h32;
+    int32_t* cnt;
+    int ncnt;
+    float* pieces;
+};
+
+// Upper bound of the per-chunk bytes of all token-group images of a call.
+template <class CFG>
+size_t group_chunk_bound(int rows, int E, int nsub)
+{
+    const size_t G = (size_t)(rows + CFG::NT - 1) / CFG::NT + (size_t)(rows < E ? rows : E);
+    const size_t n = (size_t)CFG::T * rows + 7 * G;          // image rows
+    return 128 * n + (size_t)nsub * 512 * (G + n / 128 + 1);
+}
+
+size_t fp4_ws_layout(const moe_shape* s, int rows, void* base, Fp4Ws* w)
+{
+    size_t o = 0;
+    auto take = [&](size_t b) { size_t at = o; o = align_up(o + b, 256); return at; };
+    const int R = rows > 0 ? rows : 1, E = s->experts, nsub = s->wfmt == MOE_W_MXFP4 ? 2 : 4;
+    const size_t per_chunk =
+        group_chunk_bound<DecodeCfg>(R, E, nsub) > group_chunk_bound<PrefillCfg>(R, E, nsub)
+            ? group_chunk_bound<DecodeCfg>(R, E, nsub)
+            : group_chunk_bound<PrefillCfg>(R, E, nsub);
+    const size_t ogp = take(4 * (size_t)(E + 1));
+    const size_t obo = take(4 * (size_t)(E + 1));
+    const size_t orx = take(4 * (size_t)R);
+    const size_t orh = take(4 * (size_t)R);
+    const size_t obx = take(per_chunk * (s->hidden / 256));
+    const size_t obh = take(per_chunk * (s->ffn / 256));
+    const size_t oh = take(4 * (size_t)R * s->ffn);
+    const long RBmax = (2 * s->ffn > s->hidden ? 2 * s->ffn : s->hidden) / 128;
+    const long ncnt = ((long)(R + DecodeCfg::NT - 1) / DecodeCfg::NT + (R < E ? R : E)) * RBmax;
+    const size_t oc = take(4 * (size_t)ncnt);
+    const size_t op = take(4 * (size_t)kMaxCtas * 2 * 128 * DecodeCfg::NMAX);
+    if (w) {
+        char* b = static_cast<char*>(base);
+        w->gpre = reinterpret_cast<int32_t*>(b + ogp);
+        w->boffc = reinterpret_cast<int32_t*>(b + obo);
+        w->rex_x = reinterpret_cast<int32_t*>(b + orx);
+        w->rex_h = reinterpret_cast<int32_t*>(b + orh);
+        w->bx = b + obx;
+        w->bh = b + obh;
+        w->h32 = reinterpret_cast<float*>(b + oh);
+        w->cnt = reinterpret_cast<int32_t*>(b + oc);
+        w->ncnt = (int)ncnt;
+        w->pieces = reinterpret_cast<float*>(b + op);
+    }
+    return o;
+}
+
+template <int WFMT, int PHASE, class CFG>
+int set_smem_attr()
+{
+    constexpr int smem = KCfg<WFMT, CFG>::SMEM;
+    int dev = 0;
+    MOE_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+    static bool done[kMaxDevices];
+    if (!done[dev]) {
+        MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_fp4_kernel<WFMT, PHASE, CFG>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+        done[dev] = true;
+    }
+    return MOE_OK;
+}
+
+constexpr uint8_t* kNoCanon = nullptr;
+
+template <int WFMT, class CFG>
+int run_fp4(const moe_shape* s, const BlobLayout& bl, const void* pool, size_t slot_bytes, int pool_slots,
+            const int32_t* slot_of, const int32_t* offsets, int rows, uint16_t* y_perm, const Fp4Ws& w,
+            const RowSource& src, int sms, cudaStream_t st)
+{
+    using FM = Fmt<WFMT>;
+    const int E = s->experts, H = s->hidden, F = s->ffn;
+    // per-chunk image offsets must stay 32-bit
+    if (group_chunk_bound<CFG>(rows, E, FM::NSUB) >= (size_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+    int rc;
+    if ((rc = set_smem_attr<WFMT, 1, CFG>())) return rc;
+    if ((rc = set_smem_attr<WFMT, 2, CFG>())) return rc;
+    MOE_CUDA_TRY(launch_pdl(fp4_plan_kernel, 1, 256, 0, st, offsets, slot_of, E, rows, pool_slots, CFG::NT, CFG::T,
+                            FM::NSUB, w.gpre, w.boffc, w.cnt, w.ncnt));
+    const int qgrid = rows < sms * 16 ? rows : sms * 16;
+    if (src.x_dtype == MOE_DT_F32)
+        MOE_CUDA_TRY(launch_pdl(fp4_terms_kernel<WFMT, CFG::T, true>, qgrid, kQuantThreads, 0, st, src.x, rows, H,
+                                src.assign_of, src.k, offsets, slot_of, E, pool_slots, w.boffc, CFG::NT, w.bx, w.rex_x,
+                                kNoCanon, kNoCanon));
+    else
+        MOE_CUDA_TRY(launch_pdl(fp4_terms_kernel<WFMT, CFG::T, false>, qgrid, kQuantThreads, 0, st, src.x, rows, H,
+                                src.assign_of, src.k, offsets, slot_of, E, pool_slots, w.boffc, CFG::NT, w.bx, w.rex_x,
+                                kNoCanon, kNoCanon));
+    Fp4Args a{};
+    a.pool = static_cast<const char*>(pool);
+    a.slot_bytes = slot_bytes;
+    a.ts_off = bl.ts;
+    a.E = E;
+    a.rows = rows;
+    a.pool_slots = pool_slots;
+    a.slot_of = slot_of;
+    a.offsets = offsets;
+    a.gpre = w.gpre;
+    a.boffc = w.boffc;
+    a.cnt = w.cnt;
+    a.pieces = w.pieces;
+    const int grid = sms < kMaxCtas ? sms : kMaxCtas;
+    constexpr int smem = KCfg<WFMT, CFG>::SMEM;
+    a.w_off = bl.w13;
+    a.R = 2 * F;
+    a.K = H;
+    a.bimg = w.bx;
+    a.rex = WFMT == MOE_W_NVFP4 ? w.rex_x : nullptr;
+    a.out_h = w.h32;
+    MOE_CUDA_TRY(launch_pdl(ffn_fp4_kernel<WFMT, 1, CFG>, grid, kThreads, smem, st, a));
+    MOE_CUDA_TRY(launch_pdl(fp4_terms_kernel<WFMT, CFG::T, true>, qgrid, kQuantThreads, 0, st,
+                            static_cast<const void*>(w.h32), rows, F, static_cast<const int32_t*>(nullptr), 1,
+                            offsets, slot_of, E, pool_slots, w.boffc, CFG::NT, w.bh, w.rex_h, kNoCanon, kNoCanon));
+    Fp4Args b = a;
+    b.w_off = bl.w2;
+    b.R = H;
+    b.K = F;
+    b.bimg = w.bh;
+    b.rex = WFMT == MOE_W_NVFP4 ? w.rex_h : nullptr;
+    b.out_h = nullptr;
+    b.out_y = y_perm;
+    MOE_CUDA_TRY(launch_pdl(ffn_fp4_kernel<WFMT, 2, CFG>, grid, kThreads, smem, st, b));
+    return MOE_OK;
+}
+
+// Prefill tiles once groups are large (four rows per expert on average);
+// MOE_FFN_TILE=decode|prefill overrides the choice.
+bool use_prefill_tiles(const moe_shape* s, int rows)
+{
+    const char* force = getenv("MOE_FFN_TILE");
+    if (force && !strcmp(force, "decode")) return false;
+    if (force && !strcmp(force, "prefill")) return true;
+    return rows >= 4 * s->experts;
+}
+
+}  // namespace
+
+size_t ffn_fp4_ws_bytes(const moe_shape* s, int rows) { return fp4_ws_layout(s, rows, nullptr, nullptr) + 256; }
+
+int ffn_fp4_device_error(int clear)
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_fp4_error, sizeof v) != cudaSuccess) return MOE_ERR_CUDA;
+    if (clear && v) {
+        int z = 0;
+        if (cudaMemcpyToSymbol(g_fp4_error, &z, sizeof z) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    return v;
+}
+
+int launch_ffn_fp4(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
+                   const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,
+                   cudaStream_t st, const RowSource* gather)
+{
+    Fp4Ws w;
+    fp4_ws_layout(s, rows, ws, &w);
+    int dev = 0, sms = 148;
+    MOE_CUDA_TRY(cudaGetDevice(&dev));
+    MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    const RowSource src = gather ? *gather : RowSource{x_perm, MOE_DT_BF16, nullptr, 1};
+    const BlobLayout bl = blob_layout(s);
+    prof_count(MOE_PROF_FFN, 5);
+    const bool pre = use_prefill_tiles(s, rows);
+    if (s->wfmt == MOE_W_MXFP4)
+        return pre ? run_fp4<MOE_W_MXFP4, PrefillCfg>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, rows,
+                                                      y_perm, w, src, sms, st)
+                   : run_fp4<MOE_W_MXFP4, DecodeCfg>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, rows,
+                                                     y_perm, w, src, sms, st);
+    if (s->wfmt == MOE_W_NVFP4)
+        return pre ? run_fp4<MOE_W_NVFP4, PrefillCfg>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, rows,
+                                                      y_perm, w, src, sms, st)
+                   : run_fp4<MOE_W_NVFP4, DecodeCfg>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, rows,
+                                                     y_perm, w, src, sms, st);
+    return MOE_ERR_INVALID_ARG;
+}
+
+}  // namespace moe
+
+extern "C" int moe_act_terms(const void* d_x, int32_t x_dtype, int32_t rows, int32_t K, int32_t wfmt,
+                             int32_t terms, uint8_t* d_codes, uint8_t* d_scales, int32_t* d_row_exp, void* stream)
+{
+    using namespace moe;
+    if (rows < 0 || K <= 0 || K % 32) return MOE_ERR_INVALID_ARG;
+    if (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
+    if (wfmt != MOE_W_MXFP4 && wfmt != MOE_W_NVFP4) return MOE_ERR_INVALID_ARG;
+    if (terms != 3 && terms != 4) return MOE_ERR_UNSUPPORTED;
+    if (rows == 0) return MOE_OK;
+    if (!d_x || !d_codes || !d_scales || !d_row_exp || ((uintptr_t)d_x & 15)) return MOE_ERR_INVALID_ARG;
+    int dev = 0, sms = 148;
+    MOE_CUDA_TRY(cudaGetDevice(&dev));
+    MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    const int grid = rows < sms * 16 ? rows : sms * 16;
+    cudaStream_t st = as_stream(stream);
+    const bool f32 = x_dtype == MOE_DT_F32;
+#define MOE_TERMS_LAUNCH(W, TT, F)                                                                                 \
+    fp4_terms_kernel<W, TT, F, true><<<grid, kQuantThreads, 0, st>>>(d_x, rows, K, nullptr, 1, nullptr, nullptr, 0, \
+                                                                      0, nullptr, 1, nullptr, d_row_exp, d_codes,  \
+                                                                      d_scales)
+    if (wfmt == MOE_W_MXFP4) {
+        if (terms == 3) { if (f32) MOE_TERMS_LAUNCH(MOE_W_MXFP4, 3, true); else MOE_TERMS_LAUNCH(MOE_W_MXFP4, 3, false); }
+        else { if (f32) MOE_TERMS_LAUNCH(MOE_W_MXFP4, 4, true); else MOE_TERMS_LAUNCH(MOE_W_MXFP4, 4, false); }
+    } else {
+        if (terms == 3) { if (f32) MOE_TERMS_LAUNCH(MOE_W_NVFP4, 3, true); else MOE_TERMS_LAUNCH(MOE_W_NVFP4, 3, false); }
+        else { if (f32) MOE_TERMS_LAUNCH(MOE_W_NVFP4, 4, true); else MOE_TERMS_LAUNCH(MOE_W_NVFP4, 4, false); }
+    }
+#undef MOE_TERMS_LAUNCH
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}

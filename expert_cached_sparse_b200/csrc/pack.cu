@@ -13,7 +13,7 @@
 
 namespace {
 
-// canonical row of packed W13 row p: tile rows 0..7 gate f, 8..15 up f
+// BF16: canonical row of packed W13 row p (tile rows 0..7 gate f, 8..15 up f)
 inline int w13_canon_row(int p, int F)
 {
     int rt = p / 16, r = p % 16;
@@ -21,40 +21,40 @@ inline int w13_canon_row(int p, int F)
     return r < 8 ? f : F + f;
 }
 
-// FP4 tile: lane L = 4g+t holds 8 bytes of row g then 8 of row g+8; its byte
-// p is the row's byte 4p+t of this 64-column block (columns 8p+2t, +1), i.e.
-// bytes 2j and 2j+1 are the mma.sync A-fragment pairs of k16 step j.
-void pack_fp4_matrix(const uint8_t* q, int R, int K, bool w13, int F, uint8_t* out)
+// FP4: canonical row of row r of W13 row block G (per 32 rows: 16 gate rows,
+// then the 16 matching up rows)
+inline int w13_canon_row(int G, int r, int F)
 {
-    const int KT = K / 64;
-    for (int rt = 0; rt < R / 16; rt++)
-        for (int kt = 0; kt < KT; kt++) {
-            uint8_t* tile = out + moe::tile_index(rt, kt, R / 16, KT) * 512;
-            for (int L = 0; L < 32; L++) {
-                int g = L >> 2, t = L & 3;
-                for (int half = 0; half < 2; half++) {
-                    int p = 16 * rt + g + 8 * half;
-                    int cr = w13 ? w13_canon_row(p, F) : p;
-                    const uint8_t* src = q + (size_t)cr * (K / 2) + 32 * kt;
-                    for (int b = 0; b < 8; b++) tile[16 * L + 8 * half + b] = src[4 * b + t];
-                }
-            }
-        }
+    const int q = r / 32, i = r % 32;
+    const int f = 64 * G + 16 * q + (i % 16);
+    return i < 16 ? f : F + f;
 }
 
-void pack_fp4_scales(const uint8_t* sc, int R, int K, bool w13, int F, bool mx, uint8_t* out)
+// FP4 matrix [R][K] (codes two per byte, scales [R][K / vs]) -> chunk images
+// (common.cuh): per 128-row block and 256-column chunk, the rows' code bytes
+// in the 128-byte swizzle, then the unsigned block scales in tensor-memory
+// copy order.  NVFP4 blocks with a negative scale get their codes negated.
+void pack_fp4_matrix(const uint8_t* q, const uint8_t* sc, int R, int K, bool w13, int F, int wfmt, uint8_t* out)
 {
-    const int KT = K / 64, per = mx ? 32 : 16, nb = K / per, bpt = 64 / per, stile = mx ? 32 : 64;
-    for (int rt = 0; rt < R / 16; rt++)
-        for (int kt = 0; kt < KT; kt++) {
-            uint8_t* tile = out + moe::tile_index(rt, kt, R / 16, KT) * stile;
-            for (int g = 0; g < 8; g++)
-                for (int half = 0; half < 2; half++) {
-                    int p = 16 * rt + g + 8 * half;
-                    int cr = w13 ? w13_canon_row(p, F) : p;
-                    for (int b = 0; b < bpt; b++)
-                        tile[2 * bpt * g + bpt * half + b] = sc[(size_t)cr * nb + bpt * kt + b];
+    const bool nv = wfmt == MOE_W_NVFP4;
+    const int vs = nv ? 16 : 32, KC = K / 256, spc = 256 / vs;   // scales per row per chunk
+    const size_t cb = (size_t)moe::fp4_chunk_bytes(wfmt);
+    for (int G = 0; G < R / 128; G++)
+        for (int c = 0; c < KC; c++) {
+            uint8_t* img = out + ((size_t)G * KC + c) * cb;
+            for (int r = 0; r < 128; r++) {
+                const int cr = w13 ? w13_canon_row(G, r, F) : 128 * G + r;
+                const uint8_t* src = q + (size_t)cr * (K / 2) + 128 * c;
+                const uint8_t* srow = sc + (size_t)cr * (K / vs) + (size_t)spc * c;
+                for (int b = 0; b < 128; b++) {
+                    uint8_t v = src[b];
+                    if (nv && (srow[b / 8] & 0x80)) v ^= 0x88;   // 8 bytes per 16-column block
+                    img[1024 * (r / 8) + 128 * (r % 8) + 16 * ((b / 16) ^ (r % 8)) + (b % 16)] = v;
                 }
+                for (int si = 0; si < spc; si++)
+                    img[16384 + 512 * (si / 4) + 16 * (r % 32) + 4 * (r / 32) + (si % 4)] =
+                        nv ? (uint8_t)(srow[si] & 0x7F) : srow[si];
+            }
         }
 }
 
@@ -81,12 +81,11 @@ void pack_bf16_matrix(const uint16_t* w, int R, int K, bool w13, int F, uint8_t*
         }
 }
 
-// E8M0 block scales 2^-13 .. 2^13: E2M1 x scale is then exact in f16 (the
-// tensor-core operand type) as well as in bf16.
+// E8M0 code 255 is NaN; every other code is a finite power of two.
 bool mx_codes_ok(const uint8_t* sc, size_t n)
 {
     for (size_t i = 0; i < n; i++)
-        if (sc[i] < 114 || sc[i] > 140) return false;
+        if (sc[i] == 255) return false;
     return true;
 }
 
@@ -131,10 +130,8 @@ extern "C" int moe_pack_expert(const moe_shape* s, const void* h_w13, const uint
         for (int i = 0; i < 2; i++)
             if (!isfinite(h_tensor_scales[i])) return MOE_ERR_UNSUPPORTED;
     }
-    pack_fp4_matrix(static_cast<const uint8_t*>(h_w13), 2 * F, H, true, F, out + bl.w13);
-    pack_fp4_matrix(static_cast<const uint8_t*>(h_w2), H, F, false, F, out + bl.w2);
-    pack_fp4_scales(h_w13_scales, 2 * F, H, true, F, mx, out + bl.s13);
-    pack_fp4_scales(h_w2_scales, H, F, false, F, mx, out + bl.s2);
+    pack_fp4_matrix(static_cast<const uint8_t*>(h_w13), h_w13_scales, 2 * F, H, true, F, s->wfmt, out + bl.w13);
+    pack_fp4_matrix(static_cast<const uint8_t*>(h_w2), h_w2_scales, H, F, false, F, s->wfmt, out + bl.w2);
     if (!mx) memcpy(out + bl.ts, h_tensor_scales, 2 * sizeof(float));
     return MOE_OK;
 }

@@ -38,8 +38,9 @@
  *    Argument errors are detected on the host before anything is enqueued.
  *  - Row-major everywhere.  Integer tensors are int32.  bf16 tensors are
  *    passed as uint16_t bit patterns.
- *  - Limits: hidden % 64 == 0, ffn % 64 == 0, 1 <= top_k <= experts <= 4096,
- *    capacity <= 8192, layers * experts < 65536.
+ *  - Limits: hidden % 64 == 0, ffn % 64 == 0 (FP4 formats: hidden % 256 ==
+ *    0 and ffn % 256 == 0), 1 <= top_k <= experts <= 4096, capacity <= 8192,
+ *    layers * experts < 65536.
  */
 #ifndef MOE_H
 #define MOE_H
@@ -158,10 +159,14 @@ size_t moe_layer_workspace_bytes(const moe_shape* shape, int32_t n);
  *   (fp32 scales of the whole W13 and W2); other formats ignore it (may be
  *   NULL).  BF16: w13/w2 are uint16 bit patterns, scales NULL.
  * blob_out: moe_slot_bytes(shape) bytes.
- * Errors: MOE_ERR_UNSUPPORTED for NaN scale codes, MXFP4 scale codes
- * outside [114, 140] (block scales 2^-13 .. 2^13, the range in which every
- * E2M1 x scale product is an exact f16 and bf16 number) or non-finite NVFP4
- * tensor scales.
+ * Errors: MOE_ERR_UNSUPPORTED for NaN scale codes (E8M0 255, E4M3
+ * S.1111.111) or non-finite NVFP4 tensor scales.  Every other code is
+ * accepted; a negative NVFP4 block scale is stored as its magnitude with the
+ * block's 16 codes negated (exact).
+ * Pages: the runtime keeps expert banks in its own layout so start-up does
+ * no repacking ("FreeToken linux", section "Prepara los pesos del modelo",
+ * the FTW format); the formats are named in "FreeToken quantization",
+ * section "Formatos compatibles, hardware y perfil de rendimiento".
  */
 int moe_pack_expert(const moe_shape* shape, const void* h_w13, const uint8_t* h_w13_scales,
                     const void* h_w2, const uint8_t* h_w2_scales, const float* h_tensor_scales,
@@ -170,7 +175,10 @@ int moe_pack_expert(const moe_shape* shape, const void* h_w13, const uint8_t* h_
 /* ---------------------------------------------------------------- cache */
 
 /*
- * Creates a cache of `capacity` slots over the caller's device memory:
+ * Creates a cache of `capacity` slots over the caller's device memory
+ * (pages: VRAM holds expert slots used as an LRU cache shared across MoE
+ * layers while the full expert set stays in host RAM, "FreeToken linux",
+ * section "Como gestiona FreeToken la memoria MoE"):
  *   d_meta: moe_cache_meta_bytes() bytes, 256-byte aligned;
  *   d_slot_pool: capacity * moe_slot_bytes() bytes, 256-byte aligned;
  *   h_blobs: layers*experts pointers, h_blobs[l*E+e] = packed blob of expert
@@ -205,6 +213,11 @@ int moe_cache_create(const moe_shape* shape, void* d_meta, size_t meta_bytes, vo
  * `layer` is already resident (then nothing is read back).
  * MOE_ERR_CAPACITY if more distinct experts are requested than slots exist;
  * the state is unchanged (the host learns this at the same sync point).
+ * Pages: hits run directly on the GPU and misses are brought in ("FreeToken
+ * 290b model", section "Como gestiona FreeToken el prellenado y la
+ * decodificacion"); a cache entry is a logical (layer, expert) pair
+ * ("FreeToken rtx 4090", section "Como funciona la jerarquia de memoria
+ * MoE").
  */
 int moe_cache_lookup_update(moe_cache* cache, int32_t layer, const int32_t* d_idx, int32_t count,
                             int32_t* d_slot_of_expert, void* stream, void* copy_stream);
@@ -216,6 +229,9 @@ int moe_cache_lookup_update(moe_cache* cache, int32_t layer, const int32_t* d_id
  * d_pool_new, and moves the bookkeeping to d_meta_new (either may equal the
  * old buffer when large enough; the survivors only ever move to lower
  * slots, so an in-place pool works).  Emits EVICT / MOVE trace records.
+ * Pages: the cache is rebuilt at scheduler safe points ("FreeToken
+ * quantization", section "Flujo de configuracion de la cuantizacion de
+ * FreeToken").
  */
 int moe_cache_resize(moe_cache* cache, void* d_meta_new, size_t meta_bytes, void* d_pool_new,
                      int32_t new_capacity, void* stream);
@@ -251,6 +267,10 @@ int moe_cache_destroy(moe_cache* cache);
  *   all experts renormalised over the top-k).
  * d_logits [n][experts] float32 is scratch the caller provides, and holds
  * the logits afterwards.
+ * Pages: each token is sent to a few of a layer's routed experts (6 of 256
+ * for DeepSeek-V4-Flash, "FreeToken linux", section "Como gestiona
+ * FreeToken la memoria MoE"); the softmax / top-k / renormalisation reading
+ * is this library's (the pages print no formula).
  */
 int moe_router_topk(const void* d_x, int32_t x_dtype, const uint16_t* d_wg, const float* d_bias,
                     int32_t n, int32_t hidden, int32_t experts, int32_t k, float* d_logits,
@@ -266,6 +286,8 @@ int moe_router_topk(const void* d_x, int32_t x_dtype, const uint16_t* d_wg, cons
  * moe_permute_workspace_bytes() bytes.  An index outside [0, experts) is
  * the caller's error: that assignment gets row_of = -1 and no row, and
  * offsets[experts] counts only the valid ones.
+ * Pages: no passage; the step that groups each expert's tokens so the
+ * experts run as a grouped GEMM.
  */
 int moe_permute(const int32_t* d_topk_idx, int32_t n, int32_t experts, int32_t k, const void* d_x,
                 int32_t x_dtype, int32_t hidden, int32_t* d_expert_offsets, int32_t* d_row_of,
@@ -309,18 +331,22 @@ int moe_permute_noalloc(const int32_t* d_topk_idx, int32_t n, int32_t experts, i
  *   y = h W2^T                    (fp32 accumulation, y rounded to bf16)
  * is written to d_y_perm rows.  Rows of experts with any other slot value
  * (-1 in particular), or whose range does not lie inside [0, rows), are left
- * untouched, so hits and misses can run as two passes.  d_ws: moe_ffn_workspace_bytes() bytes (operand copies of x and
- * h, h itself, and the partial sums of work split across CTAs).  The MMAs
- * take f16 operands: FP4 weights are expanded exactly (E2M1 times its block
- * scale is exact in f16 for the accepted scale codes), x and h rows are
- * scaled by a power of two so their largest magnitude lands in [2^14, 2^15)
- * (exact for bf16 x, 11 significant bits for h); the row scale and the
- * NVFP4 tensor scales are undone in fp32.  Results are deterministic: the
- * same inputs give the same bits on every call.
- * Kernel choice: FP4 formats with at least 4 rows per expert on average run
- * the tcgen05 grouped GEMM, everything else the weight-streaming kernels;
- * the environment variable MOE_FFN_PATH=mma or =tc forces one of them (read
- * at every call; intended for testing).
+ * untouched, so hits and misses can run as two passes.
+ * d_ws: moe_ffn_workspace_bytes() bytes.
+ * FP4 weights (MXFP4, NVFP4) run on the block-scaled tensor cores: the E2M1
+ * weights and their block scales are multiplied as stored; each x and h row
+ * is first written as T E2M1 terms with block scales of the weights' scale
+ * type (moe_act_terms: T = 4 when the call has few rows per expert, 3 when
+ * it averages at least 4; relative error about 2e-4 and 2e-3 per row), the
+ * terms' products are summed in fp32, and the NVFP4 row and tensor scales
+ * are undone in fp32.  BF16 weights run on bf16 MMAs with x and h rounded to
+ * bf16.  Results are deterministic: the same inputs give the same bits on
+ * every call.  MOE_FFN_TILE=decode or =prefill forces the FP4 tile shape
+ * (read at every call; intended for testing).
+ * Pages: experts found in VRAM execute on the GPU ("FreeToken
+ * quantization", section "Como se desplazan los pesos MoE cuantizados por la
+ * memoria"); SwiGLU is this library's reading (the pages name no
+ * activation).
  */
 int moe_grouped_ffn(const moe_shape* shape, const void* d_slot_pool, int32_t pool_slots,
                     const int32_t* d_slot_of_expert, const int32_t* d_expert_offsets,
@@ -331,6 +357,7 @@ int moe_grouped_ffn(const moe_shape* shape, const void* d_slot_pool, int32_t poo
  * Combine.  out[t] = sum over j = 0..k-1, in that order, of
  * w[t][j] * y_perm[row_of[t*k+j]], accumulated in fp32 and stored as
  * out_dtype.  Deterministic (no atomics).
+ * Pages: no passage; the gate-weighted sum of a routed MoE layer.
  */
 int moe_combine(const uint16_t* d_y_perm, const int32_t* d_row_of, const float* d_topk_w, int32_t n,
                 int32_t k, int32_t hidden, void* d_out, int32_t out_dtype, void* stream);
@@ -345,11 +372,39 @@ int moe_combine(const uint16_t* d_y_perm, const int32_t* d_row_of, const float* 
  * Blocks the host once, for the miss list, unless every expert of the layer
  * is resident; in that case nothing is read back and the call can be
  * captured in a CUDA graph.
+ * Pages: hits execute on the GPU while misses are brought in ("FreeToken
+ * 290b model", section "Como gestiona FreeToken el prellenado y la
+ * decodificacion"); data movement overlaps computation ("FreeToken linux",
+ * mechanism table in section "Como gestiona FreeToken la memoria MoE").
  */
 int moe_layer_forward(moe_cache* cache, int32_t layer, const void* d_x, int32_t x_dtype,
                       const uint16_t* d_wg, const float* d_bias, int32_t n, void* d_out,
                       void* d_ws, size_t ws_bytes, void* stream, void* copy_stream,
                       int32_t* d_topk_idx_out, float* d_topk_w_out);
+
+/*
+ * The operand encoding the FP4 grouped FFN applies to its activation rows,
+ * exposed for inspection and testing: d_x [rows][K] (x_dtype, K % 32 == 0,
+ * 16-byte aligned).  For wfmt MXFP4 every 32-column block, for NVFP4 every
+ * 16-column block, is written as `terms` (3 or 4) E2M1 terms, each with its
+ * own block scale (E8M0, resp. unsigned E4M3): term t takes the smallest
+ * scale s of the format with 6 s >= the block's largest remaining
+ * magnitude m (E8M0 codes 1..254; E4M3 codes 1..0x7E against m / 6 in
+ * fp32; code 127 / 0x38 when m is 0), the E2M1 code nearest to r / s (ties
+ * to the even code) for each element, and leaves r - e2m1 * s to the next
+ * term, all in fp32.  NVFP4 rows are first multiplied by 2^p with 2^p times
+ * the row's largest magnitude in [2^10, 2^11) (p clamped to [-100, 100]).
+ * Outputs (device): d_codes [rows][terms][K] one code per byte,
+ * d_scales [rows][terms][K / vs] scale codes, d_row_exp [rows] p (0 for
+ * MXFP4).  Row i is 2^-p sum_t e2m1(codes) * scale.  Errors:
+ * MOE_ERR_INVALID_ARG for bad sizes, dtypes or pointers, MOE_ERR_UNSUPPORTED
+ * for other term counts.
+ * Pages: none; the pages name the weight formats ("FreeToken quantization",
+ * section "Formatos compatibles, hardware y perfil de rendimiento"), this
+ * encoding is how this library feeds them to FP4 tensor cores.
+ */
+int moe_act_terms(const void* d_x, int32_t x_dtype, int32_t rows, int32_t K, int32_t wfmt, int32_t terms,
+                  uint8_t* d_codes, uint8_t* d_scales, int32_t* d_row_exp, void* stream);
 
 /* ---------------------------------------------------------------- profiling */
 

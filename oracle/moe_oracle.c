@@ -126,6 +126,103 @@ void orc_dequant_bf16(const uint16_t* w, size_t count, double* out)
 }
 
 /* ------------------------------------------------------------------ */
+/* activation terms: the operand encoding of the FP4 tensor-core path   */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The FP4 tensor cores multiply E2M1 values with a block scale on both
+ * operands, so the GPU path writes each activation row as a short sum of
+ * E2M1 terms.  The pages name the weight formats only ("FreeToken
+ * quantization", "Formatos compatibles, hardware y perfil de rendimiento");
+ * this encoding is the library's own, and what it must match is stated
+ * here, step by step, in fp32 with one rounding per operation:
+ *
+ *  - blocks of vs columns: vs = 32 with E8M0 scales (MXFP4 weights), vs = 16
+ *    with unsigned E4M3 scales (NVFP4 weights);
+ *  - NVFP4 only: the row is first multiplied by 2^p, p the integer with
+ *    2^10 <= 2^p max|x| < 2^11 (p = 0 for an all-zero row), clamped to
+ *    [-100, 100];
+ *  - each block starts with r = x; term t = 0..T-1 takes m = max |r|, the
+ *    scale s = the smallest positive value of the scale format with
+ *    6 s >= m (E8M0: codes 1..254; E4M3: codes 1..0x7E, against m / 6
+ *    rounded to fp32; the largest code if none qualifies), or code 127
+ *    (E8M0) / 0x38 (E4M3) when m is 0; then for each element the E2M1 code
+ *    nearest to r / s (ties to the code with an even mantissa bit, +0 for
+ *    zero), and r <- r - e2m1(code) * s.
+ *
+ * codes: [T][K] one E2M1 code per byte; scales: [T][K / vs] scale codes;
+ * *p_out: the row exponent.  Brute-force searches throughout.
+ */
+static int e2m1_nearest_code(float x)
+{
+    const float a = fabsf(x);
+    int best = 0;
+    float bd = INFINITY;
+    for (int c = 0; c < 8; c++) {
+        const float d = fabsf(a - (float)orc_e2m1(c));
+        if (d < bd || (d == bd && (c & 1) == 0)) {
+            bd = d;
+            best = c;
+        }
+    }
+    if (x < 0.0f && best != 0) best |= 8;
+    return best;
+}
+
+static int term_scale_code(int wfmt, float m)
+{
+    if (!(m > 0.0f)) return wfmt == 1 ? 127 : 0x38;
+    if (wfmt == 1) {
+        for (int c = 1; c <= 254; c++)
+            if (6.0 * orc_e8m0(c) >= (double)m) return c;
+        return 254;
+    }
+    const float target = m / 6.0f;
+    for (int c = 1; c <= 0x7E; c++)
+        if ((float)orc_e4m3(c) >= target) return c;
+    return 0x7E;
+}
+
+int orc_act_terms(const float* x, int K, int wfmt, int T, uint8_t* codes, uint8_t* scales, int* p_out)
+{
+    if (K <= 0 || T <= 0 || (wfmt != 1 && wfmt != 2)) return ORC_ERR_ARG;
+    const int vs = wfmt == 1 ? 32 : 16;
+    if (K % vs) return ORC_ERR_ARG;
+    int p = 0;
+    if (wfmt == 2) {
+        float mx = 0.0f;
+        for (int i = 0; i < K; i++) mx = fmaxf(mx, fabsf(x[i]));
+        if (mx > 0.0f && mx <= 3.4e38f) {
+            p = 0;
+            while (ldexp((double)mx, p) >= 2048.0) p--;
+            while (ldexp((double)mx, p) < 1024.0) p++;
+            if (p < -100) p = -100;
+            if (p > 100) p = 100;
+        }
+    }
+    *p_out = p;
+    const float sc = (float)ldexp(1.0, p);
+    float r[32];
+    for (int b = 0; b < K / vs; b++) {
+        for (int i = 0; i < vs; i++) r[i] = wfmt == 2 ? x[b * vs + i] * sc : x[b * vs + i];
+        for (int t = 0; t < T; t++) {
+            float m = 0.0f;
+            for (int i = 0; i < vs; i++) m = fmaxf(m, fabsf(r[i]));
+            const int sc_code = term_scale_code(wfmt, m);
+            const float s = m > 0.0f ? (float)(wfmt == 1 ? orc_e8m0(sc_code) : orc_e4m3(sc_code)) : 1.0f;
+            scales[(size_t)t * (K / vs) + b] = (uint8_t)sc_code;
+            for (int i = 0; i < vs; i++) {
+                const int q = e2m1_nearest_code(r[i] / s);
+                codes[(size_t)t * K + b * vs + i] = (uint8_t)q;
+                const float qs = (float)orc_e2m1(q) * s;
+                r[i] = r[i] - qs;
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
 /* router: logits, top-k, renormalised softmax weights                 */
 /* ------------------------------------------------------------------ */
 

@@ -70,6 +70,7 @@ def lib():
         L.orc_permute.argtypes = [P, i32, i32, i32, P, P, P]
         L.orc_expert_ffn.argtypes = [P, P, i32, i32, P, P]
         L.orc_combine.argtypes = [P, P, i32, i32, i32, P]
+        L.orc_act_terms.argtypes = [P, i32, i32, i32, P, P, P]
         _lib = L
     return _lib
 
@@ -121,6 +122,31 @@ def dequant_expert(wfmt: int, ew, hidden: int, ffn: int):
     w13 = dequant_matrix(wfmt, ew.w13, ew.w13_scales, ew.tensor_scales[0], 2 * ffn, hidden)
     w2 = dequant_matrix(wfmt, ew.w2, ew.w2_scales, ew.tensor_scales[1], hidden, ffn)
     return w13, w2
+
+
+# ------------------------------------------------------------------ activation terms
+def act_terms(x, wfmt: int, terms: int):
+    """Rows of activations (float32, or bf16 bits) as sums of E2M1 terms.
+
+    Returns (codes uint8 [n, T, K], scales uint8 [n, T, K/vs], p int32 [n]):
+    row i is approximately 2^-p[i] * sum_t e2m1(codes[i, t]) * scale(scales[i, t]).
+    """
+    xf = as_f32(np.atleast_2d(x))
+    n, k = xf.shape
+    vs = 32 if wfmt == 1 else 16
+    codes = np.empty((n, terms, k), np.uint8)
+    scales = np.empty((n, terms, k // vs), np.uint8)
+    p = np.empty(n, np.int32)
+    pi = C.c_int(0)
+    for i in range(n):
+        row = np.ascontiguousarray(xf[i])
+        c = np.empty((terms, k), np.uint8)
+        s = np.empty((terms, k // vs), np.uint8)
+        rc = lib().orc_act_terms(_p(row), k, wfmt, terms, _p(c), _p(s), C.byref(pi))
+        if rc:
+            raise ValueError(f"orc_act_terms: {rc}")
+        codes[i], scales[i], p[i] = c, s, pi.value
+    return codes, scales, p
 
 
 # ------------------------------------------------------------------ router

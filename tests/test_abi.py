@@ -68,15 +68,17 @@ def test_workspace_sizes_grow_with_tokens():
 
 
 def test_pack_rejects_bad_scale_codes():
-    cfg = W.scaled(W.DS_DECODE, hidden=128, ffn=64, experts=4, top_k=2)
+    cfg = W.scaled(W.DS_DECODE, hidden=256, ffn=256, experts=4, top_k=2)
     s = A.shape_of(cfg)
     ew = W.gen_expert(cfg, 0, 0, 0)
     A.moe_pack_expert(s, ew)   # valid
-    ew.w13_scales[3, 1] = 150  # 2^23: outside the supported block-scale range
+    ew.w13_scales[3, 1] = 150  # 2^23: any finite E8M0 code is accepted
+    A.moe_pack_expert(s, ew)
+    ew.w13_scales[3, 1] = 255  # E8M0 NaN
     with pytest.raises(A.MoeError) as e:
         A.moe_pack_expert(s, ew)
     assert e.value.code == L.MOE_ERR_UNSUPPORTED
-    cfg2 = W.scaled(W.TRACE40, layers=1, hidden=128, ffn=64, experts=4, top_k=2)
+    cfg2 = W.scaled(W.TRACE40, layers=1, hidden=256, ffn=256, experts=4, top_k=2)
     s2 = A.shape_of(cfg2)
     ew2 = W.gen_expert(cfg2, 0, 0, 0)
     A.moe_pack_expert(s2, ew2)
@@ -87,7 +89,7 @@ def test_pack_rejects_bad_scale_codes():
 
 def test_pack_is_a_byte_permutation_fp4():
     """FP4 packing moves whole bytes (nibble pairs) and scale bytes; nothing is lost."""
-    cfg = W.scaled(W.DS_DECODE, hidden=128, ffn=64, experts=4, top_k=2)
+    cfg = W.scaled(W.DS_DECODE, hidden=256, ffn=256, experts=4, top_k=2)
     s = A.shape_of(cfg)
     ew = W.gen_expert(cfg, 1, 0, 2)
     blob = A.moe_pack_expert(s, ew)

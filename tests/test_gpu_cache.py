@@ -53,7 +53,7 @@ def _requests(rng, cfg, steps):
 
 
 def test_trace_and_state_match_oracle(orc):
-    cfg = W.scaled(W.DS_DECODE, layers=3, experts=16, hidden=64, ffn=64, top_k=3, capacity=10)
+    cfg = W.scaled(W.DS_DECODE, layers=3, experts=16, hidden=256, ffn=256, top_k=3, capacity=10)
     L = Layer(cfg, 0)
     cache = make_cache(L)
     lru = orc.Lru(cfg.layers, cfg.experts, cfg.capacity)
@@ -81,7 +81,7 @@ def test_trace_and_state_match_oracle(orc):
 
 
 def test_capacity_error_changes_nothing(orc):
-    cfg = W.scaled(W.DS_DECODE, layers=2, experts=16, hidden=64, ffn=64, top_k=2, capacity=4)
+    cfg = W.scaled(W.DS_DECODE, layers=2, experts=16, hidden=256, ffn=256, top_k=2, capacity=4)
     L = Layer(cfg, 0)
     cache = make_cache(L)
     cs = torch.cuda.Stream()
@@ -102,7 +102,7 @@ def test_capacity_error_changes_nothing(orc):
 
 @pytest.mark.parametrize("in_place", [False, True])
 def test_resize_matches_oracle(orc, in_place):
-    cfg = W.scaled(W.DS_DECODE, layers=2, experts=24, hidden=64, ffn=64, top_k=2, capacity=12)
+    cfg = W.scaled(W.DS_DECODE, layers=2, experts=24, hidden=256, ffn=256, top_k=2, capacity=12)
     L = Layer(cfg, 0)
     cache = make_cache(L)
     lru = orc.Lru(cfg.layers, cfg.experts, cfg.capacity)
@@ -131,7 +131,7 @@ def test_resize_matches_oracle(orc, in_place):
 
 def test_trace40_scale_lru(orc):
     """The 40-layer, 1024-slot cache at full size: 256 steps x 40 layers of 6 experts each."""
-    cfg = W.scaled(W.TRACE40, hidden=64, ffn=64)   # tiny blobs, full cache geometry
+    cfg = W.scaled(W.TRACE40, hidden=256, ffn=256)   # tiny blobs, full cache geometry
     L = Layer(cfg, 0, distinct=32)
     cache = make_cache(L, trace_capacity=1 << 20)
     lru = orc.Lru(cfg.layers, cfg.experts, cfg.capacity)
@@ -158,7 +158,7 @@ def test_trace40_scale_lru(orc):
 
 
 def test_injected_fill_failure_is_rolled_back(orc, monkeypatch):
-    cfg = W.scaled(W.DS_DECODE, layers=1, experts=8, hidden=64, ffn=64, top_k=2, capacity=4)
+    cfg = W.scaled(W.DS_DECODE, layers=1, experts=8, hidden=256, ffn=256, top_k=2, capacity=4)
     L = Layer(cfg, 0)
     monkeypatch.setenv("MOE_FAULT_INJECT", "fill_fail:3")
     cache = make_cache(L)

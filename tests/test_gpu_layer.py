@@ -183,7 +183,7 @@ def test_resident_layer_replays_from_a_cuda_graph(orc):
     """With every expert of the layer resident, moe_layer_forward reads
     nothing back to the host, so a whole layer step can be captured in a CUDA
     graph and replayed; replays with fresh inputs match eager calls exactly."""
-    cfg = W.scaled(W.DS_DECODE, experts=16, hidden=256, ffn=128, top_k=4, capacity=16)
+    cfg = W.scaled(W.DS_DECODE, experts=16, hidden=256, ffn=256, top_k=4, capacity=16)
     R = Runner(cfg)
     preload(R.cache, cfg)
     wg, bias = R.router(0)

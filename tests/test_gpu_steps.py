@@ -146,7 +146,7 @@ def _ffn_case(orc, cfg, counts, slots, pool_slots, seed=0, passes=1):
     return worst
 
 
-SMALL = dict(hidden=256, ffn=128, experts=8, top_k=2, layers=1)
+SMALL = dict(hidden=256, ffn=256, experts=8, top_k=2, layers=1)
 
 
 @pytest.mark.parametrize("base", [W.TINY, W.DS_DECODE, W.TRACE40], ids=["bf16", "mxfp4", "nvfp4"])
@@ -172,11 +172,11 @@ def test_grouped_ffn_full_size(orc, base):
 @pytest.mark.parametrize("base", [W.DS_DECODE, W.TRACE40, W.QWEN_BF16], ids=["mxfp4", "nvfp4", "bf16"])
 @pytest.mark.parametrize("passes", [1, 2])
 def test_grouped_ffn_split_k(orc, base, passes, monkeypatch):
-    """Full expert shapes with fewer work units than CTAs: the streaming
-    kernels cut the units' K stages into equal ranges over the CTAs and add the
-    pieces up; rows of a skipped expert stay untouched, and a second pass over
-    the other experts keeps the first's."""
-    monkeypatch.setenv("MOE_FFN_PATH", "mma")
+    """Full expert shapes with decode tiles: the units' K chunks are cut into
+    equal ranges over the CTAs and the pieces added up; rows of a skipped
+    expert stay untouched, and a second pass over the other experts keeps the
+    first's."""
+    monkeypatch.setenv("MOE_FFN_TILE", "decode")
     cfg = W.scaled(base, experts=6, top_k=2, layers=1)
     counts = [1, 3, 2, 9, 0, 1]
     slots = [4, -1, 0, 2, 5, 3]
@@ -190,6 +190,36 @@ def test_grouped_ffn_slot_out_of_range_is_skipped(orc):
     counts = [2, 2, 0, 0, 0, 0, 0, 1]
     slots = [0, 50, -1, -1, -1, -1, -1, 1]   # 50 >= pool_slots: skipped, not read
     _ffn_case(orc, cfg, counts, slots, pool_slots=2)
+
+
+# ------------------------------------------------------------------ activation terms
+@pytest.mark.parametrize("xd", ["bf16", "f32"])
+@pytest.mark.parametrize("terms", [3, 4])
+@pytest.mark.parametrize("wfmt", [W.W_MXFP4, W.W_NVFP4], ids=["mxfp4", "nvfp4"])
+def test_act_terms_bit_exact(orc, wfmt, terms, xd):
+    """The FP4 path's activation encoding (codes, block scales, row exponent)
+    is bit-exact with the oracle's: both take every rounding decision in fp32."""
+    rng = np.random.default_rng(10 * wfmt + terms)
+    n, K = 12, 1024
+    x = rng.standard_normal((n, K)).astype(np.float32)
+    x[1] *= np.float32(1e-6)
+    x[2] *= np.float32(1e5)
+    x[3, ::3] = 0.0
+    x[4] = np.round(x[4] * 4) / 4                     # exact ties on the grids
+    x[5] = 0.0
+    x[6] = (rng.standard_normal(K) * 3).astype(np.float32) ** 3   # heavy tails, like h
+    x[7, :512] *= np.float32(1e-4)                    # blocks far below the row maximum
+    xo = W.f32_to_bf16_bits(x) if xd == "bf16" else x
+    vs = 32 if wfmt == W.W_MXFP4 else 16
+    codes = torch.empty(n, terms, K, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(n, terms, K // vs, dtype=torch.uint8, device="cuda")
+    rex = torch.empty(n, dtype=torch.int32, device="cuda")
+    A.moe_act_terms(dev(xo), n, K, wfmt, terms, codes, scales, rex)
+    torch.cuda.synchronize()
+    c_ref, s_ref, p_ref = orc.act_terms(xo, wfmt, terms)
+    np.testing.assert_array_equal(host(rex), p_ref)
+    np.testing.assert_array_equal(host(scales), s_ref)
+    np.testing.assert_array_equal(host(codes), c_ref)
 
 
 # ------------------------------------------------------------------ combine
@@ -216,19 +246,21 @@ def test_combine_parity(orc, n, k, H, out):
 
 
 TC_CASES = {
-    # ragged groups, an expert of 300 rows (two token blocks) and one of 256
+    # ragged groups, an expert of 300 rows (five token groups) and one of 256
     "ragged": ([0, 1, 17, 300, 33, 70, 3, 256], [3, 9, 0, 4, 5, 2, 7, 1]),
-    # token-block boundaries: one full block, one row over, two full blocks, one over
-    "block_edges": ([192, 193, 384, 385, 16, 15, 1, 0], [1, 0, 3, 2, 5, 4, 7, 6]),
+    # token-group boundaries: one full group, one row over, two full groups, one over
+    "block_edges": ([64, 65, 128, 129, 16, 15, 1, 0], [1, 0, 3, 2, 5, 4, 7, 6]),
 }
 
 
 @pytest.mark.parametrize("case", sorted(TC_CASES))
 @pytest.mark.parametrize("base", [W.DS_DECODE, W.TRACE40], ids=["mxfp4", "nvfp4"])
-def test_grouped_ffn_tensor_core_path(orc, base, case, monkeypatch):
-    """The tcgen05 grouped GEMM (prefill path), forced on small shapes."""
-    monkeypatch.setenv("MOE_FFN_PATH", "tc")
-    cfg = W.scaled(base, hidden=256, ffn=128, experts=8, top_k=2, layers=1)
+def test_grouped_ffn_prefill_tiles(orc, base, case, monkeypatch):
+    """The block-scaled grouped GEMM with prefill tiles (64 tokens x 3 terms per
+    tile, whole units), forced on small shapes: ragged groups, several token
+    groups per expert, and group sizes on and around the tile edge."""
+    monkeypatch.setenv("MOE_FFN_TILE", "prefill")
+    cfg = W.scaled(base, hidden=256, ffn=256, experts=8, top_k=2, layers=1)
     counts, slots = TC_CASES[case]
     worst = _ffn_case(orc, cfg, counts, slots, pool_slots=10, seed=11)
     assert worst < ALARM_REL_L2, worst
@@ -238,7 +270,7 @@ def test_grouped_ffn_tensor_core_path(orc, base, case, monkeypatch):
 # ------------------------------------------------------------------ self-consistency
 def _ffn_run(cfg, blobs, counts, xb, path, monkeypatch):
     """y of one moe_grouped_ffn call with expert e in slot e (blobs: host uint8 arrays)."""
-    monkeypatch.setenv("MOE_FFN_PATH", path)
+    monkeypatch.setenv("MOE_FFN_TILE", path)
     shape = A.shape_of(cfg)
     sb = A.moe_slot_bytes(shape)
     pool = torch.from_numpy(np.concatenate(blobs)).to("cuda")
@@ -254,8 +286,8 @@ def _ffn_run(cfg, blobs, counts, xb, path, monkeypatch):
     return y.view(torch.int16).cpu().numpy()
 
 
-@pytest.mark.parametrize("path,counts", [("mma", [1, 3, 2, 9, 0, 1]), ("tc", [40, 3, 200, 9, 0, 70])],
-                         ids=["streaming", "tensor_core"])
+@pytest.mark.parametrize("path,counts", [("decode", [1, 3, 2, 9, 0, 1]), ("prefill", [40, 3, 200, 9, 0, 70])],
+                         ids=["decode_tiles", "prefill_tiles"])
 def test_ffn_is_deterministic_and_scale_exact(path, counts, monkeypatch):
     """Two calls on the same inputs give the same bits (no atomics in any sum),
     and raising every W2 block-scale code by one doubles y exactly (power-of-two
