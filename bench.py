@@ -206,7 +206,7 @@ class DecodeStream:
 # stream, summed over the call's kernels (operand preps and both projections)
 # and averaged over the calls of an ncu capture of that workload.  Valid only
 # for the FFN code it was measured on (comments aside): other code reports null.
-FFN_TRAFFIC = {"source_sha1": "143f05209e80d8a0e7fb9735c80bce06b7535686", "bytes_per_call": 205387936}
+FFN_TRAFFIC = {"source_sha1": None, "bytes_per_call": None}
 
 
 def ffn_source_sha1():
@@ -214,7 +214,7 @@ def ffn_source_sha1():
     the traffic was measured on; comment edits do not change it)."""
     import hashlib
     import re
-    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "expert_cached_sparse_b200", "csrc", "ffn.cu")
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "expert_cached_sparse_b200", "csrc", "ffn_fp4.cu")
     with open(path) as f:
         src = f.read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
@@ -393,7 +393,7 @@ def run_ours(args, cfg, world, rank, local_rank):
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": Wm,
             "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic", "config": workload_config(cfg, n, world)}
-    line["roofline"] = {"kernel": "grouped SwiGLU FFN (ffn_kernel gate-up + down, weight streaming)",
+    line["roofline"] = {"kernel": "grouped SwiGLU FFN (ffn_fp4_kernel gate-up + down, block-scaled tcgen05)",
                         "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                         "frac": achieved / hbm_peak, "peak_kind": peak_kind, "traffic": ffn_traffic(),
                         "algorithmic_bytes_per_call": ffn_bytes / ffn_calls,

@@ -47,7 +47,7 @@ namespace {
 
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 32 * (2 + kEpiWarps);
-constexpr int kQuantThreads = 128;
+constexpr int kQuantThreads = 256;
 constexpr long long kWaitCycles = 4000000000ll;   // ~2 s before a wait gives up
 constexpr int kMaxCtas = 160;                      // persistent grid: one CTA per SM at most
 constexpr int kSmemBudget = 227 * 1024;
@@ -137,6 +137,12 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                  ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
+// Fire-and-forget bulk prefetch of global memory into L2.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_commit(uint32_t bar)
@@ -158,11 +164,11 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t addr)
            ((uint64_t)1 << 46);
 }
 
-// 512-byte scale image -> 4 tensor-memory columns of all 128 lanes (the
-// 32-lane pattern is replicated into the four lane quarters).
-__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint32_t saddr)
+// One 512-byte scale image (descriptor d) -> 4 tensor-memory columns of all
+// 128 lanes (the 32-lane pattern is replicated into the four lane quarters).
+__device__ __forceinline__ void tc_cp_sf_d(uint32_t taddr, uint64_t desc)
 {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc_sf(saddr)) : "memory");
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc));
 }
 
 // D[tmem] (+)= A[smem] * B[smem], E2M1 operands with block scales from tensor memory.
@@ -173,11 +179,11 @@ __device__ __forceinline__ void tc_mma_fp4(uint32_t d, uint64_t a, uint64_t b, u
     if (WFMT == MOE_W_MXFP4)
         asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
                      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-                     ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb) : "memory");
+                     ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
     else
         asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
                      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-                     ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb) : "memory");
+                     ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
 }
 
 // Instruction descriptor (block-scaled kinds): E2M1 A and B, K-major, M = 128,
@@ -220,9 +226,11 @@ __device__ __forceinline__ uint32_t term_scale(float m, float& sval)
         return WFMT == MOE_W_MXFP4 ? 127u : 0x38u;
     }
     if (WFMT == MOE_W_MXFP4) {
-        int E;
-        const float f = frexpf(m, &E);            // m = f 2^E, f in [0.5, 1)
-        int code = (f > 0.75f ? E - 2 : E - 3) + 127;   // 6 * 2^(code-127) >= m, minimal
+        // m = f 2^E with f in [0.5, 1): E = biased exponent - 126, f > 0.75
+        // exactly when the mantissa exceeds 2^22; 6 * 2^(code-127) >= m is
+        // then minimal for code = E - 2 (f > 0.75) or E - 3, plus 127
+        const uint32_t b = __float_as_uint(m);
+        int code = (int)(b >> 23) + ((b & 0x7FFFFF) > 0x400000 ? -1 : -2);
         code = code < 1 ? 1 : (code > 254 ? 254 : code);
         sval = __uint_as_float((uint32_t)code << 23);
         return (uint32_t)code;
@@ -245,20 +253,26 @@ __device__ __forceinline__ uint32_t term_scale(float m, float& sval)
     return code;
 }
 
-// Nearest E2M1 code of x (ties to the even code), |x| <= 6 expected.
-__device__ __forceinline__ uint32_t e2m1_code(float x)
+// Nearest E2M1 value of x, ties to the even code (NaN -> 0): returns the
+// code and leaves the value in *q.  |x| is rounded to the E2M1 grid by
+// adding and removing a power of two whose ulp is the grid step there (0.5
+// below 2, 1 below 4, 2 above), which rounds to the nearest even multiple
+// exactly like the even-code rule; the code is read off the result's
+// exponent and top mantissa bit (0.5 and 0 by hand).
+__device__ __forceinline__ uint32_t e2m1_round(float x, float* q)
 {
     const float a = fabsf(x);
-    uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) + (a >= 3.5f) + (a > 5.0f);
-    if (x < 0.0f && c) c |= 8u;
-    return c;
+    const float c = a < 2.0f ? 4194304.0f : (a < 4.0f ? 8388608.0f : 16777216.0f);
+    float v = fminf(__fsub_rn(__fadd_rn(a, c), c), 6.0f);
+    v = a == a ? v : 0.0f;
+    const uint32_t b = __float_as_uint(v);
+    uint32_t code = v >= 1.0f ? (b >> 22) - 252u : (v > 0.0f ? 1u : 0u);
+    if (x < 0.0f && code) code |= 8u;
+    *q = copysignf(v, x);
+    return code;
 }
 
-__device__ __forceinline__ float e2m1_val(uint32_t c)
-{
-    const float mag = (c & 7) < 4 ? 0.5f * (float)(c & 7) : (float)(1 << (((c & 7) >> 1) - 1)) * (((c & 1) ? 1.5f : 1.0f));
-    return (c & 8) ? -mag : mag;
-}
+
 
 // Per-chunk bytes of a token group's operand image with n rows (n multiple of 8).
 __host__ __device__ __forceinline__ int b_chunk_bytes(int n, int nsub)
@@ -275,11 +289,14 @@ struct Fmt {
 
 // The plan of one call: for every expert e with rows and a slot in the pool,
 // its token groups (of NT rows) are numbered from gpre[e]; the per-chunk
-// bytes of their operand images are summed in boffc (in expert order).
+// bytes of their operand images are summed in boffc (in expert order); and
+// group g's entry gtab[g] = {first row, rows, slot, per-chunk byte offset of
+// its operand image} lets the GEMM find a unit with one load.
 __global__ void __launch_bounds__(256) fp4_plan_kernel(const int32_t* __restrict__ offsets,
                                                        const int32_t* __restrict__ slot_of, int E, int rows,
                                                        int pool_slots, int NT, int T, int nsub,
                                                        int32_t* __restrict__ gpre, int32_t* __restrict__ boffc,
+                                                       int4* __restrict__ gtab,
                                                        int32_t* __restrict__ zero, int nzero)
 {
     pdl_wait();
@@ -314,22 +331,144 @@ __global__ void __launch_bounds__(256) fp4_plan_kernel(const int32_t* __restrict
     __syncthreads();
     int gr = gi - gl, br = bi - bl;
     for (int w = 0; w < wid; w++) { gr += s_g[w]; br += s_b[w]; }
+    const int bfull = b_chunk_bytes(nfull, nsub);
     for (int i = 0; i < 16; i++) {
         const int e = threadIdx.x * EPT + i;
-        if (i < EPT && e < E) { gpre[e] = gr; boffc[e] = br; }
+        if (i < EPT && e < E) {
+            gpre[e] = gr;
+            boffc[e] = br;
+            const int m = offsets[e + 1] - offsets[e], sl = slot_of[e];
+            for (int g = 0; g < gc[i]; g++)
+                gtab[gr + g] = make_int4(offsets[e] + g * NT, min(NT, m - g * NT), sl, br + g * bfull);
+        }
         gr += gc[i];
         br += bc[i];
     }
     if (threadIdx.x == 255) { gpre[E] = gr; boffc[E] = br; }
 }
 
-// One CTA per activation row (x gathered by token, or h): writes the row's T
-// E2M1 terms and their block scales into its token group's operand image,
-// and (NVFP4) the power-of-two exponent p the row was scaled by, 2^p times
-// its largest magnitude lying in [2^10, 2^11) so every term scale stays
-// inside the E4M3 range.  Rows of experts without a slot are skipped.
+// T E2M1 terms of 8 consecutive columns (a lane's share of a scale block of
+// 8 LPB columns; the LPB lanes of a block are adjacent and all active): for
+// each term the block's largest remaining magnitude (shuffles across the
+// block's lanes), its scale code, the 8 codes as one 32-bit word (column i in
+// bits 4i..4i+3) and the residual left for the next term.
+template <int WFMT, int LPB>
+__device__ __noinline__ uint32_t term8(float* v, uint32_t* scode);
+
+template <int WFMT, int T, int LPB>
+__device__ __forceinline__ void terms8(float (&v)[8], uint32_t (&word)[T], uint32_t (&scode)[T])
+{
+#pragma unroll
+    for (int t = 0; t < T; t++) {
+        float mx = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; i++) mx = fmaxf(mx, fabsf(v[i]));
+#pragma unroll
+        for (int off = 1; off < LPB; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        float sval;
+        scode[t] = term_scale<WFMT>(mx, sval);
+        // MXFP4 scales are powers of two: multiplying by the exact reciprocal is the division
+        const float inv = WFMT == MOE_W_MXFP4 ? __uint_as_float((254u - scode[t]) << 23) : 0.0f;
+        uint32_t w = 0;
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const float x = WFMT == MOE_W_MXFP4 ? __fmul_rn(v[i], inv) : __fdiv_rn(v[i], sval);
+            float q;
+            w |= e2m1_round(x, &q) << (4 * i);
+            v[i] = __fsub_rn(v[i], __fmul_rn(q, sval));
+        }
+        word[t] = w;
+    }
+}
+
+// One term of terms8 as a called function (one copy of the code for all
+// callers; the fused decode kernel runs it only a few times per launch, so
+// code size, not issue rate, decides its cost).
+template <int WFMT, int LPB>
+__device__ __noinline__ uint32_t term8(float* v, uint32_t* scode)
+{
+    float mx = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; i++) mx = fmaxf(mx, fabsf(v[i]));
+#pragma unroll
+    for (int off = 1; off < LPB; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    float sval;
+    *scode = term_scale<WFMT>(mx, sval);
+    const float inv = WFMT == MOE_W_MXFP4 ? __uint_as_float((254u - *scode) << 23) : 0.0f;
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const float x = WFMT == MOE_W_MXFP4 ? __fmul_rn(v[i], inv) : __fdiv_rn(v[i], sval);
+        float q;
+        w |= e2m1_round(x, &q) << (4 * i);
+        v[i] = __fsub_rn(v[i], __fmul_rn(q, sval));
+    }
+    return w;
+}
+
+// 8 activation values of a row (bf16 bits or fp32) as floats.  fp32 rows
+// may have been written earlier in the same kernel (h in the fused decode
+// kernel), so they are read through L2, not the read-only cache.
+template <bool IN_F32>
+__device__ __forceinline__ void load8(const void* row, int k, float (&v)[8])
+{
+    if (IN_F32) {
+        const float* f = static_cast<const float*>(row) + k;
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(f));
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(f) + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(row) + k));
+        const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int h = 0; h < 4; h++) {
+            v[2 * h] = bf16_bits_to_f32(u[h] & 0xFFFF);
+            v[2 * h + 1] = bf16_bits_to_f32(u[h] >> 16);
+        }
+    }
+}
+
+// Power-of-two exponent p of an NVFP4 activation row: 2^p times its largest
+// magnitude lands in [2^10, 2^11) (p = 0 for a zero or non-finite maximum).
+__device__ __forceinline__ int row_exponent(float mx)
+{
+    int p = 0;
+    if (mx > 0.0f && mx <= 3.4e38f) {
+        int e2;
+        frexpf(mx, &e2);          // mx = f 2^e2, f in [0.5, 1)
+        p = 11 - e2;
+        p = p < -100 ? -100 : (p > 100 ? 100 : p);
+    }
+    return p;
+}
+
+// Where a term row of a token group's operand image chunk keeps the codes of
+// columns [kin, kin+8) (kin = column inside the 256-column chunk) and the
+// scale of their block: byte offsets inside the chunk image of n rows.
+__device__ __forceinline__ int img_code_off(int row, int kin)
+{
+    return 1024 * (row >> 3) + 128 * (row & 7) + 16 * ((kin / 32) ^ (row & 7)) + (kin % 32) / 2;
+}
+template <int VS>
+__device__ __forceinline__ int img_scale_off(int n, int row, int kin)
+{
+    const int blk = kin / VS, nh = (n + 127) / 128;
+    return n * 128 + 512 * (nh * (blk / 4) + (row >> 7)) + 16 * (row & 31) + 4 * ((row & 127) >> 5) + (blk % 4);
+}
+
+// Activation rows (x gathered by token, or h) -> their T E2M1 terms and block
+// scales in the token group's operand image, and (NVFP4) the power-of-two
+// exponent p the row was scaled by, 2^p times its largest magnitude lying in
+// [2^10, 2^11) so every term scale stays inside the E4M3 range.  Rows of
+// experts without a slot are skipped.  A CTA covers kSegCols columns of one
+// row (blockIdx.x = row * segments + segment); each thread owns 8 consecutive
+// columns, so a 32-column block is 4 lanes (16 columns: 2 lanes) that share
+// their block maximum through shuffles, and a thread's 8 codes are one
+// 32-bit word of the image row.
 // CANON: no groups; row r's codes go to ccodes [rows][T][K] (one per byte),
 // its scale codes to cscales [rows][T][K / vs] and p to rex[r].
+constexpr int kSegCols = 8 * kQuantThreads;
+
 template <int WFMT, int T, bool IN_F32, bool CANON = false>
 __global__ void __launch_bounds__(kQuantThreads) fp4_terms_kernel(
     const void* __restrict__ in, int rows, int K, const int32_t* __restrict__ gather, int gk,
@@ -338,123 +477,83 @@ __global__ void __launch_bounds__(kQuantThreads) fp4_terms_kernel(
     uint8_t* __restrict__ ccodes = nullptr, uint8_t* __restrict__ cscales = nullptr)
 {
     using FM = Fmt<WFMT>;
-    constexpr int VS = FM::VS, NSUB = FM::NSUB, BPC = 256 / VS;   // blocks per chunk
+    constexpr int VS = FM::VS, NSUB = FM::NSUB, LPB = VS / 8;   // lanes per scale block
     pdl_wait();
     pdl_trigger();
     __shared__ float s_max[kQuantThreads / 32];
-    const int tid = threadIdx.x, KC = K / 256, nblk = K / VS;
+    const int tid = threadIdx.x, lane = tid & 31, KC = K / 256;
+    const int nseg = (K + kSegCols - 1) / kSegCols;
     const int nfull = ((T * NT + 7) / 8) * 8;
-    for (int r = blockIdx.x; r < rows; r += gridDim.x) {
-        int j = 0, N = 0, nh = 0, BB = 0;
+    for (int item = blockIdx.x; item < rows * nseg; item += gridDim.x) {
+        const int r = item / nseg, seg = item % nseg;
+        int j = 0, N = 0, BB = 0;
         char* base = nullptr;
         if (!CANON) {
             int lo = 0, hi = E - 1;   // expert of row r: the largest e with offsets[e] <= r
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
-                if (offsets[mid] <= r) lo = mid;
+                if (__ldg(offsets + mid) <= r) lo = mid;
                 else hi = mid - 1;
             }
-            const int e = lo, sl = slot_of[e], m = offsets[e + 1] - offsets[e];
-            if (!(m > 0 && sl >= 0 && sl < pool_slots && offsets[e] >= 0 && offsets[e + 1] <= rows)) continue;
-            const int loc = r - offsets[e], gi = loc / NT, nt = min(NT, m - gi * NT);
+            const int e = lo, sl = __ldg(slot_of + e), m = __ldg(offsets + e + 1) - __ldg(offsets + e);
+            if (!(m > 0 && sl >= 0 && sl < pool_slots && __ldg(offsets + e) >= 0 && __ldg(offsets + e + 1) <= rows))
+                continue;
+            const int loc = r - __ldg(offsets + e), gi = loc / NT, nt = min(NT, m - gi * NT);
             j = loc % NT;
             N = ((T * nt + 7) / 8) * 8;
-            nh = (N + 127) / 128;
             BB = b_chunk_bytes(N, NSUB);
-            base = bimg + (size_t)KC * ((size_t)boffc[e] + (size_t)gi * b_chunk_bytes(nfull, NSUB));
+            base = bimg + (size_t)KC * ((size_t)__ldg(boffc + e) + (size_t)gi * b_chunk_bytes(nfull, NSUB));
         }
         const size_t sr = gather ? (size_t)(__ldg(gather + r) / gk) : (size_t)r;
-        const float* inf = static_cast<const float*>(in) + sr * K;
-        const uint16_t* inb = static_cast<const uint16_t*>(in) + sr * K;
+        const void* row = IN_F32 ? static_cast<const void*>(static_cast<const float*>(in) + sr * K)
+                                 : static_cast<const void*>(static_cast<const uint16_t*>(in) + sr * K);
         int p = 0;
-        if (WFMT == MOE_W_NVFP4) {
+        if (WFMT == MOE_W_NVFP4) {   // row maximum (every segment's CTA reads the whole row)
             float mx = 0.0f;
             for (int k = tid * 8; k < K; k += kQuantThreads * 8) {
-                if (IN_F32) {
-                    const float4 a = __ldg(reinterpret_cast<const float4*>(inf + k));
-                    const float4 b = __ldg(reinterpret_cast<const float4*>(inf + k) + 1);
-                    mx = fmaxf(mx, fmaxf(fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))),
-                                         fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w)))));
-                } else {
-                    const uint4 q = __ldg(reinterpret_cast<const uint4*>(inb + k));
-                    const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+                float v[8];
+                load8<IN_F32>(row, k, v);
 #pragma unroll
-                    for (int i = 0; i < 4; i++)
-                        mx = fmaxf(mx, fmaxf(fabsf(bf16_bits_to_f32(u[i] & 0xFFFF)), fabsf(bf16_bits_to_f32(u[i] >> 16))));
-                }
+                for (int i = 0; i < 8; i++) mx = fmaxf(mx, fabsf(v[i]));
             }
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            if ((tid & 31) == 0) s_max[tid >> 5] = mx;
+            if (lane == 0) s_max[tid >> 5] = mx;
             __syncthreads();
-            mx = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
-            __syncthreads();   // s_max is reused by the next row
-            if (mx > 0.0f && mx <= 3.4e38f) {
-                int e2;
-                frexpf(mx, &e2);          // mx = f 2^e2, f in [0.5, 1)
-                p = 11 - e2;              // mx 2^p in [2^10, 2^11)
-                p = p < -100 ? -100 : (p > 100 ? 100 : p);
-            }
-            if (tid == 0) rex[r] = p;
+            mx = s_max[0];
+#pragma unroll
+            for (int w = 1; w < kQuantThreads / 32; w++) mx = fmaxf(mx, s_max[w]);
+            __syncthreads();   // s_max is reused by the next item
+            p = row_exponent(mx);
         }
-        if (CANON && WFMT == MOE_W_MXFP4 && tid == 0) rex[r] = 0;
+        if (seg == 0 && tid == 0 && (WFMT == MOE_W_NVFP4 || CANON)) rex[r] = p;
         const float sc = ldexpf(1.0f, p);
-        for (int b = tid; b < nblk; b += kQuantThreads) {
-            float v[VS];
+        const int k0 = seg * kSegCols + tid * 8;
+        if (k0 >= K) continue;          // whole scale blocks: every lane of a block is active together
+        float v[8];
+        load8<IN_F32>(row, k0, v);
+        if (WFMT == MOE_W_NVFP4)
 #pragma unroll
-            for (int i = 0; i < VS; i += 8) {
-                if (IN_F32) {
-                    const float4 a = __ldg(reinterpret_cast<const float4*>(inf + b * VS + i));
-                    const float4 c = __ldg(reinterpret_cast<const float4*>(inf + b * VS + i) + 1);
-                    v[i] = a.x; v[i + 1] = a.y; v[i + 2] = a.z; v[i + 3] = a.w;
-                    v[i + 4] = c.x; v[i + 5] = c.y; v[i + 6] = c.z; v[i + 7] = c.w;
-                } else {
-                    const uint4 q = __ldg(reinterpret_cast<const uint4*>(inb + b * VS + i));
-                    const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+            for (int i = 0; i < 8; i++) v[i] = __fmul_rn(v[i], sc);
+        uint32_t word[T], scode[T];
+        terms8<WFMT, T, LPB>(v, word, scode);
+        const int c = k0 / 256, kin = k0 % 256;   // chunk, column inside it
 #pragma unroll
-                    for (int h = 0; h < 4; h++) {
-                        v[i + 2 * h] = bf16_bits_to_f32(u[h] & 0xFFFF);
-                        v[i + 2 * h + 1] = bf16_bits_to_f32(u[h] >> 16);
-                    }
-                }
+        for (int t = 0; t < T; t++) {
+            if (CANON) {
+                uint8_t* cr = ccodes + ((size_t)r * T + t) * K + k0;
+                const uint32_t w = word[t];
+                uint2 o;
+                o.x = (w & 0xF) | ((w >> 4 & 0xF) << 8) | ((w >> 8 & 0xF) << 16) | ((w >> 12 & 0xF) << 24);
+                o.y = (w >> 16 & 0xF) | ((w >> 20 & 0xF) << 8) | ((w >> 24 & 0xF) << 16) | ((w >> 28) << 24);
+                *reinterpret_cast<uint2*>(cr) = o;
+                if ((tid % LPB) == 0) cscales[((size_t)r * T + t) * (K / VS) + k0 / VS] = (uint8_t)scode[t];
+                continue;
             }
-            if (WFMT == MOE_W_NVFP4)
-#pragma unroll
-                for (int i = 0; i < VS; i++) v[i] = __fmul_rn(v[i], sc);
-            const int c = b / BPC, bc = b % BPC, sub = bc / 4, s4 = bc % 4;
-            const int piece = (bc * VS / 2) / 16, half = (VS == 16) ? (bc & 1) : 0;
-            char* cb = CANON ? nullptr : base + (size_t)c * BB;
-#pragma unroll
-            for (int t = 0; t < T; t++) {
-                const int n = j * T + t;
-                float mx = 0.0f;
-#pragma unroll
-                for (int i = 0; i < VS; i++) mx = fmaxf(mx, fabsf(v[i]));
-                float sval;
-                const uint32_t scode = term_scale<WFMT>(mx, sval);
-                uint32_t packed[VS / 8];
-#pragma unroll
-                for (int w = 0; w < VS / 8; w++) packed[w] = 0;
-#pragma unroll
-                for (int i = 0; i < VS; i++) {
-                    const uint32_t q = e2m1_code(__fdiv_rn(v[i], sval));
-                    packed[i / 8] |= q << (4 * (i % 8));
-                    v[i] = __fsub_rn(v[i], __fmul_rn(e2m1_val(q), sval));
-                }
-                if (CANON) {
-                    uint8_t* cr = ccodes + ((size_t)r * T + t) * K + (size_t)b * VS;
-#pragma unroll
-                    for (int i = 0; i < VS; i++) cr[i] = (uint8_t)((packed[i / 8] >> (4 * (i % 8))) & 15);
-                    cscales[((size_t)r * T + t) * nblk + b] = (uint8_t)scode;
-                    continue;
-                }
-                char* dst = cb + 1024 * (n >> 3) + 128 * (n & 7) + 16 * (piece ^ (n & 7)) + 8 * half;
-                if (VS == 32)
-                    *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                else
-                    *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-                cb[N * 128 + 512 * (nh * sub + (n >> 7)) + 16 * (n & 31) + 4 * ((n & 127) >> 5) + s4] = (char)scode;
-            }
+            char* cb = base + (size_t)c * BB;
+            const int n = j * T + t;
+            *reinterpret_cast<uint32_t*>(cb + img_code_off(n, kin)) = word[t];
+            if ((tid % LPB) == 0) cb[img_scale_off<VS>(N, n, kin)] = (char)scode[t];
         }
     }
 }
@@ -469,7 +568,7 @@ struct Fp4Args {
     const int32_t* slot_of;
     const int32_t* offsets;
     const int32_t* gpre;
-    const int32_t* boffc;
+    const int4* gtab;       // per token group: first row, rows, slot, per-chunk image offset
     const char* bimg;       // operand images of this phase's activations
     const int32_t* rex;     // per-row exponents of the activations (NVFP4), else null
     float* out_h;           // phase 1: h [rows][R/2] fp32
@@ -498,9 +597,35 @@ struct KCfg {
     static_assert(STAGE % 1024 == 0, "1024-byte aligned stages");
 };
 
+// The scale-factor copies and four MMAs of one 256-column chunk whose ring
+// stage starts at shared address sa (weight image, its scale images, then
+// the token group's image with n rows and its scale images).  Descriptors of
+// the later K steps and operands are offsets of the first one: the address
+// field counts 16-byte units and the ring lies below 256 KB, so no carry.
+template <int WFMT, int A_BYTES>
+__device__ __forceinline__ void issue_chunk(uint32_t sa, int n, int nh, uint32_t dcol, uint32_t sfa, uint32_t sfb,
+                                            uint32_t id0, uint32_t id1, bool first)
+{
+    using FM = Fmt<WFMT>;
+    const uint64_t da = desc_sw128(sa), db = da + (A_BYTES >> 4);
+    const uint64_t dsa = desc_sf(sa + 16384), dsb = dsa + (uint64_t)((A_BYTES - 16384 + n * 128) >> 4);
+#pragma unroll
+    for (int s = 0; s < FM::NSUB; s++) tc_cp_sf_d(sfa + 4 * s, dsa + (uint64_t)(32 * s));
+    for (int s = 0; s < FM::NSUB * nh; s++) tc_cp_sf_d(sfb + 4 * s, dsb + (uint64_t)(32 * s));
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        // MXFP4: two 32-column scales per MMA, bytes 0-1 or 2-3 of a word;
+        // NVFP4: four 16-column scales per MMA, one image each
+        const int s = WFMT == MOE_W_MXFP4 ? (k >> 1) : k;
+        tc_mma_fp4<WFMT>(dcol, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k),
+                         (WFMT == MOE_W_MXFP4 && (k & 1)) ? id1 : id0, (!first || k > 0) ? 1u : 0u, sfa + 4 * s,
+                         sfb + 4 * nh * s);
+    }
+}
+
 // A unit: (token group of one expert, 128-row block of the weight matrix).
 struct Unit {
-    int e, G, row0, nt, n;   // n: MMA N (terms x tokens, multiple of 8)
+    int G, row0, nt, n;      // n: MMA N (terms x tokens, multiple of 8)
     const char* blob;        // the expert's slot
     const char* a;           // chunk 0 of the weight block
     const char* b;           // chunk 0 of the token group's operand image
@@ -508,29 +633,22 @@ struct Unit {
 };
 
 template <int WFMT, class CFG>
-__device__ __forceinline__ Unit unit_of(const Fp4Args& a, int u, int RB, int KC)
+__device__ __forceinline__ Unit unit_of(const Fp4Args& a, int u, int RB, int KC, int4 g)
 {
     using FM = Fmt<WFMT>;
     Unit U;
     U.G = u % RB;
-    const int gi = u / RB;
-    int lo = 0, hi = a.E - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(a.gpre + mid) <= gi) lo = mid;
-        else hi = mid - 1;
-    }
-    U.e = lo;
-    const int i = gi - __ldg(a.gpre + lo), m = __ldg(a.offsets + lo + 1) - __ldg(a.offsets + lo);
-    U.row0 = __ldg(a.offsets + lo) + i * CFG::NT;
-    U.nt = min(CFG::NT, m - i * CFG::NT);
+    U.row0 = g.x;
+    U.nt = g.y;
     U.n = ((CFG::T * U.nt + 7) / 8) * 8;
     U.bb = b_chunk_bytes(U.n, FM::NSUB);
-    U.blob = a.pool + (size_t)__ldg(a.slot_of + lo) * a.slot_bytes;
+    U.blob = a.pool + (size_t)g.z * a.slot_bytes;
     U.a = U.blob + a.w_off + (size_t)U.G * KC * FM::CB;
-    U.b = a.bimg + (size_t)KC * ((size_t)__ldg(a.boffc + lo) + (size_t)i * b_chunk_bytes(CFG::NMAX, FM::NSUB));
+    U.b = a.bimg + (size_t)KC * (size_t)g.w;
     return U;
 }
+
+__device__ __forceinline__ int4 group_of(const Fp4Args& a, int u, int RB) { return __ldg(a.gtab + u / RB); }
 
 // Segments of one CTA: whole units u = blockIdx.x + i * gridDim.x, or the
 // stream-K pieces of its stage range [pos, end): unit u, chunks [p0, p1).
@@ -584,7 +702,7 @@ __device__ __forceinline__ void finish8(const Fp4Args& a, const Unit& U, int q, 
         const bool live = tok < U.nt;
         const int row = U.row0 + tok;
         float u = tsc;
-        if (WFMT == MOE_W_NVFP4 && live) u = tsc * pow2i(-__ldg(a.rex + row));
+        if (WFMT == MOE_W_NVFP4 && live) u = tsc * pow2i(-__ldcg(a.rex + row));   // written in this grid (fused)
         v *= u;
         if (PHASE == 1) {
             const float up = __shfl_down_sync(0xffffffffu, v, 16);
@@ -643,7 +761,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     volatile int* abort_v = abort_flag;
-    pdl_wait();
+    // The plan (token groups, their table) was written by a kernel that had
+    // completed before this grid's predecessor started, so it may be read
+    // before griddepcontrol.wait; the activation images, row exponents and
+    // the outputs belong to the predecessor and are touched only after it.
     pdl_trigger();
 
     // work: whole units round-robin (prefill), or the units' K chunks cut into
@@ -658,41 +779,80 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
     const long first = whole ? (long)blockIdx.x : b0;
 
     if (warp == 0) {
-        // ============ bulk copies: weight chunk image + token group image chunk
+        // ============ bulk copies: weight chunk image + token group image chunk.
+        // The first D stages' weight copies are issued before waiting for the
+        // predecessor grid (weights do not depend on it); their activation
+        // copies follow once it has completed.
         if (lane == 0 && in_use) {
             int st = 0;
             uint32_t ph = 0;
             long issued = 0;
-            bool ok = true;
+            bool ok = true, waited = false;
+            const char* pend_src[D];
+            uint32_t pend_bytes[D];
+            int npend = 0;
+            auto release_pending = [&]() {
+                pdl_wait();
+                waited = true;
+                for (int i = 0; i < npend; i++) {
+                    bulk_g2s(smem_u32(ring + (size_t)i * STAGE + KC_::A_BYTES), pend_src[i], pend_bytes[i],
+                             smem_u32(&full[i]));
+                }
+                npend = 0;
+            };
             Seg sg{first};
-            while (ok && sg.next(whole, NU, KC, b1)) {
-                const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC);
+            bool have = sg.next(whole, NU, KC, b1);
+            int4 g = have ? group_of(a, sg.u, RB) : make_int4(0, 0, 0, 0);
+            while (ok && have) {
+                const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC, g);
+                Seg nx = sg;   // look one unit ahead: its table entry loads during this unit's copies
+                const bool have_nx = nx.next(whole, NU, KC, b1);
+                const int4 gn = have_nx ? group_of(a, nx.u, RB) : g;
                 for (int c = sg.p0; c < sg.p1; c++) {
                     if (!(ok = mbar_wait(smem_u32(&empty[st]), ph ^ 1, abort_v))) break;
                     const uint32_t bar = smem_u32(&full[st]);
                     unsigned char* sp = ring + (size_t)st * STAGE;
                     mbar_expect_tx(bar, (uint32_t)(FM::CB + U.bb));
                     bulk_g2s(smem_u32(sp), U.a + (size_t)c * FM::CB, FM::CB, bar);
-                    bulk_g2s(smem_u32(sp + KC_::A_BYTES), U.b + (size_t)c * U.bb, (uint32_t)U.bb, bar);
+                    if (waited) {
+                        bulk_g2s(smem_u32(sp + KC_::A_BYTES), U.b + (size_t)c * U.bb, (uint32_t)U.bb, bar);
+                    } else {   // first pass over the ring: stage st == issued
+                        pend_src[npend] = U.b + (size_t)c * U.bb;
+                        pend_bytes[npend++] = (uint32_t)U.bb;
+                    }
                     issued++;
                     if (++st == D) { st = 0; ph ^= 1; }
+                    if (!waited && issued == D) release_pending();
                 }
+                sg = nx;
+                have = have_nx;
+                g = gn;
             }
+            if (!waited) release_pending();
             // every issued copy lands before the CTA exits (stage i was last
             // filled in this pass if i < st, else in the previous one)
             for (int i = 0; i < D && i < issued; i++) mbar_drain(smem_u32(&full[i]), i < st ? ph : (ph ^ 1));
+        } else {
+            pdl_wait();
         }
     } else if (warp == 1) {
         // ============ scale-factor copies and MMAs (one thread)
+        const uint32_t ring_s = smem_u32(ring);
         if (lane == 0 && in_use) {
             int st = 0, it = 0;
             uint32_t ph = 0;
             long cc = 0;
             bool ok = true;
             Seg sg{first};
-            while (ok && sg.next(whole, NU, KC, b1)) {
-                const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC);
+            bool have = sg.next(whole, NU, KC, b1);
+            int4 g = have ? group_of(a, sg.u, RB) : make_int4(0, 0, 0, 0);
+            while (ok && have) {
+                const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC, g);
+                Seg nx = sg;
+                const bool have_nx = nx.next(whole, NU, KC, b1);
+                const int4 gn = have_nx ? group_of(a, nx.u, RB) : g;
                 const int ab = it & 1, nh = (U.n + 127) / 128;
+                const uint32_t id0 = idesc_fp4<WFMT>(U.n, 0), id1 = idesc_fp4<WFMT>(U.n, 2);
                 if (it >= 2) {   // the epilogue has read this accumulator's previous unit
                     if (!(ok = mbar_wait(smem_u32(&acc_empty[ab]), ((it >> 1) - 1) & 1, abort_v))) break;
                     tc_fence_after();
@@ -701,28 +861,18 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
                 for (int c = sg.p0; c < sg.p1; c++, cc++) {
                     if (!(ok = mbar_wait(smem_u32(&full[st]), ph, abort_v))) break;
                     tc_fence_after();
-                    const uint32_t sa = smem_u32(ring + (size_t)st * STAGE), sb = sa + KC_::A_BYTES;
                     const uint32_t sfa = tmem + KC_::SF_COL + (uint32_t)((cc & 1) * KC_::SF_SET);
-                    const uint32_t sfb = sfa + KC_::SF_A;
-#pragma unroll
-                    for (int s = 0; s < FM::NSUB; s++) tc_cp_sf(sfa + 4 * s, sa + 16384 + 512 * s);
-                    for (int s = 0; s < FM::NSUB * nh; s++) tc_cp_sf(sfb + 4 * s, sb + U.n * 128 + 512 * s);
-#pragma unroll
-                    for (int k = 0; k < 4; k++) {
-                        // MXFP4: two 32-column scales per MMA, bytes 0-1 or 2-3 of a word;
-                        // NVFP4: four 16-column scales per MMA, one image each
-                        const int s = WFMT == MOE_W_MXFP4 ? (k >> 1) : k;
-                        const uint32_t id = WFMT == MOE_W_MXFP4 ? 2u * (k & 1) : 0u;
-                        tc_mma_fp4<WFMT>(dcol, desc_sw128(sa + 32 * k), desc_sw128(sb + 32 * k),
-                                         idesc_fp4<WFMT>(U.n, id), (c > sg.p0 || k > 0) ? 1u : 0u, sfa + 4 * s,
-                                         sfb + 4 * nh * s);
-                    }
+                    issue_chunk<WFMT, KC_::A_BYTES>(ring_s + (uint32_t)(st * STAGE), U.n, nh, dcol, sfa,
+                                                    sfa + KC_::SF_A, id0, id1, c == sg.p0);
                     tc_commit(smem_u32(&empty[st]));   // the stage is free once these MMAs have read it
                     if (++st == D) { st = 0; ph ^= 1; }
                 }
                 if (!ok) break;
                 tc_commit(smem_u32(&acc_full[ab]));
                 it++;
+                sg = nx;
+                have = have_nx;
+                g = gn;
             }
             // every MMA issued here completes before tensor memory is released
             tc_commit(smem_u32(fin));
@@ -736,11 +886,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
         const int q = warp & 3;
         const int etid = tid - 64;   // 0..127
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        pdl_wait();
         int it = 0;
         bool ok = true;
         Seg sg{first};
         while (sg.next(whole, NU, KC, b1)) {
-            const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC);
+            const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC, group_of(a, sg.u, RB));
             const int ab = it & 1;
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[ab]), (it >> 1) & 1, abort_v));
             if (ok) tc_fence_after();
@@ -816,6 +967,579 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
     }
 }
 
+// ------------------------------------------------------------------ fused decode FFN
+// Decode calls are too small to pay one kernel boundary per step (each costs
+// several microseconds on the GPU timeline), so with decode tiles the whole
+// FFN call is one cooperative persistent kernel, one CTA per SM:
+//   plan (every CTA computes the token groups of the call for itself, in
+//   shared memory) -> x terms -> grid barrier -> gate-up GEMM -> barrier ->
+//   h terms -> barrier -> down GEMM.
+// The quantisation steps run on the four epilogue warps; the copy warp keeps
+// streaming weights across the barriers and holds back only the activation
+// copies until the barrier that publishes them has passed.  Grid barriers
+// are a global arrival counter and generation word (both back in their idle
+// state after every barrier); every wait on them is bounded.
+__device__ unsigned int g_gb_count;   // arrivals at the current grid barrier
+__device__ unsigned int g_gb_gen;     // completed grid barriers (wraps)
+__device__ int g_gb_abort;            // set when a CTA gave up; cleared with the error word
+
+constexpr int kFusedMaxE = 512;
+constexpr int kPfAhead = 12;   // weight chunks the L2 prefetch runs ahead of the shared-memory copies
+
+struct FusedArgs {
+    Fp4Args p1, p2;                 // the two GEMM phases (gpre / gtab unused)
+    const void* x;                  // input rows: token gather[r] / gk of x (row r when gather is null)
+    int x_f32;
+    const int32_t* gather;
+    int gk;
+    char* bx;                       // operand images of x and of h
+    char* bh;
+    int32_t* rex_x;
+    int32_t* rex_h;
+    int32_t* cnt2;                  // phase-2 piece counters (phase 1 uses p1.cnt)
+    int ncnt;
+};
+
+template <int WFMT>
+struct FusedCfg {
+    using K = KCfg<WFMT, DecodeCfg>;
+    static constexpr int STAGE = K::STAGE;
+    // offsets, group prefix, image offsets, slots; padded so the ring stays
+    // 1024-byte aligned (the 128-byte swizzle of the operand images needs it)
+    static constexpr int PLAN = (4 * 4 * (kFusedMaxE + 1) + 1023) / 1024 * 1024;
+    static constexpr int D = (kSmemBudget - 2048 - PLAN) / STAGE > 8 ? 8 : (kSmemBudget - 2048 - PLAN) / STAGE;
+    static constexpr int SMEM = 1024 + 1024 + PLAN + D * STAGE;
+    static_assert(PLAN % 1024 == 0 && STAGE % 1024 == 0, "1024-byte aligned ring");
+};
+
+// Bounded grid barrier for the four epilogue warps of every CTA.  Their
+// global writes before it are visible to every CTA after it (generic and
+// async proxy: operand images are read by bulk copies).
+__device__ __forceinline__ bool grid_sync_epi(int etid, volatile int* s_flag)
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __threadfence();
+    epi_bar();
+    if (etid == 0) {
+        bool ok = !*reinterpret_cast<volatile int*>(&g_gb_abort);
+        const unsigned gen = *reinterpret_cast<volatile unsigned*>(&g_gb_gen);
+        __threadfence();
+        const unsigned arrived = atomicAdd(&g_gb_count, 1u);
+        if (arrived == gridDim.x - 1) {
+            atomicExch(&g_gb_count, 0u);
+            __threadfence();
+            atomicAdd(&g_gb_gen, 1u);
+        } else {
+            const long long t0 = clock64();
+            while (*reinterpret_cast<volatile unsigned*>(&g_gb_gen) == gen) {
+                if (*reinterpret_cast<volatile int*>(&g_gb_abort)) { ok = false; break; }
+                if (clock64() - t0 > kWaitCycles) {
+                    ok = false;
+                    atomicExch(&g_gb_abort, 1);
+                    atomicCAS(&g_fp4_error, 0, (int)MOE_ERR_TIMEOUT);
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+        __threadfence();
+        *s_flag = ok ? 1 : 0;
+    }
+    epi_bar();
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    return *s_flag != 0;
+}
+
+// The call's plan in shared memory, computed by every CTA.
+struct Plan {
+    int* off;    // [E+1] row offsets
+    int* gpre;   // [E+1] first token group of each expert (experts with rows and a slot have groups)
+    int* boff;   // [E+1] per-chunk image byte offset of its first group
+    int* slot;   // [E]   slot, -1 when the expert is skipped
+    int E;
+};
+
+__device__ __forceinline__ int4 plan_group(const Plan& P, int gi, int NT, int bfull)
+{
+    int lo = 0, hi = P.E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.gpre[mid] <= gi) lo = mid;
+        else hi = mid - 1;
+    }
+    const int i = gi - P.gpre[lo], m = P.off[lo + 1] - P.off[lo];
+    return make_int4(P.off[lo] + i * NT, min(NT, m - i * NT), P.slot[lo], P.boff[lo] + i * bfull);
+}
+
+// One quantisation item of one epilogue warp: row r, 256-column chunk c of
+// its K, into the operand image of its token group (32 lanes x 8 columns).
+// qitem_load finds the item's place and loads its 8 values per lane (a warp
+// loads all its items first, so their global-memory latencies overlap);
+// qitem_store computes the terms and writes them.
+struct QItem {
+    char* cb;          // the item's chunk of its group's operand image (null: skipped row)
+    const void* row;   // the source row
+    int r, c, n0, N;   // row, chunk, first term row (j T), image rows
+    float v[8];
+};
+
+template <int WFMT, int T, bool IN_F32>
+__device__ __forceinline__ void qitem_load(QItem& it, const Plan& P, const void* in, int K, const int32_t* gather,
+                                           int gk, int r, int c, char* bimg, int lane)
+{
+    using FM = Fmt<WFMT>;
+    constexpr int NT = DecodeCfg::NT;
+    it.cb = nullptr;
+    it.r = r;
+    it.c = c;
+    int lo = 0, hi = P.E - 1;   // expert of row r
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.off[mid] <= r) lo = mid;
+        else hi = mid - 1;
+    }
+    const int e = lo;
+    if (P.slot[e] < 0) return;   // the same for the whole warp
+    const int m = P.off[e + 1] - P.off[e], loc = r - P.off[e], gi = loc / NT, j = loc % NT;
+    const int nt = min(NT, m - gi * NT);
+    it.N = ((T * nt + 7) / 8) * 8;
+    it.n0 = j * T;
+    const int KC = K / 256;
+    it.cb = bimg + (size_t)KC * ((size_t)P.boff[e] + (size_t)gi * b_chunk_bytes(DecodeCfg::NMAX, FM::NSUB)) +
+            (size_t)c * b_chunk_bytes(it.N, FM::NSUB);
+    const size_t sr = gather ? (size_t)(__ldg(gather + r) / gk) : (size_t)r;
+    it.row = IN_F32 ? static_cast<const void*>(static_cast<const float*>(in) + sr * K)
+                    : static_cast<const void*>(static_cast<const uint16_t*>(in) + sr * K);
+    load8<IN_F32>(it.row, c * 256 + lane * 8, it.v);
+}
+
+template <int WFMT, int T, bool IN_F32>
+__device__ __forceinline__ void qitem_store(QItem& it, int K, int32_t* rex, int lane)
+{
+    using FM = Fmt<WFMT>;
+    constexpr int VS = FM::VS, LPB = VS / 8;
+    if (!it.cb) return;
+    const int kin = lane * 8;
+    if (WFMT == MOE_W_NVFP4) {   // the row maximum, by this warp over the whole row
+        float mx = 0.0f;
+#pragma unroll 4
+        for (int k = lane * 8; k < K; k += 256) {
+            float u[8];
+            load8<IN_F32>(it.row, k, u);
+#pragma unroll
+            for (int i = 0; i < 8; i++) mx = fmaxf(mx, fabsf(u[i]));
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const int p = row_exponent(mx);
+        if (it.c == 0 && lane == 0) rex[it.r] = p;
+        const float sc = ldexpf(1.0f, p);
+#pragma unroll
+        for (int i = 0; i < 8; i++) it.v[i] = __fmul_rn(it.v[i], sc);
+    }
+#pragma unroll 1
+    for (int t = 0; t < T; t++) {
+        uint32_t scode;
+        const uint32_t word = term8<WFMT, LPB>(it.v, &scode);
+        const int n = it.n0 + t;
+        *reinterpret_cast<uint32_t*>(it.cb + img_code_off(n, kin)) = word;
+        if ((lane % LPB) == 0) it.cb[img_scale_off<VS>(it.N, n, kin)] = (char)scode;
+    }
+}
+
+// All quantisation items of one epilogue warp, loads first (two at a time).
+// After the first loads are issued, lane 0 arrives on `loaded` (when not
+// null): the copy warp holds its weight prefetch until then, so these few
+// loads do not queue behind megabytes of bulk copies.
+template <int WFMT, int T, bool IN_F32>
+__device__ __forceinline__ void fused_quant_items(const Plan& P, const void* in, int K, const int32_t* gather, int gk,
+                                                  char* bimg, int32_t* rex, long first, long step, long items,
+                                                  int lane, uint64_t* loaded)
+{
+    const int KC = K / 256;
+    for (long i0 = first; i0 < items; i0 += 2 * step) {
+        QItem q[2];
+#pragma unroll
+        for (int k = 0; k < 2; k++) {
+            const long i = i0 + k * step;
+            q[k].cb = nullptr;
+            if (i < items) qitem_load<WFMT, T, IN_F32>(q[k], P, in, K, gather, gk, (int)(i / KC), (int)(i % KC), bimg, lane);
+        }
+        if (loaded && i0 == first) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(loaded));
+            loaded = nullptr;
+        }
+#pragma unroll
+        for (int k = 0; k < 2; k++) qitem_store<WFMT, T, IN_F32>(q[k], K, rex, lane);
+    }
+    if (loaded && lane == 0) mbar_arrive(smem_u32(loaded));   // no items
+}
+
+template <int WFMT>
+__global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
+{
+    using FM = Fmt<WFMT>;
+    using CFG = DecodeCfg;
+    using KC_ = KCfg<WFMT, CFG>;
+    using FC = FusedCfg<WFMT>;
+    constexpr int D = FC::D, STAGE = FC::STAGE, T = CFG::T, NT = CFG::NT;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ int s_g[kThreads / 32], s_b[kThreads / 32];
+    unsigned char* smem =
+        reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // [D]
+    uint64_t* empty = full + D;                           // [D]
+    uint64_t* acc_full = empty + D;                       // [2]
+    uint64_t* acc_empty = acc_full + 2;                   // [2]
+    uint64_t* fin = acc_empty + 2;
+    uint64_t* gate = fin + 1;                             // [2]: x terms published, h terms published
+    uint64_t* xloaded = gate + 2;                         // the epilogue warps' first x loads are issued
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xloaded + 1);
+    int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+    int* s_last = abort_flag + 1;
+    int* s_flag = s_last + 1;
+    Plan P;
+    P.E = f.p1.E;
+    P.off = reinterpret_cast<int*>(smem + 1024);
+    P.gpre = P.off + (kFusedMaxE + 1);
+    P.boff = P.gpre + (kFusedMaxE + 1);
+    P.slot = P.boff + (kFusedMaxE + 1);
+    unsigned char* ring = smem + 1024 + FC::PLAN;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int E = P.E, rows = f.p1.rows;
+    const int bfull = b_chunk_bytes(CFG::NMAX, FM::NSUB);
+
+    if (tid == 0) {
+        for (int i = 0; i < D; i++) {
+            mbar_init(smem_u32(&full[i]), 1);
+            mbar_init(smem_u32(&empty[i]), 1);
+        }
+        for (int i = 0; i < 2; i++) {
+            mbar_init(smem_u32(&acc_full[i]), 1);
+            mbar_init(smem_u32(&acc_empty[i]), 32 * kEpiWarps);
+            mbar_init(smem_u32(&gate[i]), 1);
+        }
+        mbar_init(smem_u32(fin), 1);
+        mbar_init(smem_u32(xloaded), kEpiWarps);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(KC_::TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        tc_fence_before();
+    }
+    // ---- plan: the call's token groups (the same in every CTA)
+    {
+        const int EPT = (E + kThreads - 1) / kThreads;   // <= 3 for E <= 512
+        int gl = 0, bl = 0;
+        for (int i = 0; i < EPT; i++) {
+            const int e = tid * EPT + i;
+            if (e < E) {
+                const int o0 = __ldg(f.p1.offsets + e), o1 = __ldg(f.p1.offsets + e + 1);
+                const int sl = __ldg(f.p1.slot_of + e);
+                const bool ok = o1 > o0 && sl >= 0 && sl < f.p1.pool_slots && o0 >= 0 && o1 <= rows;
+                P.off[e] = o0;
+                P.slot[e] = ok ? sl : -1;
+                if (e == E - 1) P.off[E] = o1;
+                if (ok) {
+                    const int g = (o1 - o0 + NT - 1) / NT, last = o1 - o0 - (g - 1) * NT;
+                    gl += g;
+                    bl += (g - 1) * bfull + b_chunk_bytes(((T * last + 7) / 8) * 8, FM::NSUB);
+                }
+            }
+        }
+        int gi = gl, bi = bl;   // inclusive scan over the warp, then over the warps
+        for (int o = 1; o < 32; o <<= 1) {
+            const int go = __shfl_up_sync(0xffffffffu, gi, o), bo = __shfl_up_sync(0xffffffffu, bi, o);
+            if (lane >= o) { gi += go; bi += bo; }
+        }
+        if (lane == 31) { s_g[warp] = gi; s_b[warp] = bi; }
+        __syncthreads();   // also publishes P.off / P.slot
+        int gr = gi - gl, br = bi - bl;
+        for (int w = 0; w < warp; w++) { gr += s_g[w]; br += s_b[w]; }
+        for (int i = 0; i < EPT; i++) {
+            const int e = tid * EPT + i;
+            if (e < E) {
+                P.gpre[e] = gr;
+                P.boff[e] = br;
+                if (P.slot[e] >= 0) {
+                    const int m = P.off[e + 1] - P.off[e];
+                    const int g = (m + NT - 1) / NT, last = m - (g - 1) * NT;
+                    gr += g;
+                    br += (g - 1) * bfull + b_chunk_bytes(((T * last + 7) / 8) * 8, FM::NSUB);
+                }
+            }
+        }
+        if (tid == kThreads - 1) { P.gpre[E] = gr; P.boff[E] = br; }
+    }
+    // the piece counters of both phases start at zero (published by the first grid barrier)
+    for (int i = blockIdx.x * kThreads + tid; i < f.ncnt; i += gridDim.x * kThreads) {
+        f.p1.cnt[i] = 0;
+        f.cnt2[i] = 0;
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    volatile int* abort_v = abort_flag;
+    const int grid = gridDim.x;
+    const int NG = P.gpre[E];
+
+    if (warp == 0) {
+        // ============ bulk copies of both phases.  A second cursor walks the
+        // same chunk sequence kPfAhead chunks ahead and prefetches the weights
+        // into L2, so the shared-memory copies find them there (the ring's
+        // depth alone cannot cover HBM latency at full bandwidth).
+        if (lane == 0) {
+            int st = 0;
+            uint32_t ph = 0;
+            long issued = 0;
+            bool ok = mbar_wait(smem_u32(xloaded), 0, abort_v);   // the x loads go first
+            int pend_st[D];
+            const char* pend_src[D];
+            uint32_t pend_bytes[D];
+            // ---- prefetch cursor
+            int pf_phase = -1, pf_c = 0, pf_p1 = 0, pf_RB = 1, pf_KC = 1, pf_NU = 0;
+            long pf_b1 = 0;
+            Seg pf_sg{0};
+            const char* pf_a = nullptr;
+            auto pf_next = [&]() -> const char* {
+                for (;;) {
+                    if (pf_c < pf_p1) return pf_a + (size_t)(pf_c++) * FM::CB;
+                    if (pf_phase >= 0 && pf_sg.next(false, pf_NU, pf_KC, pf_b1)) {
+                        const Fp4Args& a = pf_phase ? f.p2 : f.p1;
+                        pf_a = unit_of<WFMT, CFG>(a, pf_sg.u, pf_RB, pf_KC, plan_group(P, pf_sg.u / pf_RB, NT, bfull)).a;
+                        pf_c = pf_sg.p0;
+                        pf_p1 = pf_sg.p1;
+                        continue;
+                    }
+                    if (++pf_phase > 1) return nullptr;
+                    const Fp4Args& a = pf_phase ? f.p2 : f.p1;
+                    pf_RB = a.R / 128;
+                    pf_KC = a.K / 256;
+                    pf_NU = NG * pf_RB;
+                    const long W = (long)pf_NU * pf_KC;
+                    const int gridp = (int)(W < (long)grid ? W : (long)grid);
+                    if ((int)blockIdx.x >= gridp) { pf_b1 = 0; pf_sg = Seg{0}; continue; }
+                    pf_sg = Seg{sk_bound(W, blockIdx.x, gridp)};
+                    pf_b1 = sk_bound(W, blockIdx.x + 1, gridp);
+                }
+            };
+            if (ok)
+                for (int i = 0; i < kPfAhead; i++) {
+                    const char* pa = pf_next();
+                    if (!pa) break;
+                    prefetch_l2(pa, FM::CB);
+                }
+            for (int phase = 0; phase < 2 && ok; phase++) {
+                const Fp4Args& a = phase ? f.p2 : f.p1;
+                const int RB = a.R / 128, KC = a.K / 256, NU = NG * RB;
+                const long W = (long)NU * KC;
+                const int gridp = (int)(W < (long)grid ? W : (long)grid);
+                if ((int)blockIdx.x >= gridp) continue;
+                int npend = 0;
+                bool open = false;   // this phase's activation images are published
+                auto release = [&]() -> bool {
+                    if (!mbar_wait(smem_u32(&gate[phase]), 0, abort_v)) return false;
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                    for (int i = 0; i < npend; i++)
+                        bulk_g2s(smem_u32(ring + (size_t)pend_st[i] * STAGE + KC_::A_BYTES), pend_src[i],
+                                 pend_bytes[i], smem_u32(&full[pend_st[i]]));
+                    npend = 0;
+                    open = true;
+                    return true;
+                };
+                Seg sg{sk_bound(W, blockIdx.x, gridp)};
+                const long b1 = sk_bound(W, blockIdx.x + 1, gridp);
+                while (ok && sg.next(false, NU, KC, b1)) {
+                    const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC, plan_group(P, sg.u / RB, NT, bfull));
+                    for (int c = sg.p0; c < sg.p1; c++) {
+                        // a ring full of held-back stages: wait for the gate before reusing one
+                        if (!open && npend == D && !(ok = release())) break;
+                        if (!(ok = mbar_wait(smem_u32(&empty[st]), ph ^ 1, abort_v))) break;
+                        const uint32_t bar = smem_u32(&full[st]);
+                        unsigned char* sp = ring + (size_t)st * STAGE;
+                        mbar_expect_tx(bar, (uint32_t)(FM::CB + U.bb));
+                        bulk_g2s(smem_u32(sp), U.a + (size_t)c * FM::CB, FM::CB, bar);
+                        if (const char* pa = pf_next()) prefetch_l2(pa, FM::CB);
+                        if (!open && mbar_try(smem_u32(&gate[phase]), 0) && !(ok = release())) break;
+                        if (open) {
+                            bulk_g2s(smem_u32(sp + KC_::A_BYTES), U.b + (size_t)c * U.bb, (uint32_t)U.bb, bar);
+                        } else {
+                            pend_st[npend] = st;
+                            pend_src[npend] = U.b + (size_t)c * U.bb;
+                            pend_bytes[npend++] = (uint32_t)U.bb;
+                        }
+                        issued++;
+                        if (++st == D) { st = 0; ph ^= 1; }
+                    }
+                }
+                if (ok && !open && npend > 0) ok = release();
+            }
+            // every issued copy lands before the CTA exits (a stage whose
+            // activation copy was never released completes no phase: the
+            // drain gives up on it after the time limit, which only happens
+            // after an abort)
+            for (int i = 0; i < D && i < issued; i++) mbar_drain(smem_u32(&full[i]), i < st ? ph : (ph ^ 1));
+        }
+    } else if (warp == 1) {
+        // ============ scale-factor copies and MMAs of both phases
+        const uint32_t ring_s = smem_u32(ring);
+        if (lane == 0) {
+            int st = 0, it = 0;
+            uint32_t ph = 0;
+            long cc = 0;
+            bool ok = true;
+            for (int phase = 0; phase < 2 && ok; phase++) {
+                const Fp4Args& a = phase ? f.p2 : f.p1;
+                const int RB = a.R / 128, KC = a.K / 256, NU = NG * RB;
+                const long W = (long)NU * KC;
+                const int gridp = (int)(W < (long)grid ? W : (long)grid);
+                if ((int)blockIdx.x >= gridp) continue;
+                Seg sg{sk_bound(W, blockIdx.x, gridp)};
+                const long b1 = sk_bound(W, blockIdx.x + 1, gridp);
+                while (ok && sg.next(false, NU, KC, b1)) {
+                    const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC, plan_group(P, sg.u / RB, NT, bfull));
+                    const int ab = it & 1, nh = (U.n + 127) / 128;
+                    const uint32_t id0 = idesc_fp4<WFMT>(U.n, 0), id1 = idesc_fp4<WFMT>(U.n, 2);
+                    if (it >= 2) {
+                        if (!(ok = mbar_wait(smem_u32(&acc_empty[ab]), ((it >> 1) - 1) & 1, abort_v))) break;
+                        tc_fence_after();
+                    }
+                    const uint32_t dcol = tmem + (uint32_t)(ab * CFG::NMAX);
+                    for (int c = sg.p0; c < sg.p1; c++, cc++) {
+                        if (!(ok = mbar_wait(smem_u32(&full[st]), ph, abort_v))) break;
+                        tc_fence_after();
+                        const uint32_t sfa = tmem + KC_::SF_COL + (uint32_t)((cc & 1) * KC_::SF_SET);
+                        issue_chunk<WFMT, KC_::A_BYTES>(ring_s + (uint32_t)(st * STAGE), U.n, nh, dcol, sfa,
+                                                        sfa + KC_::SF_A, id0, id1, c == sg.p0);
+                        tc_commit(smem_u32(&empty[st]));
+                        if (++st == D) { st = 0; ph ^= 1; }
+                    }
+                    if (!ok) break;
+                    tc_commit(smem_u32(&acc_full[ab]));
+                    it++;
+                }
+            }
+            tc_commit(smem_u32(fin));
+            mbar_drain(smem_u32(fin), 0);
+        }
+    } else {
+        // ============ epilogue warps: terms of x, phase-1 epilogue, terms of h, phase-2 epilogue.
+        // All four warps walk the same items and segments and meet the same
+        // barriers; after a failed wait they keep walking without waiting.
+        const int q = warp & 3;
+        const int etid = tid - 64;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        int it = 0;
+        bool ok = true;
+        for (int phase = 0; phase < 2; phase++) {
+            const Fp4Args& a = phase ? f.p2 : f.p1;
+            {   // the activation terms of this phase's input rows: (row, chunk) items per warp
+                const long items = (long)rows * (a.K / 256);
+                const long first = (long)blockIdx.x * kEpiWarps + (warp - 2), step = (long)grid * kEpiWarps;
+                if (phase == 1)
+                    fused_quant_items<WFMT, T, true>(P, f.p1.out_h, a.K, nullptr, 1, f.bh, f.rex_h, first, step, items,
+                                                     lane, nullptr);
+                else if (f.x_f32)
+                    fused_quant_items<WFMT, T, true>(P, f.x, a.K, f.gather, f.gk, f.bx, f.rex_x, first, step, items,
+                                                     lane, xloaded);
+                else
+                    fused_quant_items<WFMT, T, false>(P, f.x, a.K, f.gather, f.gk, f.bx, f.rex_x, first, step, items,
+                                                      lane, xloaded);
+            }
+            ok = grid_sync_epi(etid, s_flag) && ok;   // terms published (phase 0: counters zero)
+            if (etid == 0) mbar_arrive(smem_u32(&gate[phase]));
+            const int RB = a.R / 128, KC = a.K / 256, NU = NG * RB;
+            const long W = (long)NU * KC;
+            const int gridp = (int)(W < (long)grid ? W : (long)grid);
+            if ((int)blockIdx.x < gridp) {
+                const long b0 = sk_bound(W, blockIdx.x, gridp), b1 = sk_bound(W, blockIdx.x + 1, gridp);
+                Seg sg{b0};
+                while (sg.next(false, NU, KC, b1)) {
+                    const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC, plan_group(P, sg.u / RB, NT, bfull));
+                    const int ab = it & 1;
+                    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[ab]), (it >> 1) & 1, abort_v));
+                    if (ok) tc_fence_after();
+                    float tsc = 1.0f;
+                    if (WFMT == MOE_W_NVFP4) tsc = __ldg(reinterpret_cast<const float*>(U.blob + a.ts_off) + phase);
+                    const uint32_t dcol = tmem + lane_base + (uint32_t)(ab * CFG::NMAX);
+                    const int nch = (U.nt + 7) / 8;
+                    if (sg.p0 == 0 && sg.p1 == KC) {
+                        if (ok) {
+                            for (int ch = 0; ch < nch; ch++) {
+                                uint32_t d[8 * T];
+#pragma unroll
+                                for (int t = 0; t < T; t++) tmem_ld8(dcol + 8 * T * ch + 8 * t, d + 8 * t);
+                                tmem_wait_ld();
+                                if (phase == 0)
+                                    finish8<WFMT, 1, T>(a, U, q, lane, ch, reinterpret_cast<const float*>(d), tsc);
+                                else
+                                    finish8<WFMT, 2, T>(a, U, q, lane, ch, reinterpret_cast<const float*>(d), tsc);
+                            }
+                            tc_fence_before();
+                            mbar_arrive(smem_u32(&acc_empty[ab]));
+                        }
+                    } else {
+                        const int slot = sg.start == b0 ? 0 : 1;
+                        float* mine = a.pieces + ((size_t)blockIdx.x * 2 + slot) * (128 * CFG::NMAX);
+                        if (ok) {
+                            for (int ch = 0; ch < nch; ch++) {
+                                uint32_t d[8 * T];
+#pragma unroll
+                                for (int t = 0; t < T; t++) tmem_ld8(dcol + 8 * T * ch + 8 * t, d + 8 * t);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int i = 0; i < 8 * T; i++)
+                                    mine[(size_t)(8 * T * ch + i) * 128 + etid] = __uint_as_float(d[i]);
+                            }
+                            tc_fence_before();
+                            mbar_arrive(smem_u32(&acc_empty[ab]));
+                        }
+                        __threadfence();
+                        epi_bar();
+                        const long u_lo = (long)sg.u * KC, u_hi = u_lo + KC - 1;
+                        const int c_lo = sk_cta_of(W, u_lo, gridp), c_hi = sk_cta_of(W, u_hi, gridp);
+                        if (etid == 0) *s_last = (ok && !*abort_v && atomicAdd(a.cnt + sg.u, 1) == c_hi - c_lo) ? 1 : 0;
+                        epi_bar();
+                        if (*s_last) {
+                            __threadfence();
+                            for (int ch = 0; ch < nch; ch++) {
+                                float d[8 * T];
+#pragma unroll
+                                for (int i = 0; i < 8 * T; i++) d[i] = 0.0f;
+                                for (int c = c_lo; c <= c_hi; c++) {
+                                    const int sl = sk_bound(W, c, gridp) >= u_lo ? 0 : 1;
+                                    const float* pc = a.pieces + ((size_t)c * 2 + sl) * (128 * CFG::NMAX);
+#pragma unroll
+                                    for (int i = 0; i < 8 * T; i++)
+                                        d[i] += __ldcg(pc + (size_t)(8 * T * ch + i) * 128 + etid);
+                                }
+                                if (phase == 0) finish8<WFMT, 1, T>(a, U, q, lane, ch, d, tsc);
+                                else finish8<WFMT, 2, T>(a, U, q, lane, ch, d, tsc);
+                            }
+                            if (etid == 0) a.cnt[sg.u] = 0;
+                        }
+                        epi_bar();   // s_last is rewritten by the next piece
+                    }
+                    it++;
+                }
+            }
+            if (phase == 0) ok = grid_sync_epi(etid, s_flag) && ok;   // h complete before its terms are taken
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(KC_::TMEM_COLS)
+                     : "memory");
+    }
+}
+
 // ------------------------------------------------------------------ host side
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t st, Args... args)
@@ -836,12 +1560,14 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t sme
 struct Fp4Ws {
     int32_t* gpre;
     int32_t* boffc;
+    int4* gtab;
     int32_t* rex_x;
     int32_t* rex_h;
     char* bx;
     char* bh;
     float* h32;
     int32_t* cnt;
+    int32_t* cnt2;   // second counter set (the fused decode kernel's down projection)
     int ncnt;
     float* pieces;
 };
@@ -866,6 +1592,8 @@ size_t fp4_ws_layout(const moe_shape* s, int rows, void* base, Fp4Ws* w)
             : group_chunk_bound<PrefillCfg>(R, E, nsub);
     const size_t ogp = take(4 * (size_t)(E + 1));
     const size_t obo = take(4 * (size_t)(E + 1));
+    const size_t Gmax = (size_t)(R + DecodeCfg::NT - 1) / DecodeCfg::NT + (size_t)(R < E ? R : E);
+    const size_t ogt = take(16 * Gmax);
     const size_t orx = take(4 * (size_t)R);
     const size_t orh = take(4 * (size_t)R);
     const size_t obx = take(per_chunk * (s->hidden / 256));
@@ -874,17 +1602,20 @@ size_t fp4_ws_layout(const moe_shape* s, int rows, void* base, Fp4Ws* w)
     const long RBmax = (2 * s->ffn > s->hidden ? 2 * s->ffn : s->hidden) / 128;
     const long ncnt = ((long)(R + DecodeCfg::NT - 1) / DecodeCfg::NT + (R < E ? R : E)) * RBmax;
     const size_t oc = take(4 * (size_t)ncnt);
+    const size_t oc2 = take(4 * (size_t)ncnt);
     const size_t op = take(4 * (size_t)kMaxCtas * 2 * 128 * DecodeCfg::NMAX);
     if (w) {
         char* b = static_cast<char*>(base);
         w->gpre = reinterpret_cast<int32_t*>(b + ogp);
         w->boffc = reinterpret_cast<int32_t*>(b + obo);
+        w->gtab = reinterpret_cast<int4*>(b + ogt);
         w->rex_x = reinterpret_cast<int32_t*>(b + orx);
         w->rex_h = reinterpret_cast<int32_t*>(b + orh);
         w->bx = b + obx;
         w->bh = b + obh;
         w->h32 = reinterpret_cast<float*>(b + oh);
         w->cnt = reinterpret_cast<int32_t*>(b + oc);
+        w->cnt2 = reinterpret_cast<int32_t*>(b + oc2);
         w->ncnt = (int)ncnt;
         w->pieces = reinterpret_cast<float*>(b + op);
     }
@@ -922,8 +1653,12 @@ int run_fp4(const moe_shape* s, const BlobLayout& bl, const void* pool, size_t s
     if ((rc = set_smem_attr<WFMT, 1, CFG>())) return rc;
     if ((rc = set_smem_attr<WFMT, 2, CFG>())) return rc;
     MOE_CUDA_TRY(launch_pdl(fp4_plan_kernel, 1, 256, 0, st, offsets, slot_of, E, rows, pool_slots, CFG::NT, CFG::T,
-                            FM::NSUB, w.gpre, w.boffc, w.cnt, w.ncnt));
-    const int qgrid = rows < sms * 16 ? rows : sms * 16;
+                            FM::NSUB, w.gpre, w.boffc, w.gtab, w.cnt, w.ncnt));
+    auto qgrid_for = [&](int K) {
+        const long items = (long)rows * ((K + kSegCols - 1) / kSegCols);
+        return (int)(items < (long)sms * 8 ? items : (long)sms * 8);
+    };
+    const int qgrid = qgrid_for(H);
     if (src.x_dtype == MOE_DT_F32)
         MOE_CUDA_TRY(launch_pdl(fp4_terms_kernel<WFMT, CFG::T, true>, qgrid, kQuantThreads, 0, st, src.x, rows, H,
                                 src.assign_of, src.k, offsets, slot_of, E, pool_slots, w.boffc, CFG::NT, w.bx, w.rex_x,
@@ -942,7 +1677,7 @@ int run_fp4(const moe_shape* s, const BlobLayout& bl, const void* pool, size_t s
     a.slot_of = slot_of;
     a.offsets = offsets;
     a.gpre = w.gpre;
-    a.boffc = w.boffc;
+    a.gtab = w.gtab;
     a.cnt = w.cnt;
     a.pieces = w.pieces;
     const int grid = sms < kMaxCtas ? sms : kMaxCtas;
@@ -954,7 +1689,7 @@ int run_fp4(const moe_shape* s, const BlobLayout& bl, const void* pool, size_t s
     a.rex = WFMT == MOE_W_NVFP4 ? w.rex_x : nullptr;
     a.out_h = w.h32;
     MOE_CUDA_TRY(launch_pdl(ffn_fp4_kernel<WFMT, 1, CFG>, grid, kThreads, smem, st, a));
-    MOE_CUDA_TRY(launch_pdl(fp4_terms_kernel<WFMT, CFG::T, true>, qgrid, kQuantThreads, 0, st,
+    MOE_CUDA_TRY(launch_pdl(fp4_terms_kernel<WFMT, CFG::T, true>, qgrid_for(F), kQuantThreads, 0, st,
                             static_cast<const void*>(w.h32), rows, F, static_cast<const int32_t*>(nullptr), 1,
                             offsets, slot_of, E, pool_slots, w.boffc, CFG::NT, w.bh, w.rex_h, kNoCanon, kNoCanon));
     Fp4Args b = a;
@@ -966,6 +1701,84 @@ int run_fp4(const moe_shape* s, const BlobLayout& bl, const void* pool, size_t s
     b.out_h = nullptr;
     b.out_y = y_perm;
     MOE_CUDA_TRY(launch_pdl(ffn_fp4_kernel<WFMT, 2, CFG>, grid, kThreads, smem, st, b));
+    return MOE_OK;
+}
+
+// The whole decode-tile FFN call as one cooperative launch (one CTA per SM).
+// Returns MOE_ERR_UNSUPPORTED when the device cannot run it that way, so the
+// caller falls back to one launch per step.
+template <int WFMT>
+int run_fp4_fused(const moe_shape* s, const BlobLayout& bl, const void* pool, size_t slot_bytes, int pool_slots,
+                  const int32_t* slot_of, const int32_t* offsets, int rows, uint16_t* y_perm, const Fp4Ws& w,
+                  const RowSource& src, int sms, cudaStream_t st)
+{
+    using FC = FusedCfg<WFMT>;
+    const int E = s->experts, H = s->hidden, F = s->ffn;
+    if (E > kFusedMaxE) return MOE_ERR_UNSUPPORTED;
+    if (group_chunk_bound<DecodeCfg>(rows, E, Fmt<WFMT>::NSUB) >= (size_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+    int dev = 0, coop = 0;
+    MOE_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+    MOE_CUDA_TRY(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev));
+    if (!coop) return MOE_ERR_UNSUPPORTED;
+    static int resident[kMaxDevices];   // 0 unknown, 1 one CTA per SM fits, -1 it does not
+    if (!resident[dev]) {
+        MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_fp4_fused_kernel<WFMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          FC::SMEM));
+        int nb = 0;
+        MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, ffn_fp4_fused_kernel<WFMT>, kThreads, FC::SMEM));
+        resident[dev] = nb >= 1 ? 1 : -1;
+    }
+    if (resident[dev] < 0) return MOE_ERR_UNSUPPORTED;
+    FusedArgs f{};
+    Fp4Args& a = f.p1;
+    a.pool = static_cast<const char*>(pool);
+    a.slot_bytes = slot_bytes;
+    a.ts_off = bl.ts;
+    a.E = E;
+    a.rows = rows;
+    a.pool_slots = pool_slots;
+    a.slot_of = slot_of;
+    a.offsets = offsets;
+    a.pieces = w.pieces;
+    a.w_off = bl.w13;
+    a.R = 2 * F;
+    a.K = H;
+    a.bimg = w.bx;
+    a.rex = WFMT == MOE_W_NVFP4 ? w.rex_x : nullptr;
+    a.out_h = w.h32;
+    a.cnt = w.cnt;
+    Fp4Args& b = f.p2;
+    b = a;
+    b.w_off = bl.w2;
+    b.R = H;
+    b.K = F;
+    b.bimg = w.bh;
+    b.rex = WFMT == MOE_W_NVFP4 ? w.rex_h : nullptr;
+    b.out_h = nullptr;
+    b.out_y = y_perm;
+    b.cnt = w.cnt2;
+    f.x = src.x;
+    f.x_f32 = src.x_dtype == MOE_DT_F32;
+    f.gather = src.assign_of;
+    f.gk = src.k;
+    f.bx = w.bx;
+    f.bh = w.bh;
+    f.rex_x = w.rex_x;
+    f.rex_h = w.rex_h;
+    f.cnt2 = w.cnt2;
+    f.ncnt = w.ncnt;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sms < kMaxCtas ? sms : kMaxCtas);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = FC::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, ffn_fp4_fused_kernel<WFMT>, f));
     return MOE_OK;
 }
 
@@ -988,8 +1801,13 @@ int ffn_fp4_device_error(int clear)
     int v = 0;
     if (cudaMemcpyFromSymbol(&v, g_fp4_error, sizeof v) != cudaSuccess) return MOE_ERR_CUDA;
     if (clear && v) {
-        int z = 0;
-        if (cudaMemcpyToSymbol(g_fp4_error, &z, sizeof z) != cudaSuccess) return MOE_ERR_CUDA;
+        // the kernels are not running: put the grid barrier back in its idle state too
+        const int z = 0;
+        const unsigned zu = 0;
+        if (cudaMemcpyToSymbol(g_fp4_error, &z, sizeof z) != cudaSuccess ||
+            cudaMemcpyToSymbol(g_gb_abort, &z, sizeof z) != cudaSuccess ||
+            cudaMemcpyToSymbol(g_gb_count, &zu, sizeof zu) != cudaSuccess)
+            return MOE_ERR_CUDA;
     }
     return v;
 }
@@ -1005,8 +1823,19 @@ int launch_ffn_fp4(const moe_shape* s, const void* pool, size_t slot_bytes, int 
     MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
     const RowSource src = gather ? *gather : RowSource{x_perm, MOE_DT_BF16, nullptr, 1};
     const BlobLayout bl = blob_layout(s);
-    prof_count(MOE_PROF_FFN, 5);
     const bool pre = use_prefill_tiles(s, rows);
+    if (!pre && !getenv("MOE_FFN_UNFUSED")) {
+        const int rc = s->wfmt == MOE_W_MXFP4
+                           ? run_fp4_fused<MOE_W_MXFP4>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, rows,
+                                                        y_perm, w, src, sms, st)
+                           : run_fp4_fused<MOE_W_NVFP4>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, rows,
+                                                        y_perm, w, src, sms, st);
+        if (rc != MOE_ERR_UNSUPPORTED) {
+            if (rc == MOE_OK) prof_count(MOE_PROF_FFN, 1);
+            return rc;
+        }
+    }
+    prof_count(MOE_PROF_FFN, 5);
     if (s->wfmt == MOE_W_MXFP4)
         return pre ? run_fp4<MOE_W_MXFP4, PrefillCfg>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, rows,
                                                       y_perm, w, src, sms, st)
@@ -1035,7 +1864,8 @@ extern "C" int moe_act_terms(const void* d_x, int32_t x_dtype, int32_t rows, int
     int dev = 0, sms = 148;
     MOE_CUDA_TRY(cudaGetDevice(&dev));
     MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-    const int grid = rows < sms * 16 ? rows : sms * 16;
+    const long items = (long)rows * ((K + kSegCols - 1) / kSegCols);
+    const int grid = (int)(items < (long)sms * 8 ? items : (long)sms * 8);
     cudaStream_t st = as_stream(stream);
     const bool f32 = x_dtype == MOE_DT_F32;
 #define MOE_TERMS_LAUNCH(W, TT, F)                                                                                 \
