@@ -54,19 +54,23 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--resident-batch", default="1,4,16", help="batch sizes of the resident decode leg")
-    p.add_argument("--leg", choices=["all", "resident", "prefill", "tiny", "qwen", "trace"], default="all",
+    p.add_argument("--leg", choices=["all", "resident", "prefill", "tiny", "qwen", "trace", "device_fill"],
+                   default="all",
                    help="run only that context leg (profiling); prints its own JSON line")
     p.add_argument("--trace-steps", type=int, default=256, help="decode steps of the 40-layer trace leg")
+    p.add_argument("--fill", choices=["host", "device"], default="host",
+                   help="miss fills of the decode streams: host-issued DMA copies or the zero-copy fill kernel")
     return p.parse_args()
 
 
-def workload_config(cfg, n, world):
+def workload_config(cfg, n, world, fill="host"):
     return {"workload": "DeepSeek-V4-Flash-shaped MXFP4 MoE decode layer: 256 routed experts, top-6, "
                         "hidden 4096, expert FFN 2048, 64-slot GPU expert cache (LRU, misses filled from "
                         "pinned host RAM), Zipf(1.1) routing, continuous decode stream from a cold cache",
             "batch_tokens": n, "experts": cfg.experts, "top_k": cfg.top_k, "hidden": cfg.hidden,
             "ffn": cfg.ffn, "weights": "mxfp4", "activations": "bf16", "capacity_slots": cfg.capacity,
             "routing": "zipf(s=1.1) via router bias, seed 0", "l2": "flushed before every step (256 MiB write)",
+            "miss_fills": "zero-copy fill kernel" if fill == "device" else "host-issued DMA copies",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
@@ -187,22 +191,38 @@ class OneCore:
         return False
 
 
-def measure_bp(device, mib=64, reps=20):
-    """Pinned host -> device copy bandwidth (GB/s): median of `reps` copies of `mib` MiB."""
+def measure_bp(device, srcs, mib=64, reps=20):
+    """Pinned host -> device copy bandwidth Bp (GB/s): median of `reps` samples, each one
+    cudaMemcpyAsync per source buffer until `mib` MiB are copied.  The sources are the
+    pinned expert blobs the cache fills from: a fresh pinned buffer can land on another
+    NUMA node than the blobs and see a different PCIe path."""
     import torch
-    h = torch.empty(mib << 20, dtype=torch.uint8).pin_memory()
-    d = torch.empty(mib << 20, dtype=torch.uint8, device=device)
-    d.copy_(h, non_blocking=True)
+    todo, plan = mib << 20, []
+    for h in srcs:
+        if todo <= 0:
+            break
+        take = min(todo, h.numel())
+        plan.append((h, take))
+        todo -= take
+    total = sum(t for _, t in plan)
+    d = torch.empty(total, dtype=torch.uint8, device=device)
+
+    def once():
+        o = 0
+        for h, t in plan:
+            d[o:o + t].copy_(h[:t], non_blocking=True)
+            o += t
+    once()
     torch.cuda.synchronize()
     ts = []
     for _ in range(reps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        d.copy_(h, non_blocking=True)
+        once()
         b.record()
         torch.cuda.synchronize()
         ts.append(a.elapsed_time(b))
-    return (mib << 20) / (float(np.median(ts)) / 1000.0) / 1e9
+    return total / (float(np.median(ts)) / 1000.0) / 1e9
 
 
 # ------------------------------------------------------------------ multi-rank plumbing
@@ -247,13 +267,15 @@ def to_dev_bits(a, device):
 class DecodeStream:
     """One replica: a cache over the host blobs, device inputs for every step, workspace."""
 
-    def __init__(self, cfg, shape, blobs, wg, bias, n, steps, capacity, rank, device, tag="decode"):
+    def __init__(self, cfg, shape, blobs, wg, bias, n, steps, capacity, rank, device, tag="decode", fill="host"):
         import torch
 
         from expert_cached_sparse_b200 import api as A
         from expert_cached_sparse_b200 import workloads as W
         self.A, self.n, self.cfg, self.shape = A, n, cfg, shape
         self.cache = A.MoeCache(shape, capacity, blobs, trace_capacity=0)
+        if fill == "device":
+            self.cache.set_fill_mode(1)
         self.wg = to_dev_bits(wg, device)
         self.bias = torch.from_numpy(bias).to(device) if bias is not None else None
         xs = np.stack([W.gen_x(cfg, 1000 + rank, n, tag, s) for s in range(steps)])
@@ -329,10 +351,10 @@ def timed_steps(ds, first, k, flush, dist_ok):
 
 
 def graph_steps(ds, first, k, flush):
-    """A fully resident layer step reads nothing back to the host, so it can be
-    captured once in a CUDA graph; replays steps first..first+k-1 (inputs copied
-    into the captured input buffer before each, outside the events) and returns
-    the summed device ms."""
+    """A layer step that reads nothing back to the host (every expert resident, or
+    device fills) can be captured once in a CUDA graph; replays steps
+    first..first+k-1 (inputs copied into the captured input buffer before each,
+    outside the events) and returns the summed device ms."""
     import torch
     xin = ds.x[first].clone()
     torch.cuda.synchronize()
@@ -394,7 +416,7 @@ def run_reference(args, cfg, world):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * sec / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(cfg, args.batch, world),
+            "data": "synthetic", "config": workload_config(cfg, args.batch, world, args.fill),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "pinned_core": oc.core, **host_info(),
                              "sample": f"{args.steps} one-token samples of the decode stream (route, LRU, "
@@ -426,13 +448,15 @@ def run_ours(args, cfg, world, rank, local_rank):
     if args.leg != "all":
         res = extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=(args.leg,),
                      batches=tuple(int(b) for b in args.resident_batch.split(",")), trace_steps=args.trace_steps,
-                     cpu=not args.no_cpu_baseline)
+                     cpu=not args.no_cpu_baseline, fill=args.fill)
         if rank == 0:
             print(json.dumps({"leg": args.leg, "steps": K, "warmup": Wm, "results": res}), flush=True)
         return
 
     # ---- headline: 64-slot decode stream
-    ds = DecodeStream(cfg, shape, blobs, wg, bias, n, 2 * K + Wm, cfg.capacity, rank, device)
+    distinct_blobs = list({b.data_ptr(): b for b in blobs}.values())
+    bp0 = measure_bp(device, distinct_blobs)
+    ds = DecodeStream(cfg, shape, blobs, wg, bias, n, 2 * K + Wm, cfg.capacity, rank, device, fill=args.fill)
     for s in range(Wm):
         ds.step(s)
     torch.cuda.synchronize()
@@ -468,21 +492,26 @@ def run_ours(args, cfg, world, rank, local_rank):
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": Wm,
             "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic", "config": workload_config(cfg, n, world)}
+            "dtype": "bf16", "data": "synthetic", "config": workload_config(cfg, n, world, args.fill)}
     line["roofline"] = {"kernel": "grouped SwiGLU FFN call (ffn_fp4_fused_kernel: x terms, gate-up, h terms, "
                                   "down; block-scaled tcgen05)",
                         "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                         "frac": achieved / hbm_peak, "peak_kind": peak_kind, "traffic": ffn_traffic(),
                         "algorithmic_bytes_per_call": ffn_bytes / ffn_calls,
                         "avg_call_ms": ffn_ms / ffn_calls, "calls": ffn_calls}
-    bp = measure_bp(device)
+    # Bp before and after the timed region (the PCIe path can be shared with
+    # other traffic on the host); the bound takes the better of the two
+    bp1 = measure_bp(device, distinct_blobs)
+    bp = max(bp0, bp1)
     # the step's end-to-end bound: its HBM bytes at the measured peak plus its misses over PCIe at Bp
     step_hbm = ffn_bytes / K + cfg.experts * cfg.hidden * 2 + 2 * n * cfg.hidden * 2
     bound_ms = step_hbm / (hbm_peak * 1e9) * 1e3 + (misses / K) * slot_bytes / (bp * 1e9) * 1e3
     line["bp_GBps"] = bp
+    line["bp_GBps_before_after"] = [bp0, bp1]
     line["step_bound"] = {"ms_per_step": bound_ms, "frac": bound_ms / (ms_max / K),
                           "note": "HBM bytes of the step at the measured peak + misses x slot bytes / Bp "
-                                  "(Bp: pinned 64 MiB host->device copy, median of 20, measured in this run)"}
+                                  "(Bp: 64 MiB of the pinned expert blobs copied host->device, median of 20, measured "
+                                  "before and after the timed steps in this run, the better taken)"}
     line["gpu_launches"] = int(kernels)
     line["cache"] = {"lookups": lookups, "hit_rate": hits / max(1, hits + misses), "misses_per_step": misses / K,
                      "fill_GBps": fill_gbs, "fill_ms_per_step": fill_ms / K,
@@ -518,7 +547,8 @@ def run_ours(args, cfg, world, rank, local_rank):
     # ---- extra legs (rank 0 only, single-GPU context numbers)
     if not args.no_extras and rank == 0:
         line["extras"] = extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak,
-                                trace_steps=args.trace_steps, cpu=world == 1 and not args.no_cpu_baseline)
+                                trace_steps=args.trace_steps, cpu=world == 1 and not args.no_cpu_baseline,
+                                fill=args.fill)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         with OneCore() as oc:
@@ -617,9 +647,34 @@ def layer_leg(cfg, shape, blobs, wg, bias, n, steps, warm, flush, device, hbm_pe
     return out, ds.x_host
 
 
+def device_fill_leg(cfg, shape, blobs, wg, bias, n, K, Wm, flush, device):
+    """The headline decode stream (cold 64-slot cache) with device fills: eager calls, then
+    a fresh cache whose whole step, misses included, is one CUDA graph replayed per step."""
+    import torch
+    out = {}
+    for mode in ("eager", "cuda_graph"):
+        ds = DecodeStream(cfg, shape, blobs, wg, bias, n, K + Wm, cfg.capacity, 0, device, fill="device")
+        for s in range(Wm):
+            ds.step(s)
+        torch.cuda.synchronize()
+        st0 = ds.cache.stats()
+        ms = timed_steps(ds, Wm, K, flush, False) if mode == "eager" else graph_steps(ds, Wm, K, flush)
+        st1 = ds.cache.stats()
+        misses = st1["misses"] - st0["misses"]
+        hits = st1["hits"] - st0["hits"]
+        out[mode] = {"tokens_per_s": K * n / (ms / 1000), "ms_per_step": ms / K,
+                     "hit_rate": hits / max(1, hits + misses), "misses_per_step": misses / K,
+                     "host_syncs": st1["host_syncs"] - st0["host_syncs"]}
+        ds.cache.close()
+        del ds
+    out["note"] = ("misses copied by the zero-copy fill kernel from mapped pinned blobs; nothing is read back, "
+                   "so the graph holds the whole step; L2 flushed before each step")
+    return out
+
+
 def extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=("resident", "prefill", "tiny", "qwen",
-                                                                              "trace"),
-           batches=(1, 4, 16), trace_steps=256, cpu=True):
+                                                                              "trace", "device_fill"),
+           batches=(1, 4, 16), trace_steps=256, cpu=True, fill="host"):
     """Context legs: every other workload of the layer, each with its roofline fraction and the oracle's
     single-core rate on a bounded sample."""
     import torch
@@ -628,6 +683,9 @@ def extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=("r
     from expert_cached_sparse_b200 import workloads as W
     out = {}
     tensor_peak, tensor_kind = measured_bf16_tflops()
+    # ---- the headline stream with device-initiated fills
+    if "device_fill" in legs:
+        out["decode_b16_device_fill"] = device_fill_leg(cfg, shape, blobs, wg, bias, 16, K, Wm, flush, device)
     # ---- the DeepSeek-shaped MXFP4 layer, every expert resident (decode, HBM-bound)
     for n in (batches if "resident" in legs else ()):
         r, _ = layer_leg(cfg, shape, blobs, wg, bias, n, K, Wm, flush, device, hbm_peak, "resident")
@@ -698,11 +756,11 @@ def extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=("r
         del qblobs
     # ---- the 40-layer NVFP4 decode trace: shared 1024-slot cache, misses filled over PCIe
     if "trace" in legs:
-        out["trace40"] = trace_leg(trace_steps, flush, device, hbm_peak, cpu)
+        out["trace40"] = trace_leg(trace_steps, flush, device, hbm_peak, cpu, fill=fill)
     return out
 
 
-def trace_leg(steps, flush, device, hbm_peak, cpu=True, distinct=64):
+def trace_leg(steps, flush, device, hbm_peak, cpu=True, distinct=64, fill="host"):
     """256 one-token decode steps through 40 NVFP4 layers (per-layer Zipf(1.0) routing with 10% rank
     drift every 32 steps) sharing one 1024-slot cache, cold; misses filled from pinned host RAM.
     Host blobs are aliased to `distinct` weight sets (cache behaviour does not depend on contents)."""
@@ -714,6 +772,8 @@ def trace_leg(steps, flush, device, hbm_peak, cpu=True, distinct=64):
     shape, blobs = pinned_blobs(cfg, 0, distinct)
     sb = A.moe_slot_bytes(shape)
     cache = A.MoeCache(shape, cfg.capacity, blobs, trace_capacity=0)
+    if fill == "device":
+        cache.set_fill_mode(1)
     wgs = [to_dev_bits(W.gen_wg(cfg, 0, l), device) for l in range(cfg.layers)]
     nep = (steps + cfg.drift_every - 1) // cfg.drift_every
     biases = {(l, ep): torch.from_numpy(W.gen_bias(cfg, 0, l, ep)).to(device)

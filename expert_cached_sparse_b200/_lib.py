@@ -26,6 +26,7 @@ MOE_ERR_UNSUPPORTED = -6
 MOE_ERR_STATE = -7
 DT_F32, DT_BF16 = 0, 1
 W_BF16, W_MXFP4, W_NVFP4 = 0, 1, 2
+FILL_HOST, FILL_DEVICE = 0, 1
 
 EXPORTS = [
     "moe_status_str", "moe_version", "moe_slot_bytes", "moe_cache_meta_bytes",
@@ -34,7 +35,8 @@ EXPORTS = [
     "moe_cache_read_trace", "moe_cache_get_stats", "moe_cache_snapshot", "moe_cache_capacity",
     "moe_cache_destroy", "moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine",
     "moe_layer_forward", "moe_profile_enable", "moe_profile_read", "moe_get_device_error",
-    "moe_permute_noalloc", "moe_act_terms",
+    "moe_permute_noalloc", "moe_act_terms", "moe_cache_set_fill_mode", "moe_cache_fill_mode",
+    "moe_cache_device_status",
 ]
 PROF_KINDS = ["router", "lookup", "permute", "ffn", "combine", "fill"]
 
@@ -95,6 +97,9 @@ def _load():
         "moe_profile_read": (C.c_int, [C.POINTER(MoeProf), C.c_int, C.c_int]),
         "moe_get_device_error": (C.c_int, [C.c_int]),
         "moe_act_terms": (C.c_int, [P, I32, I32, I32, I32, I32, P, P, P, P]),
+        "moe_cache_set_fill_mode": (C.c_int, [P, I32, P]),
+        "moe_cache_fill_mode": (I32, [P]),
+        "moe_cache_device_status": (C.c_int, [P, I32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)

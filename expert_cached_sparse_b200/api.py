@@ -161,6 +161,21 @@ class MoeCache:
         check("moe_cache_resize", rc)
         self.meta, self.pool = meta, pool
 
+    def set_fill_mode(self, mode: int, stream=None):
+        """L.FILL_HOST (host-issued DMA copies) or L.FILL_DEVICE (zero-copy fill kernel)."""
+        check("moe_cache_set_fill_mode", L.lib.moe_cache_set_fill_mode(self.handle, mode, stream_handle(stream)))
+
+    @property
+    def fill_mode(self) -> int:
+        return L.lib.moe_cache_fill_mode(self.handle)
+
+    def device_status(self, clear: bool = False) -> int:
+        """First error a lookup kernel recorded since the last clear (0 if none)."""
+        rc = L.lib.moe_cache_device_status(self.handle, 1 if clear else 0)
+        if rc in (L.MOE_ERR_CUDA,):
+            raise MoeError("moe_cache_device_status", rc)
+        return rc
+
     def read_trace(self, cap: int | None = None) -> np.ndarray:
         cap = self.trace_capacity if cap is None else cap
         buf = np.zeros(cap, L.TRACE_DTYPE)

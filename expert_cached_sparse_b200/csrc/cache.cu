@@ -10,6 +10,13 @@
 // ("FreeToken 290b model", section "Prepara el conjunto de expertos del
 // host").  Resize at scheduler safe points ("FreeToken quantization",
 // section "Flujo de configuracion de la cuantizacion de FreeToken").
+//
+// Two ways to bring misses in.  Host fills: the host reads the miss list
+// back and issues one DMA copy per miss.  Device fills: a copy kernel reads
+// the miss list where the lookup kernel left it and loads each blob from
+// pinned host memory mapped into the device's address space (zero-copy
+// loads over PCIe), so no call blocks and a decode step with misses can be
+// captured in a CUDA graph.
 #include <stdlib.h>
 #include <string.h>
 
@@ -33,6 +40,7 @@ struct MissEnt {
 };
 struct DevStats {
     unsigned long long lookups, hits, misses, evictions, trace_dropped;
+    unsigned long long dev_fills;   // blobs copied by fill_kernel
 };
 
 struct MetaPtrs {
@@ -47,10 +55,11 @@ struct MetaPtrs {
     int32_t* slot_hit;      // [E] hits only
     int32_t* slot_miss;     // [E] misses only
     moe_trace_rec* trace;   // [trace_cap]
+    const char** src_of;    // [L*E] device address of each key's mapped host blob (device fills)
 };
 
 struct MetaLayout {
-    size_t hdr, stats, tcount, slot_table, key_of, stamp, slot_all, slot_hit, slot_miss, trace, bytes;
+    size_t hdr, stats, tcount, slot_table, key_of, stamp, slot_all, slot_hit, slot_miss, trace, src, bytes;
 };
 
 static MetaLayout meta_layout(const moe_shape* s, int C, int trace_cap)
@@ -68,6 +77,7 @@ static MetaLayout meta_layout(const moe_shape* s, int C, int trace_cap)
     m.slot_hit = take(sizeof(int32_t) * (size_t)s->experts);
     m.slot_miss = take(sizeof(int32_t) * (size_t)s->experts);
     m.trace = take(sizeof(moe_trace_rec) * (size_t)trace_cap);
+    m.src = take(sizeof(void*) * (size_t)s->layers * s->experts);
     m.bytes = o;
     return m;
 }
@@ -87,6 +97,7 @@ static MetaPtrs meta_ptrs(void* base, const MetaLayout& l)
     p.slot_hit = reinterpret_cast<int32_t*>(b + l.slot_hit);
     p.slot_miss = reinterpret_cast<int32_t*>(b + l.slot_miss);
     p.trace = reinterpret_cast<moe_trace_rec*>(b + l.trace);
+    p.src_of = reinterpret_cast<const char**>(b + l.src);
     return p;
 }
 
@@ -220,6 +231,7 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int 
             hdr->status = MOE_ERR_CAPACITY;
             hdr->n_req = nreq_tot;
             hdr->n_hit = hdr->n_miss = hdr->n_evict = 0;
+            if (!hdr->sticky) hdr->sticky = MOE_ERR_CAPACITY;
         }
         for (int e = tid; e < E; e += NT) {
             m.slot_all[e] = m.slot_hit[e] = m.slot_miss[e] = -1;
@@ -379,6 +391,50 @@ __global__ void rollback_kernel(MetaPtrs m, int n)
     }
 }
 
+constexpr int kFillCtas = 16;
+constexpr int kFillThreads = 256;
+constexpr int kFillUnroll = 8;   // 16-byte loads in flight per thread
+
+// Device fills: copies every blob on the miss list of the last lookup from
+// mapped pinned host memory into its slot.  Runs after the lookup kernel in
+// stream order and reads what it wrote; a failed lookup leaves nothing to
+// copy.  The work is cut into rounds of kFillThreads * kFillUnroll 16-byte
+// words (32 KiB) dealt out to the CTAs; every thread issues all its loads
+// of a round before its stores, so 16 CTAs keep 512 KiB of PCIe reads in
+// flight.  Blob and slot addresses are 16-byte aligned, slot_bytes is a
+// multiple of 128.
+__global__ void __launch_bounds__(kFillThreads) fill_kernel(MetaPtrs m, int layer, int E, char* __restrict__ pool,
+                                                            size_t slot_bytes)
+{
+    const LookupHdr* h = m.hdr;
+    if (h->status != MOE_OK) return;
+    const int nm = h->n_miss;
+    if (nm <= 0) return;
+    constexpr size_t kRound = (size_t)kFillThreads * kFillUnroll;
+    const size_t n16 = slot_bytes / 16;
+    const size_t rounds = (n16 + kRound - 1) / kRound;
+    const size_t total = rounds * (size_t)nm;
+    for (size_t p = blockIdx.x; p < total; p += gridDim.x) {
+        const int i = (int)(p / rounds);
+        const size_t b = (p - (size_t)i * rounds) * kRound + threadIdx.x;
+        const MissEnt me = m.miss[i];
+        const int4* __restrict__ src = reinterpret_cast<const int4*>(m.src_of[(size_t)layer * E + me.expert]);
+        int4* __restrict__ dst = reinterpret_cast<int4*>(pool + (size_t)me.slot * slot_bytes);
+        int4 v[kFillUnroll];
+#pragma unroll
+        for (int u = 0; u < kFillUnroll; u++) {
+            const size_t w = b + (size_t)u * kFillThreads;
+            if (w < n16) v[u] = src[w];
+        }
+#pragma unroll
+        for (int u = 0; u < kFillUnroll; u++) {
+            const size_t w = b + (size_t)u * kFillThreads;
+            if (w < n16) dst[w] = v[u];
+        }
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) m.stats->dev_fills += (unsigned long long)nm;
+}
+
 }  // namespace moe
 
 // ====================================================================== host side
@@ -392,6 +448,8 @@ struct moe_cache {
     moe::MetaPtrs m;
     char* pool;
     std::vector<const void*> blobs;
+    std::vector<const char*> dsrc;       // device addresses of the blobs (device fills)
+    int fill_mode = MOE_FILL_HOST;
     std::vector<int> resident;           // host mirror: resident keys per layer
     std::vector<unsigned char> hbuf;     // LookupHdr + MissEnt[E]
     cudaEvent_t ev_lookup = nullptr, ev_fill = nullptr;
@@ -478,6 +536,38 @@ int cache_read_and_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t c
 
 cudaEvent_t cache_fill_event(const moe_cache* c) { return c->ev_fill; }
 
+int cache_fill_mode(const moe_cache* c) { return c->fill_mode; }
+
+// Device fills of the last lookup on `layer`: the copy stream waits for the
+// lookup (and so for every earlier reader of a victim slot on the compute
+// stream), runs fill_kernel and records ev_fill.  Nothing is read back.
+int cache_launch_device_fill(moe_cache* c, int layer, cudaStream_t copy)
+{
+    MOE_CUDA_TRY(cudaStreamWaitEvent(copy, c->ev_lookup, 0));
+    {
+        ProfScope ps(MOE_PROF_FILL, copy);
+        prof_count(MOE_PROF_FILL, 1);
+        fill_kernel<<<kFillCtas, kFillThreads, 0, copy>>>(c->m, layer, c->shape.experts, c->pool, c->slot_bytes);
+        MOE_LAUNCH_CHECK();
+    }
+    MOE_CUDA_TRY(cudaEventRecord(c->ev_fill, copy));
+    return MOE_OK;
+}
+
+// Host mirror of the resident keys per layer, recounted from the slot table.
+static int resync_resident(moe_cache* c, cudaStream_t st)
+{
+    const int E = c->shape.experts;
+    const size_t nkeys = (size_t)c->shape.layers * E;
+    std::vector<int32_t> table(nkeys);
+    MOE_CUDA_TRY(cudaStreamSynchronize(st));
+    MOE_CUDA_TRY(cudaMemcpy(table.data(), c->m.slot_table, 4 * nkeys, cudaMemcpyDeviceToHost));
+    c->resident.assign(c->shape.layers, 0);
+    for (size_t k = 0; k < nkeys; k++)
+        if (table[k] >= 0) c->resident[k / E]++;
+    return MOE_OK;
+}
+
 const moe_shape* cache_shape(const moe_cache* c) { return &c->shape; }
 
 int cache_capacity_int(const moe_cache* c) { return c->C; }
@@ -562,6 +652,11 @@ extern "C" int moe_cache_lookup_update(moe_cache* c, int32_t layer, const int32_
     cudaStream_t st = as_stream(stream), cp = as_stream(copy_stream);
     int rc = cache_launch_lookup(c, layer, d_idx, count, d_slot_of_expert, st);
     if (rc) return rc;
+    if (c->fill_mode == MOE_FILL_DEVICE) {
+        if ((rc = cache_launch_device_fill(c, layer, cp))) return rc;
+        MOE_CUDA_TRY(cudaStreamWaitEvent(st, c->ev_fill, 0));
+        return MOE_OK;
+    }
     if (cache_layer_resident(c, layer)) return MOE_OK;
     int nm = 0;
     rc = cache_read_and_fill(c, layer, st, cp, &nm);
@@ -596,7 +691,7 @@ extern "C" int moe_cache_get_stats(moe_cache* c, moe_cache_stats* out)
     out->misses = d.misses;
     out->evictions = d.evictions;
     out->trace_dropped = d.trace_dropped;
-    out->fill_bytes = c->fill_bytes;
+    out->fill_bytes = c->fill_bytes + d.dev_fills * (uint64_t)c->slot_bytes;
     out->host_syncs = c->host_syncs;
     return MOE_OK;
 }
@@ -626,6 +721,11 @@ extern "C" int moe_cache_resize(moe_cache* c, void* d_meta_new, size_t meta_byte
     if (meta_bytes < nl.bytes) return MOE_ERR_INVALID_ARG;
     cudaStream_t st = as_stream(stream);
     MOE_CUDA_TRY(cudaStreamSynchronize(st));
+    // device fills leave the host mirror stale: recount it first
+    if (c->fill_mode == MOE_FILL_DEVICE) {
+        int rc = resync_resident(c, st);
+        if (rc) return rc;
+    }
     const int E = c->shape.experts, C = c->C;
     const size_t nkeys = (size_t)c->shape.layers * E;
     std::vector<int32_t> table(nkeys), key(C);
@@ -708,6 +808,8 @@ extern "C" int moe_cache_resize(moe_cache* c, void* d_meta_new, size_t meta_byte
     MOE_CUDA_TRY(cudaMemcpyAsync(nm.stamp, nstamp.data(), 8 * (size_t)new_capacity, cudaMemcpyHostToDevice, st));
     if (ntc)
         MOE_CUDA_TRY(cudaMemcpyAsync(nm.trace, recs.data(), sizeof(moe_trace_rec) * ntc, cudaMemcpyHostToDevice, st));
+    if (!c->dsrc.empty())
+        MOE_CUDA_TRY(cudaMemcpyAsync(nm.src_of, c->dsrc.data(), sizeof(void*) * nkeys, cudaMemcpyHostToDevice, st));
     MOE_CUDA_TRY(cudaStreamSynchronize(st));
     c->C = new_capacity;
     c->d_meta = d_meta_new;
@@ -718,4 +820,65 @@ extern "C" int moe_cache_resize(moe_cache* c, void* d_meta_new, size_t meta_byte
     if (c->lookup_smem > 48 * 1024)
         MOE_CUDA_TRY(cudaFuncSetAttribute(lookup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, c->lookup_smem));
     return MOE_OK;
+}
+
+extern "C" int moe_cache_set_fill_mode(moe_cache* c, int32_t mode, void* stream)
+{
+    if (!c || (mode != MOE_FILL_HOST && mode != MOE_FILL_DEVICE)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    MOE_CUDA_TRY(cudaStreamSynchronize(st));
+    if (mode == MOE_FILL_DEVICE) {
+        const size_t nkeys = c->blobs.size();
+        std::vector<const char*> d(nkeys);
+        const void* last = nullptr;
+        const char* last_d = nullptr;
+        for (size_t k = 0; k < nkeys; k++) {
+            const char* b = static_cast<const char*>(c->blobs[k]);
+            if (b && b == last) { d[k] = last_d; continue; }   // keys often share a blob
+            if (!b || ((uintptr_t)b & 15)) return MOE_ERR_INVALID_ARG;
+            // both ends of the blob must be mapped host memory of one mapping
+            cudaPointerAttributes a0, a1;
+            if (cudaPointerGetAttributes(&a0, b) != cudaSuccess ||
+                cudaPointerGetAttributes(&a1, b + c->slot_bytes - 1) != cudaSuccess) {
+                cudaGetLastError();
+                return MOE_ERR_INVALID_ARG;
+            }
+            if (a0.type != cudaMemoryTypeHost || a1.type != cudaMemoryTypeHost || !a0.devicePointer ||
+                static_cast<const char*>(a1.devicePointer) !=
+                    static_cast<const char*>(a0.devicePointer) + c->slot_bytes - 1)
+                return MOE_ERR_INVALID_ARG;
+            last = b;
+            last_d = static_cast<const char*>(a0.devicePointer);
+            d[k] = last_d;
+        }
+        // The fill kernel runs beside the FFN kernels, whose CTAs need nearly
+        // all of an SM's shared memory.  An SM configures its L1 / shared
+        // split for the kernel it runs; the fill CTAs ask for the largest
+        // shared share so that FFN CTAs can join them on the same SMs.
+        MOE_CUDA_TRY(cudaFuncSetAttribute(fill_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                          (int)cudaSharedmemCarveoutMaxShared));
+        MOE_CUDA_TRY(cudaMemcpyAsync(c->m.src_of, d.data(), sizeof(void*) * nkeys, cudaMemcpyHostToDevice, st));
+        MOE_CUDA_TRY(cudaStreamSynchronize(st));
+        c->dsrc.swap(d);
+    } else if (c->fill_mode == MOE_FILL_DEVICE) {
+        int rc = resync_resident(c, st);
+        if (rc) return rc;
+    }
+    c->fill_mode = mode;
+    return MOE_OK;
+}
+
+extern "C" int32_t moe_cache_fill_mode(const moe_cache* c) { return c ? c->fill_mode : MOE_ERR_INVALID_ARG; }
+
+extern "C" int moe_cache_device_status(moe_cache* c, int32_t clear)
+{
+    if (!c) return MOE_ERR_INVALID_ARG;
+    MOE_CUDA_TRY(cudaDeviceSynchronize());
+    int32_t sticky = 0;
+    MOE_CUDA_TRY(cudaMemcpy(&sticky, &c->m.hdr->sticky, sizeof sticky, cudaMemcpyDeviceToHost));
+    if (clear && sticky) {
+        const int32_t zero = 0;
+        MOE_CUDA_TRY(cudaMemcpy(&c->m.hdr->sticky, &zero, sizeof zero, cudaMemcpyHostToDevice));
+    }
+    return sticky;
 }

@@ -1287,6 +1287,18 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
     volatile int* abort_v = abort_flag;
     const int grid = gridDim.x;
     const int NG = P.gpre[E];
+    if (NG == 0) {
+        // no expert with rows has a slot (a miss pass without misses): every
+        // CTA sees the same plan and leaves before the first grid barrier
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 1) {
+            tc_fence_after();
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(KC_::TMEM_COLS)
+                         : "memory");
+        }
+        return;
+    }
 
     if (warp == 0) {
         // ============ bulk copies of both phases.  A second cursor walks the

@@ -22,6 +22,8 @@ int cache_read_and_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t c
 cudaEvent_t cache_fill_event(const moe_cache* c);
 const moe_shape* cache_shape(const moe_cache* c);
 int cache_capacity_int(const moe_cache* c);
+int cache_fill_mode(const moe_cache* c);
+int cache_launch_device_fill(moe_cache* c, int layer, cudaStream_t copy);
 
 struct LayerWs {
     float* logits;
@@ -107,7 +109,17 @@ extern "C" int moe_layer_forward(moe_cache* c, int32_t layer, const void* d_x, i
     const char* pool = cache_pool(c);
     const size_t sb = cache_slot_bytes(c);
     const int C = cache_capacity_int(c);
-    if (cache_layer_resident(c, layer)) {
+    if (cache_fill_mode(c) == MOE_FILL_DEVICE) {
+        // the copy kernel takes the miss list from the lookup on the device:
+        // it starts first (it needs few SMs and only PCIe), the hits run
+        // beside it, the misses after it.  Nothing is read back.
+        if ((rc = cache_launch_device_fill(c, layer, cp))) return rc;
+        if ((rc = launch_ffn(s, pool, sb, C, cache_slot_hit(c), L.offsets, xp, A, L.y_perm, L.ffn_ws, st, gather)))
+            return rc;
+        MOE_CUDA_TRY(cudaStreamWaitEvent(st, cache_fill_event(c), 0));
+        if ((rc = launch_ffn(s, pool, sb, C, cache_slot_miss(c), L.offsets, xp, A, L.y_perm, L.ffn_ws, st, gather)))
+            return rc;
+    } else if (cache_layer_resident(c, layer)) {
         // every expert of this layer is resident: no miss is possible, nothing is read back
         if ((rc = launch_ffn(s, pool, sb, C, cache_slot_all(c), L.offsets, xp, A, L.y_perm, L.ffn_ws, st, gather)))
             return rc;

@@ -64,6 +64,7 @@ typedef enum {
 } moe_status;
 
 typedef enum { MOE_W_BF16 = 0, MOE_W_MXFP4 = 1, MOE_W_NVFP4 = 2 } moe_wfmt;
+typedef enum { MOE_FILL_HOST = 0, MOE_FILL_DEVICE = 1 } moe_fill_mode;
 typedef enum { MOE_DT_F32 = 0, MOE_DT_BF16 = 1 } moe_dtype;
 
 typedef struct {
@@ -98,7 +99,7 @@ typedef struct {
     uint64_t hits;         /* requested (layer, expert) pairs found resident */
     uint64_t misses;       /* requested pairs brought in */
     uint64_t evictions;
-    uint64_t fill_bytes;   /* bytes copied host -> device by fills */
+    uint64_t fill_bytes;   /* bytes copied host -> device by fills (both fill modes) */
     uint64_t host_syncs;   /* lookups that had to read the miss list on the host */
     uint64_t trace_dropped;/* records lost because the trace buffer was full */
 } moe_cache_stats;
@@ -110,12 +111,12 @@ typedef enum {
     MOE_PROF_PERMUTE = 2, /* histogram, scan, scatter/gather kernels */
     MOE_PROF_FFN = 3,     /* grouped FFN kernels (gate-up, down) */
     MOE_PROF_COMBINE = 4, /* combine kernel */
-    MOE_PROF_FILL = 5,    /* miss fills: host->device copies (not kernels) */
+    MOE_PROF_FILL = 5,    /* miss fills: host->device copies, or the device-fill kernel */
     MOE_PROF_COUNT = 6
 } moe_prof_kind;
 
 typedef struct {
-    uint64_t launches;  /* kernels launched (copies issued for MOE_PROF_FILL) */
+    uint64_t launches;  /* kernels launched (MOE_PROF_FILL: copies issued, or fill kernels) */
     uint64_t timed;     /* bracketed steps whose duration is in ms */
     double ms;          /* summed device time of the bracketed steps */
 } moe_prof_entry;
@@ -209,10 +210,14 @@ int moe_cache_create(const moe_shape* shape, void* d_meta, size_t meta_bytes, vo
  * -1 for the others.  Fills are issued on copy_stream after everything
  * already on `stream` is done, and `stream` waits for them, so work enqueued
  * on `stream` afterwards sees the weights.
- * Blocks the host until the miss list is known, except when every expert of
- * `layer` is already resident (then nothing is read back).
- * MOE_ERR_CAPACITY if more distinct experts are requested than slots exist;
- * the state is unchanged (the host learns this at the same sync point).
+ * Host fills (the default): blocks the host until the miss list is known,
+ * except when every expert of `layer` is already resident (then nothing is
+ * read back).  MOE_ERR_CAPACITY if more distinct experts are requested than
+ * slots exist; the state is unchanged (the host learns this at the same sync
+ * point).  Device fills (moe_cache_set_fill_mode): never blocks; the fill
+ * kernel runs on copy_stream and `stream` waits for it; a capacity error
+ * leaves the state unchanged, every slot_of entry -1, and is reported by
+ * moe_cache_device_status.
  * Pages: hits run directly on the GPU and misses are brought in ("FreeToken
  * 290b model", section "Como gestiona FreeToken el prellenado y la
  * decodificacion"); a cache entry is a logical (layer, expert) pair
@@ -235,6 +240,42 @@ int moe_cache_lookup_update(moe_cache* cache, int32_t layer, const int32_t* d_id
  */
 int moe_cache_resize(moe_cache* cache, void* d_meta_new, size_t meta_bytes, void* d_pool_new,
                      int32_t new_capacity, void* stream);
+
+/*
+ * Chooses how misses are brought in (default MOE_FILL_HOST).
+ *   MOE_FILL_HOST: the host reads the lookup's miss list back and issues one
+ *   cudaMemcpyAsync per miss on copy_stream (the DMA engine).
+ *   MOE_FILL_DEVICE: a copy kernel on copy_stream reads the miss list where
+ *   the lookup kernel wrote it and copies each missing blob from pinned host
+ *   memory, mapped into the device's address space, into its slot (zero-copy
+ *   loads over PCIe by 16 CTAs).  No call reads anything back, so
+ *   moe_cache_lookup_update and moe_layer_forward never block the host and a
+ *   whole decode step, misses included, can be captured in a CUDA graph.
+ *   The kernel waits for nothing on the device (stream order sequences it
+ *   after the lookup and before the miss-pass FFN), so it has no timeout.
+ *   Requires every blob of h_blobs to be 16-byte aligned page-locked host
+ *   memory mapped into the device's address space (cudaHostAlloc /
+ *   cudaMallocHost memory on a system with unified addressing, or
+ *   cudaHostRegister with cudaHostRegisterMapped), the whole blob inside one
+ *   mapping; otherwise MOE_ERR_INVALID_ARG and the mode is unchanged.  The
+ *   fill_fail testing hook of moe_cache_create applies to host fills only.
+ * The trace, the LRU state and the results are the same in both modes.
+ * Synchronises `stream`; call it at a safe point (no call of this cache in
+ * flight).
+ * Pages: misses are brought over PCIe from the host expert set into VRAM
+ * ("FreeToken 290b model", section "Como gestiona FreeToken el prellenado y
+ * la decodificacion"); who issues the copy is this library's choice.
+ */
+int moe_cache_set_fill_mode(moe_cache* cache, int32_t mode, void* stream);
+
+/* The current moe_fill_mode, or MOE_ERR_INVALID_ARG for a NULL cache. */
+int32_t moe_cache_fill_mode(const moe_cache* cache);
+
+/* First error a lookup kernel recorded since the last clear (MOE_ERR_CAPACITY,
+ * or MOE_ERR_INVALID_ARG for an expert index outside [0, E)), 0 if none;
+ * clear != 0 resets it.  The way to learn of a failed lookup under device
+ * fills, where calls do not read the lookup's status back.  Synchronous. */
+int moe_cache_device_status(moe_cache* cache, int32_t clear);
 
 /* Copies up to `cap` trace records, oldest first, into h_buf, reports how
  * many in *n_out, and clears the device trace buffer.  Synchronous. */
@@ -369,9 +410,11 @@ int moe_combine(const uint16_t* d_y_perm, const int32_t* d_row_of, const float* 
  * d_x [n][H] (x_dtype), d_wg [E][H] bf16, d_bias [E] or NULL; d_out [n][H]
  * in x_dtype.  d_ws: moe_layer_workspace_bytes() bytes.  d_topk_idx_out /
  * d_topk_w_out ([n][k], device) receive the routing when not NULL.
- * Blocks the host once, for the miss list, unless every expert of the layer
- * is resident; in that case nothing is read back and the call can be
- * captured in a CUDA graph.
+ * Host fills: blocks the host once, for the miss list, unless every expert
+ * of the layer is resident; in that case nothing is read back and the call
+ * can be captured in a CUDA graph.  Device fills (moe_cache_set_fill_mode):
+ * the fill kernel runs on copy_stream beside the hit FFN, nothing is read
+ * back, and every call can be captured in a CUDA graph.
  * Pages: hits execute on the GPU while misses are brought in ("FreeToken
  * 290b model", section "Como gestiona FreeToken el prellenado y la
  * decodificacion"); data movement overlaps computation ("FreeToken linux",
