@@ -218,6 +218,19 @@ def moe_layer_forward(cache: MoeCache, layer, x, wg, bias, out, ws, stream=None,
     check("moe_layer_forward", rc)
 
 
+# ------------------------------------------------------------------ testing hooks
+def moe_test_set_wait(cycles: int, withhold: bool = False) -> None:
+    """Bounded-wait limit (SM cycles, 0 = default) and stage withholding of later FFN launches."""
+    check("moe_test_set_wait", L.lib.moe_test_set_wait(int(cycles), 1 if withhold else 0))
+
+
+def moe_get_device_error(clear: bool = False) -> int:
+    rc = L.lib.moe_get_device_error(1 if clear else 0)
+    if rc == L.MOE_ERR_CUDA:
+        raise MoeError("moe_get_device_error", rc)
+    return rc
+
+
 # ------------------------------------------------------------------ profiling
 def moe_profile_enable(timing: bool) -> None:
     check("moe_profile_enable", L.lib.moe_profile_enable(1 if timing else 0))

@@ -163,6 +163,10 @@ struct RowSource {
     int k;
 };
 int ffn_device_error(int clear);   // BF16 streaming FFN's device error word (0: none)
+// Testing hook (moe_test_set_wait): the wait limit the FFN kernels launched
+// next get (dflt unless a test set one), and whether CTA 0 withholds a stage.
+long long test_wait_cycles(long long dflt);
+int test_withhold();
 int ffn_fp4_device_error(int clear);   // FP4 FFN's device error word (0: none)
 int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
                const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,

@@ -213,6 +213,8 @@ struct FfnArgs {
     uint16_t* out_y;        // phase 2: y [rows][R] bf16
     int32_t* cnt;           // per unit: pieces finished (units split across CTAs)
     float* pieces;          // [gridDim.x][2][kPieceFloats]
+    long long wait;         // limit of the bounded waits of the copy lane and the compute warps
+    int withhold;           // testing: CTA 0 leaves its first ring stage unfilled
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -244,17 +246,18 @@ __device__ __forceinline__ bool mbar_try_suspend(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait (about 2 s of clock), false on timeout.  With `abort` set the
-// wait also gives up as soon as another warp of the CTA has raised it, and
-// raises it itself on a timeout.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort = nullptr)
+// Bounded wait (`limit` cycles, about 2 s by default), false on timeout.
+// With `abort` set the wait also gives up as soon as another warp of the CTA
+// has raised it, and raises it itself on a timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort = nullptr,
+                                                  long long limit = kWaitCycles)
 {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
         if (mbar_try_suspend(bar, parity)) return true;
         if (abort && *abort) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             if (abort) *abort = 1;
             return false;
         }
@@ -382,11 +385,11 @@ struct Ring {
 template <int NQ>
 __device__ __forceinline__ bool run_unit(float (&acc)[2][4], const DecUnit& U, bool act, Ring& R,
                                          unsigned char* ring, uint64_t* full, uint64_t* empty, int w, int lane,
-                                         volatile int* abort)
+                                         volatile int* abort, long long limit)
 {
     const int g = lane >> 2, t = lane & 3, sw = (U.row0 + g) & 7;
     for (int kt = U.k0; kt < U.k1; kt++) {
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&full[R.st]), R.ph, abort))) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&full[R.st]), R.ph, abort, limit))) return false;
         const unsigned char* sg = ring + (size_t)R.st * kStage;
         if (act) mma_tile<NQ>(acc, sg, U.ng, w, lane, g, t, sw);
         __syncwarp();
@@ -497,17 +500,22 @@ __global__ void __launch_bounds__(kDecThreads, 3) ffn_kernel(FfnArgs a)
             uint32_t ph = 0;
             long issued = 0;
             bool ok = true;
+            int withheld = -1;   // testing: the stage left unfilled
             auto issue = [&](const DecUnit& U) {
                 for (int kt = U.k0; kt < U.k1 && ok; kt++) {
-                    if (!(ok = mbar_wait_bounded(smem_u32(&empty[st]), ph ^ 1, s_abort))) break;
+                    if (!(ok = mbar_wait_bounded(smem_u32(&empty[st]), ph ^ 1, s_abort, a.wait))) break;
                     const uint32_t bar = smem_u32(&full[st]);
                     unsigned char* sg = ring + (size_t)st * kStage;
                     const size_t ti = tile_index(8 * U.G, kt, RT, KP);
                     const uint32_t bytes = U.ng * kTile + U.nq * 1024;
-                    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                                 : "memory");
-                    bulk_copy(smem_u32(sg), U.blob + a.w_off + ti * kTile, U.ng * kTile, bar);
-                    bulk_copy(smem_u32(sg + kABytes), a.in + ((size_t)kt * RP + U.row0) * 64, U.nq * 1024, bar);
+                    if (a.withhold && blockIdx.x == 0 && issued == 0) {
+                        withheld = st;   // never filled, so the compute warps' wait for it runs out
+                    } else {
+                        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                                     : "memory");
+                        bulk_copy(smem_u32(sg), U.blob + a.w_off + ti * kTile, U.ng * kTile, bar);
+                        bulk_copy(smem_u32(sg + kABytes), a.in + ((size_t)kt * RP + U.row0) * 64, U.nq * 1024, bar);
+                    }
                     issued++;
                     if (++st == kRing) { st = 0; ph ^= 1; }
                 }
@@ -517,9 +525,10 @@ __global__ void __launch_bounds__(kDecThreads, 3) ffn_kernel(FfnArgs a)
                 issue(dec_unit(a, s_groups, sg.u, RT, RB, sg.p0, sg.p1));
             if (!ok) atomicCAS(&g_ffn_error, 0, (int)MOE_ERR_TIMEOUT);
             // let the last copies land before the CTA exits (stage i was last
-            // filled in this pass if i < st, else in the previous one)
+            // filled in this pass if i < st, else in the previous one; a
+            // withheld stage is never refilled: its consumers give up first)
             for (int i = 0; i < kRing && i < issued; i++)
-                mbar_wait_bounded(smem_u32(&full[i]), i < st ? ph : (ph ^ 1));
+                if (i != withheld) mbar_wait_bounded(smem_u32(&full[i]), i < st ? ph : (ph ^ 1));
         }
         return;
     }
@@ -535,8 +544,8 @@ __global__ void __launch_bounds__(kDecThreads, 3) ffn_kernel(FfnArgs a)
 #pragma unroll
             for (int i = 0; i < 4; i++) acc[q][i] = 0.0f;
         if (ok)
-            ok = U.nq == 1 ? run_unit<1>(acc, U, w < U.ng, R, ring, full, empty, w, lane, s_abort)
-                           : run_unit<2>(acc, U, w < U.ng, R, ring, full, empty, w, lane, s_abort);
+            ok = U.nq == 1 ? run_unit<1>(acc, U, w < U.ng, R, ring, full, empty, w, lane, s_abort, a.wait)
+                           : run_unit<2>(acc, U, w < U.ng, R, ring, full, empty, w, lane, s_abort, a.wait);
     };
     Seg sg{whole ? (long)blockIdx.x : b0};
     while (sg.next(whole, NU, KP, b1)) {
@@ -623,6 +632,8 @@ int launch_bf16(const moe_shape* s, const BlobLayout& bl, const void* pool, size
     a.rows = rows;
     a.cnt = w.cnt;
     a.pieces = w.pieces;
+    a.wait = test_wait_cycles(kWaitCycles);
+    a.withhold = test_withhold();
     const size_t smem = dec_smem_bytes(E);
     // persistent grid: as many CTAs as fit at once (recomputed when the
     // shared-memory size, which grows with E, changes); function attributes
@@ -735,6 +746,23 @@ extern "C" int moe_grouped_ffn(const moe_shape* shape, const void* d_slot_pool, 
     size_t sb = moe::blob_layout(shape).bytes;
     return moe::launch_ffn(shape, d_slot_pool, sb, pool_slots, d_slot_of_expert, d_expert_offsets, d_x_perm, rows,
                            d_y_perm, d_ws, moe::as_stream(stream));
+}
+
+namespace moe {
+namespace {
+long long g_test_wait = 0;   // 0: every kernel's default limit
+int g_test_withhold = 0;
+}  // namespace
+long long test_wait_cycles(long long dflt) { return g_test_wait > 0 ? g_test_wait : dflt; }
+int test_withhold() { return g_test_withhold; }
+}  // namespace moe
+
+extern "C" int moe_test_set_wait(int64_t cycles, int32_t withhold)
+{
+    if (cycles < 0) return MOE_ERR_INVALID_ARG;
+    moe::g_test_wait = cycles;
+    moe::g_test_withhold = withhold ? 1 : 0;
+    return MOE_OK;
 }
 
 extern "C" int moe_get_device_error(int clear)

@@ -32,7 +32,8 @@
 //  - decode cuts the concatenated K stages of all units into equal ranges
 //    per CTA (stream-K); the CTA finishing a unit sums its pieces in CTA
 //    order, so results are deterministic.  Prefill deals whole units.
-// Every wait is bounded; a timeout records MOE_ERR_TIMEOUT, raises the CTA's
+// Every wait is bounded (the limit is a kernel argument, about 2 s unless a
+// test shortens it); a timeout records MOE_ERR_TIMEOUT, raises the CTA's
 // abort flag so the other roles drain, and the kernel returns.
 #include <stdlib.h>
 #include <string.h>
@@ -48,7 +49,7 @@ namespace {
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kQuantThreads = 256;
-constexpr long long kWaitCycles = 4000000000ll;   // ~2 s before a wait gives up
+constexpr long long kWaitCycles = 4000000000ll;   // ~2 s: drains, and waits unless a test sets a limit
 constexpr int kMaxCtas = 160;                      // persistent grid: one CTA per SM at most
 constexpr int kSmemBudget = 227 * 1024;
 
@@ -104,15 +105,15 @@ __device__ __forceinline__ bool mbar_try_suspend(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 // Bounded wait: gives up when another role raised the abort flag, or after
-// kWaitCycles, in which case it records MOE_ERR_TIMEOUT and raises the flag.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag)
+// `limit` cycles, in which case it records MOE_ERR_TIMEOUT and raises the flag.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, long long limit)
 {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
         if (mbar_try_suspend(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitCycles) break;
+        if (clock64() - t0 > limit) break;
     }
     *abort_flag = 1;
     atomicCAS(&g_fp4_error, 0, (int)MOE_ERR_TIMEOUT);
@@ -575,6 +576,8 @@ struct Fp4Args {
     uint16_t* out_y;        // phase 2: y [rows][R] bf16
     int32_t* cnt;           // per unit: pieces finished (stream-K)
     float* pieces;          // [gridDim.x][2][128 * NMAX] partial accumulators (stream-K)
+    long long wait;         // limit of every bounded wait, in SM clock cycles
+    int withhold;           // testing: CTA 0 leaves its first ring stage unfilled
 };
 
 template <int WFMT, class CFG>
@@ -788,6 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
             uint32_t ph = 0;
             long issued = 0;
             bool ok = true, waited = false;
+            int withheld = -1;   // testing: the stage left unfilled
             const char* pend_src[D];
             uint32_t pend_bytes[D];
             int npend = 0;
@@ -795,8 +799,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
                 pdl_wait();
                 waited = true;
                 for (int i = 0; i < npend; i++) {
-                    bulk_g2s(smem_u32(ring + (size_t)i * STAGE + KC_::A_BYTES), pend_src[i], pend_bytes[i],
-                             smem_u32(&full[i]));
+                    if (pend_bytes[i])
+                        bulk_g2s(smem_u32(ring + (size_t)i * STAGE + KC_::A_BYTES), pend_src[i], pend_bytes[i],
+                                 smem_u32(&full[i]));
                 }
                 npend = 0;
             };
@@ -809,16 +814,23 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
                 const bool have_nx = nx.next(whole, NU, KC, b1);
                 const int4 gn = have_nx ? group_of(a, nx.u, RB) : g;
                 for (int c = sg.p0; c < sg.p1; c++) {
-                    if (!(ok = mbar_wait(smem_u32(&empty[st]), ph ^ 1, abort_v))) break;
+                    if (!(ok = mbar_wait(smem_u32(&empty[st]), ph ^ 1, abort_v, a.wait))) break;
                     const uint32_t bar = smem_u32(&full[st]);
                     unsigned char* sp = ring + (size_t)st * STAGE;
-                    mbar_expect_tx(bar, (uint32_t)(FM::CB + U.bb));
-                    bulk_g2s(smem_u32(sp), U.a + (size_t)c * FM::CB, FM::CB, bar);
-                    if (waited) {
-                        bulk_g2s(smem_u32(sp + KC_::A_BYTES), U.b + (size_t)c * U.bb, (uint32_t)U.bb, bar);
-                    } else {   // first pass over the ring: stage st == issued
-                        pend_src[npend] = U.b + (size_t)c * U.bb;
-                        pend_bytes[npend++] = (uint32_t)U.bb;
+                    if (a.withhold && blockIdx.x == 0 && issued == 0) {
+                        // testing: never filled, so the wait for it runs out
+                        withheld = st;
+                        pend_src[npend] = nullptr;
+                        pend_bytes[npend++] = 0;
+                    } else {
+                        mbar_expect_tx(bar, (uint32_t)(FM::CB + U.bb));
+                        bulk_g2s(smem_u32(sp), U.a + (size_t)c * FM::CB, FM::CB, bar);
+                        if (waited) {
+                            bulk_g2s(smem_u32(sp + KC_::A_BYTES), U.b + (size_t)c * U.bb, (uint32_t)U.bb, bar);
+                        } else {   // first pass over the ring: stage st == issued
+                            pend_src[npend] = U.b + (size_t)c * U.bb;
+                            pend_bytes[npend++] = (uint32_t)U.bb;
+                        }
                     }
                     issued++;
                     if (++st == D) { st = 0; ph ^= 1; }
@@ -830,8 +842,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
             }
             if (!waited) release_pending();
             // every issued copy lands before the CTA exits (stage i was last
-            // filled in this pass if i < st, else in the previous one)
-            for (int i = 0; i < D && i < issued; i++) mbar_drain(smem_u32(&full[i]), i < st ? ph : (ph ^ 1));
+            // filled in this pass if i < st, else in the previous one; a
+            // withheld stage is never refilled: its consumer gives up first)
+            for (int i = 0; i < D && i < issued; i++)
+                if (i != withheld) mbar_drain(smem_u32(&full[i]), i < st ? ph : (ph ^ 1));
         } else {
             pdl_wait();
         }
@@ -854,12 +868,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
                 const int ab = it & 1, nh = (U.n + 127) / 128;
                 const uint32_t id0 = idesc_fp4<WFMT>(U.n, 0), id1 = idesc_fp4<WFMT>(U.n, 2);
                 if (it >= 2) {   // the epilogue has read this accumulator's previous unit
-                    if (!(ok = mbar_wait(smem_u32(&acc_empty[ab]), ((it >> 1) - 1) & 1, abort_v))) break;
+                    if (!(ok = mbar_wait(smem_u32(&acc_empty[ab]), ((it >> 1) - 1) & 1, abort_v, a.wait))) break;
                     tc_fence_after();
                 }
                 const uint32_t dcol = tmem + (uint32_t)(ab * CFG::NMAX);
                 for (int c = sg.p0; c < sg.p1; c++, cc++) {
-                    if (!(ok = mbar_wait(smem_u32(&full[st]), ph, abort_v))) break;
+                    if (!(ok = mbar_wait(smem_u32(&full[st]), ph, abort_v, a.wait))) break;
                     tc_fence_after();
                     const uint32_t sfa = tmem + KC_::SF_COL + (uint32_t)((cc & 1) * KC_::SF_SET);
                     issue_chunk<WFMT, KC_::A_BYTES>(ring_s + (uint32_t)(st * STAGE), U.n, nh, dcol, sfa,
@@ -893,7 +907,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
         while (sg.next(whole, NU, KC, b1)) {
             const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC, group_of(a, sg.u, RB));
             const int ab = it & 1;
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[ab]), (it >> 1) & 1, abort_v));
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[ab]), (it >> 1) & 1, abort_v, a.wait));
             if (ok) tc_fence_after();
             float tsc = 1.0f;
             if (WFMT == MOE_W_NVFP4) tsc = __ldg(reinterpret_cast<const float*>(U.blob + a.ts_off) + PHASE - 1);
@@ -1015,7 +1029,7 @@ struct FusedCfg {
 // Bounded grid barrier for the four epilogue warps of every CTA.  Their
 // global writes before it are visible to every CTA after it (generic and
 // async proxy: operand images are read by bulk copies).
-__device__ __forceinline__ bool grid_sync_epi(int etid, volatile int* s_flag)
+__device__ __forceinline__ bool grid_sync_epi(int etid, volatile int* s_flag, long long limit)
 {
     asm volatile("fence.proxy.async.global;" ::: "memory");
     __threadfence();
@@ -1033,7 +1047,7 @@ __device__ __forceinline__ bool grid_sync_epi(int etid, volatile int* s_flag)
             const long long t0 = clock64();
             while (*reinterpret_cast<volatile unsigned*>(&g_gb_gen) == gen) {
                 if (*reinterpret_cast<volatile int*>(&g_gb_abort)) { ok = false; break; }
-                if (clock64() - t0 > kWaitCycles) {
+                if (clock64() - t0 > limit) {
                     ok = false;
                     atomicExch(&g_gb_abort, 1);
                     atomicCAS(&g_fp4_error, 0, (int)MOE_ERR_TIMEOUT);
@@ -1309,7 +1323,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
             int st = 0;
             uint32_t ph = 0;
             long issued = 0;
-            bool ok = mbar_wait(smem_u32(xloaded), 0, abort_v);   // the x loads go first
+            bool ok = mbar_wait(smem_u32(xloaded), 0, abort_v, f.p1.wait);   // the x loads go first
+            int withheld = -1;   // testing: the stage left unfilled
             int pend_st[D];
             const char* pend_src[D];
             uint32_t pend_bytes[D];
@@ -1355,7 +1370,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
                 int npend = 0;
                 bool open = false;   // this phase's activation images are published
                 auto release = [&]() -> bool {
-                    if (!mbar_wait(smem_u32(&gate[phase]), 0, abort_v)) return false;
+                    if (!mbar_wait(smem_u32(&gate[phase]), 0, abort_v, f.p1.wait)) return false;
                     asm volatile("fence.proxy.async.global;" ::: "memory");
                     for (int i = 0; i < npend; i++)
                         bulk_g2s(smem_u32(ring + (size_t)pend_st[i] * STAGE + KC_::A_BYTES), pend_src[i],
@@ -1371,31 +1386,44 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
                     for (int c = sg.p0; c < sg.p1; c++) {
                         // a ring full of held-back stages: wait for the gate before reusing one
                         if (!open && npend == D && !(ok = release())) break;
-                        if (!(ok = mbar_wait(smem_u32(&empty[st]), ph ^ 1, abort_v))) break;
+                        if (!(ok = mbar_wait(smem_u32(&empty[st]), ph ^ 1, abort_v, f.p1.wait))) break;
                         const uint32_t bar = smem_u32(&full[st]);
                         unsigned char* sp = ring + (size_t)st * STAGE;
-                        mbar_expect_tx(bar, (uint32_t)(FM::CB + U.bb));
-                        bulk_g2s(smem_u32(sp), U.a + (size_t)c * FM::CB, FM::CB, bar);
-                        if (const char* pa = pf_next()) prefetch_l2(pa, FM::CB);
-                        if (!open && mbar_try(smem_u32(&gate[phase]), 0) && !(ok = release())) break;
-                        if (open) {
-                            bulk_g2s(smem_u32(sp + KC_::A_BYTES), U.b + (size_t)c * U.bb, (uint32_t)U.bb, bar);
+                        if (f.p1.withhold && blockIdx.x == 0 && issued == 0) {
+                            withheld = st;   // testing: never filled, so the wait for it runs out
                         } else {
-                            pend_st[npend] = st;
-                            pend_src[npend] = U.b + (size_t)c * U.bb;
-                            pend_bytes[npend++] = (uint32_t)U.bb;
+                            mbar_expect_tx(bar, (uint32_t)(FM::CB + U.bb));
+                            bulk_g2s(smem_u32(sp), U.a + (size_t)c * FM::CB, FM::CB, bar);
+                            if (const char* pa = pf_next()) prefetch_l2(pa, FM::CB);
+                            // (the gate has passed here, so release() cannot fail)
+                            if (!open && mbar_try(smem_u32(&gate[phase]), 0)) release();
+                            if (open) {
+                                bulk_g2s(smem_u32(sp + KC_::A_BYTES), U.b + (size_t)c * U.bb, (uint32_t)U.bb, bar);
+                            } else {
+                                pend_st[npend] = st;
+                                pend_src[npend] = U.b + (size_t)c * U.bb;
+                                pend_bytes[npend++] = (uint32_t)U.bb;
+                            }
                         }
                         issued++;
                         if (++st == D) { st = 0; ph ^= 1; }
                     }
                 }
                 if (ok && !open && npend > 0) ok = release();
+                if (!ok) {
+                    // after an abort the held-back activation copies are issued
+                    // anyway (their data is not used), so that every stage whose
+                    // weight copy went out completes its phase before the drain
+                    for (int i = 0; i < npend; i++)
+                        bulk_g2s(smem_u32(ring + (size_t)pend_st[i] * STAGE + KC_::A_BYTES), pend_src[i],
+                                 pend_bytes[i], smem_u32(&full[pend_st[i]]));
+                    npend = 0;
+                }
             }
-            // every issued copy lands before the CTA exits (a stage whose
-            // activation copy was never released completes no phase: the
-            // drain gives up on it after the time limit, which only happens
-            // after an abort)
-            for (int i = 0; i < D && i < issued; i++) mbar_drain(smem_u32(&full[i]), i < st ? ph : (ph ^ 1));
+            // every issued copy lands before the CTA exits (a withheld stage
+            // is never refilled: its consumer gives up first)
+            for (int i = 0; i < D && i < issued; i++)
+                if (i != withheld) mbar_drain(smem_u32(&full[i]), i < st ? ph : (ph ^ 1));
         }
     } else if (warp == 1) {
         // ============ scale-factor copies and MMAs of both phases
@@ -1418,12 +1446,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
                     const int ab = it & 1, nh = (U.n + 127) / 128;
                     const uint32_t id0 = idesc_fp4<WFMT>(U.n, 0), id1 = idesc_fp4<WFMT>(U.n, 2);
                     if (it >= 2) {
-                        if (!(ok = mbar_wait(smem_u32(&acc_empty[ab]), ((it >> 1) - 1) & 1, abort_v))) break;
+                        if (!(ok = mbar_wait(smem_u32(&acc_empty[ab]), ((it >> 1) - 1) & 1, abort_v, f.p1.wait))) break;
                         tc_fence_after();
                     }
                     const uint32_t dcol = tmem + (uint32_t)(ab * CFG::NMAX);
                     for (int c = sg.p0; c < sg.p1; c++, cc++) {
-                        if (!(ok = mbar_wait(smem_u32(&full[st]), ph, abort_v))) break;
+                        if (!(ok = mbar_wait(smem_u32(&full[st]), ph, abort_v, f.p1.wait))) break;
                         tc_fence_after();
                         const uint32_t sfa = tmem + KC_::SF_COL + (uint32_t)((cc & 1) * KC_::SF_SET);
                         issue_chunk<WFMT, KC_::A_BYTES>(ring_s + (uint32_t)(st * STAGE), U.n, nh, dcol, sfa,
@@ -1463,7 +1491,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
                     fused_quant_items<WFMT, T, false>(P, f.x, a.K, f.gather, f.gk, f.bx, f.rex_x, first, step, items,
                                                       lane, xloaded);
             }
-            ok = grid_sync_epi(etid, s_flag) && ok;   // terms published (phase 0: counters zero)
+            ok = grid_sync_epi(etid, s_flag, f.p1.wait) && ok;   // terms published (phase 0: counters zero)
             if (etid == 0) mbar_arrive(smem_u32(&gate[phase]));
             const int RB = a.R / 128, KC = a.K / 256, NU = NG * RB;
             const long W = (long)NU * KC;
@@ -1474,7 +1502,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
                 while (sg.next(false, NU, KC, b1)) {
                     const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC, plan_group(P, sg.u / RB, NT, bfull));
                     const int ab = it & 1;
-                    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[ab]), (it >> 1) & 1, abort_v));
+                    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[ab]), (it >> 1) & 1, abort_v, f.p1.wait));
                     if (ok) tc_fence_after();
                     float tsc = 1.0f;
                     if (WFMT == MOE_W_NVFP4) tsc = __ldg(reinterpret_cast<const float*>(U.blob + a.ts_off) + phase);
@@ -1540,7 +1568,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
                     it++;
                 }
             }
-            if (phase == 0) ok = grid_sync_epi(etid, s_flag) && ok;   // h complete before its terms are taken
+            if (phase == 0) ok = grid_sync_epi(etid, s_flag, f.p1.wait) && ok;   // h complete before its terms are taken
         }
     }
     tc_fence_before();
@@ -1692,6 +1720,8 @@ int run_fp4(const moe_shape* s, const BlobLayout& bl, const void* pool, size_t s
     a.gtab = w.gtab;
     a.cnt = w.cnt;
     a.pieces = w.pieces;
+    a.wait = test_wait_cycles(kWaitCycles);
+    a.withhold = test_withhold();
     const int grid = sms < kMaxCtas ? sms : kMaxCtas;
     constexpr int smem = KCfg<WFMT, CFG>::SMEM;
     a.w_off = bl.w13;
@@ -1760,6 +1790,8 @@ int run_fp4_fused(const moe_shape* s, const BlobLayout& bl, const void* pool, si
     a.rex = WFMT == MOE_W_NVFP4 ? w.rex_x : nullptr;
     a.out_h = w.h32;
     a.cnt = w.cnt;
+    a.wait = test_wait_cycles(kWaitCycles);
+    a.withhold = test_withhold();
     Fp4Args& b = f.p2;
     b = a;
     b.w_off = bl.w2;

@@ -468,9 +468,25 @@ int moe_profile_read(moe_prof_entry* h_out, int count, int reset);
 /*
  * First error recorded by a device-side bounded wait since the last clear
  * (MOE_ERR_TIMEOUT when a kernel gave up waiting and drained instead of
- * hanging), 0 if none; clear != 0 resets it.  Synchronous.
+ * hanging), 0 if none; clear != 0 resets it.  Synchronous.  The grouped FFN
+ * results of a call that timed out, and of FP4 decode calls made while the
+ * error is set (their grid barriers give up at once), are undefined; clear
+ * the error before relying on results again.
  */
 int moe_get_device_error(int clear);
+
+/*
+ * Testing hook, process-wide, for grouped-FFN launches made afterwards:
+ * `cycles` > 0 sets the limit of the kernels' bounded waits to that many SM
+ * clock cycles (0 restores the default of about 2 s), and withhold != 0
+ * makes the first CTA's copy issuer leave its first ring stage unfilled, so
+ * that the wait for it runs out: the kernel records MOE_ERR_TIMEOUT, lets
+ * its own copies and MMAs finish and returns.  Drains of a CTA's own
+ * asynchronous work keep the default limit.  MOE_ERR_INVALID_ARG for
+ * cycles < 0.  Not thread-safe with concurrent launches.
+ * Pages: none (a robustness test of this library's bounded waits).
+ */
+int moe_test_set_wait(int64_t cycles, int32_t withhold);
 
 #ifdef __cplusplus
 }
