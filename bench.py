@@ -54,7 +54,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--resident-batch", default="1,4,16", help="batch sizes of the resident decode leg")
-    p.add_argument("--leg", choices=["all", "resident", "prefill", "tiny", "qwen", "trace", "device_fill"],
+    p.add_argument("--leg", choices=["all", "resident", "prefill", "tiny", "qwen", "trace", "device_fill",
+                                    "prefill_layers"],
                    default="all",
                    help="run only that context leg (profiling); prints its own JSON line")
     p.add_argument("--trace-steps", type=int, default=256, help="decode steps of the 40-layer trace leg")
@@ -647,6 +648,66 @@ def layer_leg(cfg, shape, blobs, wg, bias, n, steps, warm, flush, device, hbm_pe
     return out, ds.x_host
 
 
+def prefill_layers_leg(device, nl=4, n=4096, distinct=24, reps=2):
+    """4096 tokens through 4 DeepSeek-shaped MXFP4 layers (each with its own input), cold cache: with 512 slots the next layer's 256 experts stream in over PCIe while the current layer
+    computes; with 256 slots (one layer) its fills follow the compute.  Compute alone is timed on a
+    warm 1024-slot cache (every lookup hits).  Host blobs aliased to `distinct` weight sets."""
+    import torch
+
+    from expert_cached_sparse_b200 import api as A
+    from expert_cached_sparse_b200 import workloads as W
+    cfg = W.scaled(W.DS_PREFILL, layers=nl)
+    E = cfg.experts
+    shape, blobs = pinned_blobs(cfg, 0, distinct)
+    sb = A.moe_slot_bytes(shape)
+    bp = measure_bp(device, list({b.data_ptr(): b for b in blobs}.values()))
+    wgs = [to_dev_bits(W.gen_wg(cfg, 0, l), device) for l in range(nl)]
+    biases = [torch.from_numpy(W.gen_bias(cfg, 0, l, 0)).to(device) for l in range(nl)]
+    xs = [to_dev_bits(W.gen_x(cfg, 0, n, "prefill", l), device) for l in range(nl)]
+    outs = [torch.empty_like(xs[0]) for _ in range(nl)]
+    ws = torch.empty(A.moe_prefill_workspace_bytes(shape, n), dtype=torch.uint8, device=device)
+    st, cp = torch.cuda.Stream(device), torch.cuda.Stream(device)
+
+    def run(cache):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(st)
+        A.moe_prefill_forward(cache, 0, xs, wgs, biases, outs, ws, stream=st, copy_stream=cp)
+        b.record(st)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+    out = {"layers": nl, "tokens": n, "bp_GBps": bp, "layer_fill_bytes": E * sb, "host_blob_sets": distinct}
+    warm = A.MoeCache(shape, nl * E, blobs, trace_capacity=0)
+    run(warm)
+    compute_ms = min(run(warm) for _ in range(reps))
+    warm.close()
+    del warm
+    out["compute_ms"] = compute_ms
+    for name, cap in (("double_buffered_512_slots", 2 * E), ("one_layer_256_slots", E)):
+        ts = []
+        for _ in range(reps):
+            cache = A.MoeCache(shape, cap, blobs, trace_capacity=0)
+            ts.append(run(cache))
+            cache.close()
+            del cache
+        out[name] = {"ms": min(ts), "tokens_per_s": n / (min(ts) / 1000)}
+    fill_ms = E * sb / (bp * 1e9) * 1e3
+    layer_ms = compute_ms / nl
+    # the first layer's fills precede any compute; then each layer's fills hide the previous
+    # layer's compute (or the reverse); the last layer computes alone
+    pipe_ms = fill_ms + (nl - 1) * max(fill_ms, layer_ms) + layer_ms
+    out["bound"] = {"per_layer_ms": max(layer_ms, fill_ms), "pipeline_ms": pipe_ms,
+                    "sequential_ms": nl * (fill_ms + layer_ms),
+                    "note": "per layer max(compute, layer bytes / Bp); pipeline = fill + (L-1) max(fill, "
+                            "compute) + compute; sequential = L (fill + compute)"}
+    out["double_buffered_512_slots"]["frac_of_pipeline_bound"] = pipe_ms / out["double_buffered_512_slots"]["ms"]
+    out["one_layer_256_slots"]["frac_of_sequential_bound"] = out["bound"]["sequential_ms"] / \
+        out["one_layer_256_slots"]["ms"]
+    del blobs
+    return out
+
+
 def device_fill_leg(cfg, shape, blobs, wg, bias, n, K, Wm, flush, device):
     """The headline decode stream (cold 64-slot cache) with device fills: eager calls, then
     a fresh cache whose whole step, misses included, is one CUDA graph replayed per step."""
@@ -673,7 +734,8 @@ def device_fill_leg(cfg, shape, blobs, wg, bias, n, K, Wm, flush, device):
 
 
 def extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=("resident", "prefill", "tiny", "qwen",
-                                                                              "trace", "device_fill"),
+                                                                              "trace", "device_fill",
+                                                                              "prefill_layers"),
            batches=(1, 4, 16), trace_steps=256, cpu=True, fill="host"):
     """Context legs: every other workload of the layer, each with its roofline fraction and the oracle's
     single-core rate on a bounded sample."""
@@ -683,6 +745,9 @@ def extras(cfg, shape, blobs, wg, bias, K, Wm, flush, device, hbm_peak, legs=("r
     from expert_cached_sparse_b200 import workloads as W
     out = {}
     tensor_peak, tensor_kind = measured_bf16_tflops()
+    # ---- multi-layer prefill with full-layer double buffering
+    if "prefill_layers" in legs:
+        out["prefill_4x4096_double_buffered"] = prefill_layers_leg(device)
     # ---- the headline stream with device-initiated fills
     if "device_fill" in legs:
         out["decode_b16_device_fill"] = device_fill_leg(cfg, shape, blobs, wg, bias, 16, K, Wm, flush, device)

@@ -36,7 +36,7 @@ EXPORTS = [
     "moe_cache_destroy", "moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine",
     "moe_layer_forward", "moe_profile_enable", "moe_profile_read", "moe_get_device_error",
     "moe_permute_noalloc", "moe_act_terms", "moe_cache_set_fill_mode", "moe_cache_fill_mode",
-    "moe_cache_device_status", "moe_test_set_wait",
+    "moe_cache_device_status", "moe_test_set_wait", "moe_prefill_workspace_bytes", "moe_prefill_forward",
 ]
 PROF_KINDS = ["router", "lookup", "permute", "ffn", "combine", "fill"]
 
@@ -101,6 +101,8 @@ def _load():
         "moe_cache_fill_mode": (I32, [P]),
         "moe_cache_device_status": (C.c_int, [P, I32]),
         "moe_test_set_wait": (C.c_int, [C.c_int64, I32]),
+        "moe_prefill_workspace_bytes": (SZ, [SP, I32]),
+        "moe_prefill_forward": (C.c_int, [P, I32, I32, P, I32, P, P, I32, P, P, SZ, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)

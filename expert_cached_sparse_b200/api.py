@@ -218,6 +218,27 @@ def moe_layer_forward(cache: MoeCache, layer, x, wg, bias, out, ws, stream=None,
     check("moe_layer_forward", rc)
 
 
+def moe_prefill_workspace_bytes(shape, n) -> int:
+    return L.lib.moe_prefill_workspace_bytes(C.byref(shape), n)
+
+
+def moe_prefill_forward(cache: MoeCache, layer0, xs, wgs, biases, outs, ws, stream=None, copy_stream=None,
+                        topk_idx_out=None):
+    """Layers layer0 .. layer0+len(xs)-1 over one prompt; xs / wgs / biases / outs are per-layer
+    device tensors (biases may be None or hold None; outs[i] may be xs[i+1])."""
+    nl = len(xs)
+    if not (len(wgs) == len(outs) == nl) or (biases is not None and len(biases) != nl):
+        raise ValueError("per-layer lists of different lengths")
+    n = xs[0].shape[0] if nl else 0
+    arr = lambda ts: (C.c_void_p * max(1, nl))(*[ptr(t) for t in ts])
+    xa, wa, oa = arr(xs), arr(wgs), arr(outs)
+    ba = None if biases is None else arr(biases)
+    rc = L.lib.moe_prefill_forward(cache.handle, layer0, nl, xa, _dt(xs[0]) if nl else 0, wa, ba, n, oa, ptr(ws),
+                                   ws.numel() * ws.element_size(), stream_handle(stream), stream_handle(copy_stream),
+                                   ptr(topk_idx_out))
+    check("moe_prefill_forward", rc)
+
+
 # ------------------------------------------------------------------ testing hooks
 def moe_test_set_wait(cycles: int, withhold: bool = False) -> None:
     """Bounded-wait limit (SM cycles, 0 = default) and stage withholding of later FFN launches."""

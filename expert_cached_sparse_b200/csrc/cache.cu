@@ -453,6 +453,7 @@ struct moe_cache {
     std::vector<int> resident;           // host mirror: resident keys per layer
     std::vector<unsigned char> hbuf;     // LookupHdr + MissEnt[E]
     cudaEvent_t ev_lookup = nullptr, ev_fill = nullptr;
+    cudaEvent_t ev_pf[2] = {nullptr, nullptr};   // fills of the two layers a prefill has in flight
     uint64_t fill_bytes = 0, host_syncs = 0, fills_issued = 0;
     long fault_fill_at = 0;              // MOE_FAULT_INJECT=fill_fail:<n>
     int lookup_smem = 0;
@@ -488,11 +489,12 @@ size_t cache_slot_bytes(const moe_cache* c) { return c->slot_bytes; }
 
 // Host side of a lookup that may miss: wait for the lookup kernel, read the
 // miss list, issue one copy per miss on `copy` after everything before the
-// lookup on the compute stream is done, and record ev_fill.  *n_miss gets
-// the number of fills issued; the caller makes the compute stream wait on
-// ev_fill when *n_miss > 0.
-int cache_read_and_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t copy, int* n_miss)
+// lookup on the compute stream is done, and record `ev` (ev_fill by
+// default).  *n_miss gets the number of fills issued; the caller makes the
+// compute stream wait on the event when *n_miss > 0.
+int cache_read_and_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t copy, int* n_miss, cudaEvent_t ev)
 {
+    if (!ev) ev = c->ev_fill;
     *n_miss = 0;
     const int E = c->shape.experts;
     // one read-back of the header and the whole miss list, ordered after the
@@ -529,7 +531,7 @@ int cache_read_and_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t c
     }
     c->fills_issued += (uint64_t)h->n_miss;
     c->fill_bytes += (uint64_t)h->n_miss * c->slot_bytes;
-    MOE_CUDA_TRY(cudaEventRecord(c->ev_fill, copy));
+    MOE_CUDA_TRY(cudaEventRecord(ev, copy));
     *n_miss = h->n_miss;
     return MOE_OK;
 }
@@ -541,8 +543,9 @@ int cache_fill_mode(const moe_cache* c) { return c->fill_mode; }
 // Device fills of the last lookup on `layer`: the copy stream waits for the
 // lookup (and so for every earlier reader of a victim slot on the compute
 // stream), runs fill_kernel and records ev_fill.  Nothing is read back.
-int cache_launch_device_fill(moe_cache* c, int layer, cudaStream_t copy)
+int cache_launch_device_fill(moe_cache* c, int layer, cudaStream_t copy, cudaEvent_t ev)
 {
+    if (!ev) ev = c->ev_fill;
     MOE_CUDA_TRY(cudaStreamWaitEvent(copy, c->ev_lookup, 0));
     {
         ProfScope ps(MOE_PROF_FILL, copy);
@@ -550,9 +553,27 @@ int cache_launch_device_fill(moe_cache* c, int layer, cudaStream_t copy)
         fill_kernel<<<kFillCtas, kFillThreads, 0, copy>>>(c->m, layer, c->shape.experts, c->pool, c->slot_bytes);
         MOE_LAUNCH_CHECK();
     }
-    MOE_CUDA_TRY(cudaEventRecord(c->ev_fill, copy));
+    MOE_CUDA_TRY(cudaEventRecord(ev, copy));
     return MOE_OK;
 }
+
+// The fills of the lookup just enqueued on `st` for `layer`, whichever fill
+// mode the cache is in; `ev` completes once they have landed (recorded on
+// `st` itself when there is nothing to copy), so work that waits on it sees
+// every slot of the lookup filled.
+int cache_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t copy, cudaEvent_t ev)
+{
+    if (c->fill_mode == MOE_FILL_DEVICE) return cache_launch_device_fill(c, layer, copy, ev);
+    int nm = 0;
+    if (!cache_layer_resident(c, layer)) {
+        int rc = cache_read_and_fill(c, layer, st, copy, &nm, ev);
+        if (rc) return rc;
+    }
+    if (nm == 0) MOE_CUDA_TRY(cudaEventRecord(ev, st));
+    return MOE_OK;
+}
+
+cudaEvent_t cache_prefill_event(const moe_cache* c, int i) { return c->ev_pf[i & 1]; }
 
 // Host mirror of the resident keys per layer, recounted from the slot table.
 static int resync_resident(moe_cache* c, cudaStream_t st)
@@ -612,9 +633,11 @@ extern "C" int moe_cache_create(const moe_shape* shape, void* d_meta, size_t met
         if (!strncmp(fi, "fill_fail:", 10)) c->fault_fill_at = atol(fi + 10);
     }
     cudaStream_t st = as_stream(stream);
-    auto fail = [&](int rc) { delete c; return rc; };
+    auto fail = [&](int rc) { moe_cache_destroy(c); return rc; };
     if (cudaEventCreateWithFlags(&c->ev_lookup, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&c->ev_fill, cudaEventDisableTiming) != cudaSuccess)
+        cudaEventCreateWithFlags(&c->ev_fill, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c->ev_pf[0], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c->ev_pf[1], cudaEventDisableTiming) != cudaSuccess)
         return fail(MOE_ERR_CUDA);
     if (c->lookup_smem > 48 * 1024 &&
         cudaFuncSetAttribute(lookup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, c->lookup_smem) !=
@@ -638,6 +661,8 @@ extern "C" int moe_cache_destroy(moe_cache* c)
     if (!c) return MOE_ERR_INVALID_ARG;
     if (c->ev_lookup) cudaEventDestroy(c->ev_lookup);
     if (c->ev_fill) cudaEventDestroy(c->ev_fill);
+    for (cudaEvent_t e : c->ev_pf)
+        if (e) cudaEventDestroy(e);
     delete c;
     return MOE_OK;
 }

@@ -177,4 +177,22 @@ int launch_ffn_fp4(const moe_shape* s, const void* pool, size_t slot_bytes, int 
                    cudaStream_t st, const RowSource* gather);
 int launch_combine(const uint16_t* y_perm, const int32_t* row_of, const float* w, int n, int k, int H,
                    void* out, int out_dtype, cudaStream_t st);
+
+// ---------------------------------------------------------------- cache internals (cache.cu)
+int cache_launch_lookup(moe_cache* c, int layer, const int32_t* idx, int count, int32_t* slot_user, cudaStream_t st);
+bool cache_layer_resident(const moe_cache* c, int layer);
+const int32_t* cache_slot_all(const moe_cache* c);
+const int32_t* cache_slot_hit(const moe_cache* c);
+const int32_t* cache_slot_miss(const moe_cache* c);
+const char* cache_pool(const moe_cache* c);
+size_t cache_slot_bytes(const moe_cache* c);
+int cache_read_and_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t copy, int* n_miss,
+                        cudaEvent_t ev = nullptr);
+cudaEvent_t cache_fill_event(const moe_cache* c);
+const moe_shape* cache_shape(const moe_cache* c);
+int cache_capacity_int(const moe_cache* c);
+int cache_fill_mode(const moe_cache* c);
+int cache_launch_device_fill(moe_cache* c, int layer, cudaStream_t copy, cudaEvent_t ev = nullptr);
+int cache_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t copy, cudaEvent_t ev);
+cudaEvent_t cache_prefill_event(const moe_cache* c, int i);
 }  // namespace moe

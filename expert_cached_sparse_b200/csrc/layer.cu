@@ -11,20 +11,6 @@
 #include "common.cuh"
 
 namespace moe {
-int cache_launch_lookup(moe_cache* c, int layer, const int32_t* idx, int count, int32_t* slot_user, cudaStream_t st);
-bool cache_layer_resident(const moe_cache* c, int layer);
-const int32_t* cache_slot_all(const moe_cache* c);
-const int32_t* cache_slot_hit(const moe_cache* c);
-const int32_t* cache_slot_miss(const moe_cache* c);
-const char* cache_pool(const moe_cache* c);
-size_t cache_slot_bytes(const moe_cache* c);
-int cache_read_and_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t copy, int* n_miss);
-cudaEvent_t cache_fill_event(const moe_cache* c);
-const moe_shape* cache_shape(const moe_cache* c);
-int cache_capacity_int(const moe_cache* c);
-int cache_fill_mode(const moe_cache* c);
-int cache_launch_device_fill(moe_cache* c, int layer, cudaStream_t copy);
-
 struct LayerWs {
     float* logits;
     int32_t* idx;
@@ -69,9 +55,112 @@ static LayerWs layer_ws(const moe_shape* s, int n, void* base)
     return L;
 }
 
+// Router -> permutation -> grouped FFN over the experts in `slot_of` ->
+// combine, for one layer whose experts are already in their slots.
+static int layer_chain(const moe_shape* s, const LayerWs& L, const char* pool, size_t sb, int C,
+                       const int32_t* slot_of, const void* x, int x_dtype, const uint16_t* wg, const float* bias,
+                       int n, void* out, int32_t* idx, float* w, cudaStream_t st)
+{
+    const int E = s->experts, k = s->top_k, H = s->hidden, A = n * k;
+    int rc;
+    if ((rc = launch_router(x, x_dtype, wg, bias, n, H, E, k, L.logits, idx, w, st))) return rc;
+    if ((rc = launch_permute(idx, n, E, k, x, x_dtype, H, L.offsets, L.row_of, L.assign_of, nullptr, L.perm_ws, st)))
+        return rc;
+    const RowSource src{x, x_dtype, L.assign_of, k};
+    if ((rc = launch_ffn(s, pool, sb, C, slot_of, L.offsets, nullptr, A, L.y_perm, L.ffn_ws, st, &src))) return rc;
+    return launch_combine(L.y_perm, L.row_of, w, n, k, H, out, x_dtype, st);
+}
+
+// Prefill workspace: one layer's, then the expert list 0..E-1 and the slot
+// tables of the two layers in flight.
+struct PrefillWs {
+    LayerWs L;
+    int32_t* all;
+    int32_t* slot[2];
+    size_t bytes;
+};
+
+static PrefillWs prefill_ws(const moe_shape* s, int n, void* base)
+{
+    PrefillWs P{};
+    P.L = layer_ws(s, n, base);
+    const size_t e4 = align_up(4 * (size_t)s->experts, 256);
+    P.bytes = P.L.bytes + 3 * e4;
+    if (base) {
+        char* b = static_cast<char*>(base) + P.L.bytes;
+        P.all = reinterpret_cast<int32_t*>(b);
+        P.slot[0] = reinterpret_cast<int32_t*>(b + e4);
+        P.slot[1] = reinterpret_cast<int32_t*>(b + 2 * e4);
+    }
+    return P;
+}
+
+__global__ void iota_kernel(int32_t* v, int n)
+{
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) v[i] = i;
+}
+
 }  // namespace moe
 
 using namespace moe;
+
+extern "C" size_t moe_prefill_workspace_bytes(const moe_shape* shape, int32_t n)
+{
+    if (!shape_ok(shape) || n < 0) return 0;
+    return prefill_ws(shape, n, nullptr).bytes;
+}
+
+extern "C" int moe_prefill_forward(moe_cache* c, int32_t layer0, int32_t n_layers, const void* const* d_x,
+                                   int32_t x_dtype, const uint16_t* const* d_wg, const float* const* d_bias,
+                                   int32_t n, void* const* d_out, void* d_ws, size_t ws_bytes, void* stream,
+                                   void* copy_stream, int32_t* d_topk_idx_out)
+{
+    if (!c) return MOE_ERR_INVALID_ARG;
+    const moe_shape* s = cache_shape(c);
+    if (layer0 < 0 || n_layers < 0 || layer0 + (int64_t)n_layers > s->layers || n < 0) return MOE_ERR_INVALID_ARG;
+    if (x_dtype != MOE_DT_F32 && x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
+    if (n_layers == 0 || n == 0) return MOE_OK;
+    if (!d_x || !d_wg || !d_out || !d_ws) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < n_layers; i++) {
+        if (!d_x[i] || !d_wg[i] || !d_out[i]) return MOE_ERR_INVALID_ARG;
+        if (((uintptr_t)d_x[i] | (uintptr_t)d_wg[i] | (uintptr_t)d_out[i]) & 15) return MOE_ERR_INVALID_ARG;
+    }
+    if ((uintptr_t)d_ws & 15) return MOE_ERR_INVALID_ARG;
+    const PrefillWs P = prefill_ws(s, n, d_ws);
+    if (ws_bytes < P.bytes) return MOE_ERR_INVALID_ARG;
+    const int E = s->experts, k = s->top_k, C = cache_capacity_int(c);
+    if (C < E) return MOE_ERR_CAPACITY;   // a whole layer must fit
+    // Two whole layers fit: the next layer's lookup goes ahead of this
+    // layer's compute.  Its misses take the least recently used slots that
+    // it does not request; this layer's keys carry the newest stamps and at
+    // least E older keys or free slots exist, so none of them is a victim.
+    const bool overlap = C >= 2 * E;
+    cudaStream_t st = as_stream(stream), cp = as_stream(copy_stream);
+    const char* pool = cache_pool(c);
+    const size_t sb = cache_slot_bytes(c);
+    int rc;
+    iota_kernel<<<(E + 255) / 256, 256, 0, st>>>(P.all, E);
+    MOE_LAUNCH_CHECK();
+    auto bring_in = [&](int l, int b) -> int {
+        int r = cache_launch_lookup(c, l, P.all, E, P.slot[b], st);
+        return r ? r : cache_fill(c, l, st, cp, cache_prefill_event(c, b));
+    };
+    if ((rc = bring_in(layer0, 0))) return rc;
+    for (int i = 0; i < n_layers; i++) {
+        const int l = layer0 + i, b = i & 1;
+        // this layer's fills have landed (and device fills have read the
+        // miss list, which the next lookup rewrites) before anything else
+        // on the compute stream; the compute needs them anyway
+        MOE_CUDA_TRY(cudaStreamWaitEvent(st, cache_prefill_event(c, b), 0));
+        if (overlap && i + 1 < n_layers && (rc = bring_in(l + 1, b ^ 1))) return rc;
+        int32_t* idx = d_topk_idx_out ? d_topk_idx_out + (size_t)i * n * k : P.L.idx;
+        if ((rc = layer_chain(s, P.L, pool, sb, C, P.slot[b], d_x[i], x_dtype, d_wg[i], d_bias ? d_bias[i] : nullptr,
+                              n, d_out[i], idx, P.L.w, st)))
+            return rc;
+        if (!overlap && i + 1 < n_layers && (rc = bring_in(l + 1, b ^ 1))) return rc;
+    }
+    return MOE_OK;
+}
 
 extern "C" size_t moe_layer_workspace_bytes(const moe_shape* shape, int32_t n)
 {

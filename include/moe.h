@@ -146,6 +146,9 @@ size_t moe_ffn_workspace_bytes(const moe_shape* shape, int32_t rows);
 /* Device workspace bytes of moe_layer_forward for n tokens. */
 size_t moe_layer_workspace_bytes(const moe_shape* shape, int32_t n);
 
+/* Device workspace bytes of moe_prefill_forward for n tokens. */
+size_t moe_prefill_workspace_bytes(const moe_shape* shape, int32_t n);
+
 /* ---------------------------------------------------------------- packing */
 
 /*
@@ -424,6 +427,42 @@ int moe_layer_forward(moe_cache* cache, int32_t layer, const void* d_x, int32_t 
                       const uint16_t* d_wg, const float* d_bias, int32_t n, void* d_out,
                       void* d_ws, size_t ws_bytes, void* stream, void* copy_stream,
                       int32_t* d_topk_idx_out, float* d_topk_w_out);
+
+/*
+ * Multi-layer prefill with full-layer double buffering: layers layer0 ..
+ * layer0 + n_layers - 1 over one prompt of n tokens, every expert of a layer
+ * brought into the cache before the layer runs.  Layer i of the call (layer
+ * l = layer0 + i) reads d_x[i] [n][H] (x_dtype), its router d_wg[i] [E][H]
+ * bf16 and d_bias[i] [E] (d_bias, or any entry, may be NULL), and writes
+ * d_out[i] [n][H] (x_dtype) and, when d_topk_idx_out is not NULL, its
+ * routing to d_topk_idx_out + i*n*k.  d_x, d_wg, d_bias and d_out are host
+ * arrays of n_layers device pointers; d_x[i+1] may be d_out[i].  Each layer
+ * computes what moe_layer_forward computes.
+ * Cache: one lookup per layer, in layer order, requesting all E experts
+ * (ascending), with the LRU updates, trace records and fills of
+ * moe_cache_lookup_update in the cache's fill mode.  With capacity >= 2E the
+ * lookup and fills of layer l+1 are issued before layer l computes, so the
+ * next layer's experts stream over PCIe on copy_stream while the current one
+ * computes; the LRU order keeps layer l's slots out of their victims (layer
+ * l's keys are the newest, and at least E slots are free or older).  With
+ * E <= capacity < 2E the next layer's lookup follows the current layer's
+ * compute (no overlap).  MOE_ERR_CAPACITY (before anything is enqueued) when
+ * capacity < E.  Host fills block the host at every lookup that may miss,
+ * until the previous layer's fills have landed; device fills never block.
+ * d_ws: moe_prefill_workspace_bytes(shape, n) bytes.  Pointers 16-byte
+ * aligned.
+ * Pages: during prefill the whole next layer's experts stream over PCIe into
+ * a second buffer while the GPU computes the current layer, when the cache
+ * has room for it ("FreeToken linux", section "Como gestiona FreeToken la
+ * memoria MoE" and its mechanism table, "Doble bufer para la capa
+ * completa"; "FreeToken 290b model", section "Como gestiona FreeToken el
+ * prellenado y la decodificacion"); the same cache serves prefill and decode
+ * (same section of "FreeToken linux").
+ */
+int moe_prefill_forward(moe_cache* cache, int32_t layer0, int32_t n_layers, const void* const* d_x,
+                        int32_t x_dtype, const uint16_t* const* d_wg, const float* const* d_bias, int32_t n,
+                        void* const* d_out, void* d_ws, size_t ws_bytes, void* stream, void* copy_stream,
+                        int32_t* d_topk_idx_out);
 
 /*
  * The operand encoding the FP4 grouped FFN applies to its activation rows,
