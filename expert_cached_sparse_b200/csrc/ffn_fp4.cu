@@ -74,9 +74,13 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
 {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
+// Issued by one elected lane of a converged warp (the copy warps walk their
+// loops warp-uniformly; see tc_commit).
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
 {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(bar), "r"(bytes)
+                 : "memory");
 }
 __device__ __forceinline__ void mbar_arrive(uint32_t bar)
 {
@@ -132,23 +136,25 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity)
         }
 }
 
+// One elected lane of a converged warp issues the copy.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
 {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}"
                  ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
-}
-
-// Fire-and-forget bulk prefetch of global memory into L2.
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// The MMA warps issue tcgen05 operations from warp-uniform code: every lane
+// computes the operands, one lane elected by elect.sync issues (keeping the
+// operands warp-uniform roughly halves the issue cost of a chunk against a
+// lane-0-only branch).  Callers are converged warps.
 __device__ __forceinline__ void tc_commit(uint32_t bar)
 {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+                 : "memory");
 }
 
 // Shared-memory descriptor of a K-major operand in the 128-byte swizzle:
@@ -169,7 +175,8 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t addr)
 // 128 lanes (the 32-lane pattern is replicated into the four lane quarters).
 __device__ __forceinline__ void tc_cp_sf_d(uint32_t taddr, uint64_t desc)
 {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc));
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr), "l"(desc));
 }
 
 // D[tmem] (+)= A[smem] * B[smem], E2M1 operands with block scales from tensor memory.
@@ -178,12 +185,12 @@ __device__ __forceinline__ void tc_mma_fp4(uint32_t d, uint64_t a, uint64_t b, u
                                            uint32_t sfa, uint32_t sfb)
 {
     if (WFMT == MOE_W_MXFP4)
-        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                     "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
                      ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
     else
-        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                     "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
                      ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
 }
 
@@ -782,11 +789,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
     const long first = whole ? (long)blockIdx.x : b0;
 
     if (warp == 0) {
-        // ============ bulk copies: weight chunk image + token group image chunk.
-        // The first D stages' weight copies are issued before waiting for the
+        // ============ bulk copies: weight chunk image + token group image chunk
+        // (the whole warp walks the loop, one elected lane issues).  The first
+        // D stages' weight copies are issued before waiting for the
         // predecessor grid (weights do not depend on it); their activation
         // copies follow once it has completed.
-        if (lane == 0 && in_use) {
+        if (in_use) {
             int st = 0;
             uint32_t ph = 0;
             long issued = 0;
@@ -814,7 +822,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
                 const bool have_nx = nx.next(whole, NU, KC, b1);
                 const int4 gn = have_nx ? group_of(a, nx.u, RB) : g;
                 for (int c = sg.p0; c < sg.p1; c++) {
-                    if (!(ok = mbar_wait(smem_u32(&empty[st]), ph ^ 1, abort_v, a.wait))) break;
+                    if (!(ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&empty[st]), ph ^ 1, abort_v, a.wait))))
+                        break;
                     const uint32_t bar = smem_u32(&full[st]);
                     unsigned char* sp = ring + (size_t)st * STAGE;
                     if (a.withhold && blockIdx.x == 0 && issued == 0) {
@@ -850,9 +859,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
             pdl_wait();
         }
     } else if (warp == 1) {
-        // ============ scale-factor copies and MMAs (one thread)
+        // ============ scale-factor copies and MMAs (the whole warp walks the
+        // loop, one elected lane issues)
         const uint32_t ring_s = smem_u32(ring);
-        if (lane == 0 && in_use) {
+        if (in_use) {
             int st = 0, it = 0;
             uint32_t ph = 0;
             long cc = 0;
@@ -868,12 +878,13 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
                 const int ab = it & 1, nh = (U.n + 127) / 128;
                 const uint32_t id0 = idesc_fp4<WFMT>(U.n, 0), id1 = idesc_fp4<WFMT>(U.n, 2);
                 if (it >= 2) {   // the epilogue has read this accumulator's previous unit
-                    if (!(ok = mbar_wait(smem_u32(&acc_empty[ab]), ((it >> 1) - 1) & 1, abort_v, a.wait))) break;
+                    ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_empty[ab]), ((it >> 1) - 1) & 1, abort_v, a.wait));
+                    if (!ok) break;
                     tc_fence_after();
                 }
                 const uint32_t dcol = tmem + (uint32_t)(ab * CFG::NMAX);
                 for (int c = sg.p0; c < sg.p1; c++, cc++) {
-                    if (!(ok = mbar_wait(smem_u32(&full[st]), ph, abort_v, a.wait))) break;
+                    if (!(ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), ph, abort_v, a.wait)))) break;
                     tc_fence_after();
                     const uint32_t sfa = tmem + KC_::SF_COL + (uint32_t)((cc & 1) * KC_::SF_SET);
                     issue_chunk<WFMT, KC_::A_BYTES>(ring_s + (uint32_t)(st * STAGE), U.n, nh, dcol, sfa,
@@ -998,7 +1009,6 @@ __device__ unsigned int g_gb_gen;     // completed grid barriers (wraps)
 __device__ int g_gb_abort;            // set when a CTA gave up; cleared with the error word
 
 constexpr int kFusedMaxE = 512;
-constexpr int kPfAhead = 12;   // weight chunks the L2 prefetch runs ahead of the shared-memory copies
 
 struct FusedArgs {
     Fp4Args p1, p2;                 // the two GEMM phases (gpre / gtab unused)
@@ -1315,120 +1325,84 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
     }
 
     if (warp == 0) {
-        // ============ bulk copies of both phases.  A second cursor walks the
-        // same chunk sequence kPfAhead chunks ahead and prefetches the weights
-        // into L2, so the shared-memory copies find them there (the ring's
-        // depth alone cannot cover HBM latency at full bandwidth).
-        if (lane == 0) {
-            int st = 0;
-            uint32_t ph = 0;
-            long issued = 0;
-            bool ok = mbar_wait(smem_u32(xloaded), 0, abort_v, f.p1.wait);   // the x loads go first
-            int withheld = -1;   // testing: the stage left unfilled
-            int pend_st[D];
-            const char* pend_src[D];
-            uint32_t pend_bytes[D];
-            // ---- prefetch cursor
-            int pf_phase = -1, pf_c = 0, pf_p1 = 0, pf_RB = 1, pf_KC = 1, pf_NU = 0;
-            long pf_b1 = 0;
-            Seg pf_sg{0};
-            const char* pf_a = nullptr;
-            auto pf_next = [&]() -> const char* {
-                for (;;) {
-                    if (pf_c < pf_p1) return pf_a + (size_t)(pf_c++) * FM::CB;
-                    if (pf_phase >= 0 && pf_sg.next(false, pf_NU, pf_KC, pf_b1)) {
-                        const Fp4Args& a = pf_phase ? f.p2 : f.p1;
-                        pf_a = unit_of<WFMT, CFG>(a, pf_sg.u, pf_RB, pf_KC, plan_group(P, pf_sg.u / pf_RB, NT, bfull)).a;
-                        pf_c = pf_sg.p0;
-                        pf_p1 = pf_sg.p1;
-                        continue;
-                    }
-                    if (++pf_phase > 1) return nullptr;
-                    const Fp4Args& a = pf_phase ? f.p2 : f.p1;
-                    pf_RB = a.R / 128;
-                    pf_KC = a.K / 256;
-                    pf_NU = NG * pf_RB;
-                    const long W = (long)pf_NU * pf_KC;
-                    const int gridp = (int)(W < (long)grid ? W : (long)grid);
-                    if ((int)blockIdx.x >= gridp) { pf_b1 = 0; pf_sg = Seg{0}; continue; }
-                    pf_sg = Seg{sk_bound(W, blockIdx.x, gridp)};
-                    pf_b1 = sk_bound(W, blockIdx.x + 1, gridp);
-                }
+        // ============ bulk copies of both phases: the whole warp walks the
+        // chunk sequence, one elected lane issues.  A phase's activation copies
+        // wait for its gate (the grid barrier that publishes the images); the
+        // weight copies do not, up to a ring full of held-back stages.
+        int st = 0;
+        uint32_t ph = 0;
+        long issued = 0;
+        bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(xloaded), 0, abort_v, f.p1.wait));   // x loads first
+        int withheld = -1;   // testing: the stage left unfilled
+        int pend_st[D];
+        const char* pend_src[D];
+        uint32_t pend_bytes[D];
+        for (int phase = 0; phase < 2 && ok; phase++) {
+            const Fp4Args& a = phase ? f.p2 : f.p1;
+            const int RB = a.R / 128, KC = a.K / 256, NU = NG * RB;
+            const long W = (long)NU * KC;
+            const int gridp = (int)(W < (long)grid ? W : (long)grid);
+            if ((int)blockIdx.x >= gridp) continue;
+            int npend = 0;
+            bool open = false;   // this phase's activation images are published
+            auto issue_pending = [&]() {
+                for (int i = 0; i < npend; i++)
+                    bulk_g2s(smem_u32(ring + (size_t)pend_st[i] * STAGE + KC_::A_BYTES), pend_src[i], pend_bytes[i],
+                             smem_u32(&full[pend_st[i]]));
+                npend = 0;
             };
-            if (ok)
-                for (int i = 0; i < kPfAhead; i++) {
-                    const char* pa = pf_next();
-                    if (!pa) break;
-                    prefetch_l2(pa, FM::CB);
-                }
-            for (int phase = 0; phase < 2 && ok; phase++) {
-                const Fp4Args& a = phase ? f.p2 : f.p1;
-                const int RB = a.R / 128, KC = a.K / 256, NU = NG * RB;
-                const long W = (long)NU * KC;
-                const int gridp = (int)(W < (long)grid ? W : (long)grid);
-                if ((int)blockIdx.x >= gridp) continue;
-                int npend = 0;
-                bool open = false;   // this phase's activation images are published
-                auto release = [&]() -> bool {
-                    if (!mbar_wait(smem_u32(&gate[phase]), 0, abort_v, f.p1.wait)) return false;
-                    asm volatile("fence.proxy.async.global;" ::: "memory");
-                    for (int i = 0; i < npend; i++)
-                        bulk_g2s(smem_u32(ring + (size_t)pend_st[i] * STAGE + KC_::A_BYTES), pend_src[i],
-                                 pend_bytes[i], smem_u32(&full[pend_st[i]]));
-                    npend = 0;
-                    open = true;
-                    return true;
-                };
-                Seg sg{sk_bound(W, blockIdx.x, gridp)};
-                const long b1 = sk_bound(W, blockIdx.x + 1, gridp);
-                while (ok && sg.next(false, NU, KC, b1)) {
-                    const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC, plan_group(P, sg.u / RB, NT, bfull));
-                    for (int c = sg.p0; c < sg.p1; c++) {
-                        // a ring full of held-back stages: wait for the gate before reusing one
-                        if (!open && npend == D && !(ok = release())) break;
-                        if (!(ok = mbar_wait(smem_u32(&empty[st]), ph ^ 1, abort_v, f.p1.wait))) break;
-                        const uint32_t bar = smem_u32(&full[st]);
-                        unsigned char* sp = ring + (size_t)st * STAGE;
-                        if (f.p1.withhold && blockIdx.x == 0 && issued == 0) {
-                            withheld = st;   // testing: never filled, so the wait for it runs out
+            auto release = [&]() -> bool {
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&gate[phase]), 0, abort_v, f.p1.wait))) return false;
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                issue_pending();
+                open = true;
+                return true;
+            };
+            Seg sg{sk_bound(W, blockIdx.x, gridp)};
+            const long b1 = sk_bound(W, blockIdx.x + 1, gridp);
+            while (ok && sg.next(false, NU, KC, b1)) {
+                const Unit U = unit_of<WFMT, CFG>(a, sg.u, RB, KC, plan_group(P, sg.u / RB, NT, bfull));
+                for (int c = sg.p0; c < sg.p1; c++) {
+                    // a ring full of held-back stages: wait for the gate before reusing one
+                    if (!open && npend == D && !(ok = release())) break;
+                    if (!(ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&empty[st]), ph ^ 1, abort_v, f.p1.wait))))
+                        break;
+                    const uint32_t bar = smem_u32(&full[st]);
+                    unsigned char* sp = ring + (size_t)st * STAGE;
+                    if (f.p1.withhold && blockIdx.x == 0 && issued == 0) {
+                        withheld = st;   // testing: never filled, so the wait for it runs out
+                    } else {
+                        mbar_expect_tx(bar, (uint32_t)(FM::CB + U.bb));
+                        bulk_g2s(smem_u32(sp), U.a + (size_t)c * FM::CB, FM::CB, bar);
+                        // (once the gate has passed, release() cannot fail)
+                        if (!open && __any_sync(0xffffffffu, mbar_try(smem_u32(&gate[phase]), 0))) release();
+                        if (open) {
+                            bulk_g2s(smem_u32(sp + KC_::A_BYTES), U.b + (size_t)c * U.bb, (uint32_t)U.bb, bar);
                         } else {
-                            mbar_expect_tx(bar, (uint32_t)(FM::CB + U.bb));
-                            bulk_g2s(smem_u32(sp), U.a + (size_t)c * FM::CB, FM::CB, bar);
-                            if (const char* pa = pf_next()) prefetch_l2(pa, FM::CB);
-                            // (the gate has passed here, so release() cannot fail)
-                            if (!open && mbar_try(smem_u32(&gate[phase]), 0)) release();
-                            if (open) {
-                                bulk_g2s(smem_u32(sp + KC_::A_BYTES), U.b + (size_t)c * U.bb, (uint32_t)U.bb, bar);
-                            } else {
-                                pend_st[npend] = st;
-                                pend_src[npend] = U.b + (size_t)c * U.bb;
-                                pend_bytes[npend++] = (uint32_t)U.bb;
-                            }
+                            pend_st[npend] = st;
+                            pend_src[npend] = U.b + (size_t)c * U.bb;
+                            pend_bytes[npend++] = (uint32_t)U.bb;
                         }
-                        issued++;
-                        if (++st == D) { st = 0; ph ^= 1; }
                     }
-                }
-                if (ok && !open && npend > 0) ok = release();
-                if (!ok) {
-                    // after an abort the held-back activation copies are issued
-                    // anyway (their data is not used), so that every stage whose
-                    // weight copy went out completes its phase before the drain
-                    for (int i = 0; i < npend; i++)
-                        bulk_g2s(smem_u32(ring + (size_t)pend_st[i] * STAGE + KC_::A_BYTES), pend_src[i],
-                                 pend_bytes[i], smem_u32(&full[pend_st[i]]));
-                    npend = 0;
+                    issued++;
+                    if (++st == D) { st = 0; ph ^= 1; }
                 }
             }
-            // every issued copy lands before the CTA exits (a withheld stage
-            // is never refilled: its consumer gives up first)
-            for (int i = 0; i < D && i < issued; i++)
-                if (i != withheld) mbar_drain(smem_u32(&full[i]), i < st ? ph : (ph ^ 1));
+            if (ok && !open && npend > 0) ok = release();
+            // after an abort the held-back activation copies are issued anyway
+            // (their data is not used), so that every stage whose weight copy
+            // went out completes its phase before the drain
+            if (!ok) issue_pending();
         }
+        // every issued copy lands before the CTA exits (a withheld stage is
+        // never refilled: its consumer gives up first)
+        for (int i = 0; i < D && i < issued; i++)
+            if (i != withheld) mbar_drain(smem_u32(&full[i]), i < st ? ph : (ph ^ 1));
     } else if (warp == 1) {
-        // ============ scale-factor copies and MMAs of both phases
+        // ============ scale-factor copies and MMAs of both phases (the whole
+        // warp walks the loop, one elected lane issues)
         const uint32_t ring_s = smem_u32(ring);
-        if (lane == 0) {
+        {
             int st = 0, it = 0;
             uint32_t ph = 0;
             long cc = 0;
@@ -1446,12 +1420,15 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
                     const int ab = it & 1, nh = (U.n + 127) / 128;
                     const uint32_t id0 = idesc_fp4<WFMT>(U.n, 0), id1 = idesc_fp4<WFMT>(U.n, 2);
                     if (it >= 2) {
-                        if (!(ok = mbar_wait(smem_u32(&acc_empty[ab]), ((it >> 1) - 1) & 1, abort_v, f.p1.wait))) break;
+                        ok = __all_sync(0xffffffffu,
+                                        mbar_wait(smem_u32(&acc_empty[ab]), ((it >> 1) - 1) & 1, abort_v, f.p1.wait));
+                        if (!ok) break;
                         tc_fence_after();
                     }
                     const uint32_t dcol = tmem + (uint32_t)(ab * CFG::NMAX);
                     for (int c = sg.p0; c < sg.p1; c++, cc++) {
-                        if (!(ok = mbar_wait(smem_u32(&full[st]), ph, abort_v, f.p1.wait))) break;
+                        if (!(ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), ph, abort_v, f.p1.wait))))
+                            break;
                         tc_fence_after();
                         const uint32_t sfa = tmem + KC_::SF_COL + (uint32_t)((cc & 1) * KC_::SF_SET);
                         issue_chunk<WFMT, KC_::A_BYTES>(ring_s + (uint32_t)(st * STAGE), U.n, nh, dcol, sfa,
