@@ -90,3 +90,28 @@ def preload(cache: A.MoeCache, cfg: W.LayerConfig, stream=None, copy_stream=None
 
 def trace_rows(recs) -> list[tuple]:
     return [(int(r["call"]), int(r["event"]), int(r["layer"]), int(r["expert"]), int(r["slot"])) for r in recs]
+
+
+def oracle_route_trace(orc, cfg: W.LayerConfig, steps: int, prefill_tokens: int):
+    """The routing of the placement study's trace (the inputs and biases that
+    ``policy_study.route_trace`` feeds the GPU router), computed by the oracle
+    router: (decode trace [(layer, ids)] step-major, prefill trace)."""
+    E = cfg.experts
+    per_layer, prefill = {}, []
+    for l in range(cfg.layers):
+        wg = W.gen_wg(cfg, 0, l)
+        epochs = (steps + cfg.drift_every - 1) // cfg.drift_every if cfg.drift_every else 1
+        rows = []
+        for ep in range(epochs):
+            s0 = ep * cfg.drift_every if cfg.drift_every else 0
+            n = min(steps, s0 + (cfg.drift_every or steps)) - s0
+            x = np.concatenate([W.gen_x(cfg, 0, 1, "policy-decode", l, s) for s in range(s0, s0 + n)])
+            _, idx, _ = orc.router(x, wg, W.gen_bias(cfg, 0, l, ep), cfg.top_k)
+            rows.append(idx)
+        per_layer[l] = np.concatenate(rows)[:steps]
+        x = W.gen_x(cfg, 0, prefill_tokens, "policy-prefill", l)
+        _, idx, _ = orc.router(x, wg, W.gen_bias(cfg, 0, l, 0), cfg.top_k)
+        prefill.append((l, idx))
+    assert all(per_layer[l].shape == (steps, cfg.top_k) and per_layer[l].max() < E for l in per_layer)
+    decode = [(l, per_layer[l][s]) for s in range(steps) for l in range(cfg.layers)]
+    return decode, prefill
