@@ -144,6 +144,13 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                  ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
+// L2 prefetch of a weight chunk the CTA streams a little later (one elected lane).
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes)
+{
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e cp.async.bulk.prefetch.L2.global [%0], %1;\n\t}" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 // The MMA warps issue tcgen05 operations from warp-uniform code: every lane
@@ -1001,14 +1008,30 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
 //   h terms -> barrier -> down GEMM.
 // The quantisation steps run on the four epilogue warps; the copy warp keeps
 // streaming weights across the barriers and holds back only the activation
-// copies until the barrier that publishes them has passed.  Grid barriers
-// are a global arrival counter and generation word (both back in their idle
-// state after every barrier); every wait on them is bounded.
-__device__ unsigned int g_gb_count;   // arrivals at the current grid barrier
-__device__ unsigned int g_gb_gen;     // completed grid barriers (wraps)
-__device__ int g_gb_abort;            // set when a CTA gave up; cleared with the error word
+// copies until the barrier that publishes them has passed.
+// Grid barriers count arrivals on one 64-bit counter that only grows: a
+// launch whose CTAs all finish adds (barriers x CTAs) to it.  Each CTA rounds
+// the counter down to a multiple of the grid when it starts (the first
+// barrier cannot complete before every CTA has arrived, so every CTA finds
+// the same value) and barrier k completes when the counter reaches that value
+// plus (k + 1) x grid.  Arrival is one release add, waiting is acquire loads;
+// every wait is bounded.  Clearing the error word resets the counter.
+__device__ unsigned long long g_gb_count;   // grid-barrier arrivals since the last clear
+__device__ int g_gb_abort;                  // set when a CTA gave up; cleared with the error word
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p)
+{
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_add_u64(unsigned long long* p, unsigned long long v)
+{
+    asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
 
 constexpr int kFusedMaxE = 512;
+constexpr int kPfUnit = 8;     // weight chunks of the current unit prefetched into L2 ahead of its copies
 
 struct FusedArgs {
     Fp4Args p1, p2;                 // the two GEMM phases (gpre / gtab unused)
@@ -1036,39 +1059,41 @@ struct FusedCfg {
     static_assert(PLAN % 1024 == 0 && STAGE % 1024 == 0, "1024-byte aligned ring");
 };
 
+// The arrival count this CTA's first grid barrier completes at (epilogue
+// thread 0, before its first arrival).
+__device__ __forceinline__ unsigned long long grid_bar_first()
+{
+    const unsigned long long c = ld_acquire_u64(&g_gb_count);
+    return c - c % gridDim.x + gridDim.x;
+}
+
 // Bounded grid barrier for the four epilogue warps of every CTA.  Their
 // global writes before it are visible to every CTA after it (generic and
-// async proxy: operand images are read by bulk copies).
-__device__ __forceinline__ bool grid_sync_epi(int etid, volatile int* s_flag, long long limit)
+// async proxy: operand images are read by bulk copies).  `next` (meaningful
+// in epilogue thread 0) is the count this barrier completes at; it moves on
+// to the next barrier's.
+__device__ __forceinline__ bool grid_sync_epi(int etid, volatile int* s_flag, long long limit,
+                                              unsigned long long& next)
 {
     asm volatile("fence.proxy.async.global;" ::: "memory");
     __threadfence();
     epi_bar();
     if (etid == 0) {
         bool ok = !*reinterpret_cast<volatile int*>(&g_gb_abort);
-        const unsigned gen = *reinterpret_cast<volatile unsigned*>(&g_gb_gen);
-        __threadfence();
-        const unsigned arrived = atomicAdd(&g_gb_count, 1u);
-        if (arrived == gridDim.x - 1) {
-            atomicExch(&g_gb_count, 0u);
-            __threadfence();
-            atomicAdd(&g_gb_gen, 1u);
-        } else {
-            const long long t0 = clock64();
-            while (*reinterpret_cast<volatile unsigned*>(&g_gb_gen) == gen) {
-                if (*reinterpret_cast<volatile int*>(&g_gb_abort)) { ok = false; break; }
-                if (clock64() - t0 > limit) {
-                    ok = false;
-                    atomicExch(&g_gb_abort, 1);
-                    atomicCAS(&g_fp4_error, 0, (int)MOE_ERR_TIMEOUT);
-                    break;
-                }
-                __nanosleep(64);
+        red_release_add_u64(&g_gb_count, 1ull);
+        const long long t0 = clock64();
+        while (ld_acquire_u64(&g_gb_count) < next) {
+            if (*reinterpret_cast<volatile int*>(&g_gb_abort)) { ok = false; break; }
+            if (clock64() - t0 > limit) {
+                ok = false;
+                atomicExch(&g_gb_abort, 1);
+                atomicCAS(&g_fp4_error, 0, (int)MOE_ERR_TIMEOUT);
+                break;
             }
         }
-        __threadfence();
         *s_flag = ok ? 1 : 0;
     }
+    next += gridDim.x;
     epi_bar();
     asm volatile("fence.proxy.async.global;" ::: "memory");
     return *s_flag != 0;
@@ -1374,6 +1399,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
                     } else {
                         mbar_expect_tx(bar, (uint32_t)(FM::CB + U.bb));
                         bulk_g2s(smem_u32(sp), U.a + (size_t)c * FM::CB, FM::CB, bar);
+                        // the unit's chunks kPfUnit ahead go to L2 meanwhile
+                        if (c == sg.p0)
+                            for (int j = 1; j < kPfUnit && c + j < sg.p1; j++)
+                                prefetch_l2(U.a + (size_t)(c + j) * FM::CB, FM::CB);
+                        if (c + kPfUnit < sg.p1) prefetch_l2(U.a + (size_t)(c + kPfUnit) * FM::CB, FM::CB);
                         // (once the gate has passed, release() cannot fail)
                         if (!open && __any_sync(0xffffffffu, mbar_try(smem_u32(&gate[phase]), 0))) release();
                         if (open) {
@@ -1453,6 +1483,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         int it = 0;
         bool ok = true;
+        unsigned long long gb_next = etid == 0 ? grid_bar_first() : 0ull;
         for (int phase = 0; phase < 2; phase++) {
             const Fp4Args& a = phase ? f.p2 : f.p1;
             {   // the activation terms of this phase's input rows: (row, chunk) items per warp
@@ -1468,7 +1499,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
                     fused_quant_items<WFMT, T, false>(P, f.x, a.K, f.gather, f.gk, f.bx, f.rex_x, first, step, items,
                                                       lane, xloaded);
             }
-            ok = grid_sync_epi(etid, s_flag, f.p1.wait) && ok;   // terms published (phase 0: counters zero)
+            ok = grid_sync_epi(etid, s_flag, f.p1.wait, gb_next) && ok;   // terms published (phase 0: counters zero)
             if (etid == 0) mbar_arrive(smem_u32(&gate[phase]));
             const int RB = a.R / 128, KC = a.K / 256, NU = NG * RB;
             const long W = (long)NU * KC;
@@ -1545,7 +1576,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
                     it++;
                 }
             }
-            if (phase == 0) ok = grid_sync_epi(etid, s_flag, f.p1.wait) && ok;   // h complete before its terms are taken
+            if (phase == 0) ok = grid_sync_epi(etid, s_flag, f.p1.wait, gb_next) && ok;   // h complete before its terms are taken
         }
     }
     tc_fence_before();
@@ -1824,7 +1855,7 @@ int ffn_fp4_device_error(int clear)
     if (clear && v) {
         // the kernels are not running: put the grid barrier back in its idle state too
         const int z = 0;
-        const unsigned zu = 0;
+        const unsigned long long zu = 0;
         if (cudaMemcpyToSymbol(g_fp4_error, &z, sizeof z) != cudaSuccess ||
             cudaMemcpyToSymbol(g_gb_abort, &z, sizeof z) != cudaSuccess ||
             cudaMemcpyToSymbol(g_gb_count, &zu, sizeof zu) != cudaSuccess)

@@ -386,7 +386,10 @@ int moe_permute_noalloc(const int32_t* d_topk_idx, int32_t n, int32_t experts, i
  * are undone in fp32.  BF16 weights run on bf16 MMAs with x and h rounded to
  * bf16.  Results are deterministic: the same inputs give the same bits on
  * every call.  MOE_FFN_TILE=decode or =prefill forces the FP4 tile shape
- * (read at every call; intended for testing).
+ * (read at every call; intended for testing).  FP4 calls with decode tiles
+ * run as one cooperative kernel whose grid barriers use a process-wide
+ * counter of the device: such calls must not run at the same time on
+ * different streams (calls on one stream never do).
  * Pages: experts found in VRAM execute on the GPU ("FreeToken
  * quantization", section "Como se desplazan los pesos MoE cuantizados por la
  * memoria"); SwiGLU is this library's reading (the pages name no
