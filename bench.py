@@ -300,10 +300,11 @@ class DecodeStream:
 
 
 # DRAM bytes (read + write) per grouped-FFN call of the headline decode
-# stream, summed over the call's kernels (operand preps and both projections)
-# and averaged over the calls of an ncu capture of that workload.  Valid only
-# for the FFN code it was measured on (comments aside): other code reports null.
-FFN_TRAFFIC = {"source_sha1": None, "bytes_per_call": None}
+# stream (one launch of the fused decode kernel per call), averaged over the
+# four calls of an ncu capture of that workload (the hit and miss passes of
+# two steps).  Valid only for the FFN code it was measured on (comments
+# aside): other code reports null.
+FFN_TRAFFIC = {"source_sha1": "28c74927921c75799ffea0fbee673c7186816eab", "bytes_per_call": 244683840}
 
 
 def ffn_source_sha1():
