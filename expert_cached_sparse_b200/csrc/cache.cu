@@ -24,6 +24,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "route_dev.cuh"
 
 namespace moe {
 
@@ -158,12 +159,11 @@ static size_t lookup_smem_bytes(int E, int C)
 // One CTA.  All state the call needs is read into shared memory in one
 // parallel phase (one memory round trip), the decisions are made there,
 // and only the entries that change are written back.
-__global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int layer,
-                                                                const int32_t* __restrict__ idx,
-                                                                int count, int E, int C, int trace_cap,
-                                                                int32_t* __restrict__ slot_user)
+// The lookup, by every thread of a kLookupThreads CTA; smem: lookup_smem_bytes(E, C).
+__device__ __forceinline__ void lookup_body(MetaPtrs m, int layer, const int32_t* __restrict__ idx, int count,
+                                            int E, int C, int trace_cap, int32_t* __restrict__ slot_user,
+                                            unsigned char* smem)
 {
-    extern __shared__ __align__(16) unsigned char smem[];
     unsigned char* p = smem;
     int* s_row = reinterpret_cast<int*>(p);                     p += align_up(sizeof(int) * E, 16);
     int* s_key = reinterpret_cast<int*>(p);                     p += align_up(sizeof(int) * C, 16);
@@ -378,6 +378,37 @@ __global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int 
     }
 }
 
+__global__ void __launch_bounds__(kLookupThreads) lookup_kernel(MetaPtrs m, int layer,
+                                                                const int32_t* __restrict__ idx,
+                                                                int count, int E, int C, int trace_cap,
+                                                                int32_t* __restrict__ slot_user)
+{
+    extern __shared__ __align__(16) unsigned char smem[];
+    lookup_body(m, layer, idx, count, E, C, trace_cap, slot_user, smem);
+}
+
+// The front of a decode-sized layer call in one launch: top-k of the n <= 32
+// tokens (a warp per token, from the logits the router kernel wrote), the
+// lookup of their experts, and the token -> expert permutation; the same code
+// as the separate router top-k, lookup and permutation kernels.
+template <int EPL>
+__global__ void __launch_bounds__(kLookupThreads) front_kernel(MetaPtrs m, int layer, const float* __restrict__ logits,
+                                                               int n, int k, int E, int C, int trace_cap,
+                                                               int32_t* __restrict__ idx, float* __restrict__ w,
+                                                               int32_t* __restrict__ offsets,
+                                                               int32_t* __restrict__ row_of,
+                                                               int32_t* __restrict__ assign_of)
+{
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ PermSmem S;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp < n) topk_token<EPL>(logits + (size_t)warp * E, E, k, lane, idx + (size_t)warp * k, w + (size_t)warp * k);
+    __syncthreads();   // the indices (global) are complete and visible to the whole CTA
+    lookup_body(m, layer, idx, n * k, E, C, trace_cap, nullptr, smem);
+    __syncthreads();
+    perm_small_body(idx, n * k, E, offsets, row_of, assign_of, S);
+}
+
 // Undo the installs of a call whose fills could not be issued: the keys
 // become non-resident and their slots free.  Victims stay evicted.
 __global__ void rollback_kernel(MetaPtrs m, int n)
@@ -457,6 +488,7 @@ struct moe_cache {
     uint64_t fill_bytes = 0, host_syncs = 0, fills_issued = 0;
     long fault_fill_at = 0;              // MOE_FAULT_INJECT=fill_fail:<n>
     int lookup_smem = 0;
+    int front_smem_set = 0;   // dynamic shared memory the front kernels are allowed (per cache)
 };
 
 namespace moe {
@@ -475,6 +507,43 @@ int cache_launch_lookup(moe_cache* c, int layer, const int32_t* idx, int count, 
     }
     // everything before this point on `st` (earlier readers of any victim
     // slot included) is complete once ev_lookup fires
+    MOE_CUDA_TRY(cudaEventRecord(c->ev_lookup, st));
+    return MOE_OK;
+}
+
+// Whether a call of n tokens is small enough for the fused front kernel.
+bool cache_front_fits(const moe_cache* c, int n)
+{
+    const int E = c->shape.experts, k = c->shape.top_k;
+    return n > 0 && n <= kLookupThreads / 32 && E <= 1024 && n * k <= kSmallA && E <= kSmallE;
+}
+
+// The fused front (top-k + lookup + permutation) for n tokens, when
+// cache_front_fits; MOE_ERR_UNSUPPORTED otherwise (nothing enqueued).
+int cache_launch_front(moe_cache* c, int layer, const float* logits, int n, int32_t* idx, float* w,
+                       int32_t* offsets, int32_t* row_of, int32_t* assign_of, cudaStream_t st)
+{
+    const int E = c->shape.experts, k = c->shape.top_k;
+    if (!cache_front_fits(c, n)) return MOE_ERR_UNSUPPORTED;
+    if (c->front_smem_set < c->lookup_smem) {
+        if (c->lookup_smem > 48 * 1024) {
+            MOE_CUDA_TRY(cudaFuncSetAttribute(front_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, c->lookup_smem));
+            MOE_CUDA_TRY(cudaFuncSetAttribute(front_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, c->lookup_smem));
+        }
+        c->front_smem_set = c->lookup_smem;
+    }
+    {
+        ProfScope ps(MOE_PROF_LOOKUP, st);
+        prof_count(MOE_PROF_LOOKUP, 1);
+        if (E <= 256)
+            front_kernel<8><<<1, kLookupThreads, c->lookup_smem, st>>>(c->m, layer, logits, n, k, E, c->C, c->trace_cap,
+                                                                       idx, w, offsets, row_of, assign_of);
+        else
+            front_kernel<32><<<1, kLookupThreads, c->lookup_smem, st>>>(c->m, layer, logits, n, k, E, c->C,
+                                                                        c->trace_cap, idx, w, offsets, row_of,
+                                                                        assign_of);
+        MOE_LAUNCH_CHECK();
+    }
     MOE_CUDA_TRY(cudaEventRecord(c->ev_lookup, st));
     return MOE_OK;
 }

@@ -149,6 +149,8 @@ class ProfScope {
 namespace moe {
 int launch_router(const void* x, int x_dtype, const uint16_t* wg, const float* bias, int n, int H,
                   int E, int k, float* logits, int32_t* idx, float* w, cudaStream_t st);
+int launch_router_logits(const void* x, int x_dtype, const uint16_t* wg, const float* bias, int n, int H, int E,
+                         float* logits, cudaStream_t st);
 size_t permute_ws_bytes(int n, int E, int k);
 int launch_permute(const int32_t* idx, int n, int E, int k, const void* x, int x_dtype, int H,
                    int32_t* offsets, int32_t* row_of, int32_t* assign_of, uint16_t* x_perm, void* ws,
@@ -195,4 +197,7 @@ int cache_fill_mode(const moe_cache* c);
 int cache_launch_device_fill(moe_cache* c, int layer, cudaStream_t copy, cudaEvent_t ev = nullptr);
 int cache_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t copy, cudaEvent_t ev);
 cudaEvent_t cache_prefill_event(const moe_cache* c, int i);
+bool cache_front_fits(const moe_cache* c, int n);
+int cache_launch_front(moe_cache* c, int layer, const float* logits, int n, int32_t* idx, float* w,
+                       int32_t* offsets, int32_t* row_of, int32_t* assign_of, cudaStream_t st);
 }  // namespace moe

@@ -186,13 +186,20 @@ extern "C" int moe_layer_forward(moe_cache* c, int32_t layer, const void* d_x, i
     int32_t* idx = d_topk_idx_out ? d_topk_idx_out : L.idx;
     float* w = d_topk_w_out ? d_topk_w_out : L.w;
     int rc;
-    if ((rc = launch_router(d_x, x_dtype, d_wg, d_bias, n, H, E, k, L.logits, idx, w, st))) return rc;
-    if ((rc = cache_launch_lookup(c, layer, idx, A, nullptr, st))) return rc;
     // Both FFN paths gather the token rows straight from x into their own
     // operand copies, so the permutation writes no x_perm.
     uint16_t* xp = nullptr;
-    if ((rc = launch_permute(idx, n, E, k, d_x, x_dtype, H, L.offsets, L.row_of, L.assign_of, xp, L.perm_ws, st)))
-        return rc;
+    if (cache_front_fits(c, n)) {
+        // decode-sized calls: top-k, lookup and permutation in one launch after the logits
+        if ((rc = launch_router_logits(d_x, x_dtype, d_wg, d_bias, n, H, E, L.logits, st))) return rc;
+        if ((rc = cache_launch_front(c, layer, L.logits, n, idx, w, L.offsets, L.row_of, L.assign_of, st)))
+            return rc;
+    } else {
+        if ((rc = launch_router(d_x, x_dtype, d_wg, d_bias, n, H, E, k, L.logits, idx, w, st))) return rc;
+        if ((rc = cache_launch_lookup(c, layer, idx, A, nullptr, st))) return rc;
+        if ((rc = launch_permute(idx, n, E, k, d_x, x_dtype, H, L.offsets, L.row_of, L.assign_of, xp, L.perm_ws, st)))
+            return rc;
+    }
     const RowSource src{d_x, x_dtype, L.assign_of, k};
     const RowSource* gather = &src;
     const char* pool = cache_pool(c);

@@ -9,6 +9,7 @@
 // counts are scanned per expert across chunks; offsets come from a block
 // scan of the totals.
 #include "common.cuh"
+#include "route_dev.cuh"
 
 namespace moe {
 namespace {
@@ -171,67 +172,12 @@ __global__ void perm_scatter_gather_kernel(const int32_t* __restrict__ idx, int 
 // counts, an exclusive block scan for the offsets, and for every assignment
 // its rank among earlier assignments to the same expert (a scan over the
 // call's indices held in shared memory).
-constexpr int kSmallA = 1024;
-constexpr int kSmallE = 1024;
-
 __global__ void __launch_bounds__(1024) perm_small_kernel(const int32_t* __restrict__ idx, int A, int E,
                                                           int32_t* __restrict__ offsets, int32_t* __restrict__ row_of,
                                                           int32_t* __restrict__ assign_of)
 {
-    __shared__ int s_idx[kSmallA];
-    __shared__ int s_cnt[kSmallE];
-    __shared__ int s_warp[32];
-    __shared__ int s_tot;
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
-    __syncthreads();
-    for (int a = tid; a < A; a += blockDim.x) {
-        int e = idx[a];
-        if (e < 0 || e >= E) e = -1;          // out-of-range experts get no row
-        s_idx[a] = e;
-        if (e >= 0) atomicAdd(&s_cnt[e], 1);  // integer counts: order-independent
-    }
-    __syncthreads();
-    // offsets: exclusive scan of the counts (E <= blockDim.x)
-    const int v = (tid < E) ? s_cnt[tid] : 0;
-    int inc = v;
-    for (int off = 1; off < 32; off <<= 1) {
-        int o = __shfl_up_sync(0xffffffffu, inc, off);
-        if (lane >= off) inc += o;
-    }
-    if (lane == 31) s_warp[w] = inc;
-    __syncthreads();
-    if (w == 0) {
-        int x = (lane < (int)(blockDim.x >> 5)) ? s_warp[lane] : 0;
-        int xi = x;
-        for (int off = 1; off < 32; off <<= 1) {
-            int o = __shfl_up_sync(0xffffffffu, xi, off);
-            if (lane >= off) xi += o;
-        }
-        s_warp[lane] = xi - x;
-        if (lane == 31) s_tot = xi;
-    }
-    __syncthreads();
-    const int excl = s_warp[w] + inc - v;
-    __syncthreads();
-    if (tid < E) {
-        offsets[tid] = excl;
-        s_cnt[tid] = excl;                    // reuse as the base row of each expert
-    }
-    if (tid == 0) offsets[E] = s_tot;
-    __syncthreads();
-    for (int a = tid; a < A; a += blockDim.x) {
-        const int e = s_idx[a];
-        if (e < 0) {
-            row_of[a] = -1;
-            continue;
-        }
-        int rank = 0;
-        for (int b = 0; b < a; b++) rank += (s_idx[b] == e);
-        const int row = s_cnt[e] + rank;
-        row_of[a] = row;
-        assign_of[row] = a;
-    }
+    __shared__ PermSmem S;
+    perm_small_body(idx, A, E, offsets, row_of, assign_of, S);
 }
 
 // x_perm[row] = bf16(x[assign_of[row] / k]): one warp per row.

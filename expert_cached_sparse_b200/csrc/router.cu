@@ -8,6 +8,7 @@
 // multiply-adds in ascending order; an xor butterfly (16, 8, 4, 2, 1)
 // then sums the lanes, leaving the same value in all of them.
 #include "common.cuh"
+#include "route_dev.cuh"
 
 namespace moe {
 namespace {
@@ -233,16 +234,6 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(const void* __
     }
 }
 
-// a ranks above b: larger logit; ties -> lower index; NaN below everything.
-__device__ __forceinline__ bool ranks_above(float a, int ia, float b, int ib)
-{
-    bool na = isnan(a), nb = isnan(b);
-    if (na != nb) return nb;
-    if (na) return ia < ib;
-    if (a != b) return a > b;
-    return ia < ib;
-}
-
 // Warp per token: k rounds of arg-max, then exp(l - lmax) renormalised.
 __global__ void __launch_bounds__(128) router_topk_kernel(const float* __restrict__ logits, int n,
                                                           int E, int k, int32_t* __restrict__ idx,
@@ -287,9 +278,7 @@ __global__ void __launch_bounds__(128) router_topk_kernel(const float* __restric
     }
 }
 
-// Warp per token with the token's logits in registers (EPL per lane, expert
-// lane + 32 i in slot i): k rounds of arg-max over the experts not yet taken,
-// then the same weights as router_topk_kernel.
+// Warp per token with the token's logits in registers (topk_token).
 template <int EPL>
 __global__ void __launch_bounds__(128) router_topk_reg_kernel(const float* __restrict__ logits, int n, int E, int k,
                                                               int32_t* __restrict__ idx, float* __restrict__ w)
@@ -297,43 +286,7 @@ __global__ void __launch_bounds__(128) router_topk_reg_kernel(const float* __res
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= n) return;
-    const float* lt = logits + (size_t)t * E;
-    float v[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; i++) v[i] = (lane + 32 * i < E) ? __ldg(lt + lane + 32 * i) : 0.0f;
-    uint32_t avail = 0;   // bit i: expert lane + 32 i exists and is not taken
-#pragma unroll
-    for (int i = 0; i < EPL; i++)
-        if (lane + 32 * i < E) avail |= 1u << i;
-    float my_l = 0.0f;
-    int my_i = 0;
-    for (int r = 0; r < k; r++) {
-        float bv = 0.0f;
-        int bi = -1;
-#pragma unroll
-        for (int i = 0; i < EPL; i++)
-            if (((avail >> i) & 1) && (bi < 0 || ranks_above(v[i], lane + 32 * i, bv, bi))) {
-                bv = v[i];
-                bi = lane + 32 * i;
-            }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            if (oi >= 0 && (bi < 0 || ranks_above(ov, oi, bv, bi))) { bv = ov; bi = oi; }
-        }
-        if ((bi & 31) == lane) avail &= ~(1u << (bi >> 5));
-        if (lane == r) { my_l = bv; my_i = bi; }
-    }
-    const float lmax = __shfl_sync(0xffffffffu, my_l, 0);
-    float p = (lane < k) ? expf(my_l - lmax) : 0.0f;
-    float z = p;
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-    if (lane < k) {
-        idx[(size_t)t * k + lane] = my_i;
-        w[(size_t)t * k + lane] = p / z;
-    }
+    topk_token<EPL>(logits + (size_t)t * E, E, k, lane, idx + (size_t)t * k, w + (size_t)t * k);
 }
 
 template <bool XF32>
@@ -359,6 +312,17 @@ int launch_logits(const void* x, const uint16_t* wg, const float* bias, int n, i
 }
 
 }  // namespace
+
+// The logits kernel alone (the decode front kernel takes the top-k).
+int launch_router_logits(const void* x, int x_dtype, const uint16_t* wg, const float* bias, int n, int H, int E,
+                         float* logits, cudaStream_t st)
+{
+    if (n == 0) return MOE_OK;
+    ProfScope ps(MOE_PROF_ROUTER, st);
+    prof_count(MOE_PROF_ROUTER, 1);
+    return (x_dtype == MOE_DT_F32) ? launch_logits<true>(x, wg, bias, n, H, E, logits, st)
+                                   : launch_logits<false>(x, wg, bias, n, H, E, logits, st);
+}
 
 int launch_router(const void* x, int x_dtype, const uint16_t* wg, const float* bias, int n, int H,
                   int E, int k, float* logits, int32_t* idx, float* w, cudaStream_t st)

@@ -416,6 +416,9 @@ int moe_combine(const uint16_t* d_y_perm, const int32_t* d_row_of, const float* 
  * d_x [n][H] (x_dtype), d_wg [E][H] bf16, d_bias [E] or NULL; d_out [n][H]
  * in x_dtype.  d_ws: moe_layer_workspace_bytes() bytes.  d_topk_idx_out /
  * d_topk_w_out ([n][k], device) receive the routing when not NULL.
+ * Calls of at most 32 tokens (with E <= 1024 and n*k <= 1024) run the top-k,
+ * the lookup and the permutation as one kernel after the logits kernel; the
+ * results are those of the separate steps.
  * Host fills: blocks the host once, for the miss list, unless every expert
  * of the layer is resident; in that case nothing is read back and the call
  * can be captured in a CUDA graph.  Device fills (moe_cache_set_fill_mode):
