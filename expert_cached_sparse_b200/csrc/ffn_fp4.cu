@@ -48,6 +48,15 @@ namespace {
 
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 32 * (2 + kEpiWarps);
+// Epilogue warps of the separate GEMM kernel: with prefill tiles (64 tokens
+// per unit) reading back and finishing a unit takes longer than its MMAs, so
+// two warps share each tensor-memory lane quarter, one per half of the
+// unit's 8-token chunks.
+template <class CFG>
+struct SepCfg {
+    static constexpr int EW = CFG::SPLIT ? kEpiWarps : 2 * kEpiWarps;
+    static constexpr int THREADS = 32 * (2 + EW);
+};
 constexpr int kQuantThreads = 256;
 constexpr long long kWaitCycles = 4000000000ll;   // ~2 s: drains, and waits unless a test sets a limit
 constexpr int kMaxCtas = 160;                      // persistent grid: one CTA per SM at most
@@ -734,7 +743,7 @@ __device__ __forceinline__ void finish8(const Fp4Args& a, const Unit& U, int q, 
 }
 
 template <int WFMT, int PHASE, class CFG>
-__global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
+__global__ void __launch_bounds__(SepCfg<CFG>::THREADS, 1) ffn_fp4_kernel(Fp4Args a)
 {
     using FM = Fmt<WFMT>;
     using KC_ = KCfg<WFMT, CFG>;
@@ -762,7 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
         }
         for (int i = 0; i < 2; i++) {
             mbar_init(smem_u32(&acc_full[i]), 1);
-            mbar_init(smem_u32(&acc_empty[i]), 32 * kEpiWarps);
+            mbar_init(smem_u32(&acc_empty[i]), 32 * SepCfg<CFG>::EW);
         }
         mbar_init(smem_u32(fin), 1);
         *abort_flag = 0;
@@ -911,7 +920,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
             mbar_drain(smem_u32(fin), 0);
         }
     } else if (in_use) {
-        // ============ epilogue: warps 2..5, tensor-memory lane quarter q.
+        // ============ epilogue: warps 2.., tensor-memory lane quarter q = warp % 4;
+        // with 8 epilogue warps, warp w takes the unit's chunks ch = (w - 2) / 4 mod 2.
         // All four warps walk the same segments and meet the same named
         // barriers; after a failed wait a warp keeps walking without waiting
         // or touching tensor memory, so the barriers still match.
@@ -933,7 +943,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_kernel(Fp4Args a)
             const int nch = (U.nt + 7) / 8;
             if (whole || (sg.p0 == 0 && sg.p1 == KC)) {
                 if (ok) {
-                    for (int ch = 0; ch < nch; ch++) {
+                    constexpr int EH = SepCfg<CFG>::EW / 4;
+                    for (int ch = (warp - 2) / 4; ch < nch; ch += EH) {
                         uint32_t d[8 * T];
 #pragma unroll
                         for (int t = 0; t < T; t++) tmem_ld8(dcol + 8 * T * ch + 8 * t, d + 8 * t);
@@ -1738,7 +1749,7 @@ int run_fp4(const moe_shape* s, const BlobLayout& bl, const void* pool, size_t s
     a.bimg = w.bx;
     a.rex = WFMT == MOE_W_NVFP4 ? w.rex_x : nullptr;
     a.out_h = w.h32;
-    MOE_CUDA_TRY(launch_pdl(ffn_fp4_kernel<WFMT, 1, CFG>, grid, kThreads, smem, st, a));
+    MOE_CUDA_TRY(launch_pdl(ffn_fp4_kernel<WFMT, 1, CFG>, grid, SepCfg<CFG>::THREADS, smem, st, a));
     MOE_CUDA_TRY(launch_pdl(fp4_terms_kernel<WFMT, CFG::T, true>, qgrid_for(F), kQuantThreads, 0, st,
                             static_cast<const void*>(w.h32), rows, F, static_cast<const int32_t*>(nullptr), 1,
                             offsets, slot_of, E, pool_slots, w.boffc, CFG::NT, w.bh, w.rex_h, kNoCanon, kNoCanon));
@@ -1750,7 +1761,7 @@ int run_fp4(const moe_shape* s, const BlobLayout& bl, const void* pool, size_t s
     b.rex = WFMT == MOE_W_NVFP4 ? w.rex_h : nullptr;
     b.out_h = nullptr;
     b.out_y = y_perm;
-    MOE_CUDA_TRY(launch_pdl(ffn_fp4_kernel<WFMT, 2, CFG>, grid, kThreads, smem, st, b));
+    MOE_CUDA_TRY(launch_pdl(ffn_fp4_kernel<WFMT, 2, CFG>, grid, SepCfg<CFG>::THREADS, smem, st, b));
     return MOE_OK;
 }
 
