@@ -304,7 +304,7 @@ class DecodeStream:
 # four calls of an ncu capture of that workload (the hit and miss passes of
 # two steps).  Valid only for the FFN code it was measured on (comments
 # aside): other code reports null.
-FFN_TRAFFIC = {"source_sha1": "28c74927921c75799ffea0fbee673c7186816eab", "bytes_per_call": 244683840}
+FFN_TRAFFIC = {"source_sha1": "70725fa1423008d4dc351207abe4d4af39b2a0c0", "bytes_per_call": 244677120}
 
 
 def ffn_source_sha1():
