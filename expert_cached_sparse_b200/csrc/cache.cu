@@ -54,13 +54,12 @@ struct MetaPtrs {
     unsigned long long* stamp;  // [C]
     int32_t* slot_all;      // [E] slot of each requested expert of the last call
     int32_t* slot_hit;      // [E] hits only
-    int32_t* slot_miss;     // [E] misses only
     moe_trace_rec* trace;   // [trace_cap]
     const char** src_of;    // [L*E] device address of each key's mapped host blob (device fills)
 };
 
 struct MetaLayout {
-    size_t hdr, stats, tcount, slot_table, key_of, stamp, slot_all, slot_hit, slot_miss, trace, src, bytes;
+    size_t hdr, stats, tcount, slot_table, key_of, stamp, slot_all, slot_hit, trace, src, bytes;
 };
 
 static MetaLayout meta_layout(const moe_shape* s, int C, int trace_cap)
@@ -76,7 +75,6 @@ static MetaLayout meta_layout(const moe_shape* s, int C, int trace_cap)
     m.stamp = take(sizeof(unsigned long long) * (size_t)C);
     m.slot_all = take(sizeof(int32_t) * (size_t)s->experts);
     m.slot_hit = take(sizeof(int32_t) * (size_t)s->experts);
-    m.slot_miss = take(sizeof(int32_t) * (size_t)s->experts);
     m.trace = take(sizeof(moe_trace_rec) * (size_t)trace_cap);
     m.src = take(sizeof(void*) * (size_t)s->layers * s->experts);
     m.bytes = o;
@@ -96,7 +94,6 @@ static MetaPtrs meta_ptrs(void* base, const MetaLayout& l)
     p.stamp = reinterpret_cast<unsigned long long*>(b + l.stamp);
     p.slot_all = reinterpret_cast<int32_t*>(b + l.slot_all);
     p.slot_hit = reinterpret_cast<int32_t*>(b + l.slot_hit);
-    p.slot_miss = reinterpret_cast<int32_t*>(b + l.slot_miss);
     p.trace = reinterpret_cast<moe_trace_rec*>(b + l.trace);
     p.src_of = reinterpret_cast<const char**>(b + l.src);
     return p;
@@ -208,7 +205,7 @@ __device__ __forceinline__ void lookup_body(MetaPtrs m, int layer, const int32_t
             if (!hdr->sticky) hdr->sticky = MOE_ERR_INVALID_ARG;
         }
         for (int e = tid; e < E; e += NT) {
-            m.slot_all[e] = m.slot_hit[e] = m.slot_miss[e] = -1;
+            m.slot_all[e] = m.slot_hit[e] = -1;
             if (slot_user) slot_user[e] = -1;
         }
         return;
@@ -234,7 +231,7 @@ __device__ __forceinline__ void lookup_body(MetaPtrs m, int layer, const int32_t
             if (!hdr->sticky) hdr->sticky = MOE_ERR_CAPACITY;
         }
         for (int e = tid; e < E; e += NT) {
-            m.slot_all[e] = m.slot_hit[e] = m.slot_miss[e] = -1;
+            m.slot_all[e] = m.slot_hit[e] = -1;
             if (slot_user) slot_user[e] = -1;
         }
         return;
@@ -253,7 +250,7 @@ __device__ __forceinline__ void lookup_body(MetaPtrs m, int layer, const int32_t
         int hr = hit_base, mr = miss_base;
         for (int e = e0; e < e0 + EPT && e < E; e++) {
             if (!req[e]) {
-                m.slot_all[e] = m.slot_hit[e] = m.slot_miss[e] = -1;
+                m.slot_all[e] = m.slot_hit[e] = -1;
                 if (slot_user) slot_user[e] = -1;
                 continue;
             }
@@ -264,7 +261,6 @@ __device__ __forceinline__ void lookup_body(MetaPtrs m, int layer, const int32_t
                 put_rec(m.trace, trace_cap, (long)base + hr, (uint32_t)T, s, layer * E + e, E, MOE_EV_HIT);
                 hr++;
                 m.slot_all[e] = m.slot_hit[e] = s;
-                m.slot_miss[e] = -1;
                 if (slot_user) slot_user[e] = s;
             } else {
                 s_list[mr++] = e;
@@ -352,7 +348,7 @@ __device__ __forceinline__ void lookup_body(MetaPtrs m, int layer, const int32_t
         m.slot_table[key] = s;
         m.key_of[s] = key;
         m.stamp[s] = T;
-        m.slot_all[e] = m.slot_miss[e] = s;
+        m.slot_all[e] = s;
         m.slot_hit[e] = -1;
         if (slot_user) slot_user[e] = s;
     }
@@ -426,28 +422,30 @@ constexpr int kFillCtas = 16;
 constexpr int kFillThreads = 256;
 constexpr int kFillUnroll = 8;   // 16-byte loads in flight per thread
 
-// Device fills: copies every blob on the miss list of the last lookup from
-// mapped pinned host memory into its slot.  Runs after the lookup kernel in
-// stream order and reads what it wrote; a failed lookup leaves nothing to
-// copy.  The work is cut into rounds of kFillThreads * kFillUnroll 16-byte
+// Device fills: copies the blobs on the miss list of the last lookup from
+// mapped pinned host memory into their slots: the whole list (group < 0) or
+// the misses of one miss group.  Runs after the lookup kernel in stream
+// order and reads what it wrote; a failed lookup leaves nothing to copy.  The work is cut into rounds of kFillThreads * kFillUnroll 16-byte
 // words (32 KiB) dealt out to the CTAs; every thread issues all its loads
 // of a round before its stores, so 16 CTAs keep 512 KiB of PCIe reads in
 // flight.  Blob and slot addresses are 16-byte aligned, slot_bytes is a
 // multiple of 128.
 __global__ void __launch_bounds__(kFillThreads) fill_kernel(MetaPtrs m, int layer, int E, char* __restrict__ pool,
-                                                            size_t slot_bytes)
+                                                            size_t slot_bytes, int group)
 {
     const LookupHdr* h = m.hdr;
     if (h->status != MOE_OK) return;
     const int nm = h->n_miss;
-    if (nm <= 0) return;
+    int i0 = 0, i1 = nm;
+    if (group >= 0) miss_group(nm, group, &i0, &i1);
+    if (i1 <= i0) return;
     constexpr size_t kRound = (size_t)kFillThreads * kFillUnroll;
     const size_t n16 = slot_bytes / 16;
     const size_t rounds = (n16 + kRound - 1) / kRound;
-    const size_t total = rounds * (size_t)nm;
+    const size_t total = rounds * (size_t)(i1 - i0);
     for (size_t p = blockIdx.x; p < total; p += gridDim.x) {
-        const int i = (int)(p / rounds);
-        const size_t b = (p - (size_t)i * rounds) * kRound + threadIdx.x;
+        const int i = i0 + (int)(p / rounds);
+        const size_t b = (p - (size_t)(i - i0) * rounds) * kRound + threadIdx.x;
         const MissEnt me = m.miss[i];
         const int4* __restrict__ src = reinterpret_cast<const int4*>(m.src_of[(size_t)layer * E + me.expert]);
         int4* __restrict__ dst = reinterpret_cast<int4*>(pool + (size_t)me.slot * slot_bytes);
@@ -463,7 +461,25 @@ __global__ void __launch_bounds__(kFillThreads) fill_kernel(MetaPtrs m, int laye
             if (w < n16) dst[w] = v[u];
         }
     }
-    if (blockIdx.x == 0 && threadIdx.x == 0) m.stats->dev_fills += (unsigned long long)nm;
+    if (blockIdx.x == 0 && threadIdx.x == 0) m.stats->dev_fills += (unsigned long long)(i1 - i0);
+}
+
+// Slot tables of the miss groups of the last lookup: out[g][e] is the slot
+// of expert e when e is a miss of group g, else -1.  A failed lookup leaves
+// every entry -1.
+__global__ void group_slots_kernel(MetaPtrs m, int E, int32_t* __restrict__ out)
+{
+    for (int i = threadIdx.x; i < kMissGroups * E; i += blockDim.x) out[i] = -1;
+    __syncthreads();
+    const int nm = m.hdr->status == MOE_OK ? m.hdr->n_miss : 0;
+    for (int g = 0; g < kMissGroups; g++) {
+        int b, e;
+        miss_group(nm, g, &b, &e);
+        for (int i = b + threadIdx.x; i < e; i += blockDim.x) {
+            const MissEnt me = m.miss[i];
+            if (me.expert >= 0 && me.expert < E) out[g * E + me.expert] = me.slot;
+        }
+    }
 }
 
 }  // namespace moe
@@ -485,6 +501,7 @@ struct moe_cache {
     std::vector<unsigned char> hbuf;     // LookupHdr + MissEnt[E]
     cudaEvent_t ev_lookup = nullptr, ev_fill = nullptr;
     cudaEvent_t ev_pf[2] = {nullptr, nullptr};   // fills of the two layers a prefill has in flight
+    cudaEvent_t ev_grp[moe::kMissGroups] = {};         // fills of each miss group of a layer call
     uint64_t fill_bytes = 0, host_syncs = 0, fills_issued = 0;
     long fault_fill_at = 0;              // MOE_FAULT_INJECT=fill_fail:<n>
     int lookup_smem = 0;
@@ -552,7 +569,6 @@ bool cache_layer_resident(const moe_cache* c, int layer) { return c->resident[la
 
 const int32_t* cache_slot_all(const moe_cache* c) { return c->m.slot_all; }
 const int32_t* cache_slot_hit(const moe_cache* c) { return c->m.slot_hit; }
-const int32_t* cache_slot_miss(const moe_cache* c) { return c->m.slot_miss; }
 const char* cache_pool(const moe_cache* c) { return c->pool; }
 size_t cache_slot_bytes(const moe_cache* c) { return c->slot_bytes; }
 
@@ -561,7 +577,8 @@ size_t cache_slot_bytes(const moe_cache* c) { return c->slot_bytes; }
 // lookup on the compute stream is done, and record `ev` (ev_fill by
 // default).  *n_miss gets the number of fills issued; the caller makes the
 // compute stream wait on the event when *n_miss > 0.
-int cache_read_and_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t copy, int* n_miss, cudaEvent_t ev)
+int cache_read_and_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t copy, int* n_miss, cudaEvent_t ev,
+                        bool groups)
 {
     if (!ev) ev = c->ev_fill;
     *n_miss = 0;
@@ -591,12 +608,19 @@ int cache_read_and_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t c
     }
     ProfScope ps(MOE_PROF_FILL, copy);
     prof_count(MOE_PROF_FILL, h->n_miss);
-    for (int i = 0; i < h->n_miss; i++) {
-        const void* src = c->blobs[(size_t)layer * E + ms[i].expert];
-        if (!src) return MOE_ERR_STATE;
-        MOE_CUDA_TRY(cudaMemcpyAsync(c->pool + (size_t)ms[i].slot * c->slot_bytes, src, c->slot_bytes,
-                                     cudaMemcpyHostToDevice, copy));
-        c->resident[layer]++;
+    // in miss-list order; with groups, each non-empty group's copies are
+    // followed by its event
+    for (int g = 0; g < (groups ? kMissGroups : 1); g++) {
+        int b = 0, e = h->n_miss;
+        if (groups) miss_group(h->n_miss, g, &b, &e);
+        for (int i = b; i < e; i++) {
+            const void* src = c->blobs[(size_t)layer * E + ms[i].expert];
+            if (!src) return MOE_ERR_STATE;
+            MOE_CUDA_TRY(cudaMemcpyAsync(c->pool + (size_t)ms[i].slot * c->slot_bytes, src, c->slot_bytes,
+                                         cudaMemcpyHostToDevice, copy));
+            c->resident[layer]++;
+        }
+        if (groups && e > b) MOE_CUDA_TRY(cudaEventRecord(c->ev_grp[g], copy));
     }
     c->fills_issued += (uint64_t)h->n_miss;
     c->fill_bytes += (uint64_t)h->n_miss * c->slot_bytes;
@@ -605,26 +629,65 @@ int cache_read_and_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t c
     return MOE_OK;
 }
 
-cudaEvent_t cache_fill_event(const moe_cache* c) { return c->ev_fill; }
-
 int cache_fill_mode(const moe_cache* c) { return c->fill_mode; }
 
-// Device fills of the last lookup on `layer`: the copy stream waits for the
-// lookup (and so for every earlier reader of a victim slot on the compute
-// stream), runs fill_kernel and records ev_fill.  Nothing is read back.
-int cache_launch_device_fill(moe_cache* c, int layer, cudaStream_t copy, cudaEvent_t ev)
+// Device fills of the last lookup on `layer` (all misses, or miss group
+// `group`): the copy stream waits for the lookup (and so for every earlier
+// reader of a victim slot on the compute stream), runs fill_kernel and
+// records ev (ev_fill by default).  Nothing is read back.
+int cache_launch_device_fill(moe_cache* c, int layer, cudaStream_t copy, cudaEvent_t ev, int group)
 {
     if (!ev) ev = c->ev_fill;
     MOE_CUDA_TRY(cudaStreamWaitEvent(copy, c->ev_lookup, 0));
     {
         ProfScope ps(MOE_PROF_FILL, copy);
         prof_count(MOE_PROF_FILL, 1);
-        fill_kernel<<<kFillCtas, kFillThreads, 0, copy>>>(c->m, layer, c->shape.experts, c->pool, c->slot_bytes);
+        fill_kernel<<<kFillCtas, kFillThreads, 0, copy>>>(c->m, layer, c->shape.experts, c->pool, c->slot_bytes,
+                                                          group);
         MOE_LAUNCH_CHECK();
     }
     MOE_CUDA_TRY(cudaEventRecord(ev, copy));
     return MOE_OK;
 }
+
+// The fills of the lookup just enqueued for `layer`, as miss groups: group
+// g's slots have landed once cache_group_event(c, g) fires.  *live gets the
+// groups that may hold misses: with device fills all of them (the miss list
+// stays on the device; an empty group's kernel copies nothing), with host
+// fills the non-empty ones (the host reads the miss list back).
+int cache_group_fills(moe_cache* c, int layer, cudaStream_t st, cudaStream_t copy, unsigned* live)
+{
+    *live = 0;
+    if (c->fill_mode == MOE_FILL_DEVICE) {
+        for (int g = 0; g < kMissGroups; g++) {
+            int rc = cache_launch_device_fill(c, layer, copy, c->ev_grp[g], g);
+            if (rc) return rc;
+        }
+        *live = (1u << kMissGroups) - 1;
+        return MOE_OK;
+    }
+    int nm = 0;
+    int rc = cache_read_and_fill(c, layer, st, copy, &nm, nullptr, true);
+    if (rc) return rc;
+    for (int g = 0; g < kMissGroups; g++) {
+        int b, e;
+        miss_group(nm, g, &b, &e);
+        if (e > b) *live |= 1u << g;
+    }
+    return MOE_OK;
+}
+
+// group_slots_kernel for the last lookup, on `st`: grp_slots [kMissGroups][E].
+int cache_launch_group_slots(moe_cache* c, int32_t* grp_slots, cudaStream_t st)
+{
+    ProfScope ps(MOE_PROF_LOOKUP, st);
+    prof_count(MOE_PROF_LOOKUP, 1);
+    group_slots_kernel<<<1, 256, 0, st>>>(c->m, c->shape.experts, grp_slots);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+cudaEvent_t cache_group_event(const moe_cache* c, int g) { return c->ev_grp[g]; }
 
 // The fills of the lookup just enqueued on `st` for `layer`, whichever fill
 // mode the cache is in; `ev` completes once they have landed (recorded on
@@ -708,6 +771,8 @@ extern "C" int moe_cache_create(const moe_shape* shape, void* d_meta, size_t met
         cudaEventCreateWithFlags(&c->ev_pf[0], cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&c->ev_pf[1], cudaEventDisableTiming) != cudaSuccess)
         return fail(MOE_ERR_CUDA);
+    for (cudaEvent_t& e : c->ev_grp)
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return fail(MOE_ERR_CUDA);
     if (c->lookup_smem > 48 * 1024 &&
         cudaFuncSetAttribute(lookup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, c->lookup_smem) !=
             cudaSuccess)
@@ -731,6 +796,8 @@ extern "C" int moe_cache_destroy(moe_cache* c)
     if (c->ev_lookup) cudaEventDestroy(c->ev_lookup);
     if (c->ev_fill) cudaEventDestroy(c->ev_fill);
     for (cudaEvent_t e : c->ev_pf)
+        if (e) cudaEventDestroy(e);
+    for (cudaEvent_t e : c->ev_grp)
         if (e) cudaEventDestroy(e);
     delete c;
     return MOE_OK;

@@ -180,21 +180,44 @@ int launch_ffn_fp4(const moe_shape* s, const void* pool, size_t slot_bytes, int 
 int launch_combine(const uint16_t* y_perm, const int32_t* row_of, const float* w, int n, int k, int H,
                    void* out, int out_dtype, cudaStream_t st);
 
+// ---------------------------------------------------------------- miss groups
+// The misses of a decode layer call are filled, and their FFN run, in up to
+// kMissGroups groups in miss-list order.  The last groups hold one miss
+// each, so only the last miss's FFN waits for the last fill; every earlier
+// group computes while later blobs are still being copied.  Groups are
+// right-aligned: with nm misses, groups g < kMissGroups - min(nm,
+// kMissGroups) are empty, and group g covers misses [*b, *e) of the list.
+constexpr int kMissGroups = 4;
+
+__host__ __device__ static inline void miss_group(int nm, int g, int* b, int* e)
+{
+    const int ng = nm < kMissGroups ? nm : kMissGroups;
+    const int j = g - (kMissGroups - ng);   // index among the ng non-empty groups
+    if (nm <= 0 || j < 0 || g >= kMissGroups) {
+        *b = *e = 0;
+        return;
+    }
+    const int first = nm - ng + 1;           // misses of the first non-empty group
+    *b = j == 0 ? 0 : first + j - 1;
+    *e = j == 0 ? first : first + j;
+}
+
 // ---------------------------------------------------------------- cache internals (cache.cu)
 int cache_launch_lookup(moe_cache* c, int layer, const int32_t* idx, int count, int32_t* slot_user, cudaStream_t st);
 bool cache_layer_resident(const moe_cache* c, int layer);
 const int32_t* cache_slot_all(const moe_cache* c);
 const int32_t* cache_slot_hit(const moe_cache* c);
-const int32_t* cache_slot_miss(const moe_cache* c);
 const char* cache_pool(const moe_cache* c);
 size_t cache_slot_bytes(const moe_cache* c);
 int cache_read_and_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t copy, int* n_miss,
-                        cudaEvent_t ev = nullptr);
-cudaEvent_t cache_fill_event(const moe_cache* c);
+                        cudaEvent_t ev = nullptr, bool groups = false);
+int cache_group_fills(moe_cache* c, int layer, cudaStream_t st, cudaStream_t copy, unsigned* live);
+int cache_launch_group_slots(moe_cache* c, int32_t* grp_slots, cudaStream_t st);
+cudaEvent_t cache_group_event(const moe_cache* c, int g);
 const moe_shape* cache_shape(const moe_cache* c);
 int cache_capacity_int(const moe_cache* c);
 int cache_fill_mode(const moe_cache* c);
-int cache_launch_device_fill(moe_cache* c, int layer, cudaStream_t copy, cudaEvent_t ev = nullptr);
+int cache_launch_device_fill(moe_cache* c, int layer, cudaStream_t copy, cudaEvent_t ev = nullptr, int group = -1);
 int cache_fill(moe_cache* c, int layer, cudaStream_t st, cudaStream_t copy, cudaEvent_t ev);
 cudaEvent_t cache_prefill_event(const moe_cache* c, int i);
 bool cache_front_fits(const moe_cache* c, int n);

@@ -19,6 +19,7 @@ struct LayerWs {
     int32_t* row_of;
     int32_t* assign_of;
     uint16_t* y_perm;
+    int32_t* grp_slots;   // [kMissGroups][E]: slot tables of the miss groups
     void* ffn_ws;
     void* perm_ws;
     size_t bytes;
@@ -37,6 +38,7 @@ static LayerWs layer_ws(const moe_shape* s, int n, void* base)
     size_t o_row = take(4 * A);
     size_t o_asg = take(4 * A);
     size_t o_yp = take(2 * A * H);
+    size_t o_grp = take(4 * (size_t)kMissGroups * E);
     size_t o_ffn = take(ffn_ws_bytes(s, (int)A));
     size_t o_perm = take(permute_ws_bytes(n, s->experts, s->top_k));
     L.bytes = o;
@@ -49,6 +51,7 @@ static LayerWs layer_ws(const moe_shape* s, int n, void* base)
         L.row_of = reinterpret_cast<int32_t*>(b + o_row);
         L.assign_of = reinterpret_cast<int32_t*>(b + o_asg);
         L.y_perm = reinterpret_cast<uint16_t*>(b + o_yp);
+        L.grp_slots = reinterpret_cast<int32_t*>(b + o_grp);
         L.ffn_ws = b + o_ffn;
         L.perm_ws = b + o_perm;
     }
@@ -205,30 +208,32 @@ extern "C" int moe_layer_forward(moe_cache* c, int32_t layer, const void* d_x, i
     const char* pool = cache_pool(c);
     const size_t sb = cache_slot_bytes(c);
     const int C = cache_capacity_int(c);
-    if (cache_fill_mode(c) == MOE_FILL_DEVICE) {
-        // the copy kernel takes the miss list from the lookup on the device:
-        // it starts first (it needs few SMs and only PCIe), the hits run
-        // beside it, the misses after it.  Nothing is read back.
-        if ((rc = cache_launch_device_fill(c, layer, cp))) return rc;
-        if ((rc = launch_ffn(s, pool, sb, C, cache_slot_hit(c), L.offsets, xp, A, L.y_perm, L.ffn_ws, st, gather)))
-            return rc;
-        MOE_CUDA_TRY(cudaStreamWaitEvent(st, cache_fill_event(c), 0));
-        if ((rc = launch_ffn(s, pool, sb, C, cache_slot_miss(c), L.offsets, xp, A, L.y_perm, L.ffn_ws, st, gather)))
-            return rc;
-    } else if (cache_layer_resident(c, layer)) {
+    const bool dev_fill = cache_fill_mode(c) == MOE_FILL_DEVICE;
+    if (!dev_fill && cache_layer_resident(c, layer)) {
         // every expert of this layer is resident: no miss is possible, nothing is read back
         if ((rc = launch_ffn(s, pool, sb, C, cache_slot_all(c), L.offsets, xp, A, L.y_perm, L.ffn_ws, st, gather)))
             return rc;
     } else {
-        // hits first, while the host learns the miss list and issues the fills
+        // Device fills take the miss list from the lookup on the device: the
+        // copy kernels start first (few SMs, only PCIe) and nothing is read
+        // back.  Host fills: the hits run while the host learns the miss list
+        // and issues the copies.  Either way the misses run in miss groups,
+        // each as soon as its blobs have landed, so the FFN of all but the
+        // last miss overlaps the later copies.
+        unsigned live = 0;
+        if (dev_fill && (rc = cache_group_fills(c, layer, st, cp, &live))) return rc;
         if ((rc = launch_ffn(s, pool, sb, C, cache_slot_hit(c), L.offsets, xp, A, L.y_perm, L.ffn_ws, st, gather)))
             return rc;
-        int nm = 0;
-        if ((rc = cache_read_and_fill(c, layer, st, cp, &nm))) return rc;
-        if (nm > 0) {
-            MOE_CUDA_TRY(cudaStreamWaitEvent(st, cache_fill_event(c), 0));
-            if ((rc = launch_ffn(s, pool, sb, C, cache_slot_miss(c), L.offsets, xp, A, L.y_perm, L.ffn_ws, st, gather)))
-                return rc;
+        if (!dev_fill && (rc = cache_group_fills(c, layer, st, cp, &live))) return rc;
+        if (live) {
+            if ((rc = cache_launch_group_slots(c, L.grp_slots, st))) return rc;
+            for (int g = 0; g < kMissGroups; g++) {
+                if (!((live >> g) & 1)) continue;
+                MOE_CUDA_TRY(cudaStreamWaitEvent(st, cache_group_event(c, g), 0));
+                if ((rc = launch_ffn(s, pool, sb, C, L.grp_slots + (size_t)g * E, L.offsets, xp, A, L.y_perm,
+                                     L.ffn_ws, st, gather)))
+                    return rc;
+            }
         }
     }
     return launch_combine(L.y_perm, L.row_of, w, n, k, H, d_out, x_dtype, st);

@@ -107,7 +107,7 @@ typedef struct {
 /* Profiling categories: kernels of each step, and the host->device fills. */
 typedef enum {
     MOE_PROF_ROUTER = 0,  /* router logits + top-k kernels */
-    MOE_PROF_LOOKUP = 1,  /* cache lookup kernel */
+    MOE_PROF_LOOKUP = 1,  /* cache lookup kernel (or the decode front kernel), miss-group slot tables */
     MOE_PROF_PERMUTE = 2, /* histogram, scan, scatter/gather kernels */
     MOE_PROF_FFN = 3,     /* grouped FFN kernels (gate-up, down) */
     MOE_PROF_COMBINE = 4, /* combine kernel */
@@ -413,6 +413,12 @@ int moe_combine(const uint16_t* d_y_perm, const int32_t* d_row_of, const float* 
  * The whole layer for `layer`: router -> cache lookup -> permute -> grouped
  * FFN over the hits -> (fills of the misses on copy_stream, overlapped with
  * the hit FFN) -> grouped FFN over the misses -> combine.
+ * Misses run in up to 4 miss groups in miss-list order (the last groups one
+ * miss each; with nm misses the first non-empty group holds nm - 3 when
+ * nm > 4): each group's FFN call starts once its own blobs have landed, so
+ * only the last miss's FFN follows the last fill.  Results depend on the
+ * grouping (the FFN's split of the work over the SMs does), and are the same
+ * in both fill modes.
  * d_x [n][H] (x_dtype), d_wg [E][H] bf16, d_bias [E] or NULL; d_out [n][H]
  * in x_dtype.  d_ws: moe_layer_workspace_bytes() bytes.  d_topk_idx_out /
  * d_topk_w_out ([n][k], device) receive the routing when not NULL.

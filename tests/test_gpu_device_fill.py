@@ -2,7 +2,8 @@
 
 A copy kernel takes the miss list from the lookup on the device and loads
 the blobs from mapped pinned host memory, so no call reads anything back and
-a decode step with misses can be captured in a CUDA graph.  Checked against
+a decode step with misses can be captured in a CUDA graph.  Misses run in
+miss groups, each FFN pass after its own fills.  Checked against
 the oracle: routing and the cache trace bit-exact on every call, outputs
 within the layer tolerance, slot contents equal to the blobs; and against
 host fills: the same bits.
@@ -224,3 +225,45 @@ def test_device_fill_rejects_pageable_blobs():
     assert ei.value.code == L.MOE_ERR_INVALID_ARG
     assert cache.fill_mode == L.FILL_HOST
     cache.close()
+
+
+@pytest.fixture
+def profiling():
+    A.moe_profile_enable(True)
+    A.moe_profile_read(reset=True)
+    yield
+    A.moe_profile_enable(False)
+    A.moe_profile_read(reset=True)
+
+
+@pytest.mark.parametrize("fill", [L.FILL_HOST, L.FILL_DEVICE], ids=["host", "device"])
+def test_misses_run_in_miss_groups(orc, profiling, fill):
+    """With nm misses a call runs its hit pass, then one FFN pass per miss group:
+    min(nm, 4) with host fills (the host knows nm), always 4 with device fills
+    (the empty ones compute nothing).  Seed 12's stream has calls with 0, 1, 2,
+    3, 4, 5 and 8 misses (oracle router and LRU), so every grouping occurs;
+    outputs and the trace as the oracle gives them."""
+    cfg = SMALL
+    Ly = Layer(cfg, 12)
+    cache = make_cache(Ly)
+    if fill == L.FILL_DEVICE:
+        cache.set_fill_mode(fill)
+    st = Step(cache, cfg, Ly.shape, 4, 12)
+    lru = orc.Lru(1, cfg.experts, cfg.capacity)
+    seen = set()
+    for s in range(12):
+        x = W.gen_x(cfg, 12, 4, "decode", s)
+        out, idx = st.run(x)
+        passes = A.moe_profile_read(reset=True)["ffn"]["timed"]
+        rc, recs, _ = lru.call(0, idx)
+        assert rc == 0
+        assert trace_rows(cache.read_trace()) == _rows(recs), s
+        nm = sum(1 for r in recs if int(r["event"]) == 1)
+        seen.add(nm)
+        assert passes == 1 + (4 if fill == L.FILL_DEVICE else min(nm, 4)), (s, nm, passes)
+        ref, i_ref, _, _ = _oracle_out(orc, Ly, cfg, st, x)
+        np.testing.assert_array_equal(idx, i_ref)
+        err = rel_l2(out, ref)
+        assert err < TOL_REL_L2 and err < ALARM_REL_L2, (s, nm, err)
+    assert {0, 1, 2, 3, 4, 5, 8} <= seen
+    _check_slots(cache, Ly, cfg)
