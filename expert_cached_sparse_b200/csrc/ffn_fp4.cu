@@ -296,6 +296,38 @@ __device__ __forceinline__ uint32_t e2m1_round(float x, float* q)
     return code;
 }
 
+// The E4M3-scaled (NVFP4) counterpart without the division: the nearest
+// E2M1 code of v / s from |v| against the midpoints between neighbouring
+// E2M1 magnitudes times s (mid[], at most 7 significant bits: exact
+// products).  > at the midpoints whose lower neighbour has the even code
+// (0.25, 1.25, 2.5, 5), >= at the others (0.75, 1.75, 3.5): exact ties go to
+// the even code.  The same code e2m1_round takes from the IEEE quotient:
+// rounding is monotone, and for fp32 v other than m s, |v - m s| >= ulp(m s)
+// (when m s is not a power of two; else s is one and the quotient is exact)
+// with s < 2^(e+1) (s = sigma 2^e) keeps |v/s - m| above half an ulp of m,
+// so no quotient rounds onto a midpoint.  NaN -> 0.
+__device__ __forceinline__ uint32_t e2m1_round_scaled(float v, const float (&mid)[7], float* q)
+{
+    const float a = fabsf(v);
+    const uint32_t k = (uint32_t)(a > mid[0]) + (uint32_t)(a >= mid[1]) + (uint32_t)(a > mid[2]) +
+                       (uint32_t)(a >= mid[3]) + (uint32_t)(a > mid[4]) + (uint32_t)(a >= mid[5]) +
+                       (uint32_t)(a > mid[6]);
+    const float mag = k < 4 ? 0.5f * (float)k : (k == 7 ? 6.0f : (float)(k - 2));
+    *q = copysignf(mag, v);
+    return (v < 0.0f && k) ? (k | 8u) : k;
+}
+
+__device__ __forceinline__ void e2m1_midpoints(float s, float (&mid)[7])
+{
+    mid[0] = __fmul_rn(0.25f, s);
+    mid[1] = __fmul_rn(0.75f, s);
+    mid[2] = __fmul_rn(1.25f, s);
+    mid[3] = __fmul_rn(1.75f, s);
+    mid[4] = __fmul_rn(2.5f, s);
+    mid[5] = __fmul_rn(3.5f, s);
+    mid[6] = __fmul_rn(5.0f, s);
+}
+
 
 
 // Per-chunk bytes of a token group's operand image with n rows (n multiple of 8).
@@ -393,12 +425,14 @@ __device__ __forceinline__ void terms8(float (&v)[8], uint32_t (&word)[T], uint3
         scode[t] = term_scale<WFMT>(mx, sval);
         // MXFP4 scales are powers of two: multiplying by the exact reciprocal is the division
         const float inv = WFMT == MOE_W_MXFP4 ? __uint_as_float((254u - scode[t]) << 23) : 0.0f;
+        float mid[7];
+        if (WFMT != MOE_W_MXFP4) e2m1_midpoints(sval, mid);
         uint32_t w = 0;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            const float x = WFMT == MOE_W_MXFP4 ? __fmul_rn(v[i], inv) : __fdiv_rn(v[i], sval);
             float q;
-            w |= e2m1_round(x, &q) << (4 * i);
+            w |= (WFMT == MOE_W_MXFP4 ? e2m1_round(__fmul_rn(v[i], inv), &q) : e2m1_round_scaled(v[i], mid, &q))
+                 << (4 * i);
             v[i] = __fsub_rn(v[i], __fmul_rn(q, sval));
         }
         word[t] = w;
@@ -407,7 +441,9 @@ __device__ __forceinline__ void terms8(float (&v)[8], uint32_t (&word)[T], uint3
 
 // One term of terms8 as a called function (one copy of the code for all
 // callers; the fused decode kernel runs it only a few times per launch, so
-// code size, not issue rate, decides its cost).
+// code size, not issue rate, decides its cost: measured, two items'
+// terms inlined and interleaved ran no faster at batch 16 and 6 us slower
+// per call at batch 1).
 template <int WFMT, int LPB>
 __device__ __noinline__ uint32_t term8(float* v, uint32_t* scode)
 {
@@ -419,12 +455,14 @@ __device__ __noinline__ uint32_t term8(float* v, uint32_t* scode)
     float sval;
     *scode = term_scale<WFMT>(mx, sval);
     const float inv = WFMT == MOE_W_MXFP4 ? __uint_as_float((254u - *scode) << 23) : 0.0f;
+    float mid[7];
+    if (WFMT != MOE_W_MXFP4) e2m1_midpoints(sval, mid);
     uint32_t w = 0;
 #pragma unroll
     for (int i = 0; i < 8; i++) {
-        const float x = WFMT == MOE_W_MXFP4 ? __fmul_rn(v[i], inv) : __fdiv_rn(v[i], sval);
         float q;
-        w |= e2m1_round(x, &q) << (4 * i);
+        w |= (WFMT == MOE_W_MXFP4 ? e2m1_round(__fmul_rn(v[i], inv), &q) : e2m1_round_scaled(v[i], mid, &q))
+             << (4 * i);
         v[i] = __fsub_rn(v[i], __fmul_rn(q, sval));
     }
     return w;
@@ -1134,8 +1172,8 @@ __device__ __forceinline__ int4 plan_group(const Plan& P, int gi, int NT, int bf
 // One quantisation item of one epilogue warp: row r, 256-column chunk c of
 // its K, into the operand image of its token group (32 lanes x 8 columns).
 // qitem_load finds the item's place and loads its 8 values per lane (a warp
-// loads all its items first, so their global-memory latencies overlap);
-// qitem_store computes the terms and writes them.
+// loads two items before computing, so their global-memory latencies
+// overlap); fused_quant_items computes the terms and writes them.
 struct QItem {
     char* cb;          // the item's chunk of its group's operand image (null: skipped row)
     const void* row;   // the source row
@@ -1173,65 +1211,81 @@ __device__ __forceinline__ void qitem_load(QItem& it, const Plan& P, const void*
     load8<IN_F32>(it.row, c * 256 + lane * 8, it.v);
 }
 
+// Largest magnitude of a row of K activations, by one warp (8 loads per
+// lane in flight).
+template <bool IN_F32>
+__device__ __forceinline__ float row_absmax(const void* row, int K, int lane)
+{
+    float mx = 0.0f;
+#pragma unroll 8
+    for (int k = lane * 8; k < K; k += 256) {
+        float u[8];
+        load8<IN_F32>(row, k, u);
+#pragma unroll
+        for (int i = 0; i < 8; i++) mx = fmaxf(mx, fabsf(u[i]));
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    return mx;
+}
+
+// The quantisation items first, first + step, ... (below end) of one
+// epilogue warp, two at a time: both items' loads first, then their terms.
+// An NVFP4 row's scale 2^p comes from its largest magnitude, taken once per
+// source row the warp meets (NVFP4 warps take consecutive items: chunks of
+// a row, then of the next; MXFP4 warps every step-th).  After the first loads are issued, lane 0 arrives on
+// `loaded` (when not null): the copy warp holds its weight prefetch until
+// then, so these few loads do not queue behind megabytes of bulk copies.
 template <int WFMT, int T, bool IN_F32>
-__device__ __forceinline__ void qitem_store(QItem& it, int K, int32_t* rex, int lane)
+__device__ __forceinline__ void fused_quant_items(const Plan& P, const void* in, int K, const int32_t* gather, int gk,
+                                                  char* bimg, int32_t* rex, long first, long step, long end,
+                                                  int lane, uint64_t* loaded)
 {
     using FM = Fmt<WFMT>;
     constexpr int VS = FM::VS, LPB = VS / 8;
-    if (!it.cb) return;
-    const int kin = lane * 8;
-    if (WFMT == MOE_W_NVFP4) {   // the row maximum, by this warp over the whole row
-        float mx = 0.0f;
-#pragma unroll 4
-        for (int k = lane * 8; k < K; k += 256) {
-            float u[8];
-            load8<IN_F32>(it.row, k, u);
-#pragma unroll
-            for (int i = 0; i < 8; i++) mx = fmaxf(mx, fabsf(u[i]));
-        }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const int p = row_exponent(mx);
-        if (it.c == 0 && lane == 0) rex[it.r] = p;
-        const float sc = ldexpf(1.0f, p);
-#pragma unroll
-        for (int i = 0; i < 8; i++) it.v[i] = __fmul_rn(it.v[i], sc);
-    }
-#pragma unroll 1
-    for (int t = 0; t < T; t++) {
-        uint32_t scode;
-        const uint32_t word = term8<WFMT, LPB>(it.v, &scode);
-        const int n = it.n0 + t;
-        *reinterpret_cast<uint32_t*>(it.cb + img_code_off(n, kin)) = word;
-        if ((lane % LPB) == 0) it.cb[img_scale_off<VS>(it.N, n, kin)] = (char)scode;
-    }
-}
-
-// All quantisation items of one epilogue warp, loads first (two at a time).
-// After the first loads are issued, lane 0 arrives on `loaded` (when not
-// null): the copy warp holds its weight prefetch until then, so these few
-// loads do not queue behind megabytes of bulk copies.
-template <int WFMT, int T, bool IN_F32>
-__device__ __forceinline__ void fused_quant_items(const Plan& P, const void* in, int K, const int32_t* gather, int gk,
-                                                  char* bimg, int32_t* rex, long first, long step, long items,
-                                                  int lane, uint64_t* loaded)
-{
-    const int KC = K / 256;
-    for (long i0 = first; i0 < items; i0 += 2 * step) {
+    const int KC = K / 256, kin = lane * 8;
+    const void* p_row = nullptr;   // NVFP4: the source row whose exponent is p (scale sc)
+    int p = 0;
+    float sc = 1.0f;
+    for (long i0 = first; i0 < end; i0 += 2 * step) {
         QItem q[2];
 #pragma unroll
         for (int k = 0; k < 2; k++) {
             const long i = i0 + k * step;
             q[k].cb = nullptr;
-            if (i < items) qitem_load<WFMT, T, IN_F32>(q[k], P, in, K, gather, gk, (int)(i / KC), (int)(i % KC), bimg, lane);
+            if (i < end) qitem_load<WFMT, T, IN_F32>(q[k], P, in, K, gather, gk, (int)(i / KC), (int)(i % KC), bimg, lane);
         }
         if (loaded && i0 == first) {
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(loaded));
             loaded = nullptr;
         }
+        if (WFMT == MOE_W_NVFP4) {
 #pragma unroll
-        for (int k = 0; k < 2; k++) qitem_store<WFMT, T, IN_F32>(q[k], K, rex, lane);
+            for (int k = 0; k < 2; k++) {
+                if (!q[k].cb) continue;   // the same for the whole warp
+                if (q[k].row != p_row) {
+                    p = row_exponent(row_absmax<IN_F32>(q[k].row, K, lane));
+                    sc = ldexpf(1.0f, p);
+                    p_row = q[k].row;
+                }
+                if (q[k].c == 0 && lane == 0) rex[q[k].r] = p;
+#pragma unroll
+                for (int j = 0; j < 8; j++) q[k].v[j] = __fmul_rn(q[k].v[j], sc);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 2; k++) {
+            if (!q[k].cb) continue;
+#pragma unroll 1
+            for (int t = 0; t < T; t++) {
+                uint32_t scode;
+                const uint32_t word = term8<WFMT, LPB>(q[k].v, &scode);
+                const int n = q[k].n0 + t;
+                *reinterpret_cast<uint32_t*>(q[k].cb + img_code_off(n, kin)) = word;
+                if ((lane % LPB) == 0) q[k].cb[img_scale_off<VS>(q[k].N, n, kin)] = (char)scode;
+            }
+        }
     }
     if (loaded && lane == 0) mbar_arrive(smem_u32(loaded));   // no items
 }
@@ -1497,17 +1551,24 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
         unsigned long long gb_next = etid == 0 ? grid_bar_first() : 0ull;
         for (int phase = 0; phase < 2; phase++) {
             const Fp4Args& a = phase ? f.p2 : f.p1;
-            {   // the activation terms of this phase's input rows: (row, chunk) items per warp
-                const long items = (long)rows * (a.K / 256);
-                const long first = (long)blockIdx.x * kEpiWarps + (warp - 2), step = (long)grid * kEpiWarps;
+            {   // the activation terms of this phase's input rows: (row, chunk) items; NVFP4
+                // warps take equal ranges of consecutive items, MXFP4 warps every nw-th
+                const long items = (long)rows * (a.K / 256), nw = (long)grid * kEpiWarps;
+                const long w_ = (long)blockIdx.x * kEpiWarps + (warp - 2), per = (items + nw - 1) / nw;
+                long first = w_, step = nw, end = items;
+                if (WFMT == MOE_W_NVFP4) {
+                    first = w_ * per < items ? w_ * per : items;
+                    step = 1;
+                    end = first + per < items ? first + per : items;
+                }
                 if (phase == 1)
-                    fused_quant_items<WFMT, T, true>(P, f.p1.out_h, a.K, nullptr, 1, f.bh, f.rex_h, first, step, items,
+                    fused_quant_items<WFMT, T, true>(P, f.p1.out_h, a.K, nullptr, 1, f.bh, f.rex_h, first, step, end,
                                                      lane, nullptr);
                 else if (f.x_f32)
-                    fused_quant_items<WFMT, T, true>(P, f.x, a.K, f.gather, f.gk, f.bx, f.rex_x, first, step, items,
+                    fused_quant_items<WFMT, T, true>(P, f.x, a.K, f.gather, f.gk, f.bx, f.rex_x, first, step, end,
                                                      lane, xloaded);
                 else
-                    fused_quant_items<WFMT, T, false>(P, f.x, a.K, f.gather, f.gk, f.bx, f.rex_x, first, step, items,
+                    fused_quant_items<WFMT, T, false>(P, f.x, a.K, f.gather, f.gk, f.bx, f.rex_x, first, step, end,
                                                       lane, xloaded);
             }
             ok = grid_sync_epi(etid, s_flag, f.p1.wait, gb_next) && ok;   // terms published (phase 0: counters zero)

@@ -14,7 +14,7 @@ import torch
 from expert_cached_sparse_b200 import api as A
 from expert_cached_sparse_b200 import workloads as W
 
-from helpers import ALARM_REL_L2, TOL_REL_L2, Layer, bf16_bits, dev, host, rel_l2
+from helpers import ALARM_REL_L2, TOL_REL_L2, Layer, bf16_bits, dev, host, make_cache, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -308,3 +308,55 @@ def test_ffn_is_deterministic_and_scale_exact(path, counts, monkeypatch):
     f1 = W.bf16_bits_to_f32(y1.view(np.uint16))
     f3 = W.bf16_bits_to_f32(y3.view(np.uint16))
     np.testing.assert_array_equal(f3, 2 * f1)
+
+
+@pytest.mark.parametrize("base", [W.DS_DECODE, W.TRACE40], ids=["mxfp4", "nvfp4"])
+def test_fused_decode_ffn_matches_the_separate_kernels_bitwise(base, monkeypatch):
+    """The fused decode kernel encodes x and h itself (two items per warp,
+    interleaved; NVFP4 row exponents once per row a warp meets); the separate
+    decode-tile kernels take both encodings from fp4_terms_kernel, whose codes
+    are bit-exact with the oracle (test_act_terms_bit_exact).  With the same
+    stream-K split the two paths must give the same bits, at full expert size,
+    for ragged groups, single rows, and rows of every expert."""
+    monkeypatch.setenv("MOE_FFN_TILE", "decode")
+    cfg = W.scaled(base, experts=6, top_k=2, layers=1)
+    shape = A.shape_of(cfg)
+    blobs = [A.moe_pack_expert(shape, W.gen_expert(cfg, 11, 0, e)) for e in range(cfg.experts)]
+    rng = np.random.default_rng(21)
+    for counts in ([1, 3, 2, 9, 0, 1], [16, 0, 1, 5, 12, 2], [1, 0, 0, 0, 0, 0], [4, 4, 4, 4, 4, 4]):
+        x = rng.standard_normal((int(sum(counts)), cfg.hidden)).astype(np.float32)
+        x[0] *= 1e-3                                  # a row far below the others (NVFP4 row exponent)
+        xb = W.f32_to_bf16_bits(x)
+        monkeypatch.delenv("MOE_FFN_UNFUSED", raising=False)
+        y_fused = _ffn_run(cfg, blobs, counts, xb, "decode", monkeypatch)
+        monkeypatch.setenv("MOE_FFN_UNFUSED", "1")
+        y_sep = _ffn_run(cfg, blobs, counts, xb, "decode", monkeypatch)
+        np.testing.assert_array_equal(y_fused, y_sep)
+        assert A.L.lib.moe_get_device_error(1) == 0
+
+
+def test_fused_decode_layer_matches_the_separate_kernels_bitwise(monkeypatch):
+    """The same through moe_layer_forward, where the fused kernel gathers x rows
+    from the tokens (a token routed to k experts is one source row of k items)."""
+    cfg = W.scaled(W.TRACE40, experts=32, top_k=4, layers=1, capacity=32)
+    Ly = Layer(cfg, 13)
+    wg, bias = dev(W.gen_wg(cfg, 13, 0)), dev(W.gen_bias(cfg, 13, 0, 0))
+    outs = []
+    for unfused in (False, True):
+        if unfused:
+            monkeypatch.setenv("MOE_FFN_UNFUSED", "1")
+        else:
+            monkeypatch.delenv("MOE_FFN_UNFUSED", raising=False)
+        cache = make_cache(Ly)
+        res = []
+        for s in range(3):
+            x = dev(W.gen_x(cfg, 13, 16, "decode", s))
+            out = torch.empty(16, cfg.hidden, dtype=torch.bfloat16, device="cuda")
+            ws = torch.empty(A.moe_layer_workspace_bytes(Ly.shape, 16), dtype=torch.uint8, device="cuda")
+            A.moe_layer_forward(cache, 0, x, wg, bias, out, ws)
+            torch.cuda.synchronize()
+            res.append(host(out))
+        outs.append(res)
+        cache.close()
+    for a, b in zip(*outs):
+        np.testing.assert_array_equal(a, b)
