@@ -299,12 +299,14 @@ class DecodeStream:
                                  copy_stream=self.copy, topk_idx_out=self.idx[s])
 
 
-# DRAM bytes (read + write) per grouped-FFN call of the headline decode
-# stream (one launch of the fused decode kernel per call), averaged over the
-# four calls of an ncu capture of that workload (the hit and miss passes of
-# two steps).  Valid only for the FFN code it was measured on (comments
-# aside): other code reports null.
-FFN_TRAFFIC = {"source_sha1": "70725fa1423008d4dc351207abe4d4af39b2a0c0", "bytes_per_call": 244677120}
+# DRAM bytes (read + write) of the grouped-FFN calls of the headline decode
+# stream (one launch of the fused decode kernel per call: the hit pass and
+# the miss groups) over their algorithmic bytes, both summed over every call
+# of the timed steps of an ncu capture of that workload.  Calls differ in
+# size by two orders of magnitude, so the ratio, times this run's
+# algorithmic bytes per call, is what is reported per call.  Valid only for
+# the FFN code it was measured on (comments aside): other code reports null.
+FFN_TRAFFIC = {"source_sha1": "", "dram_over_algorithmic": None}
 
 
 def ffn_source_sha1():
@@ -321,8 +323,11 @@ def ffn_source_sha1():
     return hashlib.sha1(code.encode()).hexdigest()
 
 
-def ffn_traffic():
-    return FFN_TRAFFIC["bytes_per_call"] if ffn_source_sha1() == FFN_TRAFFIC["source_sha1"] else None
+def ffn_traffic(algorithmic_bytes_per_call):
+    r = FFN_TRAFFIC["dram_over_algorithmic"]
+    if r is None or ffn_source_sha1() != FFN_TRAFFIC["source_sha1"]:
+        return None
+    return r * algorithmic_bytes_per_call
 
 
 def ffn_algorithmic_bytes(idx_steps, cfg, slot_bytes):
@@ -498,7 +503,8 @@ def run_ours(args, cfg, world, rank, local_rank):
     line["roofline"] = {"kernel": "grouped SwiGLU FFN call (ffn_fp4_fused_kernel: x terms, gate-up, h terms, "
                                   "down; block-scaled tcgen05)",
                         "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                        "frac": achieved / hbm_peak, "peak_kind": peak_kind, "traffic": ffn_traffic(),
+                        "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+                        "traffic": ffn_traffic(ffn_bytes / ffn_calls),
                         "algorithmic_bytes_per_call": ffn_bytes / ffn_calls,
                         "avg_call_ms": ffn_ms / ffn_calls, "calls": ffn_calls}
     # Bp before and after the timed region (the PCIe path can be shared with

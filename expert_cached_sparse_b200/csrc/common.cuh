@@ -170,13 +170,15 @@ int ffn_device_error(int clear);   // BF16 streaming FFN's device error word (0:
 long long test_wait_cycles(long long dflt);
 int test_withhold();
 int ffn_fp4_device_error(int clear);   // FP4 FFN's device error word (0: none)
+// one_expert: the pass computes at most one expert (a miss group after the
+// first), so the FP4 decode tiles run on a grid sized for one expert's work.
 int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
                const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,
-               cudaStream_t st, const RowSource* gather = nullptr);
+               cudaStream_t st, const RowSource* gather = nullptr, bool one_expert = false);
 size_t ffn_fp4_ws_bytes(const moe_shape* s, int rows);
 int launch_ffn_fp4(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
                    const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,
-                   cudaStream_t st, const RowSource* gather);
+                   cudaStream_t st, const RowSource* gather, bool one_expert);
 int launch_combine(const uint16_t* y_perm, const int32_t* row_of, const float* w, int n, int k, int H,
                    void* out, int out_dtype, cudaStream_t st);
 

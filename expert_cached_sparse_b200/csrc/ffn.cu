@@ -709,12 +709,13 @@ int ffn_device_error(int clear)
 
 int launch_ffn(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
                const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,
-               cudaStream_t st, const RowSource* gather)
+               cudaStream_t st, const RowSource* gather, bool one_expert)
 {
     if (rows == 0) return MOE_OK;
     ProfScope ps(MOE_PROF_FFN, st);
     if (s->wfmt != MOE_W_BF16)
-        return launch_ffn_fp4(s, pool, slot_bytes, pool_slots, slot_of, offsets, x_perm, rows, y_perm, ws, st, gather);
+        return launch_ffn_fp4(s, pool, slot_bytes, pool_slots, slot_of, offsets, x_perm, rows, y_perm, ws, st, gather,
+                              one_expert);
     FfnWs w;
     ffn_ws_layout(s, rows, ws, &w);
     int dev = 0, sms = 148;

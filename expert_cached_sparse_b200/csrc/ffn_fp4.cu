@@ -35,6 +35,7 @@
 // Every wait is bounded (the limit is a kernel argument, about 2 s unless a
 // test shortens it); a timeout records MOE_ERR_TIMEOUT, raises the CTA's
 // abort flag so the other roles drain, and the kernel returns.
+#include <algorithm>
 #include <stdlib.h>
 #include <string.h>
 
@@ -1065,7 +1066,11 @@ __global__ void __launch_bounds__(SepCfg<CFG>::THREADS, 1) ffn_fp4_kernel(Fp4Arg
 // the same value) and barrier k completes when the counter reaches that value
 // plus (k + 1) x grid.  Arrival is one release add, waiting is acquire loads;
 // every wait is bounded.  Clearing the error word resets the counter.
-__device__ unsigned long long g_gb_count;   // grid-barrier arrivals since the last clear
+// Grid-barrier arrivals since the last clear, one counter per grid size: a
+// launch finds its base by rounding its counter down to a multiple of its
+// grid, which holds only if every earlier launch on that counter had the
+// same grid (a one-expert pass runs on fewer CTAs than a full one).
+__device__ unsigned long long g_gb_count[kMaxCtas + 1];
 __device__ int g_gb_abort;                  // set when a CTA gave up; cleared with the error word
 
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p)
@@ -1112,7 +1117,7 @@ struct FusedCfg {
 // thread 0, before its first arrival).
 __device__ __forceinline__ unsigned long long grid_bar_first()
 {
-    const unsigned long long c = ld_acquire_u64(&g_gb_count);
+    const unsigned long long c = ld_acquire_u64(&g_gb_count[gridDim.x]);
     return c - c % gridDim.x + gridDim.x;
 }
 
@@ -1129,9 +1134,9 @@ __device__ __forceinline__ bool grid_sync_epi(int etid, volatile int* s_flag, lo
     epi_bar();
     if (etid == 0) {
         bool ok = !*reinterpret_cast<volatile int*>(&g_gb_abort);
-        red_release_add_u64(&g_gb_count, 1ull);
+        red_release_add_u64(&g_gb_count[gridDim.x], 1ull);
         const long long t0 = clock64();
-        while (ld_acquire_u64(&g_gb_count) < next) {
+        while (ld_acquire_u64(&g_gb_count[gridDim.x]) < next) {
             if (*reinterpret_cast<volatile int*>(&g_gb_abort)) { ok = false; break; }
             if (clock64() - t0 > limit) {
                 ok = false;
@@ -1927,10 +1932,10 @@ int ffn_fp4_device_error(int clear)
     if (clear && v) {
         // the kernels are not running: put the grid barrier back in its idle state too
         const int z = 0;
-        const unsigned long long zu = 0;
+        const unsigned long long zu[kMaxCtas + 1] = {};
         if (cudaMemcpyToSymbol(g_fp4_error, &z, sizeof z) != cudaSuccess ||
             cudaMemcpyToSymbol(g_gb_abort, &z, sizeof z) != cudaSuccess ||
-            cudaMemcpyToSymbol(g_gb_count, &zu, sizeof zu) != cudaSuccess)
+            cudaMemcpyToSymbol(g_gb_count, zu, sizeof zu) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
     return v;
@@ -1938,7 +1943,7 @@ int ffn_fp4_device_error(int clear)
 
 int launch_ffn_fp4(const moe_shape* s, const void* pool, size_t slot_bytes, int pool_slots, const int32_t* slot_of,
                    const int32_t* offsets, const uint16_t* x_perm, int rows, uint16_t* y_perm, void* ws,
-                   cudaStream_t st, const RowSource* gather)
+                   cudaStream_t st, const RowSource* gather, bool one_expert)
 {
     Fp4Ws w;
     fp4_ws_layout(s, rows, ws, &w);
@@ -1948,6 +1953,14 @@ int launch_ffn_fp4(const moe_shape* s, const void* pool, size_t slot_bytes, int 
     const RowSource src = gather ? *gather : RowSource{x_perm, MOE_DT_BF16, nullptr, 1};
     const BlobLayout bl = blob_layout(s);
     const bool pre = use_prefill_tiles(s, rows);
+    if (one_expert && !pre) {
+        // One expert's decode pass is latency-bound: about 16 gate-up chunks
+        // per CTA (32 CTAs for H = 4096, F = 2048) beat one chunk-sliver per SM
+        // (measured, one expert and two rows: 45 us on 148 CTAs, 37 on 64, 31.5
+        // on 32).  The stream-K split, and so the bits, follow the grid.
+        const int cap = (2 * s->ffn / 128) * (s->hidden / 256) / 16;
+        sms = std::min(sms, std::max(8, cap));
+    }
     if (!pre && !getenv("MOE_FFN_UNFUSED")) {
         const int rc = s->wfmt == MOE_W_MXFP4
                            ? run_fp4_fused<MOE_W_MXFP4>(s, bl, pool, slot_bytes, pool_slots, slot_of, offsets, rows,

@@ -230,8 +230,9 @@ extern "C" int moe_layer_forward(moe_cache* c, int32_t layer, const void* d_x, i
             for (int g = 0; g < kMissGroups; g++) {
                 if (!((live >> g) & 1)) continue;
                 MOE_CUDA_TRY(cudaStreamWaitEvent(st, cache_group_event(c, g), 0));
+                // groups after the first hold one miss at most (miss_group)
                 if ((rc = launch_ffn(s, pool, sb, C, L.grp_slots + (size_t)g * E, L.offsets, xp, A, L.y_perm,
-                                     L.ffn_ws, st, gather)))
+                                     L.ffn_ws, st, gather, g > 0)))
                     return rc;
             }
         }
