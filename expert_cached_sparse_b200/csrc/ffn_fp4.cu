@@ -1407,7 +1407,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_fp4_fused_kernel(FusedArgs f)
     const int grid = gridDim.x;
     const int NG = P.gpre[E];
     if (NG == 0) {
-        // no expert with rows has a slot (a miss pass without misses): every
+        // no expert with rows has a slot (an empty miss-group pass): every
         // CTA sees the same plan and leaves before the first grid barrier
         tc_fence_before();
         __syncthreads();

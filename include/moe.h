@@ -251,11 +251,13 @@ int moe_cache_resize(moe_cache* cache, void* d_meta_new, size_t meta_bytes, void
  *   MOE_FILL_DEVICE: a copy kernel on copy_stream reads the miss list where
  *   the lookup kernel wrote it and copies each missing blob from pinned host
  *   memory, mapped into the device's address space, into its slot (zero-copy
- *   loads over PCIe by 16 CTAs).  No call reads anything back, so
+ *   loads over PCIe by 16 CTAs; moe_layer_forward launches it once per miss
+ *   group, each launch copying its group's part of the list).  No call reads
+ *   anything back, so
  *   moe_cache_lookup_update and moe_layer_forward never block the host and a
  *   whole decode step, misses included, can be captured in a CUDA graph.
  *   The kernel waits for nothing on the device (stream order sequences it
- *   after the lookup and before the miss-pass FFN), so it has no timeout.
+ *   after the lookup and before the misses' FFN passes), so it has no timeout.
  *   Requires every blob of h_blobs to be 16-byte aligned page-locked host
  *   memory mapped into the device's address space (cudaHostAlloc /
  *   cudaMallocHost memory on a system with unified addressing, or
