@@ -234,6 +234,100 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(const void* __
     }
 }
 
+// The same block of logits for bf16 x, with the operand slices copied
+// raw (bf16) by cp.async into two buffers: the copies of slice s+1 are in
+// flight while slice s is multiplied, and each lane widens its own x and
+// gate chunks exactly when it reads them.  Lane l still owns chunk l of
+// every slice and multiplies its 8 elements in order, so every logit is
+// the same fp32 value as above.  Rows past n (or E) and chunks past H are
+// zero-filled by the copy itself (source size 0).
+__device__ __forceinline__ void cp_async16(void* smem, const void* src, uint32_t bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+                 "l"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void widen8(uint4 q, float v[8])
+{
+    const uint32_t u4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        v[2 * j] = __uint_as_float(u4[j] << 16);
+        v[2 * j + 1] = __uint_as_float(u4[j] & 0xFFFF0000u);
+    }
+}
+
+__global__ void __launch_bounds__(256, 2) router_logits_pipe_kernel(const uint16_t* __restrict__ x,
+                                                                    const uint16_t* __restrict__ wg,
+                                                                    const float* __restrict__ bias, int n, int H,
+                                                                    int E, float* __restrict__ logits)
+{
+    __shared__ __align__(16) uint16_t xs[2][RT_TOK][RT_K];
+    __shared__ __align__(16) uint16_t ws[2][RT_EXP][RT_K];
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int t0 = blockIdx.x * RT_TOK, e0 = blockIdx.y * RT_EXP;
+    const int nsl = (H + RT_K - 1) / RT_K;
+    auto stage = [&](int buf, int k0) {
+        for (int i = tid; i < RT_TOK * RT_K / 8; i += 256) {
+            const int r = i / (RT_K / 8), c = i % (RT_K / 8), t = t0 + r, k = k0 + 8 * c;
+            const bool ok = t < n && k < H;
+            cp_async16(&xs[buf][r][8 * c], ok ? x + (size_t)t * H + k : x, ok ? 16u : 0u);
+        }
+        for (int i = tid; i < RT_EXP * RT_K / 8; i += 256) {
+            const int r = i / (RT_K / 8), c = i % (RT_K / 8), e = e0 + r, k = k0 + 8 * c;
+            const bool ok = e < E && k < H;
+            cp_async16(&ws[buf][r][8 * c], ok ? wg + (size_t)e * H + k : wg, ok ? 16u : 0u);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    float acc[4][RT_EXP];
+#pragma unroll
+    for (int a = 0; a < 4; a++)
+#pragma unroll
+        for (int b = 0; b < RT_EXP; b++) acc[a][b] = 0.0f;
+    stage(0, 0);
+    for (int s = 0; s < nsl; s++) {
+        const int buf = s & 1, k0 = s * RT_K;
+        if (s + 1 < nsl) {
+            stage(buf ^ 1, k0 + RT_K);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");   // slice s has landed
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();
+        if (k0 + 8 * lane < H) {   // lane's chunk exists in this slice
+            float xv[4][8];
+#pragma unroll
+            for (int a = 0; a < 4; a++) widen8(*reinterpret_cast<const uint4*>(&xs[buf][4 * w + a][8 * lane]), xv[a]);
+#pragma unroll
+            for (int b = 0; b < RT_EXP; b++) {
+                float wv[8];
+                widen8(*reinterpret_cast<const uint4*>(&ws[buf][b][8 * lane]), wv);
+#pragma unroll
+                for (int a = 0; a < 4; a++)
+#pragma unroll
+                    for (int i = 0; i < 8; i++) acc[a][b] = __fmaf_rn(xv[a][i], wv[i], acc[a][b]);
+            }
+        }
+        __syncthreads();   // buffer `buf` is refilled by the next iteration's copies
+    }
+#pragma unroll
+    for (int a = 0; a < 4; a++)
+#pragma unroll
+        for (int b = 0; b < RT_EXP; b++)
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1)
+                acc[a][b] = __fadd_rn(acc[a][b], __shfl_xor_sync(0xffffffffu, acc[a][b], off));
+#pragma unroll
+    for (int a = 0; a < 4; a++) {
+        const int t = t0 + 4 * w + a;
+#pragma unroll
+        for (int b = 0; b < RT_EXP; b++)
+            if (lane == b && t < n && e0 + b < E)
+                logits[(size_t)t * E + e0 + b] = bias ? __fadd_rn(acc[a][b], __ldg(bias + e0 + b)) : acc[a][b];
+    }
+}
+
 // Warp per token: k rounds of arg-max, then exp(l - lmax) renormalised.
 __global__ void __launch_bounds__(128) router_topk_kernel(const float* __restrict__ logits, int n,
                                                           int E, int k, int32_t* __restrict__ idx,
@@ -299,7 +393,11 @@ int launch_logits(const void* x, const uint16_t* wg, const float* bias, int n, i
     const int threads = 256, wpb = threads / 32;
     if (n >= 64) {
         dim3 grid((n + RT_TOK - 1) / RT_TOK, (E + RT_EXP - 1) / RT_EXP);
-        router_logits_tiled_kernel<XF32><<<grid, 256, 0, st>>>(x, wg, bias, n, H, E, logits);
+        if constexpr (XF32)
+            router_logits_tiled_kernel<XF32><<<grid, 256, 0, st>>>(x, wg, bias, n, H, E, logits);
+        else
+            router_logits_pipe_kernel<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), wg, bias, n, H, E,
+                                                             logits);
     } else {
         constexpr int TB = 1, EB = 1;
         long units = (long)E * n;
