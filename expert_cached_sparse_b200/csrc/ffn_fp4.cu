@@ -278,23 +278,37 @@ __device__ __forceinline__ uint32_t term_scale(float m, float& sval)
     return code;
 }
 
-// Nearest E2M1 value of x, ties to the even code (NaN -> 0): returns the
-// code and leaves the value in *q.  |x| is rounded to the E2M1 grid by
-// adding and removing a power of two whose ulp is the grid step there (0.5
-// below 2, 1 below 4, 2 above), which rounds to the nearest even multiple
-// exactly like the even-code rule; the code is read off the result's
-// exponent and top mantissa bit (0.5 and 0 by hand).
-__device__ __forceinline__ uint32_t e2m1_round(float x, float* q)
+// Nearest E2M1 codes of 8 values |x| <= 6, ties to the even code (the
+// hardware's round-to-nearest-even conversion to E2M1, which is that rule),
+// NaN taken as 0 and a zero magnitude with the + sign (code 0); column i in
+// bits 4i..4i+3 of the result, the codes' values in q[].
+__device__ __forceinline__ uint32_t e2m1x8_round(const float (&x)[8], float (&q)[8])
 {
-    const float a = fabsf(x);
-    const float c = a < 2.0f ? 4194304.0f : (a < 4.0f ? 8388608.0f : 16777216.0f);
-    float v = fminf(__fsub_rn(__fadd_rn(a, c), c), 6.0f);
-    v = a == a ? v : 0.0f;
-    const uint32_t b = __float_as_uint(v);
-    uint32_t code = v >= 1.0f ? (b >> 22) - 252u : (v > 0.0f ? 1u : 0u);
-    if (x < 0.0f && code) code |= 8u;
-    *q = copysignf(v, x);
-    return code;
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) y[i] = x[i] == x[i] ? x[i] : 0.0f;
+    uint32_t w;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(w)
+        : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+    const uint32_t m = w & 0x77777777u;
+    w = m | (w & ((m + 0x77777777u) & 0x88888888u));   // -0 -> +0: sign kept only on a nonzero magnitude
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 h0, h1, h2, h3;\n\t"
+        ".reg .b16 l0, u0, l1, u1, l2, u2, l3, u3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %8;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h0, b0;\n\tcvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h2, b2;\n\tcvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
+        "mov.b32 {l0, u0}, h0;\n\tmov.b32 {l1, u1}, h1;\n\tmov.b32 {l2, u2}, h2;\n\tmov.b32 {l3, u3}, h3;\n\t"
+        "cvt.f32.f16 %0, l0;\n\tcvt.f32.f16 %1, u0;\n\tcvt.f32.f16 %2, l1;\n\tcvt.f32.f16 %3, u1;\n\t"
+        "cvt.f32.f16 %4, l2;\n\tcvt.f32.f16 %5, u2;\n\tcvt.f32.f16 %6, l3;\n\tcvt.f32.f16 %7, u3;\n\t}"
+        : "=f"(q[0]), "=f"(q[1]), "=f"(q[2]), "=f"(q[3]), "=f"(q[4]), "=f"(q[5]), "=f"(q[6]), "=f"(q[7])
+        : "r"(w));
+    return w;
 }
 
 // The E4M3-scaled (NVFP4) counterpart without the division: the nearest
@@ -302,7 +316,7 @@ __device__ __forceinline__ uint32_t e2m1_round(float x, float* q)
 // E2M1 magnitudes times s (mid[], at most 7 significant bits: exact
 // products).  > at the midpoints whose lower neighbour has the even code
 // (0.25, 1.25, 2.5, 5), >= at the others (0.75, 1.75, 3.5): exact ties go to
-// the even code.  The same code e2m1_round takes from the IEEE quotient:
+// the even code.  The same code as the nearest one to the IEEE quotient:
 // rounding is monotone, and for fp32 v other than m s, |v - m s| >= ulp(m s)
 // (when m s is not a power of two; else s is one and the quotient is exact)
 // with s < 2^(e+1) (s = sigma 2^e) keeps |v/s - m| above half an ulp of m,
@@ -426,15 +440,23 @@ __device__ __forceinline__ void terms8(float (&v)[8], uint32_t (&word)[T], uint3
         scode[t] = term_scale<WFMT>(mx, sval);
         // MXFP4 scales are powers of two: multiplying by the exact reciprocal is the division
         const float inv = WFMT == MOE_W_MXFP4 ? __uint_as_float((254u - scode[t]) << 23) : 0.0f;
-        float mid[7];
-        if (WFMT != MOE_W_MXFP4) e2m1_midpoints(sval, mid);
         uint32_t w = 0;
+        if (WFMT == MOE_W_MXFP4) {
+            float x[8], q[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-            float q;
-            w |= (WFMT == MOE_W_MXFP4 ? e2m1_round(__fmul_rn(v[i], inv), &q) : e2m1_round_scaled(v[i], mid, &q))
-                 << (4 * i);
-            v[i] = __fsub_rn(v[i], __fmul_rn(q, sval));
+            for (int i = 0; i < 8; i++) x[i] = __fmul_rn(v[i], inv);
+            w = e2m1x8_round(x, q);
+#pragma unroll
+            for (int i = 0; i < 8; i++) v[i] = __fsub_rn(v[i], __fmul_rn(q[i], sval));
+        } else {
+            float mid[7];
+            e2m1_midpoints(sval, mid);
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                float q;
+                w |= e2m1_round_scaled(v[i], mid, &q) << (4 * i);
+                v[i] = __fsub_rn(v[i], __fmul_rn(q, sval));
+            }
         }
         word[t] = w;
     }
@@ -456,15 +478,23 @@ __device__ __noinline__ uint32_t term8(float* v, uint32_t* scode)
     float sval;
     *scode = term_scale<WFMT>(mx, sval);
     const float inv = WFMT == MOE_W_MXFP4 ? __uint_as_float((254u - *scode) << 23) : 0.0f;
-    float mid[7];
-    if (WFMT != MOE_W_MXFP4) e2m1_midpoints(sval, mid);
     uint32_t w = 0;
+    if (WFMT == MOE_W_MXFP4) {
+        float x[8], q[8];
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-        float q;
-        w |= (WFMT == MOE_W_MXFP4 ? e2m1_round(__fmul_rn(v[i], inv), &q) : e2m1_round_scaled(v[i], mid, &q))
-             << (4 * i);
-        v[i] = __fsub_rn(v[i], __fmul_rn(q, sval));
+        for (int i = 0; i < 8; i++) x[i] = __fmul_rn(v[i], inv);
+        w = e2m1x8_round(x, q);
+#pragma unroll
+        for (int i = 0; i < 8; i++) v[i] = __fsub_rn(v[i], __fmul_rn(q[i], sval));
+    } else {
+        float mid[7];
+        e2m1_midpoints(sval, mid);
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            float q;
+            w |= e2m1_round_scaled(v[i], mid, &q) << (4 * i);
+            v[i] = __fsub_rn(v[i], __fmul_rn(q, sval));
+        }
     }
     return w;
 }

@@ -399,11 +399,19 @@ int launch_logits(const void* x, const uint16_t* wg, const float* bias, int n, i
             router_logits_pipe_kernel<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), wg, bias, n, H, E,
                                                              logits);
     } else {
-        constexpr int TB = 1, EB = 1;
-        long units = (long)E * n;
-        int grid = (int)((units + wpb - 1) / wpb);
-        if (grid > sms * 8) grid = sms * 8;
-        router_logits_kernel<XF32, TB, EB, 8><<<grid, threads, 0, st>>>(x, wg, bias, n, H, E, logits);
+        // from 8 tokens a warp takes 2 tokens x 2 experts: each gate-row load
+        // serves two tokens and each activation load two experts (measured 2.6 us
+        // faster per 16-token call; 2.4 us slower at 1-4 tokens, which keep a warp
+        // per pair).  The per-lane order, and so every logit, is the same.
+        auto grid_for = [&](int TB, int EB) {
+            const long units = (long)((E + EB - 1) / EB) * ((n + TB - 1) / TB);
+            const int g = (int)((units + wpb - 1) / wpb);
+            return g > sms * 8 ? sms * 8 : g;
+        };
+        if (n >= 8)
+            router_logits_kernel<XF32, 2, 2, 4><<<grid_for(2, 2), threads, 0, st>>>(x, wg, bias, n, H, E, logits);
+        else
+            router_logits_kernel<XF32, 1, 1, 8><<<grid_for(1, 1), threads, 0, st>>>(x, wg, bias, n, H, E, logits);
     }
     MOE_LAUNCH_CHECK();
     return MOE_OK;
